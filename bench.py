@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the fused WTConv layer on B200: one step = forward +
+input gradient + weight gradient over one synthetic batch.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload stage1|stage2|train_bf16|tiny]
+
+Prints one JSON line (rank 0).  Metric: modeled minimum HBM bytes of the three
+calls divided by their device time (GB/s), the achieved fraction of the
+measured HBM peak, and microseconds per call.  Modeled bytes per step:
+6*N*e + 4*P (x read + y written, dy read + dx written, x and dy read; P the
+float32 parameter bytes, read by every call and written once as gradients).
+
+Timing: CUDA events on the launching stream around each call, after W warm-up
+steps; L2 is flushed (a 256 MiB write) before every call; K steps between a
+barrier + synchronize on both sides; the max over ranks.  With N > 1 every
+rank runs its own batch (weak scaling) and the weight gradients are summed
+over ranks with one NCCL all-reduce per step (data parallel).
+
+`--impl reference` times the CPU oracle (the reference arm) on the host cores
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "WTConv fwd+bwd HBM GB/s and % of 8 TB/s roofline; µs/call at WTConvNeXt shapes"
+FALLBACK_HBM_GBS = 6650.0
+SMS, FP32_LANES, MAX_SM_MHZ = 148, 128, 1965.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="stage1")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# Workload arithmetic (the modeled minimum traffic and the conv FMA count).
+# --------------------------------------------------------------------------
+def param_floats(c) -> int:
+    return c.C * c.k * c.k * (1 + 4 * c.L) + 2 * c.C + 4 * c.L * c.C
+
+
+def modeled_bytes(c) -> dict:
+    N, e, P = c.numel, c.esize, 4 * param_floats(c)
+    return {"fwd": 2 * N * e + P, "bwd_in": 2 * N * e + P, "bwd_w": 2 * N * e + 2 * P}
+
+
+def conv_fmas(c) -> float:
+    """Algorithmic multiply-adds of one call: base conv + every subband conv."""
+    return c.numel * c.k * c.k * (1.0 + sum(4.0 ** -l for l in range(c.L)))
+
+
+def workload_name(c) -> str:
+    return (f"{c.name}: B={c.B} C={c.C} H={c.H} W={c.W} k={c.k} L={c.L} {c.dtype} NCHW, "
+            f"forward + backward_input + backward_weight")
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------------
+# Clock sampling during the timed region.
+# --------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, enabled: bool, gpu_index: int):
+        self.proc = None
+        self.path = None
+        self.gpu = gpu_index
+        if enabled:
+            try:
+                fd, self.path = tempfile.mkstemp(suffix=".csv")
+                os.close(fd)
+                self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                              "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                time.sleep(0.3)
+            except Exception:
+                self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8 or not f[0].isdigit() or int(f[0]) != self.gpu:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[4:8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
+        top = max(r[0] for r in rows)
+        under_load = [r[0] for r in rows if r[0] >= 0.5 * top] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(under_load), "sm_max_mhz": rows[0][1], "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# Distributed plumbing.
+# --------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def physical_gpu_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids) and ids[local].isdigit():
+            return int(ids[local])
+    return local
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the reported CPU baseline).
+# --------------------------------------------------------------------------
+def oracle_sample(case, seconds: float, max_planes: int | None = None):
+    """Time the oracle's three calls on whole batch elements (all channels),
+    one batch element at a time, until `seconds` elapse.  Returns (modeled
+    bytes processed, wall seconds, planes, cores, description)."""
+    import numpy as np
+
+    import oracle
+    from wtconv_inputs import make_inputs
+
+    orc = oracle.default()
+    sub = case.with_(B=1)
+    done_planes, t_total, nbytes = 0, 0.0, 0
+    b = 0
+    mb = modeled_bytes(sub)
+    per_b = sum(mb.values())
+    while True:
+        inp = make_inputs(sub.with_(seed=case.seed + b))
+        p = {k: inp[k].double().numpy() for k in ("base_w", "base_b", "base_scale", "wt_w", "wt_scale")}
+        x, dy = inp["x"].double().numpy(), inp["dy"].double().numpy()
+        t0 = time.perf_counter()
+        orc.forward(x, p["base_w"], p["base_b"], p["base_scale"], p["wt_w"], p["wt_scale"], case.L)
+        orc.backward_input(dy, p["base_w"], p["base_scale"], p["wt_w"], p["wt_scale"], case.L)
+        orc.backward_weight(x, dy, p["base_w"], p["base_b"], p["base_scale"], p["wt_w"], p["wt_scale"], case.L)
+        t_total += time.perf_counter() - t0
+        nbytes += per_b
+        done_planes += case.C
+        b += 1
+        if t_total >= seconds or b >= case.B or (max_planes and done_planes >= max_planes):
+            break
+    desc = (f"{b} of {case.B} batch elements x all {case.C} channels "
+            f"({done_planes} planes), forward + backward_input + backward_weight in float64")
+    return nbytes, t_total, done_planes, orc.num_threads(), desc
+
+
+def run_reference(args, case):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    # Calibrate one batch element, then size each step to keep the run short.
+    nbytes, t1, _, cores, _ = oracle_sample(case, 0.0)
+    budget = 120.0
+    steps = max(1, args.steps)
+    per_step_target = max(0.05, budget / (steps + args.warmup))
+    n_b = max(1, min(case.B, int(per_step_target / max(t1, 1e-6))))
+    sub = case.with_(B=n_b)
+    for _ in range(args.warmup):
+        oracle_sample(sub, 0.0, max_planes=1)
+    t_sum, b_sum = 0.0, 0
+    for _ in range(steps):
+        nb, t, _, _, _ = oracle_sample(sub, 1e9)
+        t_sum += t
+        b_sum += nb
+    value = b_sum / t_sum / 1e9
+    ms = 1e3 * t_sum / steps
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(case), "sample_batch_per_step": n_b},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_b} of {case.B} batch elements x all {case.C} channels per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# The CUDA path.
+# --------------------------------------------------------------------------
+def run_ours(args, case):
+    import torch
+    import torch.distributed as dist
+
+    import memory_bound_cnn_wtconv_b200 as wt
+    from wtconv_inputs import make_inputs
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wt.load_library()
+
+    my_case = case.with_(seed=case.seed + 7919 * rank)
+    inp = make_inputs(my_case)
+    g = {k: v.to(dev) for k, v in inp.items()}
+    L = case.L
+    y = torch.empty_like(g["x"])
+    dx = torch.empty_like(g["dy"])
+    grads = dict(base_w=torch.empty_like(g["base_w"]), base_b=torch.empty_like(g["base_b"]),
+                 base_scale=torch.empty_like(g["base_scale"]), wt_w=torch.empty_like(g["wt_w"]),
+                 wt_scale=torch.empty_like(g["wt_scale"]))
+    flat = torch.empty(sum(v.numel() for v in grads.values()), device=dev)
+    ws = torch.empty(max(16, wt.workspace_bytes(g["x"].shape, case.k, L, g["x"].dtype)), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        wt.forward(g["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L, y=y, stream=stream)
+
+    def bwd_in():
+        wt.backward_input(g["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], L, dx=dx, stream=stream)
+
+    def bwd_w():
+        wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
+                           grads=grads, workspace=ws, stream=stream)
+
+    def allreduce():
+        torch.cat([v.reshape(-1) for v in grads.values()], out=flat)
+        dist.all_reduce(flat)
+
+    calls = [("fwd", fwd), ("bwd_in", bwd_in), ("bwd_w", bwd_w)]
+    if world > 1:
+        calls.append(("allreduce", allreduce))
+
+    for _ in range(args.warmup):
+        for _, f in calls:
+            flush.zero_()
+            f()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(K)]
+    clocks = Clocks(not args.no_clocks, physical_gpu_index(local))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.perf_counter()
+    for s in range(K):
+        for i, (_, f) in enumerate(calls):
+            flush.zero_()
+            ev[s][i][0].record(stream)
+            f()
+            ev[s][i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+
+    per_call = {name: sum(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(K)) / K
+                for i, (name, _) in enumerate(calls)}
+    step_ms = sum(per_call.values())
+    if world > 1:
+        t = torch.tensor([step_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+
+    mb = modeled_bytes(case)
+    step_bytes = sum(mb.values())
+    value = step_bytes * world / (step_ms * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+
+    # Dominant kernel (largest share of the step) and its roofline.
+    dom = max(("fwd", "bwd_in", "bwd_w"), key=lambda n: per_call[n])
+    dom_s = per_call[dom] * 1e-3
+    flops = 2.0 * conv_fmas(case)
+    alu_peak = SMS * FP32_LANES * 2 * MAX_SM_MHZ * 1e6 / 1e12  # TFLOP/s
+    alu_achieved = flops / dom_s / 1e12
+    hbm_achieved = mb[dom] / dom_s / 1e9
+    t_alu, t_hbm = flops / (alu_peak * 1e12), mb[dom] / (peak * 1e9)
+    kernel_names = {"fwd": "wtconv_fused_kernel (forward)", "bwd_in": "wtconv_fused_kernel (input gradient)",
+                    "bwd_w": "wtconv_bwdw_partial_kernel + wtconv_bwdw_finish_kernel"}
+    if t_alu >= t_hbm:
+        roof = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                "frac": alu_achieved / alu_peak, "traffic": None, "kernel": kernel_names[dom],
+                "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 x 1965 MHz (unit counts x max clock)",
+                "flops_per_launch": flops}
+    else:
+        roof = {"bound": "hbm", "achieved": hbm_achieved, "peak": peak, "unit": "GB/s", "frac": hbm_achieved / peak,
+                "traffic": None, "kernel": kernel_names[dom], "peak_source": peak_kind,
+                "bytes_per_launch": mb[dom]}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if case.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": workload_name(case), "global_batch": case.B * world,
+                   "parallelism": f"dp{world}", "l2": "flushed before every call (256 MiB write)",
+                   "modeled_bytes_per_step": step_bytes},
+        "hbm_frac_of_peak": value / world / peak, "hbm_peak_gbs": peak, "hbm_peak_source": peak_kind,
+        "frac_of_8tbs": value / world / 8000.0,
+        "us_per_call": {k: v * 1e3 for k, v in per_call.items()},
+        "gbs_per_call": {k: mb[k] / (per_call[k] * 1e-3) / 1e9 for k in mb},
+        "roofline": roof,
+        "alu_frac_per_call": {k: 2.0 * conv_fmas(case) / (per_call[k] * 1e-3) / 1e12 / alu_peak
+                              for k in ("fwd", "bwd_in", "bwd_w")},
+        "gpu_launches": K * 4, "wall_s_timed_region": wall,
+    }
+    if clk is not None:
+        line["clocks"] = clk
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, case, g, y, dx, grads, ws, dev, stream, world, calls)
+    if world > 1:
+        dist.barrier()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nb, t, planes, cores, desc = oracle_sample(case, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": nb / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": t}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e(args, case, g, y, dx, grads, ws, dev, stream, world, calls):
+    """Same metric through the public API with host buffers: pinned host ->
+    device copies of x and dy, the three calls, device -> host copies of y,
+    dx and the gradients, every step."""
+    import torch
+    import torch.distributed as dist
+
+    xh = g["x"].cpu().pin_memory()
+    dyh = g["dy"].cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    dxh = torch.empty_like(dyh).pin_memory()
+    gh = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()}
+    K = args.e2e_steps
+
+    def step():
+        g["x"].copy_(xh, non_blocking=True)
+        g["dy"].copy_(dyh, non_blocking=True)
+        for name, f in calls:
+            f()
+        yh.copy_(y, non_blocking=True)
+        dxh.copy_(dx, non_blocking=True)
+        for k in grads:
+            gh[k].copy_(grads[k], non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / K
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    step_bytes = sum(modeled_bytes(case).values())
+    h2d = xh.numel() * xh.element_size() + dyh.numel() * dyh.element_size()
+    d2h = yh.numel() * yh.element_size() + dxh.numel() * dxh.element_size() + sum(
+        v.numel() * 4 for v in gh.values())
+    return {"value": step_bytes * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K}
+
+
+def main():
+    args = parse()
+    from wtconv_inputs import NAMED
+    if args.workload not in NAMED:
+        raise SystemExit(f"unknown workload {args.workload}; choose from {sorted(NAMED)}")
+    case = NAMED[args.workload]
+    if case.name == "tiny":
+        case = case.with_(calls=("fwd", "bwd_in", "bwd_w"))
+    if args.impl == "reference":
+        return run_reference(args, case)
+    return run_ours(args, case)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,127 @@
+/*
+ * wtconv.h -- C ABI of the B200 (sm_100a) wavelet-convolution (WTConv) library.
+ *
+ * The layer (arXiv 2608.10805, "Fast and Memory-Efficient Wavelet
+ * Convolutions via I/O-Aware Reformulation", Abstract) is, per sample b and
+ * channel c, the sum of two branches on an H x W plane:
+ *
+ *   base branch:     yb = base_scale[c] * (dwconv(x, base_w[c]) + base_b[c])
+ *   wavelet branch:  an L-level orthonormal 2-D Haar analysis that splits the
+ *                    plane into LL/LH/HL/HH subbands and recurses on the raw
+ *                    LL subband; every subband s of level l gets its own
+ *                    depthwise k x k conv scaled by wt_scale[l][c][s]; the
+ *                    inverse Haar synthesis adds each coarser level's
+ *                    reconstruction into the next finer LL.
+ *   y = yb + (wavelet branch)
+ *
+ * dwconv is cross-correlation with "same" zero padding (p = k/2) at each
+ * subband's own resolution.  Subband order: 0 = LL, 1 = LH (high-pass along
+ * H, i.e. between rows), 2 = HL (high-pass along W), 3 = HH.  One Haar step
+ * maps the 2x2 block (a b / c d) to ((a+b+c+d), (a+b-c-d), (a-b+c-d),
+ * (a-b-c+d)) / 2.
+ *
+ * The kernels apply the abstract's three reformulations: the Haar analysis
+ * is recomputed on chip for every level (nothing but x is read from HBM), the
+ * synthesis is one pass over the output indexed by the bits of the output
+ * coordinates (nothing but y is written), and the per-channel and
+ * per-subband scales are folded into the conv weights before the convs run.
+ *
+ * Conventions for every entry point:
+ *   - Layouts.  Activations are NCHW, contiguous, stored as float32 or bf16
+ *     (desc->dtype); arithmetic is float32.  Parameters and gradients are
+ *     float32, contiguous:  base_w [C][k][k], base_b [C], base_scale [C],
+ *     wt_w [L][C][4][k][k], wt_scale [L][C][4].
+ *   - Pointers are DEVICE pointers on the current device; activation pointers
+ *     must be 16-byte aligned and W must be a multiple of 4.
+ *   - Ownership.  The caller owns every buffer.  The library allocates
+ *     nothing, keeps no pointer after returning, and never synchronises: all
+ *     work is enqueued on `stream` (0 = the legacy default stream).
+ *   - Gradients are overwritten, not accumulated.
+ *   - Errors.  Arguments are validated on the host before any launch; a
+ *     non-OK status means nothing was enqueued and no output was touched.
+ *     A launch failure returns WTCONV_ERR_CUDA.  Faults of an enqueued kernel
+ *     surface at the caller's next synchronisation, as for any CUDA call.
+ *   - Limits: k in {1, 3, 5, 7}; 0 <= L <= 6; H and W divisible by 2^L;
+ *     planes too large for the on-chip staging return WTCONV_ERR_UNSUPPORTED.
+ *   - L = 0 is the base branch only; wt_w and wt_scale may then be NULL.
+ *   - Calls are reentrant; the library holds no global state.
+ */
+#ifndef WTCONV_H
+#define WTCONV_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *wtconv_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    WTCONV_OK = 0,
+    WTCONV_ERR_NULLPTR = 1,     /* a required pointer is NULL */
+    WTCONV_ERR_BAD_SHAPE = 2,   /* B, C, H or W <= 0, or H, W not divisible by 2^L, or W % 4 != 0 */
+    WTCONV_ERR_BAD_K = 3,       /* k not in {1, 3, 5, 7} */
+    WTCONV_ERR_BAD_L = 4,       /* L < 0 or L > 6 */
+    WTCONV_ERR_MISALIGNED = 5,  /* an activation pointer is not 16-byte aligned */
+    WTCONV_ERR_DTYPE = 6,       /* unknown activation dtype */
+    WTCONV_ERR_WORKSPACE = 7,   /* workspace missing or smaller than wtconv_workspace_bytes() */
+    WTCONV_ERR_UNSUPPORTED = 8, /* valid shape that this build cannot stage on chip */
+    WTCONV_ERR_CUDA = 9         /* a CUDA runtime call or kernel launch failed */
+} wtconv_status_t;
+
+typedef enum { WTCONV_F32 = 0, WTCONV_BF16 = 1 } wtconv_dtype_t; /* activation storage */
+
+typedef struct {
+    int B, C, H, W; /* batch, channels, height, width */
+    int k;          /* odd depthwise kernel size, shared by the base and subband convs */
+    int L;          /* number of wavelet decomposition levels */
+    int dtype;      /* a wtconv_dtype_t value */
+} wtconv_desc_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *wtconv_status_string(wtconv_status_t s);
+
+/* Bytes of device workspace wtconv_backward_weight needs for `d` (0 if `d`
+ * is invalid).  The forward and input-gradient calls need none. */
+size_t wtconv_workspace_bytes(const wtconv_desc_t *d);
+
+/* Forward pass: y = WTConv(x).  x, y: [B][C][H][W] in desc->dtype; x and y
+ * must not overlap.  Reads x once and writes y once. */
+wtconv_status_t wtconv_forward(const wtconv_desc_t *d, const void *x,
+                               const float *base_w, const float *base_b, const float *base_scale,
+                               const float *wt_w, const float *wt_scale,
+                               void *y, wtconv_stream_t stream);
+
+/* Gradient with respect to the input: dx = J^T dy, the transpose of the
+ * forward map (the same pass run on dy with every kernel rotated by 180
+ * degrees and no bias).  dy, dx: [B][C][H][W] in desc->dtype; must not
+ * overlap. */
+wtconv_status_t wtconv_backward_input(const wtconv_desc_t *d, const void *dy,
+                                      const float *base_w, const float *base_scale,
+                                      const float *wt_w, const float *wt_scale,
+                                      void *dx, wtconv_stream_t stream);
+
+/* Gradients with respect to every parameter, summed over the batch and all
+ * positions (overwritten):
+ *   d_base_w[c][u][v]   = base_scale[c] * sum dy[h][w] x[h+u-p][w+v-p]
+ *   d_base_b[c]         = base_scale[c] * sum dy
+ *   d_base_scale[c]     = sum dy * (dwconv(x, base_w[c]) + base_b[c])
+ *   d_wt_w[l][c][s]     = wt_scale[l][c][s] * sum D_{l,s}[i][j] S_{l,s}[i+u-p][j+v-p]
+ *   d_wt_scale[l][c][s] = sum D_{l,s} * dwconv(S_{l,s}, wt_w[l][c][s])
+ * with S / D the Haar subbands of x / dy.  The reduction order is fixed, so
+ * repeated calls return bitwise-identical results.  `workspace` (device,
+ * at least wtconv_workspace_bytes(d) bytes) holds per-block partial sums. */
+wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, const void *dy,
+                                       const float *base_w, const float *base_b, const float *base_scale,
+                                       const float *wt_w, const float *wt_scale,
+                                       float *d_base_w, float *d_base_b, float *d_base_scale,
+                                       float *d_wt_w, float *d_wt_scale,
+                                       void *workspace, size_t workspace_bytes,
+                                       wtconv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WTCONV_H */

@@ -1,0 +1,186 @@
+// C ABI of the WTConv library: argument validation, on-chip planning and
+// kernel dispatch.  Declarations and contracts: include/wtconv.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "../../include/wtconv.h"
+#include "wtconv_kernels.cuh"
+#include "wtconv_launch.h"
+#include "wtconv_plan.h"
+#include "wtconv_planner.h"
+
+namespace wtc {
+
+namespace {
+
+cudaError_t launch_fused(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cudaStream_t s) {
+    switch (P.k) {
+        case 1: return launch_fused_k1(P, dtype, bwd, a, s);
+        case 3: return launch_fused_k3(P, dtype, bwd, a, s);
+        case 5: return launch_fused_k5(P, dtype, bwd, a, s);
+        case 7: return launch_fused_k7(P, dtype, bwd, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_bwdw(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
+    switch (P.k) {
+        case 1: return launch_bwdw_k1(P, dtype, a, s);
+        case 3: return launch_bwdw_k3(P, dtype, a, s);
+        case 5: return launch_bwdw_k5(P, dtype, a, s);
+        case 7: return launch_bwdw_k7(P, dtype, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+size_t workspace_floats(const Plan& P) { return (size_t)P.C * P.groups * P.nv; }
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Weight gradient, stage 2: one CTA per channel sums the groups' partials in
+// a fixed order and turns them into the five parameter gradients.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) wtconv_bwdw_finish_kernel(
+    const float* __restrict__ part, int groups, int nv, int C, int k, int L,
+    const float* __restrict__ base_w, const float* __restrict__ base_b, const float* __restrict__ base_scale,
+    const float* __restrict__ wt_w, const float* __restrict__ wt_scale, float* __restrict__ d_base_w,
+    float* __restrict__ d_base_b, float* __restrict__ d_base_scale, float* __restrict__ d_wt_w,
+    float* __restrict__ d_wt_scale) {
+    extern __shared__ float gsum[];
+    const int c = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const int KK = k * k, ncls = 1 + 4 * L;
+    for (int t = tid; t < nv; t += nt) {
+        float s = 0.f;
+        for (int g = 0; g < groups; ++g) s += part[((size_t)c * groups + g) * nv + t];
+        gsum[t] = s;
+    }
+    __syncthreads();
+    const float sdy = gsum[ncls * KK];
+    const float bs = base_scale[c];
+    for (int t = tid; t < KK; t += nt) d_base_w[c * KK + t] = bs * gsum[t];
+    if (tid == 0) {
+        d_base_b[c] = bs * sdy;
+        float s = 0.f;
+        for (int t = 0; t < KK; ++t) s = fmaf(base_w[c * KK + t], gsum[t], s);
+        d_base_scale[c] = fmaf(base_b[c], sdy, s);
+    }
+    for (int t = tid; t < 4 * L * KK; t += nt) {
+        const int k2 = t / KK, tap = t - k2 * KK;
+        const int l = k2 >> 2, s = k2 & 3;
+        const int pi = (l * C + c) * 4 + s;
+        d_wt_w[pi * KK + tap] = wt_scale[pi] * (gsum[(1 + k2) * KK + tap] * quarter_pow(l));
+    }
+    for (int t = tid; t < 4 * L; t += nt) {
+        const int l = t >> 2, s = t & 3;
+        const int pi = (l * C + c) * 4 + s;
+        const float q = quarter_pow(l);
+        float a = 0.f;
+        for (int tap = 0; tap < KK; ++tap) a = fmaf(wt_w[pi * KK + tap], gsum[(1 + t) * KK + tap] * q, a);
+        d_wt_scale[pi] = a;
+    }
+}
+
+cudaError_t launch_bwdw_finish(const Plan& P, const float* part, const float* base_w, const float* base_b,
+                               const float* base_scale, const float* wt_w, const float* wt_scale,
+                               float* d_base_w, float* d_base_b, float* d_base_scale, float* d_wt_w,
+                               float* d_wt_scale, cudaStream_t s) {
+    wtconv_bwdw_finish_kernel<<<P.C, 128, (size_t)P.nv * 4, s>>>(part, P.groups, P.nv, P.C, P.k, P.L, base_w,
+                                                                 base_b, base_scale, wt_w, wt_scale, d_base_w,
+                                                                 d_base_b, d_base_scale, d_wt_w, d_wt_scale);
+    return cudaGetLastError();
+}
+
+}  // namespace wtc
+
+using namespace wtc;
+
+extern "C" {
+
+const char* wtconv_status_string(wtconv_status_t s) {
+    switch (s) {
+        case WTCONV_OK: return "ok";
+        case WTCONV_ERR_NULLPTR: return "a required pointer is NULL";
+        case WTCONV_ERR_BAD_SHAPE: return "bad shape (B, C, H, W > 0; H, W divisible by 2^L; W % 4 == 0)";
+        case WTCONV_ERR_BAD_K: return "unsupported kernel size (k must be 1, 3, 5 or 7)";
+        case WTCONV_ERR_BAD_L: return "unsupported level count (0 <= L <= 6)";
+        case WTCONV_ERR_MISALIGNED: return "activation pointer not 16-byte aligned";
+        case WTCONV_ERR_DTYPE: return "unknown activation dtype";
+        case WTCONV_ERR_WORKSPACE: return "workspace missing or too small";
+        case WTCONV_ERR_UNSUPPORTED: return "plane too large to stage on chip for this build";
+        case WTCONV_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+size_t wtconv_workspace_bytes(const wtconv_desc_t* d) {
+    if (validate(d) != WTCONV_OK) return 0;
+    Plan P;
+    if (make_plan(d, kBackwardWeight, &P) != WTCONV_OK) return 0;
+    return workspace_floats(P) * sizeof(float);
+}
+
+wtconv_status_t wtconv_forward(const wtconv_desc_t* d, const void* x, const float* base_w, const float* base_b,
+                               const float* base_scale, const float* wt_w, const float* wt_scale, void* y,
+                               wtconv_stream_t stream) {
+    wtconv_status_t st = validate(d);
+    if (st != WTCONV_OK) return st;
+    if (!x || !y || !base_w || !base_b || !base_scale) return WTCONV_ERR_NULLPTR;
+    if (d->L > 0 && (!wt_w || !wt_scale)) return WTCONV_ERR_NULLPTR;
+    if (!aligned16(x) || !aligned16(y)) return WTCONV_ERR_MISALIGNED;
+    Plan P;
+    st = make_plan(d, kForward, &P);
+    if (st != WTCONV_OK) return st;
+    FusedArgs a{x, base_w, base_b, base_scale, wt_w, wt_scale, y};
+    return launch_fused(P, d->dtype, false, a, (cudaStream_t)stream) == cudaSuccess ? WTCONV_OK
+                                                                                   : WTCONV_ERR_CUDA;
+}
+
+wtconv_status_t wtconv_backward_input(const wtconv_desc_t* d, const void* dy, const float* base_w,
+                                      const float* base_scale, const float* wt_w, const float* wt_scale,
+                                      void* dx, wtconv_stream_t stream) {
+    wtconv_status_t st = validate(d);
+    if (st != WTCONV_OK) return st;
+    if (!dy || !dx || !base_w || !base_scale) return WTCONV_ERR_NULLPTR;
+    if (d->L > 0 && (!wt_w || !wt_scale)) return WTCONV_ERR_NULLPTR;
+    if (!aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_MISALIGNED;
+    Plan P;
+    st = make_plan(d, kBackwardInput, &P);
+    if (st != WTCONV_OK) return st;
+    // base_b is unused by the transpose; pass base_scale as a valid pointer.
+    FusedArgs a{dy, base_w, base_scale, base_scale, wt_w, wt_scale, dx};
+    return launch_fused(P, d->dtype, true, a, (cudaStream_t)stream) == cudaSuccess ? WTCONV_OK
+                                                                                  : WTCONV_ERR_CUDA;
+}
+
+wtconv_status_t wtconv_backward_weight(const wtconv_desc_t* d, const void* x, const void* dy,
+                                       const float* base_w, const float* base_b, const float* base_scale,
+                                       const float* wt_w, const float* wt_scale, float* d_base_w,
+                                       float* d_base_b, float* d_base_scale, float* d_wt_w,
+                                       float* d_wt_scale, void* workspace, size_t workspace_bytes,
+                                       wtconv_stream_t stream) {
+    wtconv_status_t st = validate(d);
+    if (st != WTCONV_OK) return st;
+    if (!x || !dy || !base_w || !base_b || !base_scale || !d_base_w || !d_base_b || !d_base_scale)
+        return WTCONV_ERR_NULLPTR;
+    if (d->L > 0 && (!wt_w || !wt_scale || !d_wt_w || !d_wt_scale)) return WTCONV_ERR_NULLPTR;
+    if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_MISALIGNED;
+    Plan P;
+    st = make_plan(d, kBackwardWeight, &P);
+    if (st != WTCONV_OK) return st;
+    if (!workspace || workspace_bytes < workspace_floats(P) * sizeof(float)) return WTCONV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
+    float* part = static_cast<float*>(workspace);
+    BwdwArgs a{x, dy, part};
+    cudaStream_t s = (cudaStream_t)stream;
+    if (launch_bwdw(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    if (launch_bwdw_finish(P, part, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                           d_wt_w, d_wt_scale, s) != cudaSuccess)
+        return WTCONV_ERR_CUDA;
+    return WTCONV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,184 @@
+// Host-side argument validation and on-chip planning for the WTConv kernels.
+// Plain C++ (no CUDA types), so that the planner can also be compiled by a
+// host compiler to check every shared-memory access the kernels make.
+#pragma once
+
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "../../include/wtconv.h"
+#include "wtconv_plan.h"
+
+namespace wtc {
+
+constexpr int kSmemLimitFloats = 227 * 1024 / 4;
+constexpr int kNumSMs = 148;  // B200; only used to size the weight-gradient grid
+
+enum Kind { kForward = 0, kBackwardInput = 1, kBackwardWeight = 2 };
+
+inline int round4(int v) { return (v + 3) & ~3; }
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Row stride (floats, multiple of 4) of a buffer read by tiles laid out
+// ntc per tile row.  Consecutive lanes walk the tile columns and wrap to the
+// next tile row (TR rows down), so TR * stride/4 == ntc (mod 8) puts each
+// quarter-warp's 16-byte accesses on 8 distinct bank groups.
+inline int pick_stride(int min_floats, int TR, int ntc) {
+    const int s = round4(min_floats);
+    for (int t = 0; t < 8; ++t) {
+        const int c = s + 4 * t;
+        if ((((TR * (c / 4) - ntc) % 8) + 8) % 8 == 0) return c;
+    }
+    return s;
+}
+
+// Work-weighted fraction of tile slack for tile height TR (smaller is better).
+inline double tile_waste(const wtconv_desc_t* d, int TR) {
+    double used = 0.0, total = 0.0;
+    used += d->H;
+    total += ceil_div(d->H, TR) * (double)TR;
+    for (int l = 0; l < d->L; ++l) {
+        const int n = d->H >> (l + 1);
+        const double w = 1.0 / (double)(1 << (2 * l));  // level-l work relative to the base conv
+        used += w * n;
+        total += w * ceil_div(n, TR) * (double)TR;
+    }
+    return total / used;
+}
+
+inline bool is_supported_k(int k) { return k == 1 || k == 3 || k == 5 || k == 7; }
+
+inline wtconv_status_t validate(const wtconv_desc_t* d) {
+    if (!d) return WTCONV_ERR_NULLPTR;
+    if (d->dtype != WTCONV_F32 && d->dtype != WTCONV_BF16) return WTCONV_ERR_DTYPE;
+    if (d->B <= 0 || d->C <= 0 || d->H <= 0 || d->W <= 0) return WTCONV_ERR_BAD_SHAPE;
+    if (!is_supported_k(d->k)) return WTCONV_ERR_BAD_K;
+    if (d->L < 0 || d->L > kMaxL) return WTCONV_ERR_BAD_L;
+    if ((d->H % (1 << d->L)) != 0 || (d->W % (1 << d->L)) != 0) return WTCONV_ERR_BAD_SHAPE;
+    if ((d->W % 4) != 0) return WTCONV_ERR_BAD_SHAPE;
+    // Index arithmetic in the kernels is 32-bit within a plane and 64-bit across planes.
+    if ((long long)d->H * d->W > (1LL << 30)) return WTCONV_ERR_BAD_SHAPE;
+    if ((long long)d->B * d->C > (1LL << 31) - 1) return WTCONV_ERR_BAD_SHAPE;
+    return WTCONV_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
+    memset(P, 0, sizeof(*P));
+    P->B = d->B; P->C = d->C; P->H = d->H; P->W = d->W; P->k = d->k; P->L = d->L;
+    const int p = d->k / 2, k = d->k, L = d->L, H = d->H, W = d->W;
+    P->p = p;
+    P->TC = 4;
+    P->TR = tile_waste(d, 7) < tile_waste(d, 8) ? 7 : 8;
+    const int TR = P->TR, TC = P->TC;
+    const int WV4 = 4 * ((TC + k - 1 + 3) / 4);  // floats read per window row
+
+    P->ntr[kMaxL] = ceil_div(H, TR);
+    P->ntc[kMaxL] = ceil_div(W, TC);
+    for (int l = 0; l < L; ++l) {
+        P->ntr[l] = ceil_div(H >> (l + 1), TR);
+        P->ntc[l] = ceil_div(W >> (l + 1), TC);
+    }
+
+    long long off = 0;
+    const int ncls = 1 + 4 * L;
+    if (kind != kBackwardWeight) {
+        P->wcls = round4(k * k);
+        P->wbase = (int)off;
+        off += (long long)ncls * P->wcls;
+        P->bias = (int)off;
+        off += 4;
+    }
+    // Padded input plane.
+    {
+        const int ntc = P->ntc[kMaxL];
+        const int rows = P->ntr[kMaxL] * TR + 2 * p;
+        const int need = std::max(W + 2 * p, (ntc - 1) * TC + WV4);
+        P->X.stride = pick_stride(need, TR, ntc);
+        P->X.base = (int)off;
+        off += round4(rows * P->X.stride);
+    }
+    // Padded subbands of every level.
+    for (int l = 0; l < L; ++l) {
+        const int m = W >> (l + 1);
+        const int ntc = P->ntc[l];
+        const int rows = P->ntr[l] * TR + 2 * p;
+        const int need = std::max(m + 2 * p, (ntc - 1) * TC + WV4);
+        P->S[l].stride = pick_stride(need, TR, ntc);
+        P->S[l].sub = round4(rows * P->S[l].stride);
+        P->S[l].base = (int)off;
+        off += 4LL * P->S[l].sub;
+    }
+    // Tile-rounded, unpadded planes: conv outputs (forward) or dy subbands.
+    for (int l = 0; l < L; ++l) {
+        const int ntc = P->ntc[l];
+        const int rows = P->ntr[l] * TR;
+        P->Q[l].stride = pick_stride(ntc * TC, TR, ntc);
+        P->Q[l].sub = round4(rows * P->Q[l].stride);
+        P->Q[l].base = (int)off;
+        off += 4LL * P->Q[l].sub;
+    }
+    if (kind != kBackwardWeight) {
+        if (L >= 2) {
+            // Coarse-level sum at half resolution; S[0] is dead by then.
+            P->Z.stride = round4(W >> 1);
+            P->Z.base = P->S[0].base;
+            if ((long long)(H >> 1) * P->Z.stride > 4LL * P->S[0].sub) return WTCONV_ERR_UNSUPPORTED;
+        }
+    } else {
+        const int ntc = P->ntc[kMaxL];
+        const int rows = P->ntr[kMaxL] * TR;
+        P->DY.stride = pick_stride(ntc * TC, TR, ntc);
+        P->DY.base = (int)off;
+        off += round4(rows * P->DY.stride);
+    }
+
+    // Tiles and threads.
+    int nsub = 0;
+    P->sub_begin[0] = 0;
+    for (int l = 0; l < L; ++l)
+        for (int s = 0; s < 4; ++s) {
+            nsub += P->ntr[l] * P->ntc[l];
+            P->sub_begin[1 + 4 * l + s] = nsub;
+        }
+    P->n_sub_tiles = nsub;
+    P->n_base_tiles = P->ntr[kMaxL] * P->ntc[kMaxL];
+    P->cls_begin[0] = 0;
+    P->cls_begin[1] = P->n_base_tiles;
+    for (int cl = 1; cl < ncls; ++cl) {
+        const int l = (cl - 1) >> 2;
+        P->cls_begin[cl + 1] = P->cls_begin[cl] + P->ntr[l] * P->ntc[l];
+    }
+    P->n_all_tiles = P->cls_begin[ncls];
+    P->nv = ncls * k * k + 1;
+
+    if (kind == kBackwardWeight) {
+        const int nt = ceil_div(P->n_all_tiles, 32) * 32;
+        if (nt > 512) return WTCONV_ERR_UNSUPPORTED;
+        P->nthreads = std::max(nt, 64);
+        // Reduction scratch aliases the (then dead) buffers from offset 0.
+        P->red = 0;
+        const long long red_need = (long long)P->nthreads * (k * k + 1);
+        off = std::max(off, red_need);
+        // Batch groups: about two CTAs per SM, and a divisor of B so every
+        // group walks the same number of planes.
+        const int target = std::max(1, ceil_div(2 * kNumSMs, d->C));
+        int g = 1;
+        for (int cand = 1; cand <= std::min(target, d->B); ++cand)
+            if (d->B % cand == 0) g = cand;
+        P->groups = g;
+    } else {
+        const int nt = ceil_div(std::max(P->n_sub_tiles, P->n_base_tiles), 32) * 32;
+        P->nthreads = std::min(std::max(nt, 64), 512);
+        P->groups = 1;
+    }
+    off = round4((int)std::min<long long>(off, 1LL << 30));
+    if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
+    P->smem_floats = (int)off;
+    return WTCONV_OK;
+}
+
+}  // namespace wtc

@@ -1,0 +1,117 @@
+"""C ABI checks that need no GPU.
+
+The library must load and export every function declared in include/wtconv.h,
+and argument validation (done on the host before any CUDA call) must return
+the documented status codes.  Pointers passed here are never dereferenced:
+each case fails validation before any launch.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import memory_bound_cnn_wtconv_b200 as w
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wtconv.h")
+
+OK, NULLPTR, BAD_SHAPE, BAD_K, BAD_L, MISALIGNED, DTYPE, WORKSPACE, UNSUPPORTED, CUDA = range(10)
+FAKE = 0x10000  # 16-byte aligned, never dereferenced
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(wtconv_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for n in ("wtconv_forward", "wtconv_backward_input", "wtconv_backward_weight", "wtconv_workspace_bytes",
+              "wtconv_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(cuda_lib):
+    for name in declared_functions():
+        assert hasattr(cuda_lib, name), name
+
+
+def _desc(B=2, C=3, H=16, W=16, k=5, L=2, dtype=0):
+    return w.Desc(B, C, H, W, k, L, dtype)
+
+
+def _fwd(lib, d, x=FAKE, y=FAKE, ww=FAKE, ws=FAKE):
+    p = ctypes.c_void_p
+    return lib.wtconv_forward(ctypes.byref(d) if d is not None else None, p(x), p(FAKE), p(FAKE), p(FAKE),
+                              p(ww), p(ws), p(y), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), BAD_SHAPE), (dict(C=-1), BAD_SHAPE), (dict(H=0), BAD_SHAPE),
+    (dict(k=4), BAD_K), (dict(k=9), BAD_K), (dict(k=0), BAD_K),
+    (dict(L=-1), BAD_L), (dict(L=7), BAD_L),
+    (dict(H=12, L=3), BAD_SHAPE), (dict(W=20, L=3), BAD_SHAPE), (dict(W=6, L=1), BAD_SHAPE),
+    (dict(dtype=2), DTYPE),
+])
+def test_forward_validation(cuda_lib, kw, code):
+    assert _fwd(cuda_lib, _desc(**kw)) == code
+
+
+def test_null_and_alignment(cuda_lib):
+    assert _fwd(cuda_lib, None) == NULLPTR
+    assert _fwd(cuda_lib, _desc(), x=0) == NULLPTR
+    assert _fwd(cuda_lib, _desc(), ww=0) == NULLPTR
+    assert _fwd(cuda_lib, _desc(), x=FAKE + 4) == MISALIGNED
+    assert _fwd(cuda_lib, _desc(), y=FAKE + 8) == MISALIGNED
+
+
+def test_unsupported_plane(cuda_lib):
+    assert _fwd(cuda_lib, _desc(H=256, W=256, L=4)) == UNSUPPORTED
+
+
+def test_backward_input_validation(cuda_lib):
+    p = ctypes.c_void_p
+    d = _desc(k=2)
+    assert cuda_lib.wtconv_backward_input(ctypes.byref(d), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE),
+                                          None) == BAD_K
+    d = _desc()
+    assert cuda_lib.wtconv_backward_input(ctypes.byref(d), p(0), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE),
+                                          None) == NULLPTR
+
+
+def test_backward_weight_workspace(cuda_lib):
+    p = ctypes.c_void_p
+    d = _desc()
+    need = cuda_lib.wtconv_workspace_bytes(ctypes.byref(d))
+    assert need > 0
+    args = [p(FAKE)] * 12
+    assert cuda_lib.wtconv_backward_weight(ctypes.byref(d), *args, p(FAKE), ctypes.c_size_t(need - 4),
+                                           None) == WORKSPACE
+    assert cuda_lib.wtconv_backward_weight(ctypes.byref(d), *args, p(0), ctypes.c_size_t(need), None) == WORKSPACE
+    bad = _desc(L=9)
+    assert cuda_lib.wtconv_workspace_bytes(ctypes.byref(bad)) == 0
+
+
+def test_status_strings(cuda_lib):
+    for code in range(10):
+        s = cuda_lib.wtconv_status_string(code)
+        assert s and len(s) > 1
+    assert cuda_lib.wtconv_status_string(999) == b"unknown status"
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(w, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(w, "_lib", None)
+    with pytest.raises(w.WTConvLibraryMissing):
+        w.load_library()
+
+
+def test_product_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "memory_bound_cnn_wtconv_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "wtconv_oracle" not in text and "liboracle" not in text, f

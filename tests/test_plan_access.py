@@ -1,0 +1,48 @@
+"""Host replay of every kernel memory access against the library's plan (CPU).
+
+plan_access_check.cpp includes the library's planner and walks the kernels'
+loops with their index arithmetic; see its header for what is checked.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from wtconv_inputs import NAMED, sweep_cases
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "plan_access_check.cpp")
+
+EDGE = [
+    (3, 5, 56, 56, 5, 3, 0), (1, 1, 8, 8, 5, 3, 0), (1, 1, 16, 16, 7, 4, 0), (2, 3, 24, 40, 3, 3, 0),
+    (1, 2, 32, 32, 3, 4, 0), (1, 2, 64, 64, 5, 4, 0), (1, 2, 12, 8, 1, 0, 0), (1, 2, 4, 4, 7, 2, 0),
+    (2, 2, 8, 4, 3, 2, 1), (1, 1, 64, 4, 7, 2, 0), (5, 3, 20, 12, 5, 2, 1), (1, 1, 2, 4, 3, 1, 0),
+    (1, 1, 64, 64, 7, 6, 0), (1, 1, 4, 4, 1, 1, 1),
+]
+
+
+@pytest.fixture(scope="module")
+def checker():
+    d = tempfile.mkdtemp()
+    exe = os.path.join(d, "plan_access_check")
+    subprocess.run(["g++", "-O2", "-std=c++17", "-o", exe, SRC], check=True, capture_output=True)
+    return exe
+
+
+def _cases():
+    out = [(c.B, c.C, c.H, c.W, c.k, c.L, 1 if c.dtype == "bf16" else 0) for c in NAMED.values()]
+    out += EDGE
+    seen = set()
+    for c in sweep_cases():  # the sweep's distinct plane geometries (B and C do not change the plan)
+        key = (c.H, c.W, c.k, c.L)
+        if key not in seen:
+            seen.add(key)
+            out.append((2, 3, c.H, c.W, c.k, c.L, 0))
+    return out
+
+
+@pytest.mark.parametrize("case", _cases(), ids=lambda c: "x".join(map(str, c)))
+def test_every_access_in_bounds(checker, case):
+    r = subprocess.run([checker, *map(str, case)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout + r.stderr
