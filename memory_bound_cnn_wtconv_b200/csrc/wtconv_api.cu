@@ -42,15 +42,19 @@ size_t workspace_floats(const Plan& P) { return (size_t)P.C * P.groups * P.nv; }
 
 // ---------------------------------------------------------------------------
 // Weight gradient, stage 2: one CTA per channel sums the groups' partials in
-// a fixed order and turns them into the five parameter gradients.
+// a fixed order and turns them into the five parameter gradients.  The
+// channel's parameters are staged in shared memory first, and each dot
+// product is one warp's fixed xor-tree.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) wtconv_bwdw_finish_kernel(
+__global__ void __launch_bounds__(128) wtconv_bwdw_finish_kernel(
     const float* __restrict__ part, int groups, int nv, int C, int k, int L,
     const float* __restrict__ base_w, const float* __restrict__ base_b, const float* __restrict__ base_scale,
     const float* __restrict__ wt_w, const float* __restrict__ wt_scale, float* __restrict__ d_base_w,
     float* __restrict__ d_base_b, float* __restrict__ d_base_scale, float* __restrict__ d_wt_w,
     float* __restrict__ d_wt_scale) {
-    extern __shared__ float gsum[];
+    extern __shared__ float fsm[];
+    float* gsum = fsm;            // nv: summed partials (un-normalised level sums)
+    float* wts = fsm + nv;        // ncls*KK: this channel's base_w then wt_w[l][c][s]
     const int c = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
     const int KK = k * k, ncls = 1 + 4 * L;
     for (int t = tid; t < nv; t += nt) {
@@ -58,29 +62,47 @@ __global__ void __launch_bounds__(256) wtconv_bwdw_finish_kernel(
         for (int g = 0; g < groups; ++g) s += part[((size_t)c * groups + g) * nv + t];
         gsum[t] = s;
     }
+    for (int t = tid; t < ncls * KK; t += nt) {
+        const int cl = t / KK, tap = t - cl * KK;
+        if (cl == 0) {
+            wts[t] = base_w[c * KK + tap];
+        } else {
+            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+            wts[t] = wt_w[((l * C + c) * 4 + s) * KK + tap];
+        }
+    }
+    __syncthreads();
+    // Level sums were accumulated on un-normalised subbands: scale by 4^-(l+1).
+    for (int t = tid; t < 4 * L * KK; t += nt) {
+        const int l = t / (4 * KK);
+        gsum[KK + t] *= quarter_pow(l);
+    }
     __syncthreads();
     const float sdy = gsum[ncls * KK];
     const float bs = base_scale[c];
     for (int t = tid; t < KK; t += nt) d_base_w[c * KK + t] = bs * gsum[t];
-    if (tid == 0) {
-        d_base_b[c] = bs * sdy;
-        float s = 0.f;
-        for (int t = 0; t < KK; ++t) s = fmaf(base_w[c * KK + t], gsum[t], s);
-        d_base_scale[c] = fmaf(base_b[c], sdy, s);
-    }
     for (int t = tid; t < 4 * L * KK; t += nt) {
         const int k2 = t / KK, tap = t - k2 * KK;
         const int l = k2 >> 2, s = k2 & 3;
         const int pi = (l * C + c) * 4 + s;
-        d_wt_w[pi * KK + tap] = wt_scale[pi] * (gsum[(1 + k2) * KK + tap] * quarter_pow(l));
+        d_wt_w[pi * KK + tap] = wt_scale[pi] * gsum[KK + t];
     }
-    for (int t = tid; t < 4 * L; t += nt) {
-        const int l = t >> 2, s = t & 3;
-        const int pi = (l * C + c) * 4 + s;
-        const float q = quarter_pow(l);
+    // Dot products: class cl -> warp (cl mod warps); lanes stride the taps.
+    const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+    for (int cl = warp; cl < ncls; cl += nw) {
         float a = 0.f;
-        for (int tap = 0; tap < KK; ++tap) a = fmaf(wt_w[pi * KK + tap], gsum[(1 + t) * KK + tap] * q, a);
-        d_wt_scale[pi] = a;
+        for (int tap = lane; tap < KK; tap += 32) a = fmaf(wts[cl * KK + tap], gsum[cl * KK + tap], a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) {
+            if (cl == 0) {
+                d_base_b[c] = bs * sdy;
+                d_base_scale[c] = fmaf(base_b[c], sdy, a);
+            } else {
+                const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+                d_wt_scale[(l * C + c) * 4 + s] = a;
+            }
+        }
     }
 }
 
@@ -88,7 +110,7 @@ cudaError_t launch_bwdw_finish(const Plan& P, const float* part, const float* ba
                                const float* base_scale, const float* wt_w, const float* wt_scale,
                                float* d_base_w, float* d_base_b, float* d_base_scale, float* d_wt_w,
                                float* d_wt_scale, cudaStream_t s) {
-    wtconv_bwdw_finish_kernel<<<P.C, 128, (size_t)P.nv * 4, s>>>(part, P.groups, P.nv, P.C, P.k, P.L, base_w,
+    wtconv_bwdw_finish_kernel<<<P.C, 128, (size_t)(P.nv + (1 + 4 * P.L) * P.k * P.k) * 4, s>>>(part, P.groups, P.nv, P.C, P.k, P.L, base_w,
                                                                  base_b, base_scale, wt_w, wt_scale, d_base_w,
                                                                  d_base_b, d_base_scale, d_wt_w, d_wt_scale);
     return cudaGetLastError();

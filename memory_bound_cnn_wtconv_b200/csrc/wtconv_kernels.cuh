@@ -8,17 +8,22 @@
 //       for every level l, the signed sum of that level's four conv outputs
 //       at (h >> (l+1), w >> (l+1)), the signs given by bit l of h and w;
 //   (3) per-channel and per-subband scales (and the orthonormal 2^-(l+1)
-//       factors of analysis and synthesis) are folded into the conv weights
-//       once per CTA, so the butterflies are pure add/sub.
+//       factors of analysis and synthesis) are folded into the conv weights,
+//       so the butterflies are pure add/sub.
 //
 // Un-normalised butterflies: U_{l,s} = 2^(l+1) S_{l,s} (S orthonormal), so a
 // level-l conv with weights  wt_scale * wt_w * 4^-(l+1)  yields exactly the
 // term  2^-(l+1) * Shat_{l,s}  that the closed-form synthesis adds.
 //
-// Depthwise convolution is not a dense contraction, so every conv here runs
-// on the FP32 FMA pipes: each thread owns a TR x TC output tile, streams the
-// (TR+K-1) input rows of its window from shared memory once with 128-bit
-// loads, and keeps the K*K folded weights in registers.
+// Depthwise convolution is not a dense contraction, so the convs run on the
+// FP32 pipes.  They are issue-bound, so every conv uses the packed f32x2 FMA
+// (64 multiply-adds per warp instruction): a thread owns a TR x 4 output tile
+// as TR x 2 column pairs, streams its window's TR+K-1 input rows from shared
+// memory once with 128-bit loads, and keeps the K*K folded weights in
+// registers.
+//
+// CTAs are persistent: each walks a run of planes; while it computes one
+// plane, cp.async copies the next one from HBM into a staging buffer.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -29,42 +34,65 @@
 
 namespace wtc {
 
+__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+    return (int)((__umulhi((uint32_t)n, f.mul) + (uint32_t)n) >> f.shift);
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
 // ---------------------------------------------------------------------------
-// Activation storage: 4 consecutive elements at a time (W % 4 == 0).
+// Asynchronous plane staging (cp.async, 16-byte chunks, no register round trip).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+__device__ __forceinline__ void stage_plane(float* stg, const void* src, int chunks, int tid, int nt) {
+    const char* g = static_cast<const char*>(src);
+    char* d = reinterpret_cast<char*>(stg);
+    for (int ch = tid; ch < chunks; ch += nt) cp_async16(d + 16 * ch, g + 16 * ch);
+}
+
+// 4 consecutive staged elements (element index e, a multiple of 4), as floats.
 template <typename T>
-struct Act;
+__device__ __forceinline__ float4 stg_load4(const float* stg, int e);
 
 template <>
-struct Act<float> {
-    static __device__ __forceinline__ float4 load4(const float* p) {
-        return __ldg(reinterpret_cast<const float4*>(p));
-    }
-    static __device__ __forceinline__ void store4(float* p, float4 v) {
-        *reinterpret_cast<float4*>(p) = v;
-    }
-};
+__device__ __forceinline__ float4 stg_load4<float>(const float* stg, int e) {
+    return *reinterpret_cast<const float4*>(stg + e);
+}
 
 template <>
-struct Act<__nv_bfloat16> {
-    static __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
-        uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
-        __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&r.x);
-        __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&r.y);
-        float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-        return make_float4(fa.x, fa.y, fb.x, fb.y);
-    }
-    static __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
-        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
-        __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
-        uint2 r;
-        r.x = *reinterpret_cast<uint32_t*>(&a);
-        r.y = *reinterpret_cast<uint32_t*>(&b);
-        *reinterpret_cast<uint2*>(p) = r;
-    }
-};
+__device__ __forceinline__ float4 stg_load4<__nv_bfloat16>(const float* stg, int e) {
+    const uint2 r = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(stg) + e);
+    const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
 
-// Store 4 floats to a shared address that is congruent to P (mod 4) floats.
+// Store 4 activations to global memory (16 bytes as float, 8 as bf16).
+template <typename T>
+__device__ __forceinline__ void gst4(T* p, float4 v);
+
+template <>
+__device__ __forceinline__ void gst4<float>(float* p, float4 v) {
+    *reinterpret_cast<float4*>(p) = v;
+}
+
+template <>
+__device__ __forceinline__ void gst4<__nv_bfloat16>(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 r;
+    r.x = *reinterpret_cast<uint32_t*>(&a);
+    r.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = r;
+}
+
+// Store 4 / 2 floats to a shared address congruent to P (mod 4) floats.
 template <int P>
 __device__ __forceinline__ void sts4(float* dst, float4 v) {
     if constexpr (P % 4 == 0) {
@@ -77,94 +105,246 @@ __device__ __forceinline__ void sts4(float* dst, float4 v) {
     }
 }
 
+template <int P>
+__device__ __forceinline__ void sts2(float* dst, float a, float b) {
+    if constexpr (P % 2 == 0) {
+        *reinterpret_cast<float2*>(dst) = make_float2(a, b);
+    } else {
+        dst[0] = a; dst[1] = b;
+    }
+}
+
 __device__ __forceinline__ void zero_smem(float* sm, int nfloats, int tid, int nt) {
     float4* s4 = reinterpret_cast<float4*>(sm);
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i = tid; i < (nfloats >> 2); i += nt) s4[i] = z;
 }
 
-// Copy an H x W plane from global memory into a shared buffer whose element
-// (0, 0) sits at `dst` (congruent to P mod 4 floats); optionally returns the
-// thread's running sum of the loaded values (weight gradient's sum of dy).
-template <typename T, int P, bool SUM>
-__device__ __forceinline__ float load_plane(const T* __restrict__ src, int H, int W, float* dst,
-                                            int stride, int tid, int nt) {
-    constexpr int U = 4;
+// ---------------------------------------------------------------------------
+// Unpack the staged H x W plane into the plane buffer (element (0,0) at
+// `dst`, congruent to PD mod 4 floats) and, if `level0`, run the level-0
+// un-normalised butterflies into the 4 subband planes at `sb` (element (0,0),
+// congruent to PD mod 2).  One work item = rows 2i, 2i+1 x columns 4q..4q+3,
+// i.e. two 2x2 blocks.  Returns the thread's sum of the unpacked values if SUM.
+// ---------------------------------------------------------------------------
+template <typename T, int PD, bool SUM>
+__device__ __forceinline__ float unpack_level0(const float* stg, int H, int W, FastDiv dq4, float* dst, int ds,
+                                               float* sb, int sbs, int sbsub, bool level0, int tid, int nt) {
     const int W4 = W >> 2;
-    const int n = H * W4;
-    float s = 0.f;
-    for (int t0 = tid; t0 < n; t0 += U * nt) {
-        float4 v[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int t = t0 + u * nt;
-            if (t < n) {
-                const int i = t / W4, j = (t - i * W4) * 4;
-                v[u] = Act<T>::load4(src + (size_t)i * W + j);
-            }
+    float sum = 0.f;
+    if (level0) {
+        const int n = (H >> 1) * W4;
+        for (int t = tid; t < n; t += nt) {
+            const int i = fdiv(t, dq4), q = t - i * W4;
+            const int r0 = 2 * i, c0 = 4 * q;
+            const float4 a = stg_load4<T>(stg, r0 * W + c0);
+            const float4 b = stg_load4<T>(stg, (r0 + 1) * W + c0);
+            sts4<PD>(dst + r0 * ds + c0, a);
+            sts4<PD>(dst + (r0 + 1) * ds + c0, b);
+            if (SUM) sum += ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
+            const float apb0 = a.x + a.y, amb0 = a.x - a.y, cpd0 = b.x + b.y, cmd0 = b.x - b.y;
+            const float apb1 = a.z + a.w, amb1 = a.z - a.w, cpd1 = b.z + b.w, cmd1 = b.z - b.w;
+            float* d = sb + i * sbs + 2 * q;
+            sts2<PD>(d, apb0 + cpd0, apb1 + cpd1);              // LL
+            sts2<PD>(d + sbsub, apb0 - cpd0, apb1 - cpd1);      // LH: difference between rows
+            sts2<PD>(d + 2 * sbsub, amb0 + cmd0, amb1 + cmd1);  // HL: difference between columns
+            sts2<PD>(d + 3 * sbsub, amb0 - cmd0, amb1 - cmd1);  // HH
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int t = t0 + u * nt;
-            if (t < n) {
-                const int i = t / W4, j = (t - i * W4) * 4;
-                sts4<P>(dst + i * stride + j, v[u]);
-                if (SUM) s += (v[u].x + v[u].y) + (v[u].z + v[u].w);
-            }
+    } else {
+        const int n = H * W4;
+        for (int t = tid; t < n; t += nt) {
+            const int i = fdiv(t, dq4), q = t - i * W4;
+            const float4 a = stg_load4<T>(stg, i * W + 4 * q);
+            sts4<PD>(dst + i * ds + 4 * q, a);
+            if (SUM) sum += (a.x + a.y) + (a.z + a.w);
         }
     }
-    return s;
+    return sum;
 }
 
 // One un-normalised 2-D Haar analysis step on chip: the (2n) x (2m) plane at
 // `src` (element (0,0), row stride `ss`) becomes 4 planes n x m at `dst`
 // (element (0,0), row stride `ds`, plane step `dsub`), order LL, LH, HL, HH.
-__device__ __forceinline__ void haar_level(const float* src, int ss, int n, int m, float* dst, int ds,
-                                           int dsub, int tid, int nt) {
+__device__ __forceinline__ void haar_level(const float* src, int ss, int n, int m, FastDiv dm, float* dst,
+                                           int ds, int dsub, int tid, int nt) {
     for (int t = tid; t < n * m; t += nt) {
-        const int i = t / m, j = t - i * m;
+        const int i = fdiv(t, dm), j = t - i * m;
         const float* s0 = src + 2 * i * ss + 2 * j;
         const float a = s0[0], b = s0[1], c = s0[ss], d = s0[ss + 1];
         const float apb = a + b, amb = a - b, cpd = c + d, cmd = c - d;
         float* d0 = dst + i * ds + j;
-        d0[0] = apb + cpd;          // LL
-        d0[dsub] = apb - cpd;       // LH: difference between rows
-        d0[2 * dsub] = amb + cmd;   // HL: difference between columns
-        d0[3 * dsub] = amb - cmd;   // HH
+        d0[0] = apb + cpd;
+        d0[dsub] = apb - cpd;
+        d0[2 * dsub] = amb + cmd;
+        d0[3 * dsub] = amb - cmd;
     }
 }
 
+// Where one analysis level writes: element (i, j) of subband s at
+// base + s*sub + i*stride + j (`base` already includes any padding offset).
+struct LevelDst {
+    float* base;
+    int stride;
+    int sub;
+};
+
+__device__ __forceinline__ void butterfly(float a, float b, float c, float d, float& ll, float& lh, float& hl,
+                                          float& hh) {
+    const float apb = a + b, amb = a - b, cpd = c + d, cmd = c - d;
+    ll = apb + cpd;  // LL
+    lh = apb - cpd;  // LH: difference between rows
+    hl = amb + cmd;  // HL: difference between columns
+    hh = amb - cmd;  // HH
+}
+
+// Analysis pyramid of one staged plane in a single pass (no CTA barrier):
+// the `np` threads [0, np) each own 4x4 pixel blocks; they unpack the block
+// into the plane buffer `dst` (element (0,0), row stride ds, congruent to PD
+// mod 4 floats), run levels 0 and 1 in registers, and levels 2 ..
+// `levels`-1 (levels <= 4) by xor-shuffles inside groups of 4^(l-1) lanes
+// that cover one 2^(l+1) x 2^(l+1) region.  Lane groups: a region of
+// (4G)^2 pixels, G = 2^lg, occupies G*G consecutive lanes (block (by, bx) of
+// the region at lane offset by*G + bx).  Returns the thread's sum of the
+// unpacked values if SUM.
+template <typename T, int PD, bool SUM>
+__device__ __forceinline__ float analysis_pyramid(const float* stg, int H, int W, int levels, int lg, FastDiv drw,
+                                                  float* dst, int ds, const LevelDst* lev, int np, int ptid) {
+    const int G = 1 << lg, G2 = G * G;
+    const int nreg_w = W >> (lg + 2);
+    const int items = (H >> (lg + 2)) * nreg_w * G2;
+    const int lane = ptid & 31;
+    float sum = 0.f;
+    for (int base = ptid & ~31; base < items; base += np) {
+        const int item = base + lane;
+        const bool valid = item < items;  // whole lane groups are valid or not
+        const int it = valid ? item : 0;
+        const int r = it >> (2 * lg), o = it & (G2 - 1);
+        const int by = o >> lg, bx = o & (G - 1);
+        const int rrow = fdiv(r, drw), rcol = r - rrow * nreg_w;
+        const int brow = rrow * G + by, bcol = rcol * G + bx;  // 4x4 block coordinates
+        const int r0 = 4 * brow, c0 = 4 * bcol;
+        float4 v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = stg_load4<T>(stg, (r0 + q) * W + c0);
+        if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sts4<PD>(dst + (r0 + q) * ds + c0, v[q]);
+            if (SUM) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sum += (v[q].x + v[q].y) + (v[q].z + v[q].w);
+            }
+        }
+        // Level 0: the block's 2x2 positions.
+        float ll[2][2];
+#pragma unroll
+        for (int pi = 0; pi < 2; ++pi) {
+            const float4 A = v[2 * pi], B = v[2 * pi + 1];
+            float l0, h0, g0, d0, l1, h1, g1, d1;
+            butterfly(A.x, A.y, B.x, B.y, l0, h0, g0, d0);
+            butterfly(A.z, A.w, B.z, B.w, l1, h1, g1, d1);
+            if (valid) {
+                float* q = lev[0].base + (2 * brow + pi) * lev[0].stride + 2 * bcol;
+                sts2<PD>(q, l0, l1);
+                sts2<PD>(q + lev[0].sub, h0, h1);
+                sts2<PD>(q + 2 * lev[0].sub, g0, g1);
+                sts2<PD>(q + 3 * lev[0].sub, d0, d1);
+            }
+            ll[pi][0] = l0;
+            ll[pi][1] = l1;
+        }
+        if (levels < 2) continue;
+        // Level 1: the block itself.
+        float mine, lh, hl, hh;
+        butterfly(ll[0][0], ll[0][1], ll[1][0], ll[1][1], mine, lh, hl, hh);
+        if (valid) {
+            float* q = lev[1].base + brow * lev[1].stride + bcol;
+            q[0] = mine; q[lev[1].sub] = lh; q[2 * lev[1].sub] = hl; q[3 * lev[1].sub] = hh;
+        }
+        // Levels 2..: the 2x2 group of lanes that differ in bit (l-2) of by / bx.
+#pragma unroll
+        for (int l = 2; l < 4; ++l) {
+            if (l >= levels) break;
+            const int sh = l - 2;
+            const float vh = __shfl_xor_sync(0xffffffffu, mine, 1 << sh);
+            const float vv = __shfl_xor_sync(0xffffffffu, mine, G << sh);
+            const float vd = __shfl_xor_sync(0xffffffffu, vh, G << sh);
+            const int py = (by >> sh) & 1, px = (bx >> sh) & 1;
+            const float a = py ? (px ? vd : vv) : (px ? vh : mine);
+            const float b = py ? (px ? vv : vd) : (px ? mine : vh);
+            const float c = py ? (px ? vh : mine) : (px ? vd : vv);
+            const float d = py ? (px ? mine : vh) : (px ? vv : vd);
+            float nll;
+            butterfly(a, b, c, d, nll, lh, hl, hh);
+            const int m = (2 << sh) - 1;
+            if (valid && (by & m) == 0 && (bx & m) == 0) {
+                float* q = lev[l].base + (brow >> (l - 1)) * lev[l].stride + (bcol >> (l - 1));
+                q[0] = nll; q[lev[l].sub] = lh; q[2 * lev[l].sub] = hl; q[3 * lev[l].sub] = hh;
+            }
+            mine = nll;
+        }
+    }
+    return sum;
+}
+
 // ---------------------------------------------------------------------------
-// Register-tiled depthwise conv of one TR x TC output tile.
+// A window row as NW2 aligned pairs e[k] = (r[2k], r[2k+1]), loaded straight
+// into register pairs with 64-bit shared loads.  For output column pair jp
+// (columns 2jp, 2jp+1) and tap v the inputs are columns 2jp+v and 2jp+v+1:
+//   v even: the pair e[jp + v/2]              -> one packed FMA;
+//   v odd:  e[jp + v/2].y and e[jp + v/2 + 1].x -> two scalar FMAs.
+// No register moves are needed to build shifted pairs.
+// ---------------------------------------------------------------------------
+template <int NW2>
+struct WinRow {
+    float2 e[NW2];
+    __device__ __forceinline__ void load(const float* rp) {
+#pragma unroll
+        for (int k = 0; k < NW2; ++k) e[k] = *reinterpret_cast<const float2*>(rp + 2 * k);
+    }
+};
+
+// acc (output columns 2jp, 2jp+1) += w * input columns (2jp+v, 2jp+v+1).
+template <int NW2>
+__device__ __forceinline__ float2 tap(float2 acc, float w, const WinRow<NW2>& row, int jp, int v) {
+    if ((v & 1) == 0) return ffma2(make_float2(w, w), row.e[jp + (v >> 1)], acc);
+    acc.x = fmaf(w, row.e[jp + (v >> 1)].y, acc.x);
+    acc.y = fmaf(w, row.e[jp + (v >> 1) + 1].x, acc.y);
+    return acc;
+}
+
+// acc (split by column parity) += d (columns 2jp, 2jp+1) * input columns (2jp+v, 2jp+v+1).
+template <int NW2>
+__device__ __forceinline__ float2 ctap(float2 acc, float2 d, const WinRow<NW2>& row, int jp, int v) {
+    if ((v & 1) == 0) return ffma2(d, row.e[jp + (v >> 1)], acc);
+    acc.x = fmaf(d.x, row.e[jp + (v >> 1)].y, acc.x);
+    acc.y = fmaf(d.y, row.e[jp + (v >> 1) + 1].x, acc.y);
+    return acc;
+}
+
+// Register-tiled depthwise conv of one TR x TC output tile (TC/2 column pairs):
 //   out[o][j] = init + sum_{u<K, v<K} w[u*K+v] * win[(o+u)*stride + j+v]
 // `win` is the 16-byte aligned window origin (input element (r0-p, c0-p)).
-// Each input row is loaded once; output row o is handed to emit(o, acc[o])
-// as soon as its last input row has been consumed.
-// ---------------------------------------------------------------------------
+// Output row o is handed to emit(o, acc[o]) once its last input row is in.
 template <int K, int TR, int TC, class Emit>
 __device__ __forceinline__ void conv_tile(const float* __restrict__ win, int stride, const float (&w)[K * K],
-                                          float init, Emit&& emit) {
-    constexpr int WV = (TC + K - 1 + 3) / 4;
-    float acc[TR][TC];
+                                          float2 init, Emit&& emit) {
+    constexpr int NP = TC / 2;
+    constexpr int NW2 = (TC + K - 1) / 2;
+    float2 acc[TR][NP];
 #pragma unroll
     for (int r = 0; r < TR + K - 1; ++r) {
-        float row[4 * WV];
-        const float* rp = win + r * stride;
-#pragma unroll
-        for (int q = 0; q < WV; ++q) {
-            const float4 v = *reinterpret_cast<const float4*>(rp + 4 * q);
-            row[4 * q + 0] = v.x; row[4 * q + 1] = v.y; row[4 * q + 2] = v.z; row[4 * q + 3] = v.w;
-        }
+        WinRow<NW2> row;
+        row.load(win + r * stride);
 #pragma unroll
         for (int u = 0; u < K; ++u) {
             const int o = r - u;
             if (o >= 0 && o < TR) {
 #pragma unroll
-                for (int j = 0; j < TC; ++j) {
-                    float a = (u == 0) ? init : acc[o][j];
+                for (int jp = 0; jp < NP; ++jp) {
+                    float2 a = (u == 0) ? init : acc[o][jp];
 #pragma unroll
-                    for (int v = 0; v < K; ++v) a = fmaf(w[u * K + v], row[j + v], a);
-                    acc[o][j] = a;
+                    for (int v = 0; v < K; ++v) a = tap<NW2>(a, w[u * K + v], row, jp, v);
+                    acc[o][jp] = a;
                 }
             }
         }
@@ -173,39 +353,33 @@ __device__ __forceinline__ void conv_tile(const float* __restrict__ win, int str
     }
 }
 
-// Correlation of one TR x TC tile of D with the K x K shifts of S:
+// Correlation of one TR x TC tile of D with the K x K shifts of S, split by
+// column parity (sum the two halves at the end):
 //   acc[u*K+v] += sum_{o<TR, j<TC} D[o][j] * S[o+u][j+v]
 // `swin` is the S window origin (element (r0-p, c0-p)), `dt` the D tile origin.
 template <int K, int TR, int TC>
 __device__ __forceinline__ void corr_tile(const float* __restrict__ swin, int sstride,
-                                          const float* __restrict__ dt, int dstride, float (&acc)[K * K]) {
-    constexpr int WV = (TC + K - 1 + 3) / 4;
-    float d[TR][TC];
+                                          const float* __restrict__ dt, int dstride, float2 (&acc)[K * K]) {
+    constexpr int NP = TC / 2;
+    constexpr int NW2 = (TC + K - 1) / 2;
+    float2 d[TR][NP];
 #pragma unroll
     for (int r = 0; r < TR + K - 1; ++r) {
         if (r < TR) {
 #pragma unroll
-            for (int q = 0; q < TC / 4; ++q) {
-                const float4 v = *reinterpret_cast<const float4*>(dt + r * dstride + 4 * q);
-                d[r][4 * q + 0] = v.x; d[r][4 * q + 1] = v.y; d[r][4 * q + 2] = v.z; d[r][4 * q + 3] = v.w;
-            }
+            for (int q = 0; q < NP; ++q) d[r][q] = *reinterpret_cast<const float2*>(dt + r * dstride + 2 * q);
         }
-        float row[4 * WV];
-        const float* rp = swin + r * sstride;
-#pragma unroll
-        for (int q = 0; q < WV; ++q) {
-            const float4 v = *reinterpret_cast<const float4*>(rp + 4 * q);
-            row[4 * q + 0] = v.x; row[4 * q + 1] = v.y; row[4 * q + 2] = v.z; row[4 * q + 3] = v.w;
-        }
+        WinRow<NW2> row;
+        row.load(swin + r * sstride);
 #pragma unroll
         for (int u = 0; u < K; ++u) {
             const int o = r - u;
             if (o >= 0 && o < TR) {
 #pragma unroll
                 for (int v = 0; v < K; ++v) {
-                    float a = acc[u * K + v];
+                    float2 a = acc[u * K + v];
 #pragma unroll
-                    for (int j = 0; j < TC; ++j) a = fmaf(d[o][j], row[j + v], a);
+                    for (int jp = 0; jp < NP; ++jp) a = ctap<NW2>(a, d[o][jp], row, jp, v);
                     acc[u * K + v] = a;
                 }
             }
@@ -233,160 +407,324 @@ __device__ __forceinline__ float quarter_pow(int l) {
 }
 
 // ---------------------------------------------------------------------------
-// Forward (BWD = false) and input gradient (BWD = true).  One CTA per plane.
+// Staging and analysis of one plane by the threads [0, np) (ptid = thread
+// index among them): the staged plane becomes the plane buffer (element
+// (0,0) at `dst`, row stride ds, congruent to PD mod 4 floats) and the Haar
+// subbands of every level (level l in bufs[l]; `pad` is the zero border of
+// those buffers).  `sync()` synchronises the np threads between the levels
+// that run one at a time (levels >= 4, or every level without the pyramid).
+// ---------------------------------------------------------------------------
+template <typename T, int PD, bool SUM, class Sync>
+__device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const float* stg, float* dst, int ds,
+                                               const Buf* bufs, int pad, int np, int ptid, Sync&& sync) {
+    const int H = P.H, W = P.W, L = P.L;
+    float sum;
+    int done;  // levels complete
+    if (P.pyr) {
+        LevelDst lev[4];
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+            const Buf& b = bufs[l < L ? l : 0];
+            lev[l] = LevelDst{sm + b.base + pad * b.stride + pad, b.stride, b.sub};
+        }
+        sum = analysis_pyramid<T, PD, SUM>(stg, H, W, P.pyr_levels, P.pyr_lg, P.div_rw, dst, ds, lev, np, ptid);
+        done = P.pyr_levels;
+    } else {
+        const Buf& b = bufs[0];
+        sum = unpack_level0<T, PD, SUM>(stg, H, W, P.div_q4, dst, ds, sm + b.base + pad * b.stride + pad, b.stride,
+                                        b.sub, L >= 1, ptid, np);
+        done = L >= 1 ? 1 : 0;
+    }
+    for (int l = done; l < L; ++l) {
+        sync();
+        const Buf& s0 = bufs[l - 1];
+        const Buf& s1 = bufs[l];
+        haar_level(sm + s0.base + pad * s0.stride + pad, s0.stride, H >> (l + 1), W >> (l + 1), P.div_m[l],
+                   sm + s1.base + pad * s1.stride + pad, s1.stride, s1.sub, ptid, np);
+    }
+    return sum;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Forward (BWD = false) and input gradient (BWD = true).
 // The input gradient is the same pass applied to dy with every kernel
 // rotated by 180 degrees and no bias: the transpose of the forward map.
 // ---------------------------------------------------------------------------
+// A subband tile, its addressing decoded once: window origin in S, output
+// origin in Q, and the folded weights of its class.
+struct SubTile {
+    int win, out, wts;  // float offsets into shared memory
+    int sstride, qstride;
+};
+
+__device__ __forceinline__ SubTile decode_subband_tile(const Plan& P, int t, int TR, int TC) {
+    int cl = 1;
+    while (t >= P.sub_begin[cl]) ++cl;  // sub_begin[cl] = end of class cl's tiles
+    const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+    const int local = t - P.sub_begin[cl - 1];
+    const int tr = fdiv(local, P.div_ntc[l]), tc = local - tr * P.ntc[l];
+    const Buf& S = P.S[l];
+    const Buf& Q = P.Q[l];
+    SubTile st;
+    st.win = S.base + s * S.sub + tr * TR * S.stride + tc * TC;
+    st.out = Q.base + s * Q.sub + tr * TR * Q.stride + tc * TC;
+    st.wts = P.wbase + cl * P.wcls;
+    st.sstride = S.stride;
+    st.qstride = Q.stride;
+    return st;
+}
+
+template <int K, int TR, int TC>
+__device__ __forceinline__ void run_subband_tile(float* sm, const SubTile& st) {
+    float w[K * K];
+    load_weights<K>(sm + st.wts, w);
+    float* out = sm + st.out;
+    const int qs = st.qstride;
+    conv_tile<K, TR, TC>(sm + st.win, st.sstride, w, make_float2(0.f, 0.f), [&](int o, float2(&a)[TC / 2]) {
+#pragma unroll
+        for (int q = 0; q < TC / 4; ++q)
+            *reinterpret_cast<float4*>(out + o * qs + 4 * q) =
+                make_float4(a[2 * q].x, a[2 * q].y, a[2 * q + 1].x, a[2 * q + 1].y);
+    });
+}
+
+// Reformulation (2), levels >= 1, evaluated Horner-style: for l = L-1 .. 1
+// every level-l position (i, j) adds its four signed sums (signs from the
+// bit pair (a, b) of the level-(l-1) position (2i+a, 2j+b)) into the LL conv
+// output of level l-1 at that position.  Level l-1's LL then carries all
+// coarser terms into its own signed sums, so after the loop Q0's LL holds,
+// at every 2x2 output block (h >> 1, w >> 1), the closed-form sum of levels
+// 1..L-1 at that block.  One step per level, `sync()` between steps.
+template <class Sync>
+__device__ __forceinline__ void coarse_cascade(float* sm, const Plan& P, int np, int ptid, Sync&& sync) {
+    for (int l = P.L - 1; l >= 1; --l) {
+        const Buf& Q = P.Q[l];
+        const Buf& D = P.Q[l - 1];
+        const int n = P.H >> (l + 1), m = P.W >> (l + 1);
+        for (int t = ptid; t < n * m; t += np) {
+            const int i = fdiv(t, P.div_m[l]), j = t - i * m;
+            const float* q = sm + Q.base + i * Q.stride + j;
+            const float q0 = q[0], q1 = q[Q.sub], q2 = q[2 * Q.sub], q3 = q[3 * Q.sub];
+            float* d = sm + D.base + (2 * i) * D.stride + 2 * j;  // LL plane of level l-1
+            const float2 top = *reinterpret_cast<const float2*>(d);
+            const float2 bot = *reinterpret_cast<const float2*>(d + D.stride);
+            const float t0 = q0 + q1, t1 = q0 - q1, t2 = q2 + q3, t3 = q2 - q3;
+            *reinterpret_cast<float2*>(d) = make_float2(top.x + (t0 + t2), top.y + (t0 - t2));
+            *reinterpret_cast<float2*>(d + D.stride) = make_float2(bot.x + (t1 + t3), bot.y + (t1 - t3));
+        }
+        sync();
+    }
+}
+
+// The rows of one base tile (4 columns w0..w0+3, w0 % 4 == 0, rows from h0):
+// add the level-0 signed sum (signs from bit 0 of h and w; Q0's LL already
+// carries the coarser levels) and store (the only HBM write).  Straight-line
+// code with predicated stores, so the rows overlap.
+template <int TR, typename T>
+__device__ __forceinline__ void finish_tile(const float* sm, const Plan& P, T* yp, int h0, int w0,
+                                            float2 (&a)[TR][2]) {
+    const Buf& Q = P.Q[0];
+    const float* qb = sm + Q.base + (w0 >> 1);
+#pragma unroll
+    for (int o = 0; o < TR; ++o) {
+        const int h = h0 + o;
+        if (P.L >= 1) {
+            const float* r = qb + (h >> 1) * Q.stride;
+            const float2 q0 = *reinterpret_cast<const float2*>(r);
+            const float2 q1 = *reinterpret_cast<const float2*>(r + Q.sub);
+            const float2 q2 = *reinterpret_cast<const float2*>(r + 2 * Q.sub);
+            const float2 q3 = *reinterpret_cast<const float2*>(r + 3 * Q.sub);
+            const float sg = (h & 1) ? -1.f : 1.f;
+            const float t0a = fmaf(sg, q1.x, q0.x), t1a = fmaf(sg, q3.x, q2.x);
+            const float t0b = fmaf(sg, q1.y, q0.y), t1b = fmaf(sg, q3.y, q2.y);
+            a[o][0].x += t0a + t1a;
+            a[o][0].y += t0a - t1a;
+            a[o][1].x += t0b + t1b;
+            a[o][1].y += t0b - t1b;
+        }
+        if (h < P.H) gst4<T>(yp + (size_t)h * P.W + w0, make_float4(a[o][0].x, a[o][0].y, a[o][1].x, a[o][1].y));
+    }
+}
+
+// One output row (the loop schedule of large planes).
+template <typename T>
+__device__ __forceinline__ void finish_row(const float* sm, const Plan& P, T* yp, int h, int w0, float2 (&a)[2]) {
+    if (P.L >= 1) {
+        const Buf& Q = P.Q[0];
+        const float* q = sm + Q.base + (h >> 1) * Q.stride + (w0 >> 1);
+        const float sg = (h & 1) ? -1.f : 1.f;
+        const float2 q0 = *reinterpret_cast<const float2*>(q);
+        const float2 q1 = *reinterpret_cast<const float2*>(q + Q.sub);
+        const float2 q2 = *reinterpret_cast<const float2*>(q + 2 * Q.sub);
+        const float2 q3 = *reinterpret_cast<const float2*>(q + 3 * Q.sub);
+        const float t0a = fmaf(sg, q1.x, q0.x), t1a = fmaf(sg, q3.x, q2.x);
+        const float t0b = fmaf(sg, q1.y, q0.y), t1b = fmaf(sg, q3.y, q2.y);
+        a[0].x += t0a + t1a;
+        a[0].y += t0a - t1a;
+        a[1].x += t0b + t1b;
+        a[1].y += t0b - t1b;
+    }
+    gst4<T>(yp + (size_t)h * P.W + w0, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
+}
+
+// Shared pieces of the two forward schedules.
+template <int K, typename T, bool BWD>
+struct FusedCtx {
+    float* sm;
+    const Plan& P;
+    const T* x;
+    const float *base_w, *base_b, *base_scale, *wt_w, *wt_scale;
+    long long units;
+    int u0, u1;
+
+    __device__ __forceinline__ size_t plane_of(int u) const {
+        const int c = u / P.B, b = u - c * P.B;
+        return (size_t)b * P.C + c;
+    }
+    __device__ __forceinline__ const T* src(int u) const { return x + plane_of(u) * ((size_t)P.H * P.W); }
+    // Reformulation (3): fold the scales (and the Haar factors) into the
+    // weights of channel c (threads [0, np)).
+    __device__ __forceinline__ void fold(int c, int np, int ptid) const {
+        constexpr int KK = K * K;
+        const int ncls = 1 + 4 * P.L;
+        for (int t = ptid; t < ncls * KK; t += np) {
+            const int cl = t / KK, tap = t - cl * KK;
+            const int src_tap = BWD ? (KK - 1 - tap) : tap;
+            float v;
+            if (cl == 0) {
+                v = base_scale[c] * base_w[c * KK + src_tap];
+            } else {
+                const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+                const int pi = (l * P.C + c) * 4 + s;
+                v = (wt_scale[pi] * wt_w[pi * KK + src_tap]) * quarter_pow(l);
+            }
+            sm[P.wbase + cl * P.wcls + tap] = v;
+        }
+        if (ptid == 0) sm[P.bias] = BWD ? 0.f : base_scale[c] * base_b[c];
+    }
+};
+
+// Forward / input gradient.  Per plane (all threads, CTA barriers between
+// phases): fold the weights when the channel changes and analyse the staged
+// plane; start staging the next plane; run every conv tile (one per thread:
+// subband tiles write Q, base tiles keep their outputs in registers); fold
+// the coarse levels into Q0's LL; base tiles add the level-0 signed sum and
+// store y.  Large planes (more tiles than threads) loop over the subband
+// tiles and then the base tiles instead.
 template <int K, int TR, int TC, typename T, bool BWD>
-__global__ void __launch_bounds__(512) wtconv_fused_kernel(
+__global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
     const T* __restrict__ x, const float* __restrict__ base_w, const float* __restrict__ base_b,
     const float* __restrict__ base_scale, const float* __restrict__ wt_w,
     const float* __restrict__ wt_scale, T* __restrict__ y, const Plan P) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
-    constexpr int p = K / 2, KK = K * K;
-    static_assert(TC % 4 == 0, "tile width must be a multiple of 4");
+    constexpr int p = K / 2, KK = K * K, NP = TC / 2;
+    static_assert(TC == 4, "4-column tiles");
     const int tid = threadIdx.x, nt = blockDim.x;
-    const int plane = blockIdx.x;
-    const int c = plane % P.C;
-    const int H = P.H, W = P.W, L = P.L;
+    const long long units = (long long)P.B * P.C;
+    FusedCtx<K, T, BWD> cx{sm, P, x, base_w, base_b, base_scale, wt_w, wt_scale, units,
+                           (int)(((long long)blockIdx.x * units) / gridDim.x),
+                           (int)(((long long)(blockIdx.x + 1) * units) / gridDim.x)};
+    const int u0 = cx.u0, u1 = cx.u1;
+    auto csync = [&]() { __syncthreads(); };
+    float* X0 = sm + P.X.base + p * P.X.stride + p;
+    const int ntcb = P.ntc[kMaxL];
+
+    // In the one-tile-per-thread schedule each thread's tile is fixed.
+    const bool sub = P.merged && tid < P.n_sub_tiles;
+    const int bt = tid - P.base_tid0;
+    const bool held = P.merged && bt >= 0 && bt < P.n_base_tiles;
+    const int btr = held ? fdiv(bt, P.div_ntc[kMaxL]) : 0;
+    const int btc = bt - btr * ntcb;
 
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
-
-    // Reformulation (3): fold the scales (and the Haar factors) into the weights.
-    const int ncls = 1 + 4 * L;
-    for (int t = tid; t < ncls * KK; t += nt) {
-        const int cl = t / KK, tap = t - cl * KK;
-        const int src = BWD ? (KK - 1 - tap) : tap;
-        float v;
-        if (cl == 0) {
-            v = base_scale[c] * base_w[c * KK + src];
-        } else {
-            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-            const int pi = (l * P.C + c) * 4 + s;
-            v = (wt_scale[pi] * wt_w[pi * KK + src]) * quarter_pow(l);
+    if (u0 < u1) stage_plane(sm + P.stg, cx.src(u0), P.plane_chunks, tid, nt);
+    cp_async_commit();
+    int cur_c = -1;
+    for (int u = u0; u < u1; ++u) {
+        const int c = u / P.B;
+        cp_async_wait_all();
+        __syncthreads();  // staged plane complete; previous plane fully finished
+        if (c != cur_c) {
+            cx.fold(c, nt, tid);
+            cur_c = c;
         }
-        sm[P.wbase + cl * P.wcls + tap] = v;
-    }
-    if (tid == 0) sm[P.bias] = BWD ? 0.f : base_scale[c] * base_b[c];
-
-    // Stage the plane (the only HBM read).
-    const size_t poff = (size_t)plane * H * W;
-    load_plane<T, p, false>(x + poff, H, W, sm + P.X.base + p * P.X.stride + p, P.X.stride, tid, nt);
-    __syncthreads();
-
-    // Reformulation (1): analysis butterflies for every level, on chip.
-    for (int l = 0; l < L; ++l) {
-        const float* src = (l == 0) ? sm + P.X.base + p * P.X.stride + p
-                                    : sm + P.S[l - 1].base + p * P.S[l - 1].stride + p;
-        const int ss = (l == 0) ? P.X.stride : P.S[l - 1].stride;
-        haar_level(src, ss, H >> (l + 1), W >> (l + 1), sm + P.S[l].base + p * P.S[l].stride + p,
-                   P.S[l].stride, P.S[l].sub, tid, nt);
+        analyse_plane<T, p, false>(sm, P, sm + P.stg, X0, P.X.stride, P.S, p, nt, tid, csync);
         __syncthreads();
-    }
+        if (u + 1 < u1) stage_plane(sm + P.stg, cx.src(u + 1), P.plane_chunks, tid, nt);
+        cp_async_commit();
 
-    // Per-subband depthwise convs, folded weights -> Q[l].
-    for (int t = tid; t < P.n_sub_tiles; t += nt) {
-        int cl = 1;
-        while (t >= P.sub_begin[cl]) ++cl;  // sub_begin[cl] = end of class cl's tiles
-        const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-        const int local = t - P.sub_begin[cl - 1];
-        const int tr = local / P.ntc[l], tc = local - tr * P.ntc[l];
-        float w[KK];
-        load_weights<K>(sm + P.wbase + cl * P.wcls, w);
-        const Buf& S = P.S[l];
-        const Buf& Q = P.Q[l];
-        const float* win = sm + S.base + s * S.sub + tr * TR * S.stride + tc * TC;
-        float* out = sm + Q.base + s * Q.sub + tr * TR * Q.stride + tc * TC;
-        conv_tile<K, TR, TC>(win, S.stride, w, 0.f, [&](int o, float(&a)[TC]) {
+        T* yp = y + cx.plane_of(u) * ((size_t)P.H * P.W);
+        if (P.merged) {
+            float2 hold[TR][NP];
+            if (sub) {
+                run_subband_tile<K, TR, TC>(sm, decode_subband_tile(P, tid, TR, TC));
+            } else if (held) {
+                float wb[KK];
+                load_weights<K>(sm + P.wbase, wb);
+                const float bias = sm[P.bias];
+                const float* win = sm + P.X.base + btr * TR * P.X.stride + btc * TC;
+                conv_tile<K, TR, TC>(win, P.X.stride, wb, make_float2(bias, bias), [&](int o, float2(&a)[NP]) {
 #pragma unroll
-            for (int q = 0; q < TC / 4; ++q)
-                *reinterpret_cast<float4*>(out + o * Q.stride + 4 * q) =
-                    make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
-        });
-    }
-    __syncthreads();
-
-    // Reformulation (2), levels >= 1: their signed sum at half resolution
-    // (constant over each 2x2 output block), indexed by the bits of (i, j).
-    const int n0 = H >> 1, m0 = W >> 1;
-    if (L >= 2) {
-        for (int t = tid; t < n0 * m0; t += nt) {
-            const int i = t / m0, j = t - i * m0;
-            float z = 0.f;
-            for (int l = 1; l < L; ++l) {
-                const Buf& Q = P.Q[l];
-                const float* q = sm + Q.base + (i >> l) * Q.stride + (j >> l);
-                const float q0 = q[0], q1 = q[Q.sub], q2 = q[2 * Q.sub], q3 = q[3 * Q.sub];
-                const int a = (i >> (l - 1)) & 1, b = (j >> (l - 1)) & 1;
-                const float t0 = a ? q0 - q1 : q0 + q1;
-                const float t1 = a ? q2 - q3 : q2 + q3;
-                z += b ? t0 - t1 : t0 + t1;
+                    for (int j = 0; j < NP; ++j) hold[o][j] = a[j];
+                });
             }
-            sm[P.Z.base + i * P.Z.stride + j] = z;
-        }
-        __syncthreads();
-    }
-
-    // Base conv + level-0 signed sum + coarse sum -> y (the only HBM write).
-    {
-        float w[KK];
-        load_weights<K>(sm + P.wbase, w);
-        const float bias = sm[P.bias];
-        const int ntc = P.ntc[kMaxL];
-        T* yp = y + poff;
-        for (int t = tid; t < P.n_base_tiles; t += nt) {
-            const int tr = t / ntc, tc = t - tr * ntc;
-            const float* win = sm + P.X.base + tr * TR * P.X.stride + tc * TC;
-            conv_tile<K, TR, TC>(win, P.X.stride, w, bias, [&](int o, float(&a)[TC]) {
-                const int h = tr * TR + o;
-                if (h >= H) return;
-                const int w0 = tc * TC;
-                if (L >= 1) {
-                    const Buf& Q = P.Q[0];
-                    const int i = h >> 1;
-                    const float sg = (h & 1) ? -1.f : 1.f;
-#pragma unroll
-                    for (int pos = 0; pos < TC / 2; ++pos) {
-                        const int j = (w0 >> 1) + pos;
-                        const float* q = sm + Q.base + i * Q.stride + j;
-                        float q0 = q[0];
-                        if (L >= 2) q0 += sm[P.Z.base + i * P.Z.stride + j];
-                        const float t0 = fmaf(sg, q[Q.sub], q0);
-                        const float t1 = fmaf(sg, q[3 * Q.sub], q[2 * Q.sub]);
-                        a[2 * pos] += t0 + t1;
-                        a[2 * pos + 1] += t0 - t1;
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < TC / 4; ++q)
-                    Act<T>::store4(yp + (size_t)h * W + w0 + 4 * q,
-                                   make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]));
-            });
+            __syncthreads();  // every Q complete
+            coarse_cascade(sm, P, nt, tid, csync);
+            if (held) finish_tile<TR, T>(sm, P, yp, btr * TR, btc * TC, hold);
+        } else {
+            for (int t = tid; t < P.n_sub_tiles; t += nt)
+                run_subband_tile<K, TR, TC>(sm, decode_subband_tile(P, t, TR, TC));
+            __syncthreads();  // every Q complete
+            coarse_cascade(sm, P, nt, tid, csync);
+            float wb[KK];
+            load_weights<K>(sm + P.wbase, wb);
+            const float bias = sm[P.bias];
+            for (int t = tid; t < P.n_base_tiles; t += nt) {
+                const int tr = fdiv(t, P.div_ntc[kMaxL]), tc = t - tr * ntcb;
+                const float* win = sm + P.X.base + tr * TR * P.X.stride + tc * TC;
+                conv_tile<K, TR, TC>(win, P.X.stride, wb, make_float2(bias, bias), [&](int o, float2(&a)[NP]) {
+                    const int h = tr * TR + o;
+                    if (h < P.H) finish_row<T>(sm, P, yp, h, tc * TC, a);
+                });
+            }
         }
     }
+    cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
 // Weight gradient, stage 1: grid (C, groups).  The CTA of (c, g) walks the
-// planes b = g, g + groups, ... of channel c.  Thread t owns one tile of one
-// class (base, or level l subband s) for the whole walk and accumulates its
-// K*K correlation sums in registers; the CTA then reduces each class over its
+// planes b = g, g + groups, ... of channel c, staging the next (x, dy) pair
+// while it computes the current one.  Thread t owns one tile of one class
+// (base, or level l subband s) for the whole walk and accumulates its K*K
+// correlation sums in registers; the CTA then reduces each class over its
 // threads in a fixed order and writes one partial vector (plus sum dy).
 // ---------------------------------------------------------------------------
 template <int K, int TR, int TC, typename T>
-__global__ void __launch_bounds__(512) wtconv_bwdw_partial_kernel(const T* __restrict__ x,
-                                                                  const T* __restrict__ dy,
-                                                                  float* __restrict__ part, const Plan P) {
+__global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel(
+    const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const Plan P) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
     constexpr int p = K / 2, KK = K * K;
     const int tid = threadIdx.x, nt = blockDim.x;
     const int c = blockIdx.x, g = blockIdx.y, G = P.groups;
-    const int H = P.H, W = P.W, L = P.L;
+    const size_t plane_elems = (size_t)P.H * P.W;
+    auto csync = [&]() { __syncthreads(); };
 
     zero_smem(sm, P.smem_floats, tid, nt);
+    __syncthreads();
+    if (g < P.B) {
+        const size_t off = ((size_t)g * P.C + c) * plane_elems;
+        stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
+        stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
+    }
+    cp_async_commit();
 
     int cl = -1, tr = 0, tc = 0;
     if (tid < P.n_all_tiles) {
@@ -394,53 +732,60 @@ __global__ void __launch_bounds__(512) wtconv_bwdw_partial_kernel(const T* __res
         while (tid >= P.cls_begin[cl + 1]) ++cl;
         const int lvl = (cl == 0) ? kMaxL : ((cl - 1) >> 2);
         const int local = tid - P.cls_begin[cl];
-        tr = local / P.ntc[lvl];
+        tr = fdiv(local, P.div_ntc[lvl]);
         tc = local - tr * P.ntc[lvl];
     }
-    float acc[KK];
+    float2 acc[KK];
 #pragma unroll
-    for (int t = 0; t < KK; ++t) acc[t] = 0.f;
-    float sdy = 0.f;
-    __syncthreads();
+    for (int t = 0; t < KK; ++t) acc[t] = make_float2(0.f, 0.f);
+    float sdy = 0.f, sdy_c = 0.f;  // compensated running sum of dy over the walk
 
+    float* X0 = sm + P.X.base + p * P.X.stride + p;
     for (int b = g; b < P.B; b += G) {
-        const size_t poff = ((size_t)b * P.C + c) * H * W;
-        load_plane<T, p, false>(x + poff, H, W, sm + P.X.base + p * P.X.stride + p, P.X.stride, tid, nt);
-        sdy += load_plane<T, 0, true>(dy + poff, H, W, sm + P.DY.base, P.DY.stride, tid, nt);
-        __syncthreads();
-        for (int l = 0; l < L; ++l) {
-            const float* xs = (l == 0) ? sm + P.X.base + p * P.X.stride + p
-                                       : sm + P.S[l - 1].base + p * P.S[l - 1].stride + p;
-            const int xss = (l == 0) ? P.X.stride : P.S[l - 1].stride;
-            haar_level(xs, xss, H >> (l + 1), W >> (l + 1), sm + P.S[l].base + p * P.S[l].stride + p,
-                       P.S[l].stride, P.S[l].sub, tid, nt);
-            const float* ds = (l == 0) ? sm + P.DY.base : sm + P.Q[l - 1].base;
-            const int dss = (l == 0) ? P.DY.stride : P.Q[l - 1].stride;
-            haar_level(ds, dss, H >> (l + 1), W >> (l + 1), sm + P.Q[l].base, P.Q[l].stride, P.Q[l].sub,
-                       tid, nt);
-            __syncthreads();
+        cp_async_wait_all();
+        __syncthreads();  // staged pair complete; previous correlations done
+        analyse_plane<T, p, false>(sm, P, sm + P.stg, X0, P.X.stride, P.S, p, nt, tid, csync);
+        const float s = analyse_plane<T, 0, true>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base, P.DY.stride,
+                                                  P.Q, 0, nt, tid, csync);
+        {
+            const float yv = s - sdy_c;
+            const float tv = sdy + yv;
+            sdy_c = (tv - sdy) - yv;
+            sdy = tv;
         }
+        __syncthreads();
+        if (b + G < P.B) {
+            const size_t off = ((size_t)(b + G) * P.C + c) * plane_elems;
+            stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
+            stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
+        }
+        cp_async_commit();
         if (cl == 0) {
             corr_tile<K, TR, TC>(sm + P.X.base + tr * TR * P.X.stride + tc * TC, P.X.stride,
                                  sm + P.DY.base + tr * TR * P.DY.stride + tc * TC, P.DY.stride, acc);
         } else if (cl > 0) {
-            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+            const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
             const Buf& S = P.S[l];
             const Buf& Q = P.Q[l];
-            corr_tile<K, TR, TC>(sm + S.base + s * S.sub + tr * TR * S.stride + tc * TC, S.stride,
-                                 sm + Q.base + s * Q.sub + tr * TR * Q.stride + tc * TC, Q.stride, acc);
+            corr_tile<K, TR, TC>(sm + S.base + s2 * S.sub + tr * TR * S.stride + tc * TC, S.stride,
+                                 sm + Q.base + s2 * Q.sub + tr * TR * Q.stride + tc * TC, Q.stride, acc);
         }
-        __syncthreads();
     }
+    cp_async_wait_all();
+    __syncthreads();
 
     // Fixed-order reduction of every class over its threads.
     float* red = sm + P.red;
 #pragma unroll
-    for (int t = 0; t < KK; ++t) red[tid * KK + t] = acc[t];
-    red[nt * KK + tid] = sdy;
+    for (int t = 0; t < KK; ++t) red[tid * KK + t] = acc[t].x + acc[t].y;
+    // sum dy: a fixed xor-tree inside each warp, then the warps in order.
+    float sw = sdy;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
+    if ((tid & 31) == 0) red[nt * KK + (tid >> 5)] = sw;
     __syncthreads();
     float* out = part + ((size_t)c * G + g) * P.nv;
-    const int ncls = 1 + 4 * L;
+    const int ncls = 1 + 4 * P.L;
     for (int t = tid; t < ncls * KK; t += nt) {
         const int k2 = t / KK, tap = t - k2 * KK;
         float s = 0.f;
@@ -449,7 +794,7 @@ __global__ void __launch_bounds__(512) wtconv_bwdw_partial_kernel(const T* __res
     }
     if (tid == 0) {
         float s = 0.f;
-        for (int th = 0; th < nt; ++th) s += red[nt * KK + th];
+        for (int w = 0; w < (nt >> 5); ++w) s += red[nt * KK + w];
         out[ncls * KK] = s;
     }
 }

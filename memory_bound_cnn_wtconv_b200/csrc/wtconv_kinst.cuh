@@ -2,6 +2,8 @@
 // wtconv_k<K>.cu with WTC_K defined.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "wtconv_kernels.cuh"
 #include "wtconv_launch.h"
 
@@ -37,7 +39,16 @@ cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
     auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
-    fn<<<P.B * P.C, P.nthreads, (size_t)P.smem_floats * 4, s>>>(
+    // Persistent grid: every resident CTA slot of the device, at most one CTA per plane.
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, P.nthreads, (size_t)P.smem_floats * 4)) !=
+        cudaSuccess)
+        return e;
+    const long long units = (long long)P.B * P.C;
+    const int grid = (int)std::min<long long>(units, (long long)sms * std::max(per_sm, 1));
+    fn<<<grid, P.nthreads, (size_t)P.smem_floats * 4, s>>>(
         static_cast<const T*>(a.x), a.base_w, a.base_b, a.base_scale, a.wt_w, a.wt_scale, static_cast<T*>(a.y),
         P);
     return cudaGetLastError();

@@ -1,17 +1,20 @@
 // Shared-memory and tile plan for the fused WTConv kernels.
 //
-// One CTA stages one whole (b, c) plane on chip.  Every buffer below lives in
-// dynamic shared memory; offsets and strides are in floats.  The plan is built
-// on the host (wtconv_plan.cpp) and passed to the kernels by value.
+// A CTA stages whole (b, c) planes on chip, one after another (persistent):
+// while it computes one plane, cp.async copies the next plane into a staging
+// buffer.  Every buffer below lives in dynamic shared memory; offsets and
+// strides are in floats.  The plan is built on the host (wtconv_planner.h)
+// and passed to the kernels by value.
 //
 // Buffers:
-//   X      padded input plane (x in the forward, dy in the input gradient,
-//          x in the weight gradient), p = k/2 zero rows/cols around it.
-//   S[l]   padded un-normalised Haar subbands of level l (4 planes).
+//   STG    raw staging of the next plane(s), as stored in HBM (float or bf16):
+//          x (forward), dy (input gradient), x then dy (weight gradient).
+//   X      padded input plane, p = k/2 zero rows/cols around it.
+//   S[l]   padded un-normalised Haar subbands of level l (4 planes) of X.
 //   Q[l]   forward: subband conv outputs of level l (4 planes, tile-rounded);
 //          weight gradient: Haar subbands of dy (4 planes, tile-rounded).
-//   Z      forward: coarse-level synthesis at half resolution (aliases S[0]).
 //   DY     weight gradient: dy plane (tile-rounded).
+//   W      forward: folded weights, one class (K*K floats) per subband and the base.
 //
 // Padded buffers: `base` is the offset of padded element (-p, -p), so a
 // conv window for the output tile whose top-left output is (r0, c0) starts
@@ -19,10 +22,37 @@
 // multiples of 4).  Unpadded buffers: element (i, j) is at base + i*stride + j.
 #pragma once
 
+#include <stdint.h>
+
 namespace wtc {
 
 constexpr int kMaxL = 6;
 constexpr int kMaxCls = 1 + 4 * kMaxL;
+
+// Division by a runtime constant d as a multiply-high and a shift:
+//   n / d == (umulhi(n, mul) + n) >> shift   for 0 <= n < 2^31,
+// with shift = ceil(log2 d) and mul = floor(2^32 (2^shift - d) / d) + 1.
+struct FastDiv {
+    uint32_t mul;
+    uint32_t shift;
+};
+
+inline uint32_t fastdiv_host(uint32_t n, FastDiv f) {
+    return (uint32_t)(((((uint64_t)n * f.mul) >> 32) + n) >> f.shift);
+}
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    FastDiv f;
+    f.shift = l;
+    f.mul = (uint32_t)(((((uint64_t)1 << l) - d) << 32) / d + 1);
+    return f;
+}
+
+// Thread budgets (also the kernels' __launch_bounds__, two CTAs per SM).
+constexpr int kFusedMaxThreads = 320;
+constexpr int kBwdwMaxThreads = 320;
 
 struct Buf {
     int base;    // float offset (see above)
@@ -32,14 +62,19 @@ struct Buf {
 
 struct Plan {
     int B, C, H, W, k, L, p;
-    int TR, TC;          // output tile: TR rows x TC cols per thread
+    int TR, TC;          // output tile: TR rows x TC cols per thread (TC = 4: two column pairs)
+    int esize;           // bytes per stored activation (4 or 2)
     int nthreads;        // CTA size
     int smem_floats;     // dynamic shared memory, in floats (multiple of 4)
+    int grid;            // forward: number of persistent CTAs
     int groups;          // weight gradient: batch groups (grid.y)
-    int wbase, wcls;     // folded weights: class cl (0 = base, 1 + 4l + s) at wbase + cl*wcls
-    int bias;            // folded bias (forward)
-    int red;             // weight gradient: reduction scratch (aliases S / Q)
-    Buf X, DY, Z;
+    int wbase, wcls;     // forward: folded weights of class cl (0 = base, 1 + 4l + s) at wbase + cl*wcls
+    int bias;            // forward: folded bias
+    int red;             // weight gradient: reduction scratch (aliases the plane buffers)
+    int stg;             // staging buffer offset; one stored plane occupies stg_floats floats
+    int stg_floats;
+    int plane_chunks;    // 16-byte chunks per stored plane
+    Buf X, DY;
     Buf S[kMaxL], Q[kMaxL];
     int ntr[kMaxL + 1], ntc[kMaxL + 1];  // tile grid per level; index kMaxL = full resolution
     // Tile enumeration.  Forward: subband tiles in class order (l, s) first,
@@ -50,6 +85,15 @@ struct Plan {
     int cls_begin[kMaxCls + 1];
     int n_all_tiles;
     int nv;              // weight gradient: floats per partial vector = ncls*k*k + 1
+    int merged;          // forward: subband and base tiles run in one phase (one tile per thread)
+    int base_tid0;       // forward, merged: first thread of the base tiles (a warp boundary)
+    int pyr;             // analysis by the one-pass pyramid (H % 4 == 0 and L >= 1)
+    int pyr_levels;      // levels the pyramid computes (min(L, 4)); the rest run level by level
+    int pyr_lg;          // pyramid lane groups cover (4 * 2^pyr_lg)^2 pixel regions
+    FastDiv div_rw;      // (W >> (pyr_lg + 2)): pyramid regions per row
+    FastDiv div_q4;                 // W / 4: 4-column groups per row
+    FastDiv div_m[kMaxL];           // W >> (l+1)
+    FastDiv div_ntc[kMaxL + 1];     // tile columns per tile row
 };
 
 }  // namespace wtc

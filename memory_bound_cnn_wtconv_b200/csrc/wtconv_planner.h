@@ -14,7 +14,8 @@
 namespace wtc {
 
 constexpr int kSmemLimitFloats = 227 * 1024 / 4;
-constexpr int kNumSMs = 148;  // B200; only used to size the weight-gradient grid
+constexpr int kSmemPerSM = 228 * 1024;
+constexpr int kNumSMs = 148;  // B200; sizes the persistent grids
 
 enum Kind { kForward = 0, kBackwardInput = 1, kBackwardWeight = 2 };
 
@@ -34,11 +35,9 @@ inline int pick_stride(int min_floats, int TR, int ntc) {
     return s;
 }
 
-// Work-weighted fraction of tile slack for tile height TR (smaller is better).
+// Work-weighted tile slack for tile height TR (smaller is better).
 inline double tile_waste(const wtconv_desc_t* d, int TR) {
-    double used = 0.0, total = 0.0;
-    used += d->H;
-    total += ceil_div(d->H, TR) * (double)TR;
+    double used = d->H, total = ceil_div(d->H, TR) * (double)TR;
     for (int l = 0; l < d->L; ++l) {
         const int n = d->H >> (l + 1);
         const double w = 1.0 / (double)(1 << (2 * l));  // level-l work relative to the base conv
@@ -46,6 +45,33 @@ inline double tile_waste(const wtconv_desc_t* d, int TR) {
         total += w * ceil_div(n, TR) * (double)TR;
     }
     return total / used;
+}
+
+// CTAs per SM that the shared memory of one CTA allows (the register
+// budget of the launch bounds allows two).
+inline int ctas_per_sm(int smem_floats) {
+    return std::max(1, std::min(2, kSmemPerSM / (smem_floats * 4 + 1024)));
+}
+
+// Weight-gradient batch groups (grid.y): the CTA of group g walks planes
+// b = g, g + groups, ...  Chosen to minimise waves x planes-per-CTA over the
+// resident CTA slots, with at most 64 planes per CTA so every per-thread
+// running sum stays short.
+inline int pick_groups(int B, int C, int smem_floats) {
+    const long long slots = (long long)kNumSMs * ctas_per_sm(smem_floats);
+    int best = 1;
+    long long best_cost = -1;
+    for (int g = 1; g <= B; ++g) {
+        const int planes = ceil_div(B, g);
+        if (planes > 64 && g != B) continue;
+        const long long waves = (C * (long long)g + slots - 1) / slots;
+        const long long cost = waves * (planes + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = g;
+        }
+    }
+    return best;
 }
 
 inline bool is_supported_k(int k) { return k == 1 || k == 3 || k == 5 || k == 7; }
@@ -58,6 +84,9 @@ inline wtconv_status_t validate(const wtconv_desc_t* d) {
     if (d->L < 0 || d->L > kMaxL) return WTCONV_ERR_BAD_L;
     if ((d->H % (1 << d->L)) != 0 || (d->W % (1 << d->L)) != 0) return WTCONV_ERR_BAD_SHAPE;
     if ((d->W % 4) != 0) return WTCONV_ERR_BAD_SHAPE;
+    // Planes are staged in 16-byte chunks.
+    const long long esize = d->dtype == WTCONV_BF16 ? 2 : 4;
+    if (((long long)d->H * d->W * esize) % 16 != 0) return WTCONV_ERR_BAD_SHAPE;
     // Index arithmetic in the kernels is 32-bit within a plane and 64-bit across planes.
     if ((long long)d->H * d->W > (1LL << 30)) return WTCONV_ERR_BAD_SHAPE;
     if ((long long)d->B * d->C > (1LL << 31) - 1) return WTCONV_ERR_BAD_SHAPE;
@@ -69,8 +98,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     memset(P, 0, sizeof(*P));
     P->B = d->B; P->C = d->C; P->H = d->H; P->W = d->W; P->k = d->k; P->L = d->L;
-    const int p = d->k / 2, k = d->k, L = d->L, H = d->H, W = d->W;
+    const int p = d->k / 2, k = d->k, L = d->L, H = d->H, W = d->W, KK = k * k;
     P->p = p;
+    P->esize = d->dtype == WTCONV_BF16 ? 2 : 4;
     P->TC = 4;
     P->TR = tile_waste(d, 7) < tile_waste(d, 8) ? 7 : 8;
     const int TR = P->TR, TC = P->TC;
@@ -86,7 +116,7 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     long long off = 0;
     const int ncls = 1 + 4 * L;
     if (kind != kBackwardWeight) {
-        P->wcls = round4(k * k);
+        P->wcls = round4(KK);  // each class 16-byte aligned
         P->wbase = (int)off;
         off += (long long)ncls * P->wcls;
         P->bias = (int)off;
@@ -114,26 +144,25 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     }
     // Tile-rounded, unpadded planes: conv outputs (forward) or dy subbands.
     for (int l = 0; l < L; ++l) {
-        const int ntc = P->ntc[l];
         const int rows = P->ntr[l] * TR;
-        P->Q[l].stride = pick_stride(ntc * TC, TR, ntc);
+        P->Q[l].stride = round4(P->ntc[l] * TC);
         P->Q[l].sub = round4(rows * P->Q[l].stride);
         P->Q[l].base = (int)off;
         off += 4LL * P->Q[l].sub;
     }
-    if (kind != kBackwardWeight) {
-        if (L >= 2) {
-            // Coarse-level sum at half resolution; S[0] is dead by then.
-            P->Z.stride = round4(W >> 1);
-            P->Z.base = P->S[0].base;
-            if ((long long)(H >> 1) * P->Z.stride > 4LL * P->S[0].sub) return WTCONV_ERR_UNSUPPORTED;
-        }
-    } else {
-        const int ntc = P->ntc[kMaxL];
+    if (kind == kBackwardWeight) {
         const int rows = P->ntr[kMaxL] * TR;
-        P->DY.stride = pick_stride(ntc * TC, TR, ntc);
+        P->DY.stride = round4(P->ntc[kMaxL] * TC);
         P->DY.base = (int)off;
         off += round4(rows * P->DY.stride);
+    }
+    // Staging of the next plane(s), stored format.
+    {
+        const long long bytes = (long long)H * W * P->esize;
+        P->plane_chunks = (int)(bytes / 16);
+        P->stg_floats = (int)(bytes / 4);
+        P->stg = (int)off;
+        off += (kind == kBackwardWeight ? 2LL : 1LL) * P->stg_floats;
     }
 
     // Tiles and threads.
@@ -153,31 +182,44 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
         P->cls_begin[cl + 1] = P->cls_begin[cl] + P->ntr[l] * P->ntc[l];
     }
     P->n_all_tiles = P->cls_begin[ncls];
-    P->nv = ncls * k * k + 1;
+    P->nv = ncls * KK + 1;
+
+    P->pyr = (L >= 1 && H % 4 == 0) ? 1 : 0;
+    P->pyr_levels = std::min(L, 4);
+    P->pyr_lg = std::max(P->pyr_levels - 2, 0);
+    P->div_rw = make_fastdiv(std::max(W >> (P->pyr_lg + 2), 1));
+    P->div_q4 = make_fastdiv(W / 4);
+    for (int l = 0; l < L; ++l) P->div_m[l] = make_fastdiv(W >> (l + 1));
+    for (int l = 0; l <= kMaxL; ++l) P->div_ntc[l] = make_fastdiv(std::max(P->ntc[l], 1));
 
     if (kind == kBackwardWeight) {
         const int nt = ceil_div(P->n_all_tiles, 32) * 32;
-        if (nt > 512) return WTCONV_ERR_UNSUPPORTED;
+        if (nt > kBwdwMaxThreads) return WTCONV_ERR_UNSUPPORTED;
         P->nthreads = std::max(nt, 64);
         // Reduction scratch aliases the (then dead) buffers from offset 0.
         P->red = 0;
-        const long long red_need = (long long)P->nthreads * (k * k + 1);
-        off = std::max(off, red_need);
-        // Batch groups: about two CTAs per SM, and a divisor of B so every
-        // group walks the same number of planes.
-        const int target = std::max(1, ceil_div(2 * kNumSMs, d->C));
-        int g = 1;
-        for (int cand = 1; cand <= std::min(target, d->B); ++cand)
-            if (d->B % cand == 0) g = cand;
-        P->groups = g;
+        off = std::max(off, (long long)P->nthreads * (KK + 1));
     } else {
-        const int nt = ceil_div(std::max(P->n_sub_tiles, P->n_base_tiles), 32) * 32;
-        P->nthreads = std::min(std::max(nt, 64), 512);
-        P->groups = 1;
+        const int sub_pad = ceil_div(P->n_sub_tiles, 32) * 32;
+        if (sub_pad + P->n_base_tiles <= kFusedMaxThreads) {
+            P->merged = 1;
+            P->base_tid0 = sub_pad;
+            P->nthreads = std::max(64, ceil_div(sub_pad + P->n_base_tiles, 32) * 32);
+        } else {
+            P->merged = 0;
+            P->nthreads = kFusedMaxThreads;
+        }
     }
     off = round4((int)std::min<long long>(off, 1LL << 30));
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;
+    if (kind == kBackwardWeight) {
+        P->groups = pick_groups(P->B, P->C, P->smem_floats);
+    } else {
+        const long long units = (long long)P->B * P->C;
+        P->grid = (int)std::min<long long>(units, (long long)kNumSMs * ctas_per_sm(P->smem_floats));
+        P->groups = 1;
+    }
     return WTCONV_OK;
 }
 

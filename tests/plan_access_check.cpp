@@ -57,13 +57,110 @@ void check_global(long long idx, long long n, const char* what) {
     }
 }
 
-// Replays load_plane: element (i, j) -> dst + i*stride + j.
-void replay_load(Shadow& sh, const Plan& P, long long dst, int stride, long long lo, long long hi, int t) {
-    for (int i = 0; i < P.H; ++i)
-        for (int j = 0; j < P.W; j += 4) {
-            check_global((long long)i * P.W + j + 3, (long long)P.H * P.W, "plane load");
-            for (int e = 0; e < 4; ++e) sh.write(dst + (long long)i * stride + j + e, lo, hi, t, "plane store");
+// Replays stage_plane: 16-byte chunk ch of the stored plane -> staging floats [stg + 4ch, stg + 4ch + 4).
+void replay_stage(Shadow& sh, const Plan& P, long long stg, int tag) {
+    const long long plane_bytes = (long long)P.H * P.W * P.esize;
+    if (P.plane_chunks * 16LL != plane_bytes) sh.fail("plane is not a whole number of 16-byte chunks", plane_bytes);
+    if (stg % 4) sh.fail("staging not 16-byte aligned", stg);
+    for (int ch = 0; ch < P.plane_chunks; ++ch) {
+        check_global(16LL * ch + 15, plane_bytes, "staging source");
+        for (int e = 0; e < 4; ++e) sh.write(stg + 4LL * ch + e, stg, stg + P.stg_floats, tag, "staging");
+    }
+}
+
+// Replays unpack_level0: staged element e (4 at a time) -> dst (element (0,0) at `dst`, row stride ds),
+// and, if level0, the level-0 butterflies of rows 2i, 2i+1 / columns 4q..4q+3 -> the 4 subband planes.
+void replay_unpack(Shadow& sh, const Plan& P, long long stg, int stag, long long dst, int ds, long long dlo,
+                   long long dhi, int dtag, long long sb, int sbs, int sbsub, long long sblo, int (*sbtag)(int, int),
+                   bool level0) {
+    const int W = P.W;
+    auto stage_read = [&](int e) {  // 4 elements at element index e
+        if (e % 4) sh.fail("staged load not 4-element aligned", e);
+        const long long f0 = stg + (long long)e * P.esize / 4;
+        const int nf = P.esize;  // 4 elements = esize floats
+        for (int q = 0; q < nf; ++q) sh.read(f0 + q, stg, stg + P.stg_floats, stag, "staging read");
+    };
+    const int rows = level0 ? P.H / 2 : P.H;
+    for (int i = 0; i < rows; ++i)
+        for (int q = 0; q < W / 4; ++q) {
+            const int nr = level0 ? 2 : 1;
+            for (int rr = 0; rr < nr; ++rr) {
+                const int r = level0 ? 2 * i + rr : i;
+                stage_read(r * W + 4 * q);
+                for (int e = 0; e < 4; ++e) sh.write(dst + (long long)r * ds + 4 * q + e, dlo, dhi, dtag, "unpack store");
+            }
+            if (level0)
+                for (int s = 0; s < 4; ++s)
+                    for (int e = 0; e < 2; ++e)
+                        sh.write(sb + (long long)s * sbsub + (long long)i * sbs + 2 * q + e, sblo + (long long)s * sbsub,
+                                 sblo + (long long)(s + 1) * sbsub, sbtag(0, s), "level-0 store");
         }
+}
+
+void replay_haar(Shadow& sh, long long src, int ss, long long slo, long long shi, int stag, int n, int m,
+                 long long dst, int ds, int dsub, long long dlo, long long dhi, int (*dtag)(int, int), int l);
+
+// Replays analysis_pyramid: threads own 4x4 blocks (lane groups of G*G
+// lanes per (4G)^2 region), write the block into the plane buffer, levels 0
+// and 1 to their subband planes, and levels 2.. from the group leader.
+void replay_pyramid(Shadow& sh, const Plan& P, long long stg, int stag, long long dst, int ds, long long dlo,
+                    long long dhi, int dtag, const Buf* bufs, int pad, int (*sbtag)(int, int)) {
+    const int H = P.H, W = P.W, lg = P.pyr_lg, G = 1 << lg, G2 = G * G;
+    if ((4 * G) != (P.pyr_levels >= 2 ? (1 << P.pyr_levels) : 4)) sh.fail("pyramid region size", G);
+    if (H % (4 * G) || W % (4 * G)) sh.fail("pyramid regions must tile the plane", G);
+    if (32 % G2) sh.fail("pyramid lane group must divide a warp", G2);
+    const int nreg_w = W >> (lg + 2);
+    const int items = (H >> (lg + 2)) * nreg_w * G2;
+    for (int item = 0; item < items; ++item) {
+        const int r = item >> (2 * lg), o = item & (G2 - 1);
+        const int by = o >> lg, bx = o & (G - 1);
+        const int rrow = (int)fastdiv_host(r, P.div_rw), rcol = r - rrow * nreg_w;
+        if (rrow != r / nreg_w) sh.fail("region row division", r);
+        const int brow = rrow * G + by, bcol = rcol * G + bx;
+        const int r0 = 4 * brow, c0 = 4 * bcol;
+        for (int q = 0; q < 4; ++q) {
+            const long long f0 = stg + (long long)((r0 + q) * W + c0) * P.esize / 4;
+            for (int e = 0; e < P.esize; ++e) sh.read(f0 + e, stg, stg + P.stg_floats, stag, "pyramid staging read");
+            for (int e = 0; e < 4; ++e) sh.write(dst + (long long)(r0 + q) * ds + c0 + e, dlo, dhi, dtag, "pyramid plane store");
+        }
+        auto lvl_store = [&](int l, int i, int j) {
+            const Buf& b = bufs[l];
+            if (i >= (H >> (l + 1)) || j >= (W >> (l + 1))) sh.fail("pyramid subband index", l);
+            for (int s2 = 0; s2 < 4; ++s2)
+                sh.write(b.base + (long long)s2 * b.sub + (long long)(i + pad) * b.stride + (j + pad), b.base + (long long)s2 * b.sub,
+                         b.base + (long long)(s2 + 1) * b.sub, sbtag(l, s2), "pyramid subband store");
+        };
+        for (int pi = 0; pi < 2; ++pi)
+            for (int pj = 0; pj < 2; ++pj) lvl_store(0, 2 * brow + pi, 2 * bcol + pj);
+        if (P.pyr_levels >= 2) lvl_store(1, brow, bcol);
+        for (int l = 2; l < P.pyr_levels; ++l) {
+            const int sh2 = l - 2, m = (2 << sh2) - 1;
+            if ((G << sh2) >= G2) sh.fail("shuffle partner outside the lane group", l);
+            if ((by & m) == 0 && (bx & m) == 0) lvl_store(l, brow >> (l - 1), bcol >> (l - 1));
+        }
+    }
+}
+
+// Replays analyse_plane (pyramid or unpack + level 0, then the remaining levels one by one).
+void replay_analyse(Shadow& sh, const Plan& P, long long stg, int stag, long long dst, int ds, long long dlo, long long dhi,
+                    int dtag, const Buf* bufs, int pad, int (*sbtag)(int, int)) {
+    int done;
+    if (P.pyr) {
+        replay_pyramid(sh, P, stg, stag, dst, ds, dlo, dhi, dtag, bufs, pad, sbtag);
+        done = P.pyr_levels;
+    } else {
+        const Buf& b = bufs[0];
+        replay_unpack(sh, P, stg, stag, dst, ds, dlo, dhi, dtag, P.L >= 1 ? b.base + (long long)pad * b.stride + pad : 0,
+                      b.stride, b.sub, b.base, sbtag, P.L >= 1);
+        done = P.L >= 1 ? 1 : 0;
+    }
+    for (int l = done; l < P.L; ++l) {
+        const int n = P.H >> (l + 1), m = P.W >> (l + 1);
+        const Buf& s0 = bufs[l - 1];
+        const Buf& s1 = bufs[l];
+        replay_haar(sh, s0.base + (long long)pad * s0.stride + pad, s0.stride, s0.base, s0.base + s0.sub, sbtag(l - 1, 0), n, m,
+                    s1.base + (long long)pad * s1.stride + pad, s1.stride, s1.sub, s1.base, s1.base + 4LL * s1.sub, sbtag, l);
+    }
 }
 
 // Replays haar_level.
@@ -122,6 +219,26 @@ void replay_dtile(Shadow& sh, const Plan& P, long long base, int stride, long lo
         }
 }
 
+// The kernels compute n / d as fastdiv(n); check it exactly for every n the
+// kernel can pass (0 <= n < nmax).
+void check_div(FastDiv f, int d, long long nmax, const char* what) {
+    for (long long n = 0; n < nmax; ++n)
+        if ((long long)fastdiv_host((uint32_t)n, f) != n / d) {
+            std::printf("FAIL fastdiv %s: %lld / %d\n", what, n, d);
+            std::exit(1);
+        }
+}
+
+void check_divs(const Plan& P) {
+    check_div(P.div_q4, P.W / 4, (long long)P.H * (P.W / 4) + 1, "W/4");
+    for (int l = 0; l < P.L; ++l)
+        check_div(P.div_m[l], P.W >> (l + 1), (long long)(P.H >> (l + 1)) * (P.W >> (l + 1)) + 1, "level cols");
+    for (int l = 0; l <= kMaxL; ++l) {
+        if (l < kMaxL && l >= P.L) continue;
+        check_div(P.div_ntc[l], P.ntc[l], (long long)P.ntr[l] * P.ntc[l] + 1, "tile cols");
+    }
+}
+
 void check_fused(const wtconv_desc_t& d, Kind kind) {
     Plan P;
     const wtconv_status_t st = make_plan(&d, kind, &P);
@@ -135,114 +252,114 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     }
     const int K = P.k, KK = K * K, p = P.p, L = P.L, H = P.H, W = P.W, TR = P.TR, TC = P.TC;
     const int ncls = 1 + 4 * L;
+    check_divs(P);
+    if (P.nthreads % 32 || P.nthreads > kFusedMaxThreads || P.nthreads < 32) {
+        std::printf("FAIL fused thread count %d\n", P.nthreads);
+        std::exit(1);
+    }
+    if (P.merged && (P.base_tid0 % 32 || P.base_tid0 < P.n_sub_tiles || P.base_tid0 + P.n_base_tiles > P.nthreads)) {
+        std::printf("FAIL merged layout: sub %d base0 %d base %d threads %d\n", P.n_sub_tiles, P.base_tid0,
+                    P.n_base_tiles, P.nthreads);
+        std::exit(1);
+    }
     if (P.smem_floats % 4 || P.smem_floats * 4 > 227 * 1024) {
         std::printf("FAIL smem size\n");
         std::exit(1);
     }
     Shadow sh(P.smem_floats);
     const long long all = P.smem_floats;
-    sh.phase = "weights";
-    for (int cl = 0; cl < ncls; ++cl)
-        for (int t = 0; t < KK; ++t)
-            sh.write(P.wbase + (long long)cl * P.wcls + t, P.wbase, P.wbase + (long long)ncls * P.wcls, WTS, "weights");
-    sh.write(P.bias, P.bias, P.bias + 1, BIAS, "bias");
-    for (int cl = 0; cl < ncls; ++cl)
-        if ((P.wbase + cl * P.wcls) % 4) sh.fail("weight class not 16-byte aligned", P.wbase + cl * P.wcls);
-
+    if (P.grid < 1 || P.grid > (long long)P.B * P.C) sh.fail("grid", P.grid);
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
-    sh.phase = "load";
-    replay_load(sh, P, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT);
-
-    sh.phase = "analysis";
-    for (int l = 0; l < L; ++l) {
-        const int n = H >> (l + 1), m = W >> (l + 1);
-        long long src, slo, shi;
-        int ss, stag;
-        if (l == 0) {
-            src = P.X.base + (long long)p * P.X.stride + p; ss = P.X.stride; slo = xlo; shi = xhi; stag = XT;
-        } else {
-            const Buf& S = P.S[l - 1];
-            src = S.base + (long long)p * S.stride + p; ss = S.stride; slo = S.base; shi = S.base + S.sub; stag = s_tag(l - 1, 0);
+    for (int cl = 0; cl < ncls; ++cl)
+        if ((P.wbase + cl * P.wcls) % 4) sh.fail("weight class not 16-byte aligned", P.wbase + cl * P.wcls);
+    // Two planes in a row through one persistent CTA: the second must see the
+    // same zero padding and slack.
+    for (int unit = 0; unit < 2; ++unit) {
+        sh.phase = "staging";
+        replay_stage(sh, P, P.stg, XT + 10);
+        sh.phase = "weights";
+        for (int cl = 0; cl < ncls; ++cl)
+            for (int t = 0; t < KK; ++t)
+                sh.write(P.wbase + (long long)cl * P.wcls + t, P.wbase, P.wbase + (long long)ncls * P.wcls, WTS, "weights");
+        sh.write(P.bias, P.bias, P.bias + 1, BIAS, "bias");
+        sh.phase = "analysis";
+        replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S, p, s_tag);
+        sh.phase = "conv tiles";
+        for (int cl = 1; cl < ncls; ++cl) {
+            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+            const int n = H >> (l + 1), m = W >> (l + 1);
+            const int ntiles = P.sub_begin[cl] - P.sub_begin[cl - 1];
+            if (ntiles != P.ntr[l] * P.ntc[l]) sh.fail("tile count", cl);
+            for (int local = 0; local < ntiles; ++local) {
+                const int tr = (int)fastdiv_host(local, P.div_ntc[l]), tc = local - tr * P.ntc[l];
+                for (int t = 0; t < KK; ++t) sh.read(P.wbase + (long long)cl * P.wcls + t, 0, all, WTS, "weights");
+                const Buf& S = P.S[l];
+                replay_window(sh, P, S.base + (long long)s * S.sub, S.stride, S.base + (long long)s * S.sub,
+                              S.base + (long long)(s + 1) * S.sub, n, m, tr, tc, s_tag(l, s), "subband window");
+                const Buf& Q = P.Q[l];
+                const long long out = Q.base + (long long)s * Q.sub + (long long)tr * TR * Q.stride + (long long)tc * TC;
+                if (out % 4) sh.fail("Q tile not 16-byte aligned", out);
+                for (int o = 0; o < TR; ++o)
+                    for (int j = 0; j < TC; ++j)
+                        sh.write(out + (long long)o * Q.stride + j, Q.base + (long long)s * Q.sub,
+                                 Q.base + (long long)(s + 1) * Q.sub, q_tag(l, s), "Q tile");
+            }
         }
-        const Buf& S = P.S[l];
-        replay_haar(sh, src, ss, slo, shi, stag, n, m, S.base + (long long)p * S.stride + p, S.stride, S.sub, S.base,
-                    S.base + 4LL * S.sub, s_tag, l);
-    }
-
-    sh.phase = "subband convs";
-    for (int cl = 1; cl < ncls; ++cl) {
-        const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-        const int n = H >> (l + 1), m = W >> (l + 1);
-        const int ntiles = P.sub_begin[cl] - P.sub_begin[cl - 1];
-        if (ntiles != P.ntr[l] * P.ntc[l]) sh.fail("tile count", cl);
-        for (int local = 0; local < ntiles; ++local) {
-            const int tr = local / P.ntc[l], tc = local % P.ntc[l];
-            for (int t = 0; t < KK; ++t) sh.read(P.wbase + (long long)cl * P.wcls + t, 0, all, WTS, "weights");
-            const Buf& S = P.S[l];
-            replay_window(sh, P, S.base + (long long)s * S.sub, S.stride, S.base + (long long)s * S.sub,
-                          S.base + (long long)(s + 1) * S.sub, n, m, tr, tc, s_tag(l, s), "subband window");
+        const int ntc = P.ntc[kMaxL];
+        for (int t = 0; t < P.n_base_tiles; ++t) {
+            const int tr = (int)fastdiv_host(t, P.div_ntc[kMaxL]), tc = t - tr * ntc;
+            for (int q = 0; q < KK; ++q) sh.read(P.wbase + q, 0, all, WTS, "base weights");
+            sh.read(P.bias, 0, all, BIAS, "bias");
+            replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base window");
+        }
+        const int n0 = H >> 1, m0 = W >> 1;
+        sh.phase = "coarse cascade";
+        for (int l = L - 1; l >= 1; --l) {
             const Buf& Q = P.Q[l];
-            const long long out = Q.base + (long long)s * Q.sub + (long long)tr * TR * Q.stride + (long long)tc * TC;
-            if (out % 4) sh.fail("Q tile not 16-byte aligned", out);
-            for (int o = 0; o < TR; ++o)
-                for (int j = 0; j < TC; ++j)
-                    sh.write(out + (long long)o * Q.stride + j, Q.base + (long long)s * Q.sub,
-                             Q.base + (long long)(s + 1) * Q.sub, q_tag(l, s), "Q tile");
-        }
-    }
-
-    const int n0 = H >> 1, m0 = W >> 1;
-    if (L >= 2) {
-        sh.phase = "coarse synthesis";
-        std::vector<long long> zw;
-        for (int i = 0; i < n0; ++i)
-            for (int j = 0; j < m0; ++j) {
-                for (int l = 1; l < L; ++l) {
-                    const Buf& Q = P.Q[l];
-                    if ((i >> l) >= (H >> (l + 1)) || (j >> l) >= (W >> (l + 1))) sh.fail("coarse index", l);
-                    for (int s = 0; s < 4; ++s)
-                        sh.read(Q.base + (long long)(i >> l) * Q.stride + (j >> l) + (long long)s * Q.sub,
-                                Q.base + (long long)s * Q.sub, Q.base + (long long)(s + 1) * Q.sub, q_tag(l, s),
-                                "coarse Q read");
-                }
-                zw.push_back(P.Z.base + (long long)i * P.Z.stride + j);
+            const Buf& D = P.Q[l - 1];
+            const int n = H >> (l + 1), m = W >> (l + 1);
+            for (int t = 0; t < n * m; ++t) {
+                const int i = (int)fastdiv_host(t, P.div_m[l]), j = t - i * m;
+                if (i != t / m) sh.fail("cascade division", t);
+                for (int s2 = 0; s2 < 4; ++s2)
+                    sh.read(Q.base + (long long)s2 * Q.sub + (long long)i * Q.stride + j, Q.base + (long long)s2 * Q.sub,
+                            Q.base + (long long)(s2 + 1) * Q.sub, q_tag(l, s2), "cascade Q read");
+                const long long d = D.base + (long long)(2 * i) * D.stride + 2 * j;
+                if (d % 2) sh.fail("cascade pair not 8-byte aligned", d);
+                if (2 * i + 1 >= (H >> l) || 2 * j + 1 >= (W >> l)) sh.fail("cascade target index", l);
+                for (int a = 0; a < 2; ++a)
+                    for (int b = 0; b < 2; ++b)
+                        sh.read(d + (long long)a * D.stride + b, D.base, D.base + D.sub, q_tag(l - 1, 0), "cascade LL update");
             }
-        // Z overwrites dead S[0]; it must not touch X, weights, or any Q plane.
-        for (long long a : zw) {
-            sh.in_bounds(a, P.S[0].base, P.S[0].base + 4LL * P.S[0].sub, "Z write");
-            sh.tag[a] = ZT;
         }
-    }
-
-    sh.phase = "base conv + synthesis";
-    const int ntc = P.ntc[kMaxL];
-    for (int t = 0; t < P.n_base_tiles; ++t) {
-        const int tr = t / ntc, tc = t % ntc;
-        for (int q = 0; q < KK; ++q) sh.read(P.wbase + q, 0, all, WTS, "base weights");
-        sh.read(P.bias, 0, all, BIAS, "bias");
-        replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base window");
-        for (int o = 0; o < TR; ++o) {
-            const int h = tr * TR + o;
-            if (h >= H) continue;
-            const int w0 = tc * TC;
-            if (L >= 1) {
-                const Buf& Q = P.Q[0];
-                const int i = h >> 1;
-                for (int pos = 0; pos < TC / 2; ++pos) {
-                    const int j = (w0 >> 1) + pos;
-                    if (i >= n0 || j >= m0) sh.fail("level-0 synthesis index", j);
-                    for (int s = 0; s < 4; ++s)
-                        sh.read(Q.base + (long long)i * Q.stride + j + (long long)s * Q.sub, Q.base + (long long)s * Q.sub,
-                                Q.base + (long long)(s + 1) * Q.sub, q_tag(0, s), "level-0 Q read");
-                    if (L >= 2) sh.read(P.Z.base + (long long)i * P.Z.stride + j, 0, all, ZT, "Z read");
+        (void)n0;
+        sh.phase = "synthesis + store";
+        for (int t = 0; t < P.n_base_tiles; ++t) {
+            const int tr = (int)fastdiv_host(t, P.div_ntc[kMaxL]), tc = t - tr * ntc;
+            for (int o = 0; o < TR; ++o) {
+                const int h = tr * TR + o;
+                if (h >= H) continue;
+                const int w0 = tc * TC;
+                if (L >= 1) {
+                    const Buf& Q = P.Q[0];
+                    for (int g = 0; g < TC / 4; ++g)
+                        for (int s = 0; s < 4; ++s) {
+                            const long long a = Q.base + (long long)s * Q.sub + (long long)(h >> 1) * Q.stride + (w0 >> 1) + 2 * g;
+                            if (a % 2) sh.fail("level-0 pair load not 8-byte aligned", a);
+                            for (int e = 0; e < 2; ++e) {
+                                if ((w0 >> 1) + 2 * g + e >= m0) sh.fail("level-0 synthesis column", w0);
+                                sh.read(a + e, Q.base + (long long)s * Q.sub, Q.base + (long long)(s + 1) * Q.sub, q_tag(0, s),
+                                        "level-0 Q read");
+                            }
+                        }
                 }
+                for (int e = 0; e < TC; ++e) check_global((long long)h * W + w0 + e, (long long)H * W, "y store");
             }
-            for (int e = 0; e < TC; ++e) check_global((long long)h * W + w0 + e, (long long)H * W, "y store");
         }
     }
-    std::printf("fused(kind %d): smem %d B, threads %d, TR %d, tiles %d+%d\n", (int)kind, P.smem_floats * 4,
-                P.nthreads, TR, P.n_sub_tiles, P.n_base_tiles);
+    std::printf("fused(kind %d): smem %d B, threads %d, TR %d, tiles %d+%d, merged %d\n", (int)kind,
+                P.smem_floats * 4, P.nthreads, TR, P.n_sub_tiles, P.n_base_tiles, P.merged);
 }
 
 void check_bwdw(const wtconv_desc_t& d) {
@@ -258,53 +375,27 @@ void check_bwdw(const wtconv_desc_t& d) {
     }
     const int K = P.k, KK = K * K, p = P.p, L = P.L, H = P.H, W = P.W, TR = P.TR;
     const int ncls = 1 + 4 * L;
+    check_divs(P);
     Shadow sh(P.smem_floats);
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
     const long long dlo = P.DY.base, dhi = P.DY.base + (long long)P.ntr[kMaxL] * TR * P.DY.stride;
+    if (P.stg % 4 || P.stg_floats % 4) sh.fail("staging alignment", P.stg);
     // Two planes in a row: the second must see the same zero padding.
     for (int plane = 0; plane < 2; ++plane) {
-        sh.phase = "load";
-        replay_load(sh, P, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT);
-        replay_load(sh, P, P.DY.base, P.DY.stride, dlo, dhi, DYT);
+        sh.phase = "staging";
+        replay_stage(sh, P, P.stg, XT + 10);
+        replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10);
         sh.phase = "analysis";
-        for (int l = 0; l < L; ++l) {
-            const int n = H >> (l + 1), m = W >> (l + 1);
-            {
-                long long src, slo, shi;
-                int ss, stag;
-                if (l == 0) {
-                    src = P.X.base + (long long)p * P.X.stride + p; ss = P.X.stride; slo = xlo; shi = xhi; stag = XT;
-                } else {
-                    const Buf& S = P.S[l - 1];
-                    src = S.base + (long long)p * S.stride + p; ss = S.stride; slo = S.base; shi = S.base + S.sub;
-                    stag = s_tag(l - 1, 0);
-                }
-                const Buf& S = P.S[l];
-                replay_haar(sh, src, ss, slo, shi, stag, n, m, S.base + (long long)p * S.stride + p, S.stride, S.sub,
-                            S.base, S.base + 4LL * S.sub, s_tag, l);
-            }
-            {
-                long long src, slo, shi;
-                int ss, stag;
-                if (l == 0) {
-                    src = P.DY.base; ss = P.DY.stride; slo = dlo; shi = dhi; stag = DYT;
-                } else {
-                    const Buf& Q = P.Q[l - 1];
-                    src = Q.base; ss = Q.stride; slo = Q.base; shi = Q.base + Q.sub; stag = q_tag(l - 1, 0);
-                }
-                const Buf& Q = P.Q[l];
-                replay_haar(sh, src, ss, slo, shi, stag, n, m, Q.base, Q.stride, Q.sub, Q.base, Q.base + 4LL * Q.sub,
-                            q_tag, l);
-            }
-        }
+        replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S, p, s_tag);
+        replay_analyse(sh, P, P.stg + P.stg_floats, DYT + 10, P.DY.base, P.DY.stride, dlo, dhi, DYT, P.Q, 0, q_tag);
         sh.phase = "correlation";
         for (int tid = 0; tid < P.n_all_tiles; ++tid) {
             int cl = 0;
             while (tid >= P.cls_begin[cl + 1]) ++cl;
             const int lvl = (cl == 0) ? kMaxL : ((cl - 1) >> 2);
             const int local = tid - P.cls_begin[cl];
-            const int tr = local / P.ntc[lvl], tc = local % P.ntc[lvl];
+            const int tr = (int)fastdiv_host(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
             if (tr >= P.ntr[lvl]) sh.fail("tile row out of grid", tid);
             if (cl == 0) {
                 replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base S window");
@@ -324,8 +415,9 @@ void check_bwdw(const wtconv_desc_t& d) {
     sh.phase = "reduction";
     const long long red_end = (long long)P.red + (long long)P.nthreads * KK + P.nthreads;
     if (red_end > P.smem_floats) sh.fail("reduction scratch", red_end);
-    if (P.nthreads < P.n_all_tiles || P.nthreads > 512 || P.nthreads % 32) sh.fail("thread count", P.nthreads);
-    if (P.B % P.groups) sh.fail("groups must divide B", P.groups);
+    if (P.nthreads < P.n_all_tiles || P.nthreads > kBwdwMaxThreads || P.nthreads % 32) sh.fail("thread count", P.nthreads);
+    if (P.groups < 1 || P.groups > P.B) sh.fail("groups", P.groups);
+    if ((long long)P.nthreads * KK + P.nthreads / 32 > P.smem_floats) sh.fail("sum-dy scratch", P.nthreads);
     if (P.nv != ncls * KK + 1) sh.fail("partial vector length", P.nv);
     std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d, groups %d\n", P.smem_floats * 4, P.nthreads, TR,
                 P.n_all_tiles, P.groups);
