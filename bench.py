@@ -147,6 +147,28 @@ def dist_env():
     return world, rank, local
 
 
+def allreduce_weight_grads(grads: dict, flat, dist) -> None:
+    """Data parallel over the batch: sum the rank-local weight gradients over
+    all ranks (one all-reduce of the flattened tensors) and write the sums
+    back into `grads`."""
+    import torch
+    torch.cat([v.reshape(-1) for v in grads.values()], out=flat)
+    dist.all_reduce(flat)
+    off = 0
+    for v in grads.values():
+        n = v.numel()
+        v.copy_(flat[off:off + n].view_as(v))
+        off += n
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's value (timings are reported as the max over ranks)."""
+    import torch
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def physical_gpu_index(local: int) -> int:
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -269,8 +291,7 @@ def run_ours(args, case):
                            grads=grads, workspace=ws, stream=stream)
 
     def allreduce():
-        torch.cat([v.reshape(-1) for v in grads.values()], out=flat)
-        dist.all_reduce(flat)
+        allreduce_weight_grads(grads, flat, dist)
 
     calls = [("fwd", fwd), ("bwd_in", bwd_in), ("bwd_w", bwd_w)]
     if world > 1:
@@ -306,9 +327,7 @@ def run_ours(args, case):
                 for i, (name, _) in enumerate(calls)}
     step_ms = sum(per_call.values())
     if world > 1:
-        t = torch.tensor([step_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+        step_ms = max_over_ranks(step_ms, dist, dev)
 
     mb = modeled_bytes(case)
     step_bytes = sum(mb.values())
@@ -406,9 +425,7 @@ def e2e(args, case, g, y, dx, grads, ws, dev, stream, world, calls):
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / K
     if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, dev)
     step_bytes = sum(modeled_bytes(case).values())
     h2d = xh.numel() * xh.element_size() + dyh.numel() * dyh.element_size()
     d2h = yh.numel() * yh.element_size() + dxh.numel() * dxh.element_size() + sum(
