@@ -44,7 +44,9 @@
  *   - Limits: k in {1, 3, 5, 7}; 0 <= L <= 6; H and W divisible by 2^L;
  *     planes too large for the on-chip staging return WTCONV_ERR_UNSUPPORTED.
  *   - L = 0 is the base branch only; wt_w and wt_scale may then be NULL.
- *   - Calls are reentrant; the library holds no global state.
+ *   - Calls are reentrant; apart from the fixed scratch array of
+ *     wtconv_backward_weight_noalloc (see there), the library holds no
+ *     global state.
  */
 #ifndef WTCONV_H
 #define WTCONV_H
@@ -119,6 +121,30 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, co
                                        float *d_wt_w, float *d_wt_scale,
                                        void *workspace, size_t workspace_bytes,
                                        wtconv_stream_t stream);
+
+/* The paper has no counterpart to this entry point.
+ *
+ * Same result as wtconv_backward_weight, for callers that cannot allocate
+ * device memory -- for example code running inside a fixed memory budget, an
+ * allocator hook, or a runtime that forbids cudaMalloc while a stream is being
+ * captured.  Instead of a workspace argument it uses a fixed array inside this
+ * library (4 MiB of device memory per GPU that loads the library, held until
+ * the process exits) for the per-block partial sums; it calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *   - Size limit: C * groups * (k*k*(1+4L) + 1) floats must fit in 2^20 floats;
+ *     larger problems return WTCONV_ERR_WORKSPACE (use wtconv_backward_weight).
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call shares the one array: calls whose kernels overlap on the GPU
+ *     (different streams, no ordering between them) race and corrupt each
+ *     other's results.  Calls ordered on one stream are safe; each call
+ *     overwrites every partial it later reads, so nothing is cleared.
+ * Arguments, layouts and gradients as for wtconv_backward_weight. */
+wtconv_status_t wtconv_backward_weight_noalloc(const wtconv_desc_t *d, const void *x, const void *dy,
+                                               const float *base_w, const float *base_b, const float *base_scale,
+                                               const float *wt_w, const float *wt_scale,
+                                               float *d_base_w, float *d_base_b, float *d_base_scale,
+                                               float *d_wt_w, float *d_wt_scale, wtconv_stream_t stream);
 
 #ifdef __cplusplus
 }

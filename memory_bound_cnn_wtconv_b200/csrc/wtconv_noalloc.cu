@@ -1,0 +1,87 @@
+// wtconv_backward_weight_noalloc: the weight gradient without a caller-provided
+// workspace, for callers that cannot allocate device memory (see
+// include/wtconv.h).  The per-block partial sums live in a fixed-size
+// device array owned by this library instead of in a cudaMalloc'd buffer.
+#include <cuda_runtime.h>
+
+#include "../../include/wtconv.h"
+#include "wtconv_launch.h"
+#include "wtconv_plan.h"
+#include "wtconv_planner.h"
+
+namespace wtc {
+namespace {
+
+// Partial sums of the weight gradient: at most this many floats (4 MiB).
+// Every GPU that loads the library holds this array until the process exits.
+constexpr size_t kNoAllocScratchFloats = (size_t)1 << 20;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+constexpr int kMaxScratchDevices = 64;
+
+// Device address of g_noalloc_scratch, resolved once per device with that
+// device current.  The host-side name is only a stand-in for the device
+// array and must never be passed to a kernel.
+float* scratch_address(cudaError_t* err) {
+    static float* addr[kMaxScratchDevices] = {};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= kMaxScratchDevices) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<float*>(p);
+    }
+    return addr[dev];
+}
+
+cudaError_t launch_partials(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
+    switch (P.k) {
+        case 1: return launch_bwdw_k1(P, dtype, a, s);
+        case 3: return launch_bwdw_k3(P, dtype, a, s);
+        case 5: return launch_bwdw_k5(P, dtype, a, s);
+        case 7: return launch_bwdw_k7(P, dtype, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+}  // namespace wtc
+
+using namespace wtc;
+
+extern "C" wtconv_status_t wtconv_backward_weight_noalloc(
+    const wtconv_desc_t* d, const void* x, const void* dy, const float* base_w, const float* base_b,
+    const float* base_scale, const float* wt_w, const float* wt_scale, float* d_base_w, float* d_base_b,
+    float* d_base_scale, float* d_wt_w, float* d_wt_scale, wtconv_stream_t stream) {
+    wtconv_status_t st = validate(d);
+    if (st != WTCONV_OK) return st;
+    if (!x || !dy || !base_w || !base_b || !base_scale || !d_base_w || !d_base_b || !d_base_scale)
+        return WTCONV_ERR_NULLPTR;
+    if (d->L > 0 && (!wt_w || !wt_scale || !d_wt_w || !d_wt_scale)) return WTCONV_ERR_NULLPTR;
+    if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_MISALIGNED;
+    Plan P;
+    st = make_plan(d, kBackwardWeight, &P);
+    if (st != WTCONV_OK) return st;
+    // The partials need C * groups * nv floats; beyond the fixed array the
+    // call is rejected (use wtconv_backward_weight with a workspace instead).
+    if ((size_t)P.C * P.groups * P.nv > kNoAllocScratchFloats) return WTCONV_ERR_WORKSPACE;
+    cudaError_t err = cudaSuccess;
+    float* part = scratch_address(&err);
+    if (part == nullptr) return WTCONV_ERR_CUDA;
+    // Every partial slot the finish kernel reads is written by the partial
+    // kernel of the same call, so nothing has to be cleared first.
+    cudaStream_t s = (cudaStream_t)stream;
+    BwdwArgs a{x, dy, part};
+    if (launch_partials(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    if (launch_bwdw_finish(P, part, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                           d_wt_w, d_wt_scale, s) != cudaSuccess)
+        return WTCONV_ERR_CUDA;
+    return WTCONV_OK;
+}
