@@ -78,6 +78,37 @@ def workload_name(c) -> str:
             f"forward + backward_input + backward_weight")
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
+# kernel, from one ncu capture of the named workload (the command is in the
+# named profile summary).  Each figure carries the SHA-256 of the kernel
+# sources it was taken on; once those change it no longer describes the
+# kernel and is reported as null.
+KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wtconv_planner.h",
+                  "wtconv_launch.h", "wtconv_api.cu", "wtconv_k1.cu", "wtconv_k3.cu", "wtconv_k5.cu", "wtconv_k7.cu")
+MEASURED_TRAFFIC = {
+    # (workload, call): (bytes per launch, kernel, source digest, profile)
+    ("stage1", "bwd_w"): (78.780928e6, "wtconv_bwdw_partial_kernel",
+                          "5640f0ab163cf20904fe7cd454c036b827b4167b19279a98cb0c25d8353405ee",
+                          "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
+}
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "memory_bound_cnn_wtconv_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str, call: str):
+    ent = MEASURED_TRAFFIC.get((workload, call))
+    if ent is None or ent[2] != kernel_source_digest():
+        return None, None
+    return ent[0], {"kernel": ent[1], "profile": ent[3]}
+
+
 def hbm_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -181,9 +212,10 @@ def physical_gpu_index(local: int) -> int:
 # --------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the reported CPU baseline).
 # --------------------------------------------------------------------------
-def oracle_sample(case, seconds: float, max_planes: int | None = None):
+def oracle_sample(case, seconds: float, max_planes: int | None = None, wrap: bool = False):
     """Time the oracle's three calls on whole batch elements (all channels),
-    one batch element at a time, until `seconds` elapse.  Returns (modeled
+    one batch element at a time, until `seconds` elapse (or the batch ends,
+    unless `wrap` cycles over it again).  Returns (modeled
     bytes processed, wall seconds, planes, cores, description)."""
     import numpy as np
 
@@ -197,7 +229,7 @@ def oracle_sample(case, seconds: float, max_planes: int | None = None):
     mb = modeled_bytes(sub)
     per_b = sum(mb.values())
     while True:
-        inp = make_inputs(sub.with_(seed=case.seed + b))
+        inp = make_inputs(sub.with_(seed=case.seed + b % case.B))
         p = {k: inp[k].double().numpy() for k in ("base_w", "base_b", "base_scale", "wt_w", "wt_scale")}
         x, dy = inp["x"].double().numpy(), inp["dy"].double().numpy()
         t0 = time.perf_counter()
@@ -208,9 +240,9 @@ def oracle_sample(case, seconds: float, max_planes: int | None = None):
         nbytes += per_b
         done_planes += case.C
         b += 1
-        if t_total >= seconds or b >= case.B or (max_planes and done_planes >= max_planes):
+        if t_total >= seconds or (not wrap and b >= case.B) or (max_planes and done_planes >= max_planes):
             break
-    desc = (f"{b} of {case.B} batch elements x all {case.C} channels "
+    desc = (f"{b} batch elements (cycling over the {case.B} of the workload) x all {case.C} channels "
             f"({done_planes} planes), forward + backward_input + backward_weight in float64")
     return nbytes, t_total, done_planes, orc.num_threads(), desc
 
@@ -344,14 +376,17 @@ def run_ours(args, case):
     t_alu, t_hbm = flops / (alu_peak * 1e12), mb[dom] / (peak * 1e9)
     kernel_names = {"fwd": "wtconv_fused_kernel (forward)", "bwd_in": "wtconv_fused_kernel (input gradient)",
                     "bwd_w": "wtconv_bwdw_partial_kernel + wtconv_bwdw_finish_kernel"}
+    traffic, traffic_src = measured_traffic(case.name, dom)
     if t_alu >= t_hbm:
         roof = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                "frac": alu_achieved / alu_peak, "traffic": None, "kernel": kernel_names[dom],
+                "frac": alu_achieved / alu_peak, "traffic": traffic, "traffic_source": traffic_src,
+                "kernel": kernel_names[dom],
                 "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 x 1965 MHz (unit counts x max clock)",
                 "flops_per_launch": flops}
     else:
         roof = {"bound": "hbm", "achieved": hbm_achieved, "peak": peak, "unit": "GB/s", "frac": hbm_achieved / peak,
-                "traffic": None, "kernel": kernel_names[dom], "peak_source": peak_kind,
+                "traffic": traffic, "traffic_source": traffic_src, "kernel": kernel_names[dom],
+                "peak_source": peak_kind,
                 "bytes_per_launch": mb[dom]}
 
     line = {
@@ -378,7 +413,7 @@ def run_ours(args, case):
     if world > 1:
         dist.barrier()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nb, t, planes, cores, desc = oracle_sample(case, args.cpu_seconds)
+        nb, t, planes, cores, desc = oracle_sample(case, args.cpu_seconds, wrap=True)
         line["cpu_baseline"] = {"value": nb / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": desc, "seconds": t}
     if rank == 0:
