@@ -87,8 +87,8 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
                   "wtconv_launch.h", "wtconv_api.cu", "wtconv_k1.cu", "wtconv_k3.cu", "wtconv_k5.cu", "wtconv_k7.cu")
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
-    ("stage1", "bwd_w"): (78.780928e6, "wtconv_bwdw_partial_kernel",
-                          "5640f0ab163cf20904fe7cd454c036b827b4167b19279a98cb0c25d8353405ee",
+    ("stage1", "bwd_w"): (79.02336e6, "wtconv_bwdw_partial_kernel",
+                          "2ccd58ca3c396b12ccc0a389bc4b2ab8aa26480c11a07f8c6e62ab514febab89",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 

@@ -187,6 +187,9 @@ struct LevelDst {
     int stride;
     int sub;
 };
+struct Levels {
+    LevelDst d[4];  // indexed by compile-time constants only (kept in registers)
+};
 
 __device__ __forceinline__ void butterfly(float a, float b, float c, float d, float& ll, float& lh, float& hl,
                                           float& hh) {
@@ -208,7 +211,8 @@ __device__ __forceinline__ void butterfly(float a, float b, float c, float d, fl
 // unpacked values if SUM.
 template <typename T, int PD, bool SUM>
 __device__ __forceinline__ float analysis_pyramid(const float* stg, int H, int W, int levels, int lg, FastDiv drw,
-                                                  float* dst, int ds, const LevelDst* lev, int np, int ptid) {
+                                                  float* dst, int ds, const Levels& levs, int np, int ptid) {
+    const LevelDst* lev = levs.d;
     const int G = 1 << lg, G2 = G * G;
     const int nreg_w = W >> (lg + 2);
     const int items = (H >> (lg + 2)) * nreg_w * G2;
@@ -288,7 +292,9 @@ __device__ __forceinline__ float analysis_pyramid(const float* stg, int H, int W
 
 // ---------------------------------------------------------------------------
 // A window row as NW2 aligned pairs e[k] = (r[2k], r[2k+1]), loaded straight
-// into register pairs with 64-bit shared loads.  For output column pair jp
+// into register pairs with 128-bit shared loads (a trailing odd pair with a
+// 64-bit load).  Lanes walk 16-byte-apart windows, so every quarter-warp's
+// 128-bit loads hit 8 distinct bank groups.  For output column pair jp
 // (columns 2jp, 2jp+1) and tap v the inputs are columns 2jp+v and 2jp+v+1:
 //   v even: the pair e[jp + v/2]              -> one packed FMA;
 //   v odd:  e[jp + v/2].y and e[jp + v/2 + 1].x -> two scalar FMAs.
@@ -298,6 +304,17 @@ template <int NW2>
 struct WinRow {
     float2 e[NW2];
     __device__ __forceinline__ void load(const float* rp) {
+#pragma unroll
+        for (int k = 0; k < NW2 / 2; ++k) {
+            const float4 v = *reinterpret_cast<const float4*>(rp + 4 * k);
+            e[2 * k] = make_float2(v.x, v.y);
+            e[2 * k + 1] = make_float2(v.z, v.w);
+        }
+        if constexpr (NW2 % 2 == 1) e[NW2 - 1] = *reinterpret_cast<const float2*>(rp + 2 * (NW2 - 1));
+    }
+    // 64-bit loads only: looser register allocation (no 4-register groups)
+    // for the register-heavy correlation tiles.
+    __device__ __forceinline__ void load_pairs(const float* rp) {
 #pragma unroll
         for (int k = 0; k < NW2; ++k) e[k] = *reinterpret_cast<const float2*>(rp + 2 * k);
     }
@@ -370,7 +387,7 @@ __device__ __forceinline__ void corr_tile(const float* __restrict__ swin, int ss
             for (int q = 0; q < NP; ++q) d[r][q] = *reinterpret_cast<const float2*>(dt + r * dstride + 2 * q);
         }
         WinRow<NW2> row;
-        row.load(swin + r * sstride);
+        row.load_pairs(swin + r * sstride);
 #pragma unroll
         for (int u = 0; u < K; ++u) {
             const int o = r - u;
@@ -414,31 +431,35 @@ __device__ __forceinline__ float quarter_pow(int l) {
 // those buffers).  `sync()` synchronises the np threads between the levels
 // that run one at a time (levels >= 4, or every level without the pyramid).
 // ---------------------------------------------------------------------------
-template <typename T, int PD, bool SUM, class Sync>
-__device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const float* stg, float* dst, int ds,
-                                               const Buf* bufs, int pad, int np, int ptid, Sync&& sync) {
+template <typename T, int PD, bool SUM, bool TO_Q, class Sync>
+__device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const float* stg, float* dst, int ds, int pad,
+                                               int np, int ptid, Sync&& sync) {
     const int H = P.H, W = P.W, L = P.L;
+    // Level l's subbands go to P.Q[l] (TO_Q) or P.S[l]; every index below is
+    // a compile-time constant or goes through the parameter directly, so no
+    // copy of the kernel parameter is made.
+    auto buf = [&](int l) -> const Buf& { return TO_Q ? P.Q[l] : P.S[l]; };
     float sum;
     int done;  // levels complete
     if (P.pyr) {
-        LevelDst lev[4];
+        Levels lev;
 #pragma unroll
         for (int l = 0; l < 4; ++l) {
-            const Buf& b = bufs[l < L ? l : 0];
-            lev[l] = LevelDst{sm + b.base + pad * b.stride + pad, b.stride, b.sub};
+            const Buf& b = buf(l < L ? l : 0);
+            lev.d[l] = LevelDst{sm + b.base + pad * b.stride + pad, b.stride, b.sub};
         }
         sum = analysis_pyramid<T, PD, SUM>(stg, H, W, P.pyr_levels, P.pyr_lg, P.div_rw, dst, ds, lev, np, ptid);
         done = P.pyr_levels;
     } else {
-        const Buf& b = bufs[0];
+        const Buf& b = buf(0);
         sum = unpack_level0<T, PD, SUM>(stg, H, W, P.div_q4, dst, ds, sm + b.base + pad * b.stride + pad, b.stride,
                                         b.sub, L >= 1, ptid, np);
         done = L >= 1 ? 1 : 0;
     }
     for (int l = done; l < L; ++l) {
         sync();
-        const Buf& s0 = bufs[l - 1];
-        const Buf& s1 = bufs[l];
+        const Buf& s0 = buf(l - 1);
+        const Buf& s1 = buf(l);
         haar_level(sm + s0.base + pad * s0.stride + pad, s0.stride, H >> (l + 1), W >> (l + 1), P.div_m[l],
                    sm + s1.base + pad * s1.stride + pad, s1.stride, s1.sub, ptid, np);
     }
@@ -454,121 +475,108 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 // The input gradient is the same pass applied to dy with every kernel
 // rotated by 180 degrees and no bias: the transpose of the forward map.
 // ---------------------------------------------------------------------------
-// A subband tile, its addressing decoded once: window origin in S, output
-// origin in Q, and the folded weights of its class.
-struct SubTile {
-    int win, out, wts;  // float offsets into shared memory
-    int sstride, qstride;
+// One conv tile, its addressing decoded: window origin (padded S or X),
+// output origin (Q or Y), folded weights, and the initial value (the folded
+// bias for base tiles, 0 for subband tiles).
+struct TileJob {
+    int win, out, wts;  // float offsets into shared memory (out: into y when L = 0)
+    int wstride, ostride;
+    int row0;           // base tiles: first output row
+    bool base, valid;
 };
 
-__device__ __forceinline__ SubTile decode_subband_tile(const Plan& P, int t, int TR, int TC) {
-    int cl = 1;
-    while (t >= P.sub_begin[cl]) ++cl;  // sub_begin[cl] = end of class cl's tiles
-    const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-    const int local = t - P.sub_begin[cl - 1];
-    const int tr = fdiv(local, P.div_ntc[l]), tc = local - tr * P.ntc[l];
-    const Buf& S = P.S[l];
-    const Buf& Q = P.Q[l];
-    SubTile st;
-    st.win = S.base + s * S.sub + tr * TR * S.stride + tc * TC;
-    st.out = Q.base + s * Q.sub + tr * TR * Q.stride + tc * TC;
-    st.wts = P.wbase + cl * P.wcls;
-    st.sstride = S.stride;
-    st.qstride = Q.stride;
-    return st;
-}
-
-template <int K, int TR, int TC>
-__device__ __forceinline__ void run_subband_tile(float* sm, const SubTile& st) {
-    float w[K * K];
-    load_weights<K>(sm + st.wts, w);
-    float* out = sm + st.out;
-    const int qs = st.qstride;
-    conv_tile<K, TR, TC>(sm + st.win, st.sstride, w, make_float2(0.f, 0.f), [&](int o, float2(&a)[TC / 2]) {
-#pragma unroll
-        for (int q = 0; q < TC / 4; ++q)
-            *reinterpret_cast<float4*>(out + o * qs + 4 * q) =
-                make_float4(a[2 * q].x, a[2 * q].y, a[2 * q + 1].x, a[2 * q + 1].y);
-    });
-}
-
-// Reformulation (2), levels >= 1, evaluated Horner-style: for l = L-1 .. 1
-// every level-l position (i, j) adds its four signed sums (signs from the
-// bit pair (a, b) of the level-(l-1) position (2i+a, 2j+b)) into the LL conv
-// output of level l-1 at that position.  Level l-1's LL then carries all
-// coarser terms into its own signed sums, so after the loop Q0's LL holds,
-// at every 2x2 output block (h >> 1, w >> 1), the closed-form sum of levels
-// 1..L-1 at that block.  One step per level, `sync()` between steps.
-template <class Sync>
-__device__ __forceinline__ void coarse_cascade(float* sm, const Plan& P, int np, int ptid, Sync&& sync) {
-    for (int l = P.L - 1; l >= 1; --l) {
+// Tile t of the forward index space (subband tiles, then base tiles from
+// base_tid0).
+__device__ __forceinline__ TileJob decode_tile(const Plan& P, int t, int TR, int TC) {
+    TileJob j;
+    j.valid = true;
+    if (t < P.n_sub_tiles) {
+        int cl = 1;
+        while (t >= P.sub_begin[cl]) ++cl;  // sub_begin[cl] = end of class cl's tiles
+        const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+        const int local = t - P.sub_begin[cl - 1];
+        const int tr = fdiv(local, P.div_ntc[l]), tc = local - tr * P.ntc[l];
+        const Buf& S = P.S[l];
         const Buf& Q = P.Q[l];
-        const Buf& D = P.Q[l - 1];
-        const int n = P.H >> (l + 1), m = P.W >> (l + 1);
-        for (int t = ptid; t < n * m; t += np) {
-            const int i = fdiv(t, P.div_m[l]), j = t - i * m;
-            const float* q = sm + Q.base + i * Q.stride + j;
-            const float q0 = q[0], q1 = q[Q.sub], q2 = q[2 * Q.sub], q3 = q[3 * Q.sub];
-            float* d = sm + D.base + (2 * i) * D.stride + 2 * j;  // LL plane of level l-1
-            const float2 top = *reinterpret_cast<const float2*>(d);
-            const float2 bot = *reinterpret_cast<const float2*>(d + D.stride);
-            const float t0 = q0 + q1, t1 = q0 - q1, t2 = q2 + q3, t3 = q2 - q3;
-            *reinterpret_cast<float2*>(d) = make_float2(top.x + (t0 + t2), top.y + (t0 - t2));
-            *reinterpret_cast<float2*>(d + D.stride) = make_float2(bot.x + (t1 + t3), bot.y + (t1 - t3));
-        }
-        sync();
+        j.win = S.base + s * S.sub + tr * TR * S.stride + tc * TC;
+        j.out = Q.base + s * Q.sub + tr * TR * Q.stride + tc * TC;
+        j.wts = P.wbase + cl * P.wcls;
+        j.wstride = S.stride;
+        j.ostride = Q.stride;
+        j.row0 = 0;
+        j.base = false;
+    } else if (t >= P.base_tid0 && t < P.tile_end) {
+        const int bt = t - P.base_tid0;
+        const int tr = fdiv(bt, P.div_ntc[kMaxL]), tc = bt - tr * P.ntc[kMaxL];
+        j.win = P.X.base + tr * TR * P.X.stride + tc * TC;
+        j.row0 = tr * TR;
+        // L >= 1: Y in shared memory.  L = 0: the output plane itself.
+        j.out = P.L >= 1 ? P.Y.base + tr * TR * P.Y.stride + tc * TC : (tr * TR) * P.W + tc * TC;
+        j.ostride = P.L >= 1 ? P.Y.stride : P.W;
+        j.wts = P.wbase;
+        j.wstride = P.X.stride;
+        j.base = true;
+    } else {
+        j = TileJob{0, 0, 0, 0, 0, 0, false, false};
     }
+    return j;
 }
 
-// The rows of one base tile (4 columns w0..w0+3, w0 % 4 == 0, rows from h0):
-// add the level-0 signed sum (signs from bit 0 of h and w; Q0's LL already
-// carries the coarser levels) and store (the only HBM write).  Straight-line
-// code with predicated stores, so the rows overlap.
-template <int TR, typename T>
-__device__ __forceinline__ void finish_tile(const float* sm, const Plan& P, T* yp, int h0, int w0,
-                                            float2 (&a)[TR][2]) {
-    const Buf& Q = P.Q[0];
-    const float* qb = sm + Q.base + (w0 >> 1);
-#pragma unroll
-    for (int o = 0; o < TR; ++o) {
-        const int h = h0 + o;
-        if (P.L >= 1) {
-            const float* r = qb + (h >> 1) * Q.stride;
-            const float2 q0 = *reinterpret_cast<const float2*>(r);
-            const float2 q1 = *reinterpret_cast<const float2*>(r + Q.sub);
-            const float2 q2 = *reinterpret_cast<const float2*>(r + 2 * Q.sub);
-            const float2 q3 = *reinterpret_cast<const float2*>(r + 3 * Q.sub);
-            const float sg = (h & 1) ? -1.f : 1.f;
-            const float t0a = fmaf(sg, q1.x, q0.x), t1a = fmaf(sg, q3.x, q2.x);
-            const float t0b = fmaf(sg, q1.y, q0.y), t1b = fmaf(sg, q3.y, q2.y);
-            a[o][0].x += t0a + t1a;
-            a[o][0].y += t0a - t1a;
-            a[o][1].x += t0b + t1b;
-            a[o][1].y += t0b - t1b;
-        }
-        if (h < P.H) gst4<T>(yp + (size_t)h * P.W + w0, make_float4(a[o][0].x, a[o][0].y, a[o][1].x, a[o][1].y));
-    }
-}
-
-// One output row (the loop schedule of large planes).
+// Reformulation (2): the synthesis of one work item, output rows 2i, 2i+1 x
+// columns 4q..4q+3 (the level-0 positions (i, 2q) and (i, 2q+1)), added to
+// the base-branch outputs in Y and stored (the only HBM write).
+// Output (h, w) receives, for every level l, the signed sum of the four
+// level-l conv outputs at (h >> (l+1), w >> (l+1)), with LH negated when
+// bit l of h is set, HL when bit l of w is set and HH when exactly one is.
+// The levels >= 1 are gathered Horner-style along the item's path: level l's
+// signed sum for the level-(l-1) position on the path is added to that
+// position's LL term, so the level-0 butterfly carries every coarser level.
 template <typename T>
-__device__ __forceinline__ void finish_row(const float* sm, const Plan& P, T* yp, int h, int w0, float2 (&a)[2]) {
-    if (P.L >= 1) {
-        const Buf& Q = P.Q[0];
-        const float* q = sm + Q.base + (h >> 1) * Q.stride + (w0 >> 1);
-        const float sg = (h & 1) ? -1.f : 1.f;
-        const float2 q0 = *reinterpret_cast<const float2*>(q);
-        const float2 q1 = *reinterpret_cast<const float2*>(q + Q.sub);
-        const float2 q2 = *reinterpret_cast<const float2*>(q + 2 * Q.sub);
-        const float2 q3 = *reinterpret_cast<const float2*>(q + 3 * Q.sub);
-        const float t0a = fmaf(sg, q1.x, q0.x), t1a = fmaf(sg, q3.x, q2.x);
-        const float t0b = fmaf(sg, q1.y, q0.y), t1b = fmaf(sg, q3.y, q2.y);
-        a[0].x += t0a + t1a;
-        a[0].y += t0a - t1a;
-        a[1].x += t0b + t1b;
-        a[1].y += t0b - t1b;
+__device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp, int t) {
+    const int i = fdiv(t, P.div_q4), q = t - i * (P.W >> 2);
+    const int j0 = 2 * q;
+    float c0 = 0.f, c1 = 0.f;  // coarse terms for LL at (i, j0) and (i, j0 + 1)
+    if (P.L >= 2) {
+        float v = 0.f;
+#pragma unroll
+        for (int l = kMaxL - 1; l >= 1; --l) {
+            if (l >= P.L) continue;
+            const Buf& Q = P.Q[l];
+            const float* r = sm + Q.base + (i >> l) * Q.stride + (j0 >> l);
+            const float q0 = r[0] + v, q1 = r[Q.sub], q2 = r[2 * Q.sub], q3 = r[3 * Q.sub];
+            const bool bi = (i >> (l - 1)) & 1;
+            const float t0 = bi ? q0 - q1 : q0 + q1;
+            const float t1 = bi ? q2 - q3 : q2 + q3;
+            if (l > 1) {
+                v = ((j0 >> (l - 1)) & 1) ? t0 - t1 : t0 + t1;
+            } else {
+                c0 = t0 + t1;
+                c1 = t0 - t1;
+            }
+        }
     }
-    gst4<T>(yp + (size_t)h * P.W + w0, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
+    const Buf& Q = P.Q[0];
+    const float* r = sm + Q.base + i * Q.stride + j0;
+    float2 ll = *reinterpret_cast<const float2*>(r);
+    const float2 lh = *reinterpret_cast<const float2*>(r + Q.sub);
+    const float2 hl = *reinterpret_cast<const float2*>(r + 2 * Q.sub);
+    const float2 hh = *reinterpret_cast<const float2*>(r + 3 * Q.sub);
+    ll.x += c0;
+    ll.y += c1;
+    const float* yr = sm + P.Y.base + (2 * i) * P.Y.stride + 4 * q;
+    float4 top = *reinterpret_cast<const float4*>(yr);
+    float4 bot = *reinterpret_cast<const float4*>(yr + P.Y.stride);
+    {
+        const float a0 = ll.x + lh.x, b0 = hl.x + hh.x, a1 = ll.y + lh.y, b1 = hl.y + hh.y;
+        top.x += a0 + b0; top.y += a0 - b0; top.z += a1 + b1; top.w += a1 - b1;
+    }
+    {
+        const float a0 = ll.x - lh.x, b0 = hl.x - hh.x, a1 = ll.y - lh.y, b1 = hl.y - hh.y;
+        bot.x += a0 + b0; bot.y += a0 - b0; bot.z += a1 + b1; bot.w += a1 - b1;
+    }
+    T* yo = yp + (size_t)(2 * i) * P.W + 4 * q;
+    gst4<T>(yo, top);
+    gst4<T>(yo + P.W, bot);
 }
 
 // Shared pieces of the two forward schedules.
@@ -581,11 +589,11 @@ struct FusedCtx {
     long long units;
     int u0, u1;
 
-    __device__ __forceinline__ size_t plane_of(int u) const {
-        const int c = u / P.B, b = u - c * P.B;
-        return (size_t)b * P.C + c;
+    // Units run channel-major: unit u is plane (b, c) = (u mod B, u / B).
+    __device__ __forceinline__ size_t plane_of(int b, int c) const { return (size_t)b * P.C + c; }
+    __device__ __forceinline__ const T* src(int b, int c) const {
+        return x + plane_of(b, c) * ((size_t)P.H * P.W);
     }
-    __device__ __forceinline__ const T* src(int u) const { return x + plane_of(u) * ((size_t)P.H * P.W); }
     // Reformulation (3): fold the scales (and the Haar factors) into the
     // weights of channel c (threads [0, np)).
     __device__ __forceinline__ void fold(int c, int np, int ptid) const {
@@ -608,13 +616,15 @@ struct FusedCtx {
     }
 };
 
-// Forward / input gradient.  Per plane (all threads, CTA barriers between
-// phases): fold the weights when the channel changes and analyse the staged
-// plane; start staging the next plane; run every conv tile (one per thread:
-// subband tiles write Q, base tiles keep their outputs in registers); fold
-// the coarse levels into Q0's LL; base tiles add the level-0 signed sum and
-// store y.  Large planes (more tiles than threads) loop over the subband
-// tiles and then the base tiles instead.
+// Forward / input gradient.  Persistent CTAs walk a run of planes with two
+// CTA barriers per plane:
+//   phase A(u): fold the weights when the channel changes and analyse the
+//               staged plane u (writes X, S); the threads the analysis leaves
+//               idle start on the synthesis of plane u-1 (reads Q, Y; writes y);
+//   phase B(u): start staging plane u+1, then run every conv tile of plane u:
+//               subband tiles write Q, base tiles write Y (y itself if L = 0).
+// Within a phase the buffers written (A: X, S, weights; B: staging, Q, Y) and
+// the buffers read (A: staging, Q, Y; B: S, X, weights) are disjoint.
 template <int K, int TR, int TC, typename T, bool BWD>
 __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
     const T* __restrict__ x, const float* __restrict__ base_w, const float* __restrict__ base_b,
@@ -632,68 +642,70 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
     const int u0 = cx.u0, u1 = cx.u1;
     auto csync = [&]() { __syncthreads(); };
     float* X0 = sm + P.X.base + p * P.X.stride + p;
-    const int ntcb = P.ntc[kMaxL];
-
+    const size_t plane_elems = (size_t)P.H * P.W;
+    int ft = tid - P.fin_off;
+    if (ft < 0) ft += nt;
     // In the one-tile-per-thread schedule each thread's tile is fixed.
-    const bool sub = P.merged && tid < P.n_sub_tiles;
-    const int bt = tid - P.base_tid0;
-    const bool held = P.merged && bt >= 0 && bt < P.n_base_tiles;
-    const int btr = held ? fdiv(bt, P.div_ntc[kMaxL]) : 0;
-    const int btc = bt - btr * ntcb;
+    const TileJob fixed = P.merged ? decode_tile(P, tid, TR, TC) : TileJob{0, 0, 0, 0, 0, 0, false, false};
 
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
-    if (u0 < u1) stage_plane(sm + P.stg, cx.src(u0), P.plane_chunks, tid, nt);
+    // (b, c) of the plane being analysed / tiled, of the previous plane, and of the next.
+    int cur_b = u0 % P.B, cur_c = u0 / P.B;
+    int prev_b = 0, prev_c = 0;
+    if (u0 < u1) stage_plane(sm + P.stg, cx.src(cur_b, cur_c), P.plane_chunks, tid, nt);
     cp_async_commit();
-    int cur_c = -1;
-    for (int u = u0; u < u1; ++u) {
-        const int c = u / P.B;
+    int folded_c = -1;
+    for (int u = u0; u <= u1; ++u) {
         cp_async_wait_all();
-        __syncthreads();  // staged plane complete; previous plane fully finished
-        if (c != cur_c) {
-            cx.fold(c, nt, tid);
-            cur_c = c;
+        __syncthreads();  // plane u staged; every tile of plane u-1 done
+        // Phase A.
+        if (u < u1) {
+            if (cur_c != folded_c) {
+                cx.fold(cur_c, nt, tid);
+                folded_c = cur_c;
+            }
+            analyse_plane<T, p, false, false>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         }
-        analyse_plane<T, p, false>(sm, P, sm + P.stg, X0, P.X.stride, P.S, p, nt, tid, csync);
-        __syncthreads();
-        if (u + 1 < u1) stage_plane(sm + P.stg, cx.src(u + 1), P.plane_chunks, tid, nt);
+        if (u > u0 && P.L >= 1) {
+            T* yp = y + cx.plane_of(prev_b, prev_c) * plane_elems;
+            for (int t = ft; t < P.n_fin; t += nt) synth_item<T>(sm, P, yp, t);
+        }
+        if (u == u1) break;
+        __syncthreads();  // X and S of plane u ready; Q and Y of plane u-1 consumed
+        // Phase B.
+        int nb = cur_b + 1, nc = cur_c;
+        if (nb == P.B) {
+            nb = 0;
+            ++nc;
+        }
+        if (u + 1 < u1) stage_plane(sm + P.stg, cx.src(nb, nc), P.plane_chunks, tid, nt);
         cp_async_commit();
-
-        T* yp = y + cx.plane_of(u) * ((size_t)P.H * P.W);
-        if (P.merged) {
-            float2 hold[TR][NP];
-            if (sub) {
-                run_subband_tile<K, TR, TC>(sm, decode_subband_tile(P, tid, TR, TC));
-            } else if (held) {
-                float wb[KK];
-                load_weights<K>(sm + P.wbase, wb);
-                const float bias = sm[P.bias];
-                const float* win = sm + P.X.base + btr * TR * P.X.stride + btc * TC;
-                conv_tile<K, TR, TC>(win, P.X.stride, wb, make_float2(bias, bias), [&](int o, float2(&a)[NP]) {
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) hold[o][j] = a[j];
+        for (int t = tid; t < P.tile_end; t += nt) {
+            const TileJob j = P.merged ? fixed : decode_tile(P, t, TR, TC);
+            if (!j.valid) continue;
+            float w[KK];
+            load_weights<K>(sm + j.wts, w);
+            const float b0 = j.base ? sm[P.bias] : 0.f;
+            if (P.L >= 1 || !j.base) {
+                float* out = sm + j.out;
+                const int os = j.ostride;
+                conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
+                    *reinterpret_cast<float4*>(out + o * os) = make_float4(a[0].x, a[0].y, a[1].x, a[1].y);
                 });
-            }
-            __syncthreads();  // every Q complete
-            coarse_cascade(sm, P, nt, tid, csync);
-            if (held) finish_tile<TR, T>(sm, P, yp, btr * TR, btc * TC, hold);
-        } else {
-            for (int t = tid; t < P.n_sub_tiles; t += nt)
-                run_subband_tile<K, TR, TC>(sm, decode_subband_tile(P, t, TR, TC));
-            __syncthreads();  // every Q complete
-            coarse_cascade(sm, P, nt, tid, csync);
-            float wb[KK];
-            load_weights<K>(sm + P.wbase, wb);
-            const float bias = sm[P.bias];
-            for (int t = tid; t < P.n_base_tiles; t += nt) {
-                const int tr = fdiv(t, P.div_ntc[kMaxL]), tc = t - tr * ntcb;
-                const float* win = sm + P.X.base + tr * TR * P.X.stride + tc * TC;
-                conv_tile<K, TR, TC>(win, P.X.stride, wb, make_float2(bias, bias), [&](int o, float2(&a)[NP]) {
-                    const int h = tr * TR + o;
-                    if (h < P.H) finish_row<T>(sm, P, yp, h, tc * TC, a);
+            } else {
+                // L = 0: the base branch is the whole output.
+                T* yo = y + cx.plane_of(cur_b, cur_c) * plane_elems + j.out;
+                const int h0 = j.row0;
+                conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
+                    if (h0 + o < P.H) gst4<T>(yo + (size_t)o * P.W, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
                 });
             }
         }
+        prev_b = cur_b;
+        prev_c = cur_c;
+        cur_b = nb;
+        cur_c = nc;
     }
     cp_async_wait_all();
 }
@@ -744,9 +756,9 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
     for (int b = g; b < P.B; b += G) {
         cp_async_wait_all();
         __syncthreads();  // staged pair complete; previous correlations done
-        analyse_plane<T, p, false>(sm, P, sm + P.stg, X0, P.X.stride, P.S, p, nt, tid, csync);
-        const float s = analyse_plane<T, 0, true>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base, P.DY.stride,
-                                                  P.Q, 0, nt, tid, csync);
+        analyse_plane<T, p, false, false>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
+        const float s = analyse_plane<T, 0, true, true>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
+                                                        P.DY.stride, 0, nt, tid, csync);
         {
             const float yv = s - sdy_c;
             const float tv = sdy + yv;

@@ -13,6 +13,8 @@
 //   S[l]   padded un-normalised Haar subbands of level l (4 planes) of X.
 //   Q[l]   forward: subband conv outputs of level l (4 planes, tile-rounded);
 //          weight gradient: Haar subbands of dy (4 planes, tile-rounded).
+//   Y      forward (L >= 1): base-branch outputs (tile-rounded), kept until
+//          the synthesis adds the wavelet terms and stores the plane.
 //   DY     weight gradient: dy plane (tile-rounded).
 //   W      forward: folded weights, one class (K*K floats) per subband and the base.
 //
@@ -51,7 +53,7 @@ inline FastDiv make_fastdiv(uint32_t d) {
 }
 
 // Thread budgets (also the kernels' __launch_bounds__, two CTAs per SM).
-constexpr int kFusedMaxThreads = 320;
+constexpr int kFusedMaxThreads = 256;
 constexpr int kBwdwMaxThreads = 320;
 
 struct Buf {
@@ -74,7 +76,7 @@ struct Plan {
     int stg;             // staging buffer offset; one stored plane occupies stg_floats floats
     int stg_floats;
     int plane_chunks;    // 16-byte chunks per stored plane
-    Buf X, DY;
+    Buf X, Y, DY;
     Buf S[kMaxL], Q[kMaxL];
     int ntr[kMaxL + 1], ntc[kMaxL + 1];  // tile grid per level; index kMaxL = full resolution
     // Tile enumeration.  Forward: subband tiles in class order (l, s) first,
@@ -85,8 +87,14 @@ struct Plan {
     int cls_begin[kMaxCls + 1];
     int n_all_tiles;
     int nv;              // weight gradient: floats per partial vector = ncls*k*k + 1
-    int merged;          // forward: subband and base tiles run in one phase (one tile per thread)
-    int base_tid0;       // forward, merged: first thread of the base tiles (a warp boundary)
+    // Forward tile index space: subband tiles [0, n_sub_tiles), base tiles
+    // [base_tid0, tile_end); thread t takes the indices t, t + nthreads, ...
+    int base_tid0, tile_end;
+    int merged;          // forward: tile_end <= nthreads (one tile per thread)
+    // Forward synthesis work items (L >= 1): rows 2i, 2i+1 x columns 4q..4q+3;
+    // thread t takes items (t - fin_off) mod nthreads + k * nthreads, so the
+    // threads that the analysis leaves idle start first.
+    int n_fin, fin_off;
     int pyr;             // analysis by the one-pass pyramid (H % 4 == 0 and L >= 1)
     int pyr_levels;      // levels the pyramid computes (min(L, 4)); the rest run level by level
     int pyr_lg;          // pyramid lane groups cover (4 * 2^pyr_lg)^2 pixel regions

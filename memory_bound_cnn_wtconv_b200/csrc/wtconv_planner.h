@@ -35,16 +35,39 @@ inline int pick_stride(int min_floats, int TR, int ntc) {
     return s;
 }
 
-// Work-weighted tile slack for tile height TR (smaller is better).
-inline double tile_waste(const wtconv_desc_t* d, int TR) {
-    double used = d->H, total = ceil_div(d->H, TR) * (double)TR;
-    for (int l = 0; l < d->L; ++l) {
-        const int n = d->H >> (l + 1);
-        const double w = 1.0 / (double)(1 << (2 * l));  // level-l work relative to the base conv
-        used += w * n;
-        total += w * ceil_div(n, TR) * (double)TR;
+// Conv tiles of height TR (4 columns wide) over the base plane and every subband.
+inline int count_tiles(const wtconv_desc_t* d, int TR) {
+    int n = ceil_div(d->H, TR) * ceil_div(d->W, 4);
+    for (int l = 0; l < d->L; ++l) n += 4 * ceil_div(d->H >> (l + 1), TR) * ceil_div(d->W >> (l + 1), 4);
+    return n;
+}
+
+// Threads of a CTA for `tiles` conv tiles: a multiple of 4 warps (one warp
+// per SM sub-partition each) once there are more than 128 tiles, so no
+// sub-partition carries an extra warp of tiles; at most max_threads.
+inline int tile_threads(int tiles, int max_threads) {
+    const int t = tiles <= 128 ? std::max(64, ceil_div(tiles, 32) * 32) : ceil_div(tiles, 128) * 128;
+    return std::min(t, max_threads);
+}
+
+// Tile height: the one with the shorter tile phase, i.e. fewer tile rows on
+// the busiest SM sub-partition (warp-tiles per sub-partition x TR).
+inline int pick_tile_rows(const wtconv_desc_t* d, int max_threads) {
+    int best = 7;
+    long long best_cost = -1;
+    for (int TR = 7; TR <= 8; ++TR) {
+        const int tiles = count_tiles(d, TR);
+        const int threads = tile_threads(tiles, max_threads);
+        const long long warp_tiles = ceil_div(tiles, 32);
+        const long long per_smsp = ceil_div((int)std::min<long long>(warp_tiles, 1 << 30), 4);
+        const long long iters = ceil_div(tiles, threads);
+        const long long cost = std::max(per_smsp, iters) * TR;
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = TR;
+        }
     }
-    return total / used;
+    return best;
 }
 
 // CTAs per SM that the shared memory of one CTA allows (the register
@@ -102,7 +125,7 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     P->p = p;
     P->esize = d->dtype == WTCONV_BF16 ? 2 : 4;
     P->TC = 4;
-    P->TR = tile_waste(d, 7) < tile_waste(d, 8) ? 7 : 8;
+    P->TR = pick_tile_rows(d, kind == kBackwardWeight ? kBwdwMaxThreads : kFusedMaxThreads);
     const int TR = P->TR, TC = P->TC;
     const int WV4 = 4 * ((TC + k - 1 + 3) / 4);  // floats read per window row
 
@@ -150,6 +173,13 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
         P->Q[l].base = (int)off;
         off += 4LL * P->Q[l].sub;
     }
+    if (kind != kBackwardWeight && L >= 1) {
+        // Written by base tiles (lanes walk tile columns, like the windows).
+        const int ntc = P->ntc[kMaxL];
+        P->Y.stride = pick_stride(ntc * TC, TR, ntc);
+        P->Y.base = (int)off;
+        off += round4(P->ntr[kMaxL] * TR * P->Y.stride);
+    }
     if (kind == kBackwardWeight) {
         const int rows = P->ntr[kMaxL] * TR;
         P->DY.stride = round4(P->ntc[kMaxL] * TC);
@@ -193,22 +223,31 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     for (int l = 0; l <= kMaxL; ++l) P->div_ntc[l] = make_fastdiv(std::max(P->ntc[l], 1));
 
     if (kind == kBackwardWeight) {
-        const int nt = ceil_div(P->n_all_tiles, 32) * 32;
-        if (nt > kBwdwMaxThreads) return WTCONV_ERR_UNSUPPORTED;
-        P->nthreads = std::max(nt, 64);
+        // One tile per thread for the whole walk.
+        if (P->n_all_tiles > kBwdwMaxThreads) return WTCONV_ERR_UNSUPPORTED;
+        P->nthreads = tile_threads(P->n_all_tiles, kBwdwMaxThreads);
+        if (P->nthreads < P->n_all_tiles) P->nthreads = ceil_div(P->n_all_tiles, 32) * 32;
         // Reduction scratch aliases the (then dead) buffers from offset 0.
         P->red = 0;
         off = std::max(off, (long long)P->nthreads * (KK + 1));
     } else {
-        const int sub_pad = ceil_div(P->n_sub_tiles, 32) * 32;
-        if (sub_pad + P->n_base_tiles <= kFusedMaxThreads) {
-            P->merged = 1;
-            P->base_tid0 = sub_pad;
-            P->nthreads = std::max(64, ceil_div(sub_pad + P->n_base_tiles, 32) * 32);
+        // Subband and base tiles run the same code, so they share warps.
+        P->base_tid0 = P->n_sub_tiles;
+        P->tile_end = P->base_tid0 + P->n_base_tiles;
+        P->nthreads = tile_threads(P->tile_end, kFusedMaxThreads);
+        P->merged = P->tile_end <= P->nthreads ? 1 : 0;
+        P->n_fin = L >= 1 ? (H / 2) * (W / 4) : 0;
+        // Threads the analysis keeps busy (whole warps); the synthesis items
+        // start on the others.
+        long long an_items;
+        if (P->pyr) {
+            const int G = 1 << P->pyr_lg;
+            an_items = (long long)(H >> (P->pyr_lg + 2)) * (W >> (P->pyr_lg + 2)) * G * G;
         } else {
-            P->merged = 0;
-            P->nthreads = kFusedMaxThreads;
+            an_items = (long long)(L >= 1 ? H / 2 : H) * (W / 4);
         }
+        const long long busy = ceil_div((int)std::min<long long>(an_items, 1 << 30), 32) * 32LL;
+        P->fin_off = busy >= P->nthreads ? 0 : (int)busy;
     }
     off = round4((int)std::min<long long>(off, 1LL << 30));
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;

@@ -10,7 +10,10 @@
 //   - a conv / correlation window reads something other than the plane it
 //     belongs to (interior) or untouched zero (padding and tile slack),
 //   - a synthesis read sees anything but the conv output it needs,
-//   - a global load or store leaves its H x W plane.
+//   - a global load or store leaves its H x W plane,
+//   - two phases of the kernel race: the CTA barriers split the replay into
+//     phases, and no float may be written by one work item and read or
+//     written by another inside one phase.
 // Prints "OK <summary>" and exits 0, or prints the first violation and exits 1.
 #include <cstdio>
 #include <cstdlib>
@@ -23,14 +26,17 @@ using namespace wtc;
 
 namespace {
 
-enum : int { ZERO = 0, WTS = 1, BIAS = 2, XT = 3, DYT = 4, ZT = 5 };
+enum : int { ZERO = 0, WTS = 1, BIAS = 2, XT = 3, DYT = 4, ZT = 5, YT = 6, RED = 7 };
 int s_tag(int l, int s) { return 100 + 4 * l + s; }
 int q_tag(int l, int s) { return 200 + 4 * l + s; }
 
 struct Shadow {
     std::vector<int> tag;
+    std::vector<int> rd, wr;  // last phase that read / wrote each float
+    int epoch = 1;            // current phase; a CTA barrier starts the next
     const char* phase = "";
-    explicit Shadow(int n) : tag(n, ZERO) {}
+    explicit Shadow(int n) : tag(n, ZERO), rd(n, 0), wr(n, 0) {}
+    void barrier() { ++epoch; }
     [[noreturn]] void fail(const std::string& m, long long idx) {
         std::printf("FAIL [%s] %s (index %lld of %zu)\n", phase, m.c_str(), idx, tag.size());
         std::exit(1);
@@ -41,10 +47,19 @@ struct Shadow {
     }
     void write(long long i, long long lo, long long hi, int t, const char* what) {
         in_bounds(i, lo, hi, what);
+        if (rd[i] == epoch) fail(std::string(what) + ": written in the phase that reads it", i);
+        if (wr[i] == epoch) fail(std::string(what) + ": written twice in one phase", i);
+        wr[i] = epoch;
         tag[i] = t;
     }
-    void read(long long i, long long lo, long long hi, int expect, const char* what) {
+    // A load whose value is not used (vector-load slack): bounds and races only.
+    void touch(long long i, long long lo, long long hi, const char* what) {
         in_bounds(i, lo, hi, what);
+        if (wr[i] == epoch) fail(std::string(what) + ": read in the phase that writes it", i);
+        rd[i] = epoch;
+    }
+    void read(long long i, long long lo, long long hi, int expect, const char* what) {
+        touch(i, lo, hi, what);
         if (tag[i] != expect) fail(std::string(what) + ": expected tag " + std::to_string(expect) + ", found " +
                                        std::to_string(tag[i]), i);
     }
@@ -155,6 +170,7 @@ void replay_analyse(Shadow& sh, const Plan& P, long long stg, int stag, long lon
         done = P.L >= 1 ? 1 : 0;
     }
     for (int l = done; l < P.L; ++l) {
+        sh.barrier();  // sync() before every level computed on its own
         const int n = P.H >> (l + 1), m = P.W >> (l + 1);
         const Buf& s0 = bufs[l - 1];
         const Buf& s1 = bufs[l];
@@ -196,7 +212,7 @@ void replay_window(Shadow& sh, const Plan& P, long long base, int stride, long l
         for (int c = 0; c < WV4; ++c) {
             const long long a = win + (long long)r * stride + c;
             if (c >= TC + K - 1) {  // loaded but unused
-                sh.in_bounds(a, lo, hi, what);
+                sh.touch(a, lo, hi, what);
                 continue;
             }
             const int i = tr * TR + r - p, j = tc * TC + c - p;
@@ -257,9 +273,14 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
         std::printf("FAIL fused thread count %d\n", P.nthreads);
         std::exit(1);
     }
-    if (P.merged && (P.base_tid0 % 32 || P.base_tid0 < P.n_sub_tiles || P.base_tid0 + P.n_base_tiles > P.nthreads)) {
-        std::printf("FAIL merged layout: sub %d base0 %d base %d threads %d\n", P.n_sub_tiles, P.base_tid0,
-                    P.n_base_tiles, P.nthreads);
+    if (P.base_tid0 < P.n_sub_tiles || P.tile_end != P.base_tid0 + P.n_base_tiles ||
+        P.merged != (P.tile_end <= P.nthreads ? 1 : 0)) {
+        std::printf("FAIL tile index space: sub %d base0 %d base %d end %d threads %d\n", P.n_sub_tiles, P.base_tid0,
+                    P.n_base_tiles, P.tile_end, P.nthreads);
+        std::exit(1);
+    }
+    if (P.n_fin != (L >= 1 ? (H / 2) * (W / 4) : 0) || P.fin_off < 0 || P.fin_off >= P.nthreads || P.fin_off % 32) {
+        std::printf("FAIL synthesis items %d offset %d\n", P.n_fin, P.fin_off);
         std::exit(1);
     }
     if (P.smem_floats % 4 || P.smem_floats * 4 > 227 * 1024) {
@@ -271,21 +292,72 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     if (P.grid < 1 || P.grid > (long long)P.B * P.C) sh.fail("grid", P.grid);
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
+    const long long ylo = P.Y.base, yhi = P.Y.base + (long long)P.ntr[kMaxL] * TR * P.Y.stride;
     for (int cl = 0; cl < ncls; ++cl)
         if ((P.wbase + cl * P.wcls) % 4) sh.fail("weight class not 16-byte aligned", P.wbase + cl * P.wcls);
-    // Two planes in a row through one persistent CTA: the second must see the
-    // same zero padding and slack.
-    for (int unit = 0; unit < 2; ++unit) {
-        sh.phase = "staging";
-        replay_stage(sh, P, P.stg, XT + 10);
-        sh.phase = "weights";
-        for (int cl = 0; cl < ncls; ++cl)
-            for (int t = 0; t < KK; ++t)
-                sh.write(P.wbase + (long long)cl * P.wcls + t, P.wbase, P.wbase + (long long)ncls * P.wcls, WTS, "weights");
-        sh.write(P.bias, P.bias, P.bias + 1, BIAS, "bias");
-        sh.phase = "analysis";
-        replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S, p, s_tag);
-        sh.phase = "conv tiles";
+    const int ntc = P.ntc[kMaxL];
+
+    // Phase A's synthesis of the previous plane: rows 2i, 2i+1 x columns 4q..4q+3.
+    auto synthesis = [&]() {
+        for (int t = 0; t < P.n_fin; ++t) {
+            const int i = (int)fastdiv_host(t, P.div_q4), q = t - i * (W / 4);
+            if (i != t / (W / 4)) sh.fail("synthesis item division", t);
+            const int j0 = 2 * q;
+            for (int l = L - 1; l >= 1; --l) {
+                const Buf& Q = P.Q[l];
+                const int ri = i >> l, rj = j0 >> l;
+                if (ri >= (H >> (l + 1)) || rj >= (W >> (l + 1))) sh.fail("coarse synthesis index", l);
+                for (int s2 = 0; s2 < 4; ++s2)
+                    sh.read(Q.base + (long long)s2 * Q.sub + (long long)ri * Q.stride + rj, Q.base + (long long)s2 * Q.sub,
+                            Q.base + (long long)(s2 + 1) * Q.sub, q_tag(l, s2), "coarse Q read");
+            }
+            const Buf& Q = P.Q[0];
+            if (j0 + 1 >= W / 2) sh.fail("level-0 synthesis column", j0);
+            for (int s2 = 0; s2 < 4; ++s2) {
+                const long long a = Q.base + (long long)s2 * Q.sub + (long long)i * Q.stride + j0;
+                if (a % 2) sh.fail("level-0 pair load not 8-byte aligned", a);
+                for (int e = 0; e < 2; ++e)
+                    sh.read(a + e, Q.base + (long long)s2 * Q.sub, Q.base + (long long)(s2 + 1) * Q.sub, q_tag(0, s2),
+                            "level-0 Q read");
+            }
+            for (int rr = 0; rr < 2; ++rr) {
+                const long long a = P.Y.base + (long long)(2 * i + rr) * P.Y.stride + 4 * q;
+                if (a % 4) sh.fail("Y load not 16-byte aligned", a);
+                for (int e = 0; e < 4; ++e) {
+                    sh.read(a + e, ylo, yhi, YT, "Y read");
+                    check_global((long long)(2 * i + rr) * W + 4 * q + e, (long long)H * W, "y store");
+                }
+            }
+        }
+    };
+
+    // The persistent walk over two planes and the final synthesis, with the
+    // kernel's CTA barriers as phase boundaries:
+    //   stage(0) | A(0) | B(0): stage(1), tiles(0) | A(1) | B(1): tiles(1) | A(end)
+    sh.phase = "initial staging";
+    replay_stage(sh, P, P.stg, XT + 10);
+    for (int unit = 0; unit <= 2; ++unit) {
+        sh.barrier();
+        if (unit < 2) {
+            sh.phase = "A: fold";
+            for (int cl = 0; cl < ncls; ++cl)
+                for (int t = 0; t < KK; ++t)
+                    sh.write(P.wbase + (long long)cl * P.wcls + t, P.wbase, P.wbase + (long long)ncls * P.wcls, WTS,
+                             "weights");
+            sh.write(P.bias, P.bias, P.bias + 1, BIAS, "bias");
+            sh.phase = "A: analysis";
+            replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT,
+                           P.S, p, s_tag);
+        }
+        if (unit > 0 && L >= 1) {
+            sh.phase = "A: synthesis";
+            synthesis();
+        }
+        if (unit == 2) break;
+        sh.barrier();
+        sh.phase = "B: staging";
+        if (unit + 1 < 2) replay_stage(sh, P, P.stg, XT + 10);
+        sh.phase = "B: subband tiles";
         for (int cl = 1; cl < ncls; ++cl) {
             const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
             const int n = H >> (l + 1), m = W >> (l + 1);
@@ -306,55 +378,23 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
                                  Q.base + (long long)(s + 1) * Q.sub, q_tag(l, s), "Q tile");
             }
         }
-        const int ntc = P.ntc[kMaxL];
+        sh.phase = "B: base tiles";
         for (int t = 0; t < P.n_base_tiles; ++t) {
             const int tr = (int)fastdiv_host(t, P.div_ntc[kMaxL]), tc = t - tr * ntc;
             for (int q = 0; q < KK; ++q) sh.read(P.wbase + q, 0, all, WTS, "base weights");
             sh.read(P.bias, 0, all, BIAS, "bias");
             replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base window");
-        }
-        const int n0 = H >> 1, m0 = W >> 1;
-        sh.phase = "coarse cascade";
-        for (int l = L - 1; l >= 1; --l) {
-            const Buf& Q = P.Q[l];
-            const Buf& D = P.Q[l - 1];
-            const int n = H >> (l + 1), m = W >> (l + 1);
-            for (int t = 0; t < n * m; ++t) {
-                const int i = (int)fastdiv_host(t, P.div_m[l]), j = t - i * m;
-                if (i != t / m) sh.fail("cascade division", t);
-                for (int s2 = 0; s2 < 4; ++s2)
-                    sh.read(Q.base + (long long)s2 * Q.sub + (long long)i * Q.stride + j, Q.base + (long long)s2 * Q.sub,
-                            Q.base + (long long)(s2 + 1) * Q.sub, q_tag(l, s2), "cascade Q read");
-                const long long d = D.base + (long long)(2 * i) * D.stride + 2 * j;
-                if (d % 2) sh.fail("cascade pair not 8-byte aligned", d);
-                if (2 * i + 1 >= (H >> l) || 2 * j + 1 >= (W >> l)) sh.fail("cascade target index", l);
-                for (int a = 0; a < 2; ++a)
-                    for (int b = 0; b < 2; ++b)
-                        sh.read(d + (long long)a * D.stride + b, D.base, D.base + D.sub, q_tag(l - 1, 0), "cascade LL update");
-            }
-        }
-        (void)n0;
-        sh.phase = "synthesis + store";
-        for (int t = 0; t < P.n_base_tiles; ++t) {
-            const int tr = (int)fastdiv_host(t, P.div_ntc[kMaxL]), tc = t - tr * ntc;
-            for (int o = 0; o < TR; ++o) {
-                const int h = tr * TR + o;
-                if (h >= H) continue;
-                const int w0 = tc * TC;
-                if (L >= 1) {
-                    const Buf& Q = P.Q[0];
-                    for (int g = 0; g < TC / 4; ++g)
-                        for (int s = 0; s < 4; ++s) {
-                            const long long a = Q.base + (long long)s * Q.sub + (long long)(h >> 1) * Q.stride + (w0 >> 1) + 2 * g;
-                            if (a % 2) sh.fail("level-0 pair load not 8-byte aligned", a);
-                            for (int e = 0; e < 2; ++e) {
-                                if ((w0 >> 1) + 2 * g + e >= m0) sh.fail("level-0 synthesis column", w0);
-                                sh.read(a + e, Q.base + (long long)s * Q.sub, Q.base + (long long)(s + 1) * Q.sub, q_tag(0, s),
-                                        "level-0 Q read");
-                            }
-                        }
+            if (L >= 1) {
+                const long long yo = P.Y.base + (long long)tr * TR * P.Y.stride + (long long)tc * TC;
+                if (yo % 4 || P.Y.stride % 4) sh.fail("Y tile not 16-byte aligned", yo);
+                for (int o = 0; o < TR; ++o)
+                    for (int e = 0; e < TC; ++e) sh.write(yo + (long long)o * P.Y.stride + e, ylo, yhi, YT, "Y tile");
+            } else {
+                for (int o = 0; o < TR; ++o) {
+                    const int h = tr * TR + o;
+                    if (h >= H) continue;
+                    for (int e = 0; e < TC; ++e) check_global((long long)h * W + tc * TC + e, (long long)H * W, "y store");
                 }
-                for (int e = 0; e < TC; ++e) check_global((long long)h * W + w0 + e, (long long)H * W, "y store");
             }
         }
     }
@@ -381,14 +421,23 @@ void check_bwdw(const wtconv_desc_t& d) {
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
     const long long dlo = P.DY.base, dhi = P.DY.base + (long long)P.ntr[kMaxL] * TR * P.DY.stride;
     if (P.stg % 4 || P.stg_floats % 4) sh.fail("staging alignment", P.stg);
-    // Two planes in a row: the second must see the same zero padding.
+    // Two planes in a row (the second must see the same zero padding), with
+    // the kernel's CTA barriers as phase boundaries:
+    //   stage(0) | analysis(0) | stage(1), correlation(0) | analysis(1) | correlation(1) | reduction
+    sh.phase = "initial staging";
+    replay_stage(sh, P, P.stg, XT + 10);
+    replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10);
     for (int plane = 0; plane < 2; ++plane) {
-        sh.phase = "staging";
-        replay_stage(sh, P, P.stg, XT + 10);
-        replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10);
+        sh.barrier();
         sh.phase = "analysis";
         replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S, p, s_tag);
         replay_analyse(sh, P, P.stg + P.stg_floats, DYT + 10, P.DY.base, P.DY.stride, dlo, dhi, DYT, P.Q, 0, q_tag);
+        sh.barrier();
+        sh.phase = "staging";
+        if (plane == 0) {
+            replay_stage(sh, P, P.stg, XT + 10);
+            replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10);
+        }
         sh.phase = "correlation";
         for (int tid = 0; tid < P.n_all_tiles; ++tid) {
             int cl = 0;
@@ -415,6 +464,15 @@ void check_bwdw(const wtconv_desc_t& d) {
     sh.phase = "reduction";
     const long long red_end = (long long)P.red + (long long)P.nthreads * KK + P.nthreads;
     if (red_end > P.smem_floats) sh.fail("reduction scratch", red_end);
+    sh.barrier();
+    for (int tid = 0; tid < P.nthreads; ++tid)
+        for (int t = 0; t < KK; ++t) sh.write(P.red + (long long)tid * KK + t, P.red, red_end, RED, "class sums");
+    for (int w = 0; w < P.nthreads / 32; ++w)
+        sh.write(P.red + (long long)P.nthreads * KK + w, P.red, red_end, RED, "warp dy sums");
+    sh.barrier();
+    for (int k2 = 0; k2 < ncls; ++k2)
+        for (int th = P.cls_begin[k2]; th < P.cls_begin[k2 + 1]; ++th)
+            for (int t = 0; t < KK; ++t) sh.read(P.red + (long long)th * KK + t, P.red, red_end, RED, "class reduction");
     if (P.nthreads < P.n_all_tiles || P.nthreads > kBwdwMaxThreads || P.nthreads % 32) sh.fail("thread count", P.nthreads);
     if (P.groups < 1 || P.groups > P.B) sh.fail("groups", P.groups);
     if ((long long)P.nthreads * KK + P.nthreads / 32 > P.smem_floats) sh.fail("sum-dy scratch", P.nthreads);
