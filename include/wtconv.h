@@ -41,8 +41,11 @@
  *     non-OK status means nothing was enqueued and no output was touched.
  *     A launch failure returns WTCONV_ERR_CUDA.  Faults of an enqueued kernel
  *     surface at the caller's next synchronisation, as for any CUDA call.
- *   - Limits: k in {1, 3, 5, 7}; 0 <= L <= 6; H and W divisible by 2^L;
- *     planes too large for the on-chip staging return WTCONV_ERR_UNSUPPORTED.
+ *   - Limits: k in {1, 3, 5, 7}; 0 <= L <= 6; H and W divisible by 2^L.
+ *     A plane that does not fit on one SM is split into 2, 4 or 8 row strips
+ *     held by the CTAs of a thread-block cluster (strip height a multiple of
+ *     2^L and of 4); planes that still do not fit return
+ *     WTCONV_ERR_UNSUPPORTED.
  *   - L = 0 is the base branch only; wt_w and wt_scale may then be NULL.
  *   - Calls are reentrant; apart from the fixed scratch array of
  *     wtconv_backward_weight_noalloc (see there), the library holds no
@@ -131,8 +134,9 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, co
  * library (4 MiB of device memory per GPU that loads the library, held until
  * the process exits) for the per-block partial sums; it calls no cudaMalloc,
  * cudaFree or other allocating routine.
- *   - Size limit: C * groups * (k*k*(1+4L) + 1) floats must fit in 2^20 floats;
- *     larger problems return WTCONV_ERR_WORKSPACE (use wtconv_backward_weight).
+ *   - Size limit: the partial sums (wtconv_workspace_bytes(d) bytes) must fit in
+ *     2^20 floats; larger problems return WTCONV_ERR_WORKSPACE (use
+ *     wtconv_backward_weight).
  *   - The first call on each device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *   - Every call shares the one array: calls whose kernels overlap on the GPU

@@ -36,12 +36,13 @@ cudaError_t launch_bwdw(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_
     }
 }
 
-size_t workspace_floats(const Plan& P) { return (size_t)P.C * P.groups * P.nv; }
+size_t workspace_floats(const Plan& P) { return (size_t)P.C * P.parts * P.nv; }
 
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Weight gradient, stage 2: one CTA per channel sums the groups' partials in
+// Weight gradient, stage 2: one CTA per channel sums the partials (batch
+// groups x strips) in
 // a fixed order and turns them into the five parameter gradients.  The
 // channel's parameters are staged in shared memory first, and each dot
 // product is one warp's fixed xor-tree.
@@ -110,7 +111,7 @@ cudaError_t launch_bwdw_finish(const Plan& P, const float* part, const float* ba
                                const float* base_scale, const float* wt_w, const float* wt_scale,
                                float* d_base_w, float* d_base_b, float* d_base_scale, float* d_wt_w,
                                float* d_wt_scale, cudaStream_t s) {
-    wtconv_bwdw_finish_kernel<<<P.C, 128, (size_t)(P.nv + (1 + 4 * P.L) * P.k * P.k) * 4, s>>>(part, P.groups, P.nv, P.C, P.k, P.L, base_w,
+    wtconv_bwdw_finish_kernel<<<P.C, 128, (size_t)(P.nv + (1 + 4 * P.L) * P.k * P.k) * 4, s>>>(part, P.parts, P.nv, P.C, P.k, P.L, base_w,
                                                                  base_b, base_scale, wt_w, wt_scale, d_base_w,
                                                                  d_base_b, d_base_scale, d_wt_w, d_wt_scale);
     return cudaGetLastError();

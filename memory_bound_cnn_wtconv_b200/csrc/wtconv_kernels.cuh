@@ -26,6 +26,7 @@
 // plane, cp.async copies the next one from HBM into a staging buffer.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -33,6 +34,8 @@
 #include "wtconv_plan.h"
 
 namespace wtc {
+
+namespace cg = cooperative_groups;
 
 __device__ __forceinline__ int fdiv(int n, FastDiv f) {
     return (int)((__umulhi((uint32_t)n, f.mul) + (uint32_t)n) >> f.shift);
@@ -471,6 +474,71 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 }
 
 // ---------------------------------------------------------------------------
+// Planes split into strips across a thread-block cluster.
+// ---------------------------------------------------------------------------
+// Barrier of everything that shares a plane: the CTA, or the whole cluster
+// when the plane is split into strips (then it also orders the shared-memory
+// accesses of the cluster's CTAs to each other's strips).
+template <bool STRIPS>
+__device__ __forceinline__ void plane_sync() {
+    if constexpr (STRIPS) {
+        cg::this_cluster().sync();
+    } else {
+        __syncthreads();
+    }
+}
+
+// Fill the halo rows of one padded buffer of this CTA's strip: nsub planes
+// (1 or 4) of `rows` x `cols` interior elements behind `pad` border rows and
+// columns.  Halo row i (i in [-pad, 0) or [rows, rows + pad)) is plane row
+// rank*rows + i, read from the shared memory of the cluster CTA that owns it
+// (same offsets: every CTA of the cluster runs the same plan); rows outside
+// the plane are left as they are (zero).  Loads are issued in batches of 4
+// before the stores.
+__device__ __forceinline__ void copy_halo_rows(float* sm, const Buf& b, int nsub_lg, int rows, int cols, FastDiv dcols,
+                                               int pad, int rank, int nstrips, int tid, int nt) {
+    cg::cluster_group cl = cg::this_cluster();
+    const int n = (2 * pad << nsub_lg) * cols;
+    constexpr int U = 4;
+    for (int t0 = tid; t0 < n; t0 += U * nt) {
+        float v[U];
+        int dst[U];
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+            const int t = t0 + q * nt;
+            dst[q] = -1;
+            if (t < n) {
+                const int rest = fdiv(t, dcols), c = t - rest * cols;
+                const int hr = rest >> nsub_lg, s = rest - (hr << nsub_lg);
+                const int i = hr < pad ? hr - pad : rows + hr - pad;
+                const int g = rank * rows + i;
+                if (g >= 0 && g < nstrips * rows) {
+                    const int owner = g / rows, lr = g - owner * rows;
+                    const int col = b.base + s * b.sub + c + pad;
+                    const float* src = cl.map_shared_rank(sm + col + (lr + pad) * b.stride, owner);
+                    v[q] = *src;
+                    dst[q] = col + (i + pad) * b.stride;
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < U; ++q)
+            if (dst[q] >= 0) sm[dst[q]] = v[q];
+    }
+}
+
+// Halo rows of the padded input strip (X) and, for the subband convs, of
+// every level's padded subbands (S).
+__device__ __forceinline__ void copy_halos(float* sm, const Plan& P, int rank, int tid, int nt) {
+    const int p = P.p;
+    copy_halo_rows(sm, P.X, 0, P.H, P.W, P.div_w, p, rank, P.nstrips, tid, nt);
+#pragma unroll
+    for (int l = 0; l < kMaxL; ++l)
+        if (l < P.L)
+            copy_halo_rows(sm, P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), P.div_m[l], p, rank, P.nstrips, tid, nt);
+}
+
+// ---------------------------------------------------------------------------
 // Forward (BWD = false) and input gradient (BWD = true).
 // The input gradient is the same pass applied to dy with every kernel
 // rotated by 180 degrees and no bias: the transpose of the forward map.
@@ -588,12 +656,15 @@ struct FusedCtx {
     const float *base_w, *base_b, *base_scale, *wt_w, *wt_scale;
     long long units;
     int u0, u1;
+    size_t plane_elems;  // Hp * W
+    size_t strip_off;    // first element of this CTA's strip within a plane
 
     // Units run channel-major: unit u is plane (b, c) = (u mod B, u / B).
-    __device__ __forceinline__ size_t plane_of(int b, int c) const { return (size_t)b * P.C + c; }
-    __device__ __forceinline__ const T* src(int b, int c) const {
-        return x + plane_of(b, c) * ((size_t)P.H * P.W);
+    // Offset of this CTA's rows of plane (b, c).
+    __device__ __forceinline__ size_t rows_of(int b, int c) const {
+        return ((size_t)b * P.C + c) * plane_elems + strip_off;
     }
+    __device__ __forceinline__ const T* src(int b, int c) const { return x + rows_of(b, c); }
     // Reformulation (3): fold the scales (and the Haar factors) into the
     // weights of channel c (threads [0, np)).
     __device__ __forceinline__ void fold(int c, int np, int ptid) const {
@@ -625,7 +696,9 @@ struct FusedCtx {
 //               subband tiles write Q, base tiles write Y (y itself if L = 0).
 // Within a phase the buffers written (A: X, S, weights; B: staging, Q, Y) and
 // the buffers read (A: staging, Q, Y; B: S, X, weights) are disjoint.
-template <int K, int TR, int TC, typename T, bool BWD>
+// STRIPS: planes split into strips across a cluster (a separate
+// instantiation, so whole-plane walks carry no cluster code).
+template <int K, int TR, int TC, typename T, bool BWD, bool STRIPS>
 __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
     const T* __restrict__ x, const float* __restrict__ base_w, const float* __restrict__ base_b,
     const float* __restrict__ base_scale, const float* __restrict__ wt_w,
@@ -636,13 +709,16 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
     static_assert(TC == 4, "4-column tiles");
     const int tid = threadIdx.x, nt = blockDim.x;
     const long long units = (long long)P.B * P.C;
+    // With strips, the nstrips CTAs of a cluster walk the same planes.
+    const int rank = STRIPS ? (int)cg::this_cluster().block_rank() : 0;
+    const long long team = STRIPS ? blockIdx.x / P.nstrips : blockIdx.x;
+    const long long teams = STRIPS ? gridDim.x / P.nstrips : gridDim.x;
     FusedCtx<K, T, BWD> cx{sm, P, x, base_w, base_b, base_scale, wt_w, wt_scale, units,
-                           (int)(((long long)blockIdx.x * units) / gridDim.x),
-                           (int)(((long long)(blockIdx.x + 1) * units) / gridDim.x)};
+                           (int)((team * units) / teams), (int)(((team + 1) * units) / teams),
+                           (size_t)P.Hp * P.W, (size_t)rank * P.H * P.W};
     const int u0 = cx.u0, u1 = cx.u1;
     auto csync = [&]() { __syncthreads(); };
     float* X0 = sm + P.X.base + p * P.X.stride + p;
-    const size_t plane_elems = (size_t)P.H * P.W;
     int ft = tid - P.fin_off;
     if (ft < 0) ft += nt;
     // In the one-tile-per-thread schedule each thread's tile is fixed.
@@ -658,7 +734,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
     int folded_c = -1;
     for (int u = u0; u <= u1; ++u) {
         cp_async_wait_all();
-        __syncthreads();  // plane u staged; every tile of plane u-1 done
+        plane_sync<STRIPS>();  // plane u staged; every tile (and halo copy) of plane u-1 done
         // Phase A.
         if (u < u1) {
             if (cur_c != folded_c) {
@@ -668,11 +744,11 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
             analyse_plane<T, p, false, false>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         }
         if (u > u0 && P.L >= 1) {
-            T* yp = y + cx.plane_of(prev_b, prev_c) * plane_elems;
+            T* yp = y + cx.rows_of(prev_b, prev_c);
             for (int t = ft; t < P.n_fin; t += nt) synth_item<T>(sm, P, yp, t);
         }
         if (u == u1) break;
-        __syncthreads();  // X and S of plane u ready; Q and Y of plane u-1 consumed
+        plane_sync<STRIPS>();  // X and S of plane u ready (every strip); Q and Y of plane u-1 consumed
         // Phase B.
         int nb = cur_b + 1, nc = cur_c;
         if (nb == P.B) {
@@ -681,6 +757,10 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
         }
         if (u + 1 < u1) stage_plane(sm + P.stg, cx.src(nb, nc), P.plane_chunks, tid, nt);
         cp_async_commit();
+        if (STRIPS) {
+            copy_halos(sm, P, rank, tid, nt);
+            __syncthreads();  // halo rows in place
+        }
         for (int t = tid; t < P.tile_end; t += nt) {
             const TileJob j = P.merged ? fixed : decode_tile(P, t, TR, TC);
             if (!j.valid) continue;
@@ -695,7 +775,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
                 });
             } else {
                 // L = 0: the base branch is the whole output.
-                T* yo = y + cx.plane_of(cur_b, cur_c) * plane_elems + j.out;
+                T* yo = y + cx.rows_of(cur_b, cur_c) + j.out;
                 const int h0 = j.row0;
                 conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
                     if (h0 + o < P.H) gst4<T>(yo + (size_t)o * P.W, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
@@ -713,40 +793,45 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
 // ---------------------------------------------------------------------------
 // Weight gradient, stage 1: grid (C, groups).  The CTA of (c, g) walks the
 // planes b = g, g + groups, ... of channel c, staging the next (x, dy) pair
-// while it computes the current one.  Thread t owns one tile of one class
-// (base, or level l subband s) for the whole walk and accumulates its K*K
-// correlation sums in registers; the CTA then reduces each class over its
+// while it computes the current one.  Thread t owns a run of tiles of one
+// class (base, or level l subband s) for the whole walk and accumulates their
+// K*K correlation sums in registers; the CTA then reduces each class over its
 // threads in a fixed order and writes one partial vector (plus sum dy).
 // ---------------------------------------------------------------------------
-template <int K, int TR, int TC, typename T>
+// STRIPS: the plane is split into strips across a cluster (a separate
+// instantiation, so whole-plane walks keep every register for the sums).
+template <int K, int TR, int TC, typename T, bool STRIPS>
 __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel(
     const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const Plan P) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
     constexpr int p = K / 2, KK = K * K;
     const int tid = threadIdx.x, nt = blockDim.x;
-    const int c = blockIdx.x, g = blockIdx.y, G = P.groups;
-    const size_t plane_elems = (size_t)P.H * P.W;
+    // blockIdx.x = c * nstrips + (strip rank within the cluster).
+    const int rank = STRIPS ? (int)cg::this_cluster().block_rank() : 0;
+    const int c = STRIPS ? blockIdx.x / P.nstrips : blockIdx.x, g = blockIdx.y, G = P.groups;
+    const size_t plane_elems = (size_t)P.Hp * P.W;
+    const size_t strip_off = (size_t)rank * P.H * P.W;
     auto csync = [&]() { __syncthreads(); };
 
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
     if (g < P.B) {
-        const size_t off = ((size_t)g * P.C + c) * plane_elems;
+        const size_t off = ((size_t)g * P.C + c) * plane_elems + strip_off;
         stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
         stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
     }
     cp_async_commit();
 
-    int cl = -1, tr = 0, tc = 0;
-    if (tid < P.n_all_tiles) {
+    // This thread's class and its run of that class's tiles.
+    int cl = -1, first = 0, cnt = 0;
+    if (tid < P.cls_thr[1 + 4 * P.L]) {
         cl = 0;
-        while (tid >= P.cls_begin[cl + 1]) ++cl;
-        const int lvl = (cl == 0) ? kMaxL : ((cl - 1) >> 2);
-        const int local = tid - P.cls_begin[cl];
-        tr = fdiv(local, P.div_ntc[lvl]);
-        tc = local - tr * P.ntc[lvl];
+        while (tid >= P.cls_thr[cl + 1]) ++cl;
+        first = (tid - P.cls_thr[cl]) * P.tpt;
+        cnt = min(P.tpt, P.cls_tiles[cl] - first);
     }
+    const int lvl = cl <= 0 ? kMaxL : ((cl - 1) >> 2);
     float2 acc[KK];
 #pragma unroll
     for (int t = 0; t < KK; ++t) acc[t] = make_float2(0.f, 0.f);
@@ -755,7 +840,7 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
     float* X0 = sm + P.X.base + p * P.X.stride + p;
     for (int b = g; b < P.B; b += G) {
         cp_async_wait_all();
-        __syncthreads();  // staged pair complete; previous correlations done
+        plane_sync<STRIPS>();  // staged pair complete; previous correlations (and halo copies) done
         analyse_plane<T, p, false, false>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         const float s = analyse_plane<T, 0, true, true>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
                                                         P.DY.stride, 0, nt, tid, csync);
@@ -765,26 +850,34 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
             sdy_c = (tv - sdy) - yv;
             sdy = tv;
         }
-        __syncthreads();
+        plane_sync<STRIPS>();  // both analyses complete (every strip)
         if (b + G < P.B) {
-            const size_t off = ((size_t)(b + G) * P.C + c) * plane_elems;
+            const size_t off = ((size_t)(b + G) * P.C + c) * plane_elems + strip_off;
             stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
             stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
         }
         cp_async_commit();
-        if (cl == 0) {
-            corr_tile<K, TR, TC>(sm + P.X.base + tr * TR * P.X.stride + tc * TC, P.X.stride,
-                                 sm + P.DY.base + tr * TR * P.DY.stride + tc * TC, P.DY.stride, acc);
-        } else if (cl > 0) {
-            const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
-            const Buf& S = P.S[l];
-            const Buf& Q = P.Q[l];
-            corr_tile<K, TR, TC>(sm + S.base + s2 * S.sub + tr * TR * S.stride + tc * TC, S.stride,
-                                 sm + Q.base + s2 * Q.sub + tr * TR * Q.stride + tc * TC, Q.stride, acc);
+        if (STRIPS) {
+            copy_halos(sm, P, rank, tid, nt);
+            __syncthreads();  // halo rows in place
+        }
+        for (int k = 0; k < cnt; ++k) {
+            const int local = first + k;
+            const int tr = fdiv(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
+            if (cl == 0) {
+                corr_tile<K, TR, TC>(sm + P.X.base + tr * TR * P.X.stride + tc * TC, P.X.stride,
+                                     sm + P.DY.base + tr * TR * P.DY.stride + tc * TC, P.DY.stride, acc);
+            } else {
+                const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
+                const Buf& S = P.S[l];
+                const Buf& Q = P.Q[l];
+                corr_tile<K, TR, TC>(sm + S.base + s2 * S.sub + tr * TR * S.stride + tc * TC, S.stride,
+                                     sm + Q.base + s2 * Q.sub + tr * TR * Q.stride + tc * TC, Q.stride, acc);
+            }
         }
     }
     cp_async_wait_all();
-    __syncthreads();
+    plane_sync<STRIPS>();  // no CTA of the cluster reads this CTA's strip any more
 
     // Fixed-order reduction of every class over its threads.
     float* red = sm + P.red;
@@ -796,12 +889,12 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
     for (int o = 16; o > 0; o >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
     if ((tid & 31) == 0) red[nt * KK + (tid >> 5)] = sw;
     __syncthreads();
-    float* out = part + ((size_t)c * G + g) * P.nv;
+    float* out = part + ((size_t)c * P.parts + (size_t)g * P.nstrips + rank) * P.nv;
     const int ncls = 1 + 4 * P.L;
     for (int t = tid; t < ncls * KK; t += nt) {
         const int k2 = t / KK, tap = t - k2 * KK;
         float s = 0.f;
-        for (int th = P.cls_begin[k2]; th < P.cls_begin[k2 + 1]; ++th) s += red[th * KK + tap];
+        for (int th = P.cls_thr[k2]; th < P.cls_thr[k2 + 1]; ++th) s += red[th * KK + tap];
         out[t] = s;
     }
     if (tid == 0) {

@@ -22,6 +22,7 @@ constexpr int kMaxDevices = 64;
 
 // cudaFuncSetAttribute for the dynamic shared-memory opt-in, once per kernel
 // and device (idempotent; a repeated call is harmless).
+// (and the non-portable cluster-size opt-in for 16-CTA clusters).
 template <class F>
 cudaError_t opt_in_smem(F* fn, bool (&done)[kMaxDevices]) {
     int dev = 0;
@@ -29,52 +30,102 @@ cudaError_t opt_in_smem(F* fn, bool (&done)[kMaxDevices]) {
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDevices && done[dev]) return cudaSuccess;
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev] = true;
     return e;
 }
 
-template <int TR, typename T, bool BWD>
+// Launch configuration; planes split into strips run as clusters of
+// nstrips CTAs along x.
+struct Launch {
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    Launch(const Plan& P, dim3 grid, cudaStream_t s) {
+        cfg = cudaLaunchConfig_t{};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(P.nthreads);
+        cfg.dynamicSmemBytes = (size_t)P.smem_floats * 4;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 0;
+        if (P.nstrips > 1) {
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = P.nstrips;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.numAttrs = 1;
+        }
+    }
+};
+
+template <int TR, typename T, bool BWD, bool STRIPS>
 cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
     static bool done[kMaxDevices] = {};
-    auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD>;
+    auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD, STRIPS>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
-    // Persistent grid: every resident CTA slot of the device, at most one CTA per plane.
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, P.nthreads, (size_t)P.smem_floats * 4)) !=
-        cudaSuccess)
-        return e;
+    // Persistent grid: every resident CTA slot (cluster slot, for strips) of
+    // the device, at most one CTA (cluster) per plane.
     const long long units = (long long)P.B * P.C;
-    const int grid = (int)std::min<long long>(units, (long long)sms * std::max(per_sm, 1));
-    fn<<<grid, P.nthreads, (size_t)P.smem_floats * 4, s>>>(
-        static_cast<const T*>(a.x), a.base_w, a.base_b, a.base_scale, a.wt_w, a.wt_scale, static_cast<T*>(a.y),
-        P);
+    long long teams = 0;
+    Launch L(P, dim3(1), s);
+    if (P.nstrips > 1) {
+        L.cfg.gridDim = dim3(P.nstrips * 64);  // any multiple of the cluster size, for the query
+        int clusters = 0;
+        if ((e = cudaOccupancyMaxActiveClusters(&clusters, fn, &L.cfg)) != cudaSuccess) return e;
+        if (clusters < 1) return cudaErrorInvalidConfiguration;
+        teams = clusters;
+    } else {
+        int dev = 0, sms = 0, per_sm = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, P.nthreads, (size_t)P.smem_floats * 4)) !=
+            cudaSuccess)
+            return e;
+        teams = (long long)sms * std::max(per_sm, 1);
+    }
+    L.cfg.gridDim = dim3((unsigned)(std::min<long long>(units, teams) * P.nstrips));
+    e = cudaLaunchKernelEx(&L.cfg, fn, static_cast<const T*>(a.x), a.base_w, a.base_b, a.base_scale, a.wt_w,
+                           a.wt_scale, static_cast<T*>(a.y), P);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <int TR, typename T, bool STRIPS>
+cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
+    static bool done[kMaxDevices] = {};
+    auto* fn = wtconv_bwdw_partial_kernel<WTC_K, TR, 4, T, STRIPS>;
+    cudaError_t e = opt_in_smem(fn, done);
+    if (e != cudaSuccess) return e;
+    Launch L(P, dim3(P.C * P.nstrips, P.groups), s);
+    if (P.nstrips > 1) {
+        // A cluster that can never be resident is an error, not a hang.
+        int clusters = 0;
+        if ((e = cudaOccupancyMaxActiveClusters(&clusters, fn, &L.cfg)) != cudaSuccess) return e;
+        if (clusters < 1) return cudaErrorInvalidConfiguration;
+    }
+    e = cudaLaunchKernelEx(&L.cfg, fn, static_cast<const T*>(a.x), static_cast<const T*>(a.dy), a.part, P);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 template <int TR, typename T>
-cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
-    static bool done[kMaxDevices] = {};
-    auto* fn = wtconv_bwdw_partial_kernel<WTC_K, TR, 4, T>;
-    cudaError_t e = opt_in_smem(fn, done);
-    if (e != cudaSuccess) return e;
-    fn<<<dim3(P.C, P.groups), P.nthreads, (size_t)P.smem_floats * 4, s>>>(
-        static_cast<const T*>(a.x), static_cast<const T*>(a.dy), a.part, P);
-    return cudaGetLastError();
+cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s) {
+    if (P.nstrips > 1) return bwd ? fused_typed<TR, T, true, true>(P, a, s) : fused_typed<TR, T, false, true>(P, a, s);
+    return bwd ? fused_typed<TR, T, true, false>(P, a, s) : fused_typed<TR, T, false, false>(P, a, s);
 }
 
 template <int TR>
 cudaError_t fused_tr(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cudaStream_t s) {
-    if (dtype == 0) return bwd ? fused_typed<TR, float, true>(P, a, s) : fused_typed<TR, float, false>(P, a, s);
-    return bwd ? fused_typed<TR, __nv_bfloat16, true>(P, a, s) : fused_typed<TR, __nv_bfloat16, false>(P, a, s);
+    if (dtype == 0) return fused_t<TR, float>(P, bwd, a, s);
+    return fused_t<TR, __nv_bfloat16>(P, bwd, a, s);
 }
 
 template <int TR>
 cudaError_t bwdw_tr(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
-    if (dtype == 0) return bwdw_typed<TR, float>(P, a, s);
-    return bwdw_typed<TR, __nv_bfloat16>(P, a, s);
+    const bool strips = P.nstrips > 1;
+    if (dtype == 0) return strips ? bwdw_typed<TR, float, true>(P, a, s) : bwdw_typed<TR, float, false>(P, a, s);
+    return strips ? bwdw_typed<TR, __nv_bfloat16, true>(P, a, s) : bwdw_typed<TR, __nv_bfloat16, false>(P, a, s);
 }
 
 }  // namespace

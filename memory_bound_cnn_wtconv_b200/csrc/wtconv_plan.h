@@ -29,6 +29,8 @@
 namespace wtc {
 
 constexpr int kMaxL = 6;
+constexpr int kMaxStrips = 16;          // CTAs of a cluster sharing one plane
+constexpr int kMaxPortableStrips = 8;   // larger clusters need the non-portable opt-in
 constexpr int kMaxCls = 1 + 4 * kMaxL;
 
 // Division by a runtime constant d as a multiply-high and a shift:
@@ -54,7 +56,7 @@ inline FastDiv make_fastdiv(uint32_t d) {
 
 // Thread budgets (also the kernels' __launch_bounds__, two CTAs per SM).
 constexpr int kFusedMaxThreads = 256;
-constexpr int kBwdwMaxThreads = 320;
+constexpr int kBwdwMaxThreads = 256;
 
 struct Buf {
     int base;    // float offset (see above)
@@ -63,7 +65,13 @@ struct Buf {
 };
 
 struct Plan {
+    // H is the height of the rows a CTA holds: the plane, or one of its
+    // nstrips strips (a thread-block cluster of nstrips CTAs per plane, CTA
+    // rank r holding plane rows [r*H, (r+1)*H) and, in its padding rows, the
+    // neighbouring strips' halo rows).  Hp is the plane height.
     int B, C, H, W, k, L, p;
+    int Hp, nstrips;
+    int parts;           // weight gradient: partial vectors per channel (groups * nstrips)
     int TR, TC;          // output tile: TR rows x TC cols per thread (TC = 4: two column pairs)
     int esize;           // bytes per stored activation (4 or 2)
     int nthreads;        // CTA size
@@ -80,11 +88,16 @@ struct Plan {
     Buf S[kMaxL], Q[kMaxL];
     int ntr[kMaxL + 1], ntc[kMaxL + 1];  // tile grid per level; index kMaxL = full resolution
     // Tile enumeration.  Forward: subband tiles in class order (l, s) first,
-    // counted by sub_begin; base tiles separately.  Weight gradient: every
-    // class (base first) gets a contiguous thread range cls_begin[cl].
+    // counted by sub_begin; base tiles separately.  Weight gradient: class cl
+    // (0 = base, 1 + 4l + s) has cls_tiles[cl] tiles and the contiguous
+    // thread range [cls_thr[cl], cls_thr[cl+1]); its j-th thread owns the
+    // class's tiles [j*tpt, min((j+1)*tpt, cls_tiles[cl])) for the whole walk,
+    // so every thread accumulates one class only.
     int sub_begin[kMaxCls + 1];
     int n_sub_tiles, n_base_tiles;
-    int cls_begin[kMaxCls + 1];
+    int cls_tiles[kMaxCls];
+    int cls_thr[kMaxCls + 1];
+    int tpt;             // weight gradient: tiles per thread (at most)
     int n_all_tiles;
     int nv;              // weight gradient: floats per partial vector = ncls*k*k + 1
     // Forward tile index space: subband tiles [0, n_sub_tiles), base tiles
@@ -100,6 +113,7 @@ struct Plan {
     int pyr_lg;          // pyramid lane groups cover (4 * 2^pyr_lg)^2 pixel regions
     FastDiv div_rw;      // (W >> (pyr_lg + 2)): pyramid regions per row
     FastDiv div_q4;                 // W / 4: 4-column groups per row
+    FastDiv div_w;                  // W
     FastDiv div_m[kMaxL];           // W >> (l+1)
     FastDiv div_ntc[kMaxL + 1];     // tile columns per tile row
 };

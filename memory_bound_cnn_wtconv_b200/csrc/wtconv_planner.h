@@ -50,26 +50,6 @@ inline int tile_threads(int tiles, int max_threads) {
     return std::min(t, max_threads);
 }
 
-// Tile height: the one with the shorter tile phase, i.e. fewer tile rows on
-// the busiest SM sub-partition (warp-tiles per sub-partition x TR).
-inline int pick_tile_rows(const wtconv_desc_t* d, int max_threads) {
-    int best = 7;
-    long long best_cost = -1;
-    for (int TR = 7; TR <= 8; ++TR) {
-        const int tiles = count_tiles(d, TR);
-        const int threads = tile_threads(tiles, max_threads);
-        const long long warp_tiles = ceil_div(tiles, 32);
-        const long long per_smsp = ceil_div((int)std::min<long long>(warp_tiles, 1 << 30), 4);
-        const long long iters = ceil_div(tiles, threads);
-        const long long cost = std::max(per_smsp, iters) * TR;
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = TR;
-        }
-    }
-    return best;
-}
-
 // CTAs per SM that the shared memory of one CTA allows (the register
 // budget of the launch bounds allows two).
 inline int ctas_per_sm(int smem_floats) {
@@ -118,15 +98,24 @@ inline wtconv_status_t validate(const wtconv_desc_t* d) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
+// The plan for tile height TR with every plane split into `nstrips`
+// horizontal strips of H / nstrips rows (one CTA of a thread-block cluster
+// per strip; 1 = whole planes, no cluster).  Every field that describes
+// on-chip rows (H, ntr, buffers, tiles) describes one strip.
+inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, Plan* P) {
     memset(P, 0, sizeof(*P));
-    P->B = d->B; P->C = d->C; P->H = d->H; P->W = d->W; P->k = d->k; P->L = d->L;
-    const int p = d->k / 2, k = d->k, L = d->L, H = d->H, W = d->W, KK = k * k;
+    if (nstrips < 1 || nstrips > kMaxStrips || d->H % nstrips) return WTCONV_ERR_UNSUPPORTED;
+    const int Hs = d->H / nstrips;
+    if (nstrips > 1 && (Hs % (1 << d->L) != 0 || Hs % 4 != 0)) return WTCONV_ERR_UNSUPPORTED;
+    P->B = d->B; P->C = d->C; P->H = Hs; P->W = d->W; P->k = d->k; P->L = d->L;
+    P->Hp = d->H;
+    P->nstrips = nstrips;
+    const int p = d->k / 2, k = d->k, L = d->L, H = Hs, W = d->W, KK = k * k;
     P->p = p;
     P->esize = d->dtype == WTCONV_BF16 ? 2 : 4;
     P->TC = 4;
-    P->TR = pick_tile_rows(d, kind == kBackwardWeight ? kBwdwMaxThreads : kFusedMaxThreads);
-    const int TR = P->TR, TC = P->TC;
+    P->TR = TR;
+    const int TC = P->TC;
     const int WV4 = 4 * ((TC + k - 1 + 3) / 4);  // floats read per window row
 
     P->ntr[kMaxL] = ceil_div(H, TR);
@@ -205,13 +194,12 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
         }
     P->n_sub_tiles = nsub;
     P->n_base_tiles = P->ntr[kMaxL] * P->ntc[kMaxL];
-    P->cls_begin[0] = 0;
-    P->cls_begin[1] = P->n_base_tiles;
-    for (int cl = 1; cl < ncls; ++cl) {
-        const int l = (cl - 1) >> 2;
-        P->cls_begin[cl + 1] = P->cls_begin[cl] + P->ntr[l] * P->ntc[l];
+    P->n_all_tiles = 0;
+    for (int cl = 0; cl < ncls; ++cl) {
+        const int lv = cl == 0 ? kMaxL : (cl - 1) >> 2;
+        P->cls_tiles[cl] = P->ntr[lv] * P->ntc[lv];
+        P->n_all_tiles += P->cls_tiles[cl];
     }
-    P->n_all_tiles = P->cls_begin[ncls];
     P->nv = ncls * KK + 1;
 
     P->pyr = (L >= 1 && H % 4 == 0) ? 1 : 0;
@@ -219,14 +207,22 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     P->pyr_lg = std::max(P->pyr_levels - 2, 0);
     P->div_rw = make_fastdiv(std::max(W >> (P->pyr_lg + 2), 1));
     P->div_q4 = make_fastdiv(W / 4);
+    P->div_w = make_fastdiv(W);
     for (int l = 0; l < L; ++l) P->div_m[l] = make_fastdiv(W >> (l + 1));
     for (int l = 0; l <= kMaxL; ++l) P->div_ntc[l] = make_fastdiv(std::max(P->ntc[l], 1));
 
     if (kind == kBackwardWeight) {
-        // One tile per thread for the whole walk.
-        if (P->n_all_tiles > kBwdwMaxThreads) return WTCONV_ERR_UNSUPPORTED;
-        P->nthreads = tile_threads(P->n_all_tiles, kBwdwMaxThreads);
-        if (P->nthreads < P->n_all_tiles) P->nthreads = ceil_div(P->n_all_tiles, 32) * 32;
+        // The fewest tiles per thread whose class-pure thread ranges fit.
+        int tpt = 1, used = 0;
+        for (;; ++tpt) {
+            used = 0;
+            for (int cl = 0; cl < ncls; ++cl) used += ceil_div(P->cls_tiles[cl], tpt);
+            if (used <= kBwdwMaxThreads) break;
+        }
+        P->tpt = tpt;
+        P->cls_thr[0] = 0;
+        for (int cl = 0; cl < ncls; ++cl) P->cls_thr[cl + 1] = P->cls_thr[cl] + ceil_div(P->cls_tiles[cl], tpt);
+        P->nthreads = std::max(tile_threads(used, kBwdwMaxThreads), ceil_div(used, 32) * 32);
         // Reduction scratch aliases the (then dead) buffers from offset 0.
         P->red = 0;
         off = std::max(off, (long long)P->nthreads * (KK + 1));
@@ -253,11 +249,48 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;
     if (kind == kBackwardWeight) {
-        P->groups = pick_groups(P->B, P->C, P->smem_floats);
+        P->groups = pick_groups(P->B, P->C * nstrips, P->smem_floats);
+        P->parts = P->groups * nstrips;
     } else {
         const long long units = (long long)P->B * P->C;
         P->grid = (int)std::min<long long>(units, (long long)kNumSMs * ctas_per_sm(P->smem_floats));
         P->groups = 1;
+    }
+    return WTCONV_OK;
+}
+
+// Tile rows on the busiest SM sub-partition per plane and SM: the tile-phase
+// length of one CTA (its warp-tiles spread over 4 sub-partitions, times the
+// tile height), times the CTAs of a plane, over the CTAs an SM holds.
+// Cluster strips carry a halo exchange on top (weighted 15%).
+inline double plan_cost(const Plan& P, Kind kind) {
+    const int per_smsp = kind == kBackwardWeight ? P.tpt * ceil_div(ceil_div(P.cls_thr[1 + 4 * P.L], 32), 4)
+                                                 : ceil_div(ceil_div(P.tile_end, 32), 4);
+    const double c = (double)per_smsp * P.TR * P.nstrips / ctas_per_sm(P.smem_floats);
+    if (P.nstrips > kMaxPortableStrips) return 1.3 * c;  // a 16-CTA cluster needs 16 SMs of one GPC
+    return P.nstrips > 1 ? 1.15 * c : c;
+}
+
+// Chooses the strip count (whole planes, or clusters of 2, 4, 8, 16 strips)
+// and the tile height (7 or 8 rows) with the lowest plan_cost.
+inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
+    bool have = false;
+    double best = 0.0;
+    Plan cand;
+    for (int n = 1; n <= kMaxStrips; n *= 2) {
+        for (int TR = 7; TR <= 8; ++TR) {
+            if (make_plan_for(d, kind, TR, n, &cand) != WTCONV_OK) continue;
+            const double c = plan_cost(cand, kind);
+            if (!have || c < best) {
+                best = c;
+                *P = cand;
+                have = true;
+            }
+        }
+    }
+    if (!have) {
+        memset(P, 0, sizeof(*P));
+        return WTCONV_ERR_UNSUPPORTED;
     }
     return WTCONV_OK;
 }

@@ -72,13 +72,15 @@ void check_global(long long idx, long long n, const char* what) {
     }
 }
 
-// Replays stage_plane: 16-byte chunk ch of the stored plane -> staging floats [stg + 4ch, stg + 4ch + 4).
-void replay_stage(Shadow& sh, const Plan& P, long long stg, int tag) {
-    const long long plane_bytes = (long long)P.H * P.W * P.esize;
-    if (P.plane_chunks * 16LL != plane_bytes) sh.fail("plane is not a whole number of 16-byte chunks", plane_bytes);
+// Replays stage_plane: 16-byte chunk ch of this CTA's rows (strip `rank`) of
+// the stored plane -> staging floats [stg + 4ch, stg + 4ch + 4).
+void replay_stage(Shadow& sh, const Plan& P, long long stg, int tag, int rank) {
+    const long long strip_bytes = (long long)P.H * P.W * P.esize;
+    const long long plane_bytes = (long long)P.Hp * P.W * P.esize;
+    if (P.plane_chunks * 16LL != strip_bytes) sh.fail("strip is not a whole number of 16-byte chunks", strip_bytes);
     if (stg % 4) sh.fail("staging not 16-byte aligned", stg);
     for (int ch = 0; ch < P.plane_chunks; ++ch) {
-        check_global(16LL * ch + 15, plane_bytes, "staging source");
+        check_global(rank * strip_bytes + 16LL * ch + 15, plane_bytes, "staging source");
         for (int e = 0; e < 4; ++e) sh.write(stg + 4LL * ch + e, stg, stg + P.stg_floats, tag, "staging");
     }
 }
@@ -202,7 +204,7 @@ void replay_haar(Shadow& sh, long long src, int ss, long long slo, long long shi
 // Replays the window reads of conv_tile / corr_tile on a padded plane whose
 // padded element (-p, -p) sits at `base`; interior n x m must carry `itag`.
 void replay_window(Shadow& sh, const Plan& P, long long base, int stride, long long lo, long long hi, int n, int m,
-                   int tr, int tc, int itag, const char* what) {
+                   int tr, int tc, int itag, const char* what, int rank) {
     const int K = P.k, p = P.p, TR = P.TR, TC = P.TC;
     const int WV4 = 4 * ((TC + K - 1 + 3) / 4);
     const long long win = base + (long long)tr * TR * stride + (long long)tc * TC;
@@ -216,7 +218,12 @@ void replay_window(Shadow& sh, const Plan& P, long long base, int stride, long l
                 continue;
             }
             const int i = tr * TR + r - p, j = tc * TC + c - p;
-            const bool interior = i >= 0 && i < n && j >= 0 && j < m;
+            // Row i of this strip is plane row rank*n + i: its own rows and
+            // the p halo rows on each side (copied from the neighbouring
+            // strips) carry the data tag inside the plane and zero outside;
+            // rows further down only feed tile-slack outputs and stay zero.
+            const long long g = (long long)rank * n + i;
+            const bool interior = i >= -p && i < n + p && g >= 0 && g < (long long)P.nstrips * n && j >= 0 && j < m;
             sh.read(a, lo, hi, interior ? itag : ZERO, what);
         }
 }
@@ -255,6 +262,41 @@ void check_divs(const Plan& P) {
     }
 }
 
+// Replays copy_halos for strip `rank`: every halo row of X and of every
+// level's subbands is read from the CTA that owns the row (its own tag) and
+// written into this CTA's padding rows.
+void replay_halos(std::vector<Shadow>& shs, const Plan& P, int rank) {
+    Shadow& me = shs[rank];
+    auto one = [&](const Buf& b, int nsub_lg, int rows, int cols, FastDiv dcols, int tagbase, bool per_sub_tag) {
+        const int pad = P.p;
+        const int n = (2 * pad << nsub_lg) * cols;
+        const long long span = (long long)(1 << nsub_lg) * (b.sub ? b.sub : 0);
+        const long long lo = b.base, hi = nsub_lg ? b.base + span : b.base + (long long)(rows + 2 * pad) * b.stride;
+        for (int t = 0; t < n; ++t) {
+            const int rest = (int)fastdiv_host(t, dcols), c = t - rest * cols;
+            if (rest != t / cols) me.fail("halo column division", t);
+            const int hr = rest >> nsub_lg, s = rest - (hr << nsub_lg);
+            const int i = hr < pad ? hr - pad : rows + hr - pad;
+            const int g = rank * rows + i;
+            if (g < 0 || g >= P.nstrips * rows) continue;
+            const int owner = g / rows, lr = g - owner * rows;
+            if (owner == rank) me.fail("halo row owned by the copying strip", g);
+            const long long col = b.base + (long long)s * b.sub + c + pad;
+            const int tag = per_sub_tag ? tagbase + s : tagbase;
+            const long long slo = nsub_lg ? b.base + (long long)s * b.sub : lo;
+            const long long shi = nsub_lg ? b.base + (long long)(s + 1) * b.sub : hi;
+            shs[owner].read(col + (long long)(lr + pad) * b.stride, slo, shi, tag, "halo source");
+            me.write(col + (long long)(i + pad) * b.stride, slo, shi, tag, "halo row");
+        }
+    };
+    one(P.X, 0, P.H, P.W, P.div_w, XT, false);
+    for (int l = 0; l < P.L; ++l) one(P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), P.div_m[l], s_tag(l, 0), true);
+}
+
+void barrier_all(std::vector<Shadow>& shs) {
+    for (auto& sh : shs) sh.barrier();
+}
+
 void check_fused(const wtconv_desc_t& d, Kind kind) {
     Plan P;
     const wtconv_status_t st = make_plan(&d, kind, &P);
@@ -267,8 +309,13 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
         std::exit(1);
     }
     const int K = P.k, KK = K * K, p = P.p, L = P.L, H = P.H, W = P.W, TR = P.TR, TC = P.TC;
-    const int ncls = 1 + 4 * L;
+    const int ncls = 1 + 4 * L, NS = P.nstrips;
     check_divs(P);
+    check_div(P.div_w, W, (long long)(2 * p * 4) * W + 1, "W");
+    if (P.Hp != H * NS || NS < 1 || NS > kMaxStrips || (NS > 1 && (H % (1 << L) || H % 4))) {
+        std::printf("FAIL strips: Hp %d H %d n %d\n", P.Hp, H, NS);
+        std::exit(1);
+    }
     if (P.nthreads % 32 || P.nthreads > kFusedMaxThreads || P.nthreads < 32) {
         std::printf("FAIL fused thread count %d\n", P.nthreads);
         std::exit(1);
@@ -287,18 +334,19 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
         std::printf("FAIL smem size\n");
         std::exit(1);
     }
-    Shadow sh(P.smem_floats);
+    std::vector<Shadow> shs(NS, Shadow(P.smem_floats));
     const long long all = P.smem_floats;
-    if (P.grid < 1 || P.grid > (long long)P.B * P.C) sh.fail("grid", P.grid);
+    if (P.grid < 1 || P.grid > (long long)P.B * P.C) shs[0].fail("grid", P.grid);
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
     const long long ylo = P.Y.base, yhi = P.Y.base + (long long)P.ntr[kMaxL] * TR * P.Y.stride;
     for (int cl = 0; cl < ncls; ++cl)
-        if ((P.wbase + cl * P.wcls) % 4) sh.fail("weight class not 16-byte aligned", P.wbase + cl * P.wcls);
+        if ((P.wbase + cl * P.wcls) % 4) shs[0].fail("weight class not 16-byte aligned", P.wbase + cl * P.wcls);
     const int ntc = P.ntc[kMaxL];
+    const long long plane = (long long)P.Hp * W;
 
     // Phase A's synthesis of the previous plane: rows 2i, 2i+1 x columns 4q..4q+3.
-    auto synthesis = [&]() {
+    auto synthesis = [&](Shadow& sh, int rank) {
         for (int t = 0; t < P.n_fin; ++t) {
             const int i = (int)fastdiv_host(t, P.div_q4), q = t - i * (W / 4);
             if (i != t / (W / 4)) sh.fail("synthesis item division", t);
@@ -325,81 +373,113 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
                 if (a % 4) sh.fail("Y load not 16-byte aligned", a);
                 for (int e = 0; e < 4; ++e) {
                     sh.read(a + e, ylo, yhi, YT, "Y read");
-                    check_global((long long)(2 * i + rr) * W + 4 * q + e, (long long)H * W, "y store");
+                    check_global((long long)(rank * H + 2 * i + rr) * W + 4 * q + e, plane, "y store");
                 }
             }
         }
     };
 
     // The persistent walk over two planes and the final synthesis, with the
-    // kernel's CTA barriers as phase boundaries:
-    //   stage(0) | A(0) | B(0): stage(1), tiles(0) | A(1) | B(1): tiles(1) | A(end)
-    sh.phase = "initial staging";
-    replay_stage(sh, P, P.stg, XT + 10);
+    // kernel's barriers (cluster-wide with strips) as phase boundaries:
+    //   stage(0) | A(0) | B(0): stage(1), halos(0), | tiles(0) | A(1) | B(1) ... | A(end)
+    for (int r = 0; r < NS; ++r) {
+        shs[r].phase = "initial staging";
+        replay_stage(shs[r], P, P.stg, XT + 10, r);
+    }
     for (int unit = 0; unit <= 2; ++unit) {
-        sh.barrier();
-        if (unit < 2) {
-            sh.phase = "A: fold";
-            for (int cl = 0; cl < ncls; ++cl)
-                for (int t = 0; t < KK; ++t)
-                    sh.write(P.wbase + (long long)cl * P.wcls + t, P.wbase, P.wbase + (long long)ncls * P.wcls, WTS,
-                             "weights");
-            sh.write(P.bias, P.bias, P.bias + 1, BIAS, "bias");
-            sh.phase = "A: analysis";
-            replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT,
-                           P.S, p, s_tag);
-        }
-        if (unit > 0 && L >= 1) {
-            sh.phase = "A: synthesis";
-            synthesis();
-        }
-        if (unit == 2) break;
-        sh.barrier();
-        sh.phase = "B: staging";
-        if (unit + 1 < 2) replay_stage(sh, P, P.stg, XT + 10);
-        sh.phase = "B: subband tiles";
-        for (int cl = 1; cl < ncls; ++cl) {
-            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-            const int n = H >> (l + 1), m = W >> (l + 1);
-            const int ntiles = P.sub_begin[cl] - P.sub_begin[cl - 1];
-            if (ntiles != P.ntr[l] * P.ntc[l]) sh.fail("tile count", cl);
-            for (int local = 0; local < ntiles; ++local) {
-                const int tr = (int)fastdiv_host(local, P.div_ntc[l]), tc = local - tr * P.ntc[l];
-                for (int t = 0; t < KK; ++t) sh.read(P.wbase + (long long)cl * P.wcls + t, 0, all, WTS, "weights");
-                const Buf& S = P.S[l];
-                replay_window(sh, P, S.base + (long long)s * S.sub, S.stride, S.base + (long long)s * S.sub,
-                              S.base + (long long)(s + 1) * S.sub, n, m, tr, tc, s_tag(l, s), "subband window");
-                const Buf& Q = P.Q[l];
-                const long long out = Q.base + (long long)s * Q.sub + (long long)tr * TR * Q.stride + (long long)tc * TC;
-                if (out % 4) sh.fail("Q tile not 16-byte aligned", out);
-                for (int o = 0; o < TR; ++o)
-                    for (int j = 0; j < TC; ++j)
-                        sh.write(out + (long long)o * Q.stride + j, Q.base + (long long)s * Q.sub,
-                                 Q.base + (long long)(s + 1) * Q.sub, q_tag(l, s), "Q tile");
+        barrier_all(shs);
+        for (int r = 0; r < NS; ++r) {
+            Shadow& sh = shs[r];
+            if (unit < 2) {
+                sh.phase = "A: fold";
+                for (int cl = 0; cl < ncls; ++cl)
+                    for (int t = 0; t < KK; ++t)
+                        sh.write(P.wbase + (long long)cl * P.wcls + t, P.wbase, P.wbase + (long long)ncls * P.wcls, WTS,
+                                 "weights");
+                sh.write(P.bias, P.bias, P.bias + 1, BIAS, "bias");
             }
         }
-        sh.phase = "B: base tiles";
-        for (int t = 0; t < P.n_base_tiles; ++t) {
-            const int tr = (int)fastdiv_host(t, P.div_ntc[kMaxL]), tc = t - tr * ntc;
-            for (int q = 0; q < KK; ++q) sh.read(P.wbase + q, 0, all, WTS, "base weights");
-            sh.read(P.bias, 0, all, BIAS, "bias");
-            replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base window");
-            if (L >= 1) {
-                const long long yo = P.Y.base + (long long)tr * TR * P.Y.stride + (long long)tc * TC;
-                if (yo % 4 || P.Y.stride % 4) sh.fail("Y tile not 16-byte aligned", yo);
-                for (int o = 0; o < TR; ++o)
-                    for (int e = 0; e < TC; ++e) sh.write(yo + (long long)o * P.Y.stride + e, ylo, yhi, YT, "Y tile");
-            } else {
-                for (int o = 0; o < TR; ++o) {
-                    const int h = tr * TR + o;
-                    if (h >= H) continue;
-                    for (int e = 0; e < TC; ++e) check_global((long long)h * W + tc * TC + e, (long long)H * W, "y store");
+        if (unit < 2) {
+            // The analysis may have its own CTA barriers (levels computed one
+            // at a time); the synthesis runs after its last one.
+            for (int r = 0; r < NS; ++r) {
+                shs[r].phase = "A: analysis";
+                const int e0 = shs[r].epoch;
+                replay_analyse(shs[r], P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi,
+                               XT, P.S, p, s_tag);
+                if (r + 1 < NS) shs[r].epoch = e0;  // replay the next strip from the same phase
+                else for (int q = 0; q + 1 < NS; ++q) shs[q].epoch = shs[r].epoch;
+            }
+        }
+        if (unit > 0 && L >= 1)
+            for (int r = 0; r < NS; ++r) {
+                shs[r].phase = "A: synthesis";
+                synthesis(shs[r], r);
+            }
+        if (unit == 2) break;
+        barrier_all(shs);
+        for (int r = 0; r < NS; ++r) {
+            shs[r].phase = "B: staging";
+            if (unit + 1 < 2) replay_stage(shs[r], P, P.stg, XT + 10, r);
+        }
+        if (NS > 1) {
+            for (int r = 0; r < NS; ++r) {
+                shs[r].phase = "B: halo copy";
+                replay_halos(shs, P, r);
+            }
+            // Local barrier after the copy: a new phase for each CTA (the other
+            // CTAs' phase is unchanged, so remote reads still conflict with
+            // their later writes only through this CTA's epoch -- the replay
+            // keeps the cluster in lockstep, which is the stricter check).
+            barrier_all(shs);
+        }
+        for (int r = 0; r < NS; ++r) {
+            Shadow& sh = shs[r];
+            sh.phase = "B: subband tiles";
+            for (int cl = 1; cl < ncls; ++cl) {
+                const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+                const int n = H >> (l + 1), m = W >> (l + 1);
+                const int ntiles = P.sub_begin[cl] - P.sub_begin[cl - 1];
+                if (ntiles != P.ntr[l] * P.ntc[l]) sh.fail("tile count", cl);
+                for (int local = 0; local < ntiles; ++local) {
+                    const int tr = (int)fastdiv_host(local, P.div_ntc[l]), tc = local - tr * P.ntc[l];
+                    for (int t = 0; t < KK; ++t) sh.read(P.wbase + (long long)cl * P.wcls + t, 0, all, WTS, "weights");
+                    const Buf& S = P.S[l];
+                    replay_window(sh, P, S.base + (long long)s * S.sub, S.stride, S.base + (long long)s * S.sub,
+                                  S.base + (long long)(s + 1) * S.sub, n, m, tr, tc, s_tag(l, s), "subband window", r);
+                    const Buf& Q = P.Q[l];
+                    const long long out = Q.base + (long long)s * Q.sub + (long long)tr * TR * Q.stride + (long long)tc * TC;
+                    if (out % 4) sh.fail("Q tile not 16-byte aligned", out);
+                    for (int o = 0; o < TR; ++o)
+                        for (int j = 0; j < TC; ++j)
+                            sh.write(out + (long long)o * Q.stride + j, Q.base + (long long)s * Q.sub,
+                                     Q.base + (long long)(s + 1) * Q.sub, q_tag(l, s), "Q tile");
+                }
+            }
+            sh.phase = "B: base tiles";
+            for (int t = 0; t < P.n_base_tiles; ++t) {
+                const int tr = (int)fastdiv_host(t, P.div_ntc[kMaxL]), tc = t - tr * ntc;
+                for (int q = 0; q < KK; ++q) sh.read(P.wbase + q, 0, all, WTS, "base weights");
+                sh.read(P.bias, 0, all, BIAS, "bias");
+                replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base window", r);
+                if (L >= 1) {
+                    const long long yo = P.Y.base + (long long)tr * TR * P.Y.stride + (long long)tc * TC;
+                    if (yo % 4 || P.Y.stride % 4) sh.fail("Y tile not 16-byte aligned", yo);
+                    for (int o = 0; o < TR; ++o)
+                        for (int e = 0; e < TC; ++e) sh.write(yo + (long long)o * P.Y.stride + e, ylo, yhi, YT, "Y tile");
+                } else {
+                    for (int o = 0; o < TR; ++o) {
+                        const int h = tr * TR + o;
+                        if (h >= H) continue;
+                        for (int e = 0; e < TC; ++e)
+                            check_global((long long)(r * H + h) * W + tc * TC + e, plane, "y store");
+                    }
                 }
             }
         }
     }
-    std::printf("fused(kind %d): smem %d B, threads %d, TR %d, tiles %d+%d, merged %d\n", (int)kind,
-                P.smem_floats * 4, P.nthreads, TR, P.n_sub_tiles, P.n_base_tiles, P.merged);
+    std::printf("fused(kind %d): smem %d B, threads %d, TR %d, tiles %d+%d, merged %d, strips %d\n", (int)kind,
+                P.smem_floats * 4, P.nthreads, TR, P.n_sub_tiles, P.n_base_tiles, P.merged, NS);
 }
 
 void check_bwdw(const wtconv_desc_t& d) {
@@ -414,71 +494,112 @@ void check_bwdw(const wtconv_desc_t& d) {
         std::exit(1);
     }
     const int K = P.k, KK = K * K, p = P.p, L = P.L, H = P.H, W = P.W, TR = P.TR;
-    const int ncls = 1 + 4 * L;
+    const int ncls = 1 + 4 * L, NS = P.nstrips;
     check_divs(P);
-    Shadow sh(P.smem_floats);
+    check_div(P.div_w, W, (long long)(2 * p * 4) * W + 1, "W");
+    std::vector<Shadow> shs(NS, Shadow(P.smem_floats));
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
     const long long dlo = P.DY.base, dhi = P.DY.base + (long long)P.ntr[kMaxL] * TR * P.DY.stride;
-    if (P.stg % 4 || P.stg_floats % 4) sh.fail("staging alignment", P.stg);
+    if (P.stg % 4 || P.stg_floats % 4) shs[0].fail("staging alignment", P.stg);
     // Two planes in a row (the second must see the same zero padding), with
-    // the kernel's CTA barriers as phase boundaries:
-    //   stage(0) | analysis(0) | stage(1), correlation(0) | analysis(1) | correlation(1) | reduction
-    sh.phase = "initial staging";
-    replay_stage(sh, P, P.stg, XT + 10);
-    replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10);
+    // the kernel's barriers (cluster-wide with strips) as phase boundaries:
+    //   stage(0) | analysis(0) | stage(1), halos(0) | correlation(0) | analysis(1) | ... | reduction
+    for (int r = 0; r < NS; ++r) {
+        shs[r].phase = "initial staging";
+        replay_stage(shs[r], P, P.stg, XT + 10, r);
+        replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
+    }
     for (int plane = 0; plane < 2; ++plane) {
-        sh.barrier();
-        sh.phase = "analysis";
-        replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S, p, s_tag);
-        replay_analyse(sh, P, P.stg + P.stg_floats, DYT + 10, P.DY.base, P.DY.stride, dlo, dhi, DYT, P.Q, 0, q_tag);
-        sh.barrier();
-        sh.phase = "staging";
-        if (plane == 0) {
-            replay_stage(sh, P, P.stg, XT + 10);
-            replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10);
+        barrier_all(shs);
+        for (int r = 0; r < NS; ++r) {
+            Shadow& sh = shs[r];
+            sh.phase = "analysis";
+            const int e0 = sh.epoch;
+            replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S,
+                           p, s_tag);
+            replay_analyse(sh, P, P.stg + P.stg_floats, DYT + 10, P.DY.base, P.DY.stride, dlo, dhi, DYT, P.Q, 0, q_tag);
+            if (r + 1 < NS) sh.epoch = e0;
+            else for (int q = 0; q + 1 < NS; ++q) shs[q].epoch = sh.epoch;
         }
-        sh.phase = "correlation";
-        for (int tid = 0; tid < P.n_all_tiles; ++tid) {
-            int cl = 0;
-            while (tid >= P.cls_begin[cl + 1]) ++cl;
-            const int lvl = (cl == 0) ? kMaxL : ((cl - 1) >> 2);
-            const int local = tid - P.cls_begin[cl];
-            const int tr = (int)fastdiv_host(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
-            if (tr >= P.ntr[lvl]) sh.fail("tile row out of grid", tid);
-            if (cl == 0) {
-                replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base S window");
-                replay_dtile(sh, P, P.DY.base, P.DY.stride, dlo, dhi, H, W, tr, tc, DYT);
-            } else {
-                const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-                const int n = H >> (l + 1), m = W >> (l + 1);
-                const Buf& S = P.S[l];
-                const Buf& Q = P.Q[l];
-                replay_window(sh, P, S.base + (long long)s * S.sub, S.stride, S.base + (long long)s * S.sub,
-                              S.base + (long long)(s + 1) * S.sub, n, m, tr, tc, s_tag(l, s), "subband S window");
-                replay_dtile(sh, P, Q.base + (long long)s * Q.sub, Q.stride, Q.base + (long long)s * Q.sub,
-                             Q.base + (long long)(s + 1) * Q.sub, n, m, tr, tc, q_tag(l, s));
+        barrier_all(shs);
+        for (int r = 0; r < NS; ++r) {
+            shs[r].phase = "staging";
+            if (plane == 0) {
+                replay_stage(shs[r], P, P.stg, XT + 10, r);
+                replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
             }
         }
+        if (NS > 1) {
+            for (int r = 0; r < NS; ++r) {
+                shs[r].phase = "halo copy";
+                replay_halos(shs, P, r);
+            }
+            barrier_all(shs);
+        }
+        for (int r = 0; r < NS; ++r) {
+            Shadow& sh = shs[r];
+            sh.phase = "correlation";
+            int covered = 0;
+            for (int tid = 0; tid < P.cls_thr[ncls]; ++tid)
+              for (int k = 0; k < P.tpt; ++k) {
+                int cl = 0;
+                while (tid >= P.cls_thr[cl + 1]) ++cl;
+                const int lvl = (cl == 0) ? kMaxL : ((cl - 1) >> 2);
+                const int first = (tid - P.cls_thr[cl]) * P.tpt;
+                const int cnt = std::min(P.tpt, P.cls_tiles[cl] - first);
+                if (cnt < 1) sh.fail("thread without tiles", tid);
+                if (k >= cnt) continue;
+                const int local = first + k;
+                ++covered;
+                const int tr = (int)fastdiv_host(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
+                if (tr >= P.ntr[lvl]) sh.fail("tile row out of grid", tid);
+                if (cl == 0) {
+                    replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base S window", r);
+                    replay_dtile(sh, P, P.DY.base, P.DY.stride, dlo, dhi, H, W, tr, tc, DYT);
+                } else {
+                    const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+                    const int n = H >> (l + 1), m = W >> (l + 1);
+                    const Buf& S = P.S[l];
+                    const Buf& Q = P.Q[l];
+                    replay_window(sh, P, S.base + (long long)s * S.sub, S.stride, S.base + (long long)s * S.sub,
+                                  S.base + (long long)(s + 1) * S.sub, n, m, tr, tc, s_tag(l, s), "subband S window", r);
+                    replay_dtile(sh, P, Q.base + (long long)s * Q.sub, Q.stride, Q.base + (long long)s * Q.sub,
+                                 Q.base + (long long)(s + 1) * Q.sub, n, m, tr, tc, q_tag(l, s));
+                }
+              }
+            if (covered != P.n_all_tiles) sh.fail("tiles covered", covered);
+        }
     }
-    sh.phase = "reduction";
     const long long red_end = (long long)P.red + (long long)P.nthreads * KK + P.nthreads;
-    if (red_end > P.smem_floats) sh.fail("reduction scratch", red_end);
-    sh.barrier();
-    for (int tid = 0; tid < P.nthreads; ++tid)
-        for (int t = 0; t < KK; ++t) sh.write(P.red + (long long)tid * KK + t, P.red, red_end, RED, "class sums");
-    for (int w = 0; w < P.nthreads / 32; ++w)
-        sh.write(P.red + (long long)P.nthreads * KK + w, P.red, red_end, RED, "warp dy sums");
-    sh.barrier();
-    for (int k2 = 0; k2 < ncls; ++k2)
-        for (int th = P.cls_begin[k2]; th < P.cls_begin[k2 + 1]; ++th)
-            for (int t = 0; t < KK; ++t) sh.read(P.red + (long long)th * KK + t, P.red, red_end, RED, "class reduction");
-    if (P.nthreads < P.n_all_tiles || P.nthreads > kBwdwMaxThreads || P.nthreads % 32) sh.fail("thread count", P.nthreads);
+    barrier_all(shs);
+    for (int r = 0; r < NS; ++r) {
+        Shadow& sh = shs[r];
+        sh.phase = "reduction";
+        if (red_end > P.smem_floats) sh.fail("reduction scratch", red_end);
+        for (int tid = 0; tid < P.nthreads; ++tid)
+            for (int t = 0; t < KK; ++t) sh.write(P.red + (long long)tid * KK + t, P.red, red_end, RED, "class sums");
+        for (int w = 0; w < P.nthreads / 32; ++w)
+            sh.write(P.red + (long long)P.nthreads * KK + w, P.red, red_end, RED, "warp dy sums");
+    }
+    barrier_all(shs);
+    for (int r = 0; r < NS; ++r)
+        for (int k2 = 0; k2 < ncls; ++k2)
+            for (int th = P.cls_thr[k2]; th < P.cls_thr[k2 + 1]; ++th)
+                for (int t = 0; t < KK; ++t)
+                    shs[r].read(P.red + (long long)th * KK + t, P.red, red_end, RED, "class reduction");
+    Shadow& sh = shs[0];
+    if (P.nthreads < P.cls_thr[ncls] || P.nthreads > kBwdwMaxThreads || P.nthreads % 32) sh.fail("thread count", P.nthreads);
+    for (int cl = 0; cl < ncls; ++cl) {
+        const int lv = cl == 0 ? kMaxL : (cl - 1) >> 2;
+        if (P.cls_tiles[cl] != P.ntr[lv] * P.ntc[lv]) sh.fail("class tiles", cl);
+    }
     if (P.groups < 1 || P.groups > P.B) sh.fail("groups", P.groups);
+    if (P.parts != P.groups * NS) sh.fail("partial vectors", P.parts);
     if ((long long)P.nthreads * KK + P.nthreads / 32 > P.smem_floats) sh.fail("sum-dy scratch", P.nthreads);
     if (P.nv != ncls * KK + 1) sh.fail("partial vector length", P.nv);
-    std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d, groups %d\n", P.smem_floats * 4, P.nthreads, TR,
-                P.n_all_tiles, P.groups);
+    std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d (<= %d per thread), groups %d, strips %d\n",
+                P.smem_floats * 4, P.nthreads, TR, P.n_all_tiles, P.tpt, P.groups, NS);
 }
 
 }  // namespace

@@ -67,7 +67,10 @@ def test_null_and_alignment(cuda_lib):
 
 
 def test_unsupported_plane(cuda_lib):
-    assert _fwd(cuda_lib, _desc(H=256, W=256, L=4)) == UNSUPPORTED
+    # Planes up to 256 x 256 are split into cluster strips; a 64-row strip of
+    # a 1024 x 1024 plane still does not fit on one SM.
+    assert _fwd(cuda_lib, _desc(H=1024, W=1024, L=4)) == UNSUPPORTED
+    assert _fwd(cuda_lib, _desc(H=256, W=256, L=4)) != UNSUPPORTED
 
 
 def test_backward_input_validation(cuda_lib):

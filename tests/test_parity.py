@@ -138,6 +138,15 @@ SMALL = [
     Case("plane64_L4", 1, 2, 64, 64, 5, 4, "f32", 22, "normal", "normal"),
     Case("bf16_stage1_plane", 3, 2, 56, 56, 5, 3, "bf16", 23, "uniform", "normal"),
     Case("bf16_rect", 5, 3, 20, 12, 5, 2, "bf16", 24, "normal", "normal"),
+    # Two tiles per thread in the weight gradient (more tiles than threads).
+    Case("plane64_L2_two_tiles", 2, 2, 64, 64, 5, 2, "f32", 25, "normal", "normal"),
+    # Planes split into row strips across a thread-block cluster (halo rows
+    # exchanged through distributed shared memory).
+    Case("strips_128_L4", 2, 2, 128, 128, 5, 4, "f32", 26, "normal", "normal"),
+    Case("strips_128_L1_k3", 1, 3, 128, 128, 3, 1, "f32", 27, "normal", "normal"),
+    Case("strips_256_L4", 1, 1, 256, 256, 5, 4, "f32", 28, "normal", "normal"),
+    Case("strips_256_L3_k3", 2, 1, 256, 256, 3, 3, "f32", 29, "normal", "normal"),
+    Case("strips_256_L2_bf16", 1, 2, 256, 256, 5, 2, "bf16", 30, "normal", "normal"),
 ]
 
 
@@ -167,8 +176,7 @@ SWEEP_PICK = [0, 7, 9, 14, 17, 31, 40, 63, 66, 95, 105, 127]
 @pytest.mark.parametrize("idx", SWEEP_PICK)
 def test_sweep_points_sampled(oracle, idx):
     case = sweep_cases()[idx]
-    if not _supported(case):
-        pytest.skip(f"{case.name}: plane not yet staged on chip by this build")
+    assert _supported(case), f"{case.name}: no on-chip plan"
     check_sampled(oracle, case, nplanes=4, nchannels=2)
 
 
