@@ -53,6 +53,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--compare", action="store_true",
+                    help="time the unfused PyTorch layer and the plain depthwise conv beside this library "
+                         "(context lines, not the bench line)")
+    ap.add_argument("--compare-only", default="", help="with --compare: only the implementation named so")
+    ap.add_argument("--profile-one-forward", action="store_true",
+                    help="with --compare: run one forward per implementation between profiler start/stop")
     return ap.parse_args()
 
 
@@ -469,6 +475,148 @@ def e2e(args, case, g, y, dx, grads, ws, dev, stream, world, calls):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K}
 
 
+# --------------------------------------------------------------------------
+# Comparators: the same layer as separate PyTorch library ops with every
+# intermediate in memory (the unfused formulation the pages measure the
+# fused one against), and the plain depthwise conv the layer extends.
+# Context numbers only, printed by --compare; never the product path.
+# --------------------------------------------------------------------------
+def haar_filters(C: int, dtype, device):
+    """The four orthonormal 2x2 Haar analysis filters (LL, LH, HL, HH) for
+    every channel, as grouped-conv weights [4C, 1, 2, 2]."""
+    import torch
+    f = torch.tensor([[[1, 1], [1, 1]], [[1, 1], [-1, -1]], [[1, -1], [1, -1]], [[1, -1], [-1, 1]]],
+                     dtype=dtype, device=device) * 0.5
+    return f.unsqueeze(1).repeat(C, 1, 1, 1)
+
+
+def unfused_wtconv(x, base_w, base_b, base_scale, wt_w, wt_scale, L: int):
+    """The layer level by level with PyTorch ops: Haar analysis as a stride-2
+    grouped conv, one grouped conv per level for the 4C subbands, scaling,
+    and the synthesis as a stride-2 grouped transposed conv adding each
+    coarser level into the next finer LL.  Differentiable."""
+    import torch
+    import torch.nn.functional as F
+    B, C, H, W = x.shape
+    k = base_w.shape[-1]
+    p = k // 2
+    dt = x.dtype
+    y = F.conv2d(x, base_w.to(dt).unsqueeze(1), base_b.to(dt), padding=p, groups=C)
+    y = y * base_scale.to(dt).view(1, C, 1, 1)
+    if L == 0:
+        return y
+    filt = haar_filters(C, dt, x.device)
+    ll, shat = x, []
+    for l in range(L):
+        s = F.conv2d(ll, filt, stride=2, groups=C)
+        h, w = s.shape[-2:]
+        z = F.conv2d(s, wt_w[l].to(dt).reshape(4 * C, 1, k, k), padding=p, groups=4 * C)
+        shat.append(z * wt_scale[l].to(dt).reshape(1, 4 * C, 1, 1))
+        ll = s.view(B, C, 4, h, w)[:, :, 0]
+    zc = None
+    for l in range(L - 1, -1, -1):
+        z = shat[l]
+        if zc is not None:
+            h, w = z.shape[-2:]
+            z4 = z.view(B, C, 4, h, w)
+            z = torch.cat([z4[:, :, :1] + zc.unsqueeze(2), z4[:, :, 1:]], dim=2).view(B, 4 * C, h, w)
+        zc = F.conv_transpose2d(z, filt, stride=2, groups=C)
+    return y + zc
+
+
+def depthwise_conv(x, base_w, base_b):
+    """The plain depthwise k x k conv (cuDNN through PyTorch)."""
+    import torch.nn.functional as F
+    C, k = x.shape[1], base_w.shape[-1]
+    return F.conv2d(x, base_w.to(x.dtype).unsqueeze(1), base_b.to(x.dtype), padding=k // 2, groups=C)
+
+
+def run_compare(args, case):
+    """Forward and forward+backward time and the peak memory of one training
+    step: the fused library (autograd function), the unfused PyTorch layer,
+    and the plain depthwise conv; one JSON line each."""
+    import torch
+
+    import memory_bound_cnn_wtconv_b200 as wt
+    from wtconv_inputs import make_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(case)
+    g = {k: v.to(dev) for k, v in inp.items()}
+    params = {k: g[k].clone().requires_grad_(True) for k in ("base_w", "base_b", "base_scale", "wt_w", "wt_scale")}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    impls = {
+        "fused (this library)": lambda x: wt.wtconv(x, params["base_w"], params["base_b"], params["base_scale"],
+                                                    params["wt_w"], params["wt_scale"], case.L),
+        "unfused PyTorch ops": lambda x: unfused_wtconv(x, params["base_w"], params["base_b"], params["base_scale"],
+                                                        params["wt_w"], params["wt_scale"], case.L),
+        "depthwise conv only (PyTorch)": lambda x: depthwise_conv(x, params["base_w"], params["base_b"]),
+    }
+
+    def timed(fn, reps):
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(ts)
+
+    if args.compare_only:
+        impls = {k: v for k, v in impls.items() if k.startswith(args.compare_only)}
+    for name, f in impls.items():
+        x = g["x"].clone().requires_grad_(True)
+        dy = g["dy"]
+        if args.profile_one_forward:
+            # For an ncu run with --profile-from-start off: warm up, then
+            # exactly one forward between profiler start and stop.
+            for _ in range(3):
+                f(x).backward(dy)
+            torch.cuda.synchronize()
+            flush.fill_(1)
+            torch.cuda.synchronize()
+            torch.cuda.profiler.start()
+            with torch.no_grad():
+                f(x)
+            torch.cuda.synchronize()
+            torch.cuda.profiler.stop()
+            continue
+
+        def fwd():
+            with torch.no_grad():
+                f(x)
+
+        def step():
+            y = f(x)
+            y.backward(dy)
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        t_f = timed(fwd, args.steps)
+        t_s = timed(step, args.steps)
+        x.grad = None
+        for v in params.values():
+            v.grad = None
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        step()
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        print(json.dumps({"impl": "compare", "what": name, "config": {"workload": workload_name(case)},
+                          "us_forward": t_f, "us_forward_backward": t_s, "peak_extra_bytes_train_step": peak,
+                          "dtype": case.dtype, "l2": "flushed before every timed call"}), flush=True)
+        x.grad = None
+        for v in params.values():
+            v.grad = None
+    return 0
+
+
 def main():
     args = parse()
     from wtconv_inputs import NAMED
@@ -479,6 +627,8 @@ def main():
         case = case.with_(calls=("fwd", "bwd_in", "bwd_w"))
     if args.impl == "reference":
         return run_reference(args, case)
+    if args.compare:
+        return run_compare(args, case)
     return run_ours(args, case)
 
 

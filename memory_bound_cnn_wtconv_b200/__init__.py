@@ -215,3 +215,9 @@ def backward_weight(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, g
         _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
         _stream(dev, stream)), "wtconv_backward_weight")
     return grads
+
+
+# Autograd function and module (defined after the calls they wrap).
+from .module import WTConv2d, WTConvFunction, wtconv  # noqa: E402
+
+__all__ += ["WTConv2d", "WTConvFunction", "wtconv"]
