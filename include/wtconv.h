@@ -87,8 +87,9 @@ typedef struct {
 /* Human-readable name of a status code (static string, never NULL). */
 const char *wtconv_status_string(wtconv_status_t s);
 
-/* Bytes of device workspace wtconv_backward_weight needs for `d` (0 if `d`
- * is invalid).  The forward and input-gradient calls need none. */
+/* Bytes of device workspace wtconv_backward_weight and wtconv_backward need
+ * for `d` (0 if `d` is invalid); one size serves both.  The forward and
+ * input-gradient calls need none. */
 size_t wtconv_workspace_bytes(const wtconv_desc_t *d);
 
 /* Forward pass: y = WTConv(x).  x, y: [B][C][H][W] in desc->dtype; x and y
@@ -125,6 +126,20 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, co
                                        void *workspace, size_t workspace_bytes,
                                        wtconv_stream_t stream);
 
+/* Fused backward: dx (as wtconv_backward_input) and every parameter gradient
+ * (as wtconv_backward_weight, bitwise-repeatable) in one pass that reads x
+ * and dy once and writes dx once -- the backward half of the training step
+ * the Abstract's speedup refers to.  dx: [B][C][H][W] in desc->dtype, not
+ * overlapping x or dy.  Workspace as for wtconv_backward_weight.  Planes too
+ * large for one SM (split into cluster strips) are done in the two separate
+ * passes instead, with the same results. */
+wtconv_status_t wtconv_backward(const wtconv_desc_t *d, const void *x, const void *dy,
+                                const float *base_w, const float *base_b, const float *base_scale,
+                                const float *wt_w, const float *wt_scale, void *dx,
+                                float *d_base_w, float *d_base_b, float *d_base_scale,
+                                float *d_wt_w, float *d_wt_scale,
+                                void *workspace, size_t workspace_bytes, wtconv_stream_t stream);
+
 /* The paper has no counterpart to this entry point.
  *
  * Same result as wtconv_backward_weight, for callers that cannot allocate
@@ -134,8 +149,8 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, co
  * library (4 MiB of device memory per GPU that loads the library, held until
  * the process exits) for the per-block partial sums; it calls no cudaMalloc,
  * cudaFree or other allocating routine.
- *   - Size limit: the partial sums (wtconv_workspace_bytes(d) bytes) must fit in
- *     2^20 floats; larger problems return WTCONV_ERR_WORKSPACE (use
+ *   - Size limit: its partial sums (at most wtconv_workspace_bytes(d) bytes)
+ *     must fit in 2^20 floats; larger problems return WTCONV_ERR_WORKSPACE (use
  *     wtconv_backward_weight).
  *   - The first call on each device looks up the array's device address with
  *     that device current; make that first call before any stream capture.

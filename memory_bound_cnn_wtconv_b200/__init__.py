@@ -21,7 +21,7 @@ import os
 import torch
 
 __all__ = [
-    "forward", "backward_input", "backward_weight", "workspace_bytes", "WTConvError",
+    "forward", "backward_input", "backward_weight", "backward", "workspace_bytes", "WTConvError",
     "WTConvLibraryMissing", "library_path", "load_library", "Desc", "STATUS",
 ]
 
@@ -77,6 +77,8 @@ def load_library():
     lib.wtconv_backward_input.restype = ctypes.c_int
     lib.wtconv_backward_weight.argtypes = [dp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, vp, sz, vp]
     lib.wtconv_backward_weight.restype = ctypes.c_int
+    lib.wtconv_backward.argtypes = [dp, vp, vp, fp, fp, fp, fp, fp, vp, fp, fp, fp, fp, fp, vp, sz, vp]
+    lib.wtconv_backward.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -215,6 +217,41 @@ def backward_weight(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, g
         _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
         _stream(dev, stream)), "wtconv_backward_weight")
     return grads
+
+
+def backward(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, dx=None, grads=None, workspace=None,
+             stream=None):
+    """dx and the parameter gradients in one pass via ``wtconv_backward``.
+
+    Returns (dx, grads) with grads as for ``backward_weight``.
+    """
+    lib = load_library()
+    _act(x, "x")
+    _act(dy, "dy")
+    if dy.shape != x.shape or dy.dtype != x.dtype or dy.device != x.device:
+        raise ValueError("x and dy must have the same shape, dtype and device")
+    k = _params(x, base_w, base_b, base_scale, wt_w, wt_scale, L)
+    B, C, H, W = x.shape
+    dev = x.device
+    if dx is None:
+        dx = torch.empty_like(dy)
+    _act(dx, "dx")
+    if grads is None:
+        grads = dict(base_w=torch.empty((C, k, k), device=dev), base_b=torch.empty((C,), device=dev),
+                     base_scale=torch.empty((C,), device=dev),
+                     wt_w=torch.empty((L, C, 4, k, k), device=dev), wt_scale=torch.empty((L, C, 4), device=dev))
+    d = make_desc(x, k, L)
+    nbytes = int(lib.wtconv_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=dev)
+    _check(lib.wtconv_backward(
+        ctypes.byref(d), _ptr(x), _ptr(dy), _ptr(base_w), _ptr(base_b), _ptr(base_scale),
+        _ptr(wt_w if L > 0 else None), _ptr(wt_scale if L > 0 else None), _ptr(dx),
+        _ptr(grads["base_w"]), _ptr(grads["base_b"]), _ptr(grads["base_scale"]),
+        _ptr(grads["wt_w"] if L > 0 else None), _ptr(grads["wt_scale"] if L > 0 else None),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        _stream(dev, stream)), "wtconv_backward")
+    return dx, grads
 
 
 # Autograd function and module (defined after the calls they wrap).

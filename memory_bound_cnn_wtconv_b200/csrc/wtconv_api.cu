@@ -36,7 +36,26 @@ cudaError_t launch_bwdw(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_
     }
 }
 
+cudaError_t launch_bwd(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s) {
+    switch (P.k) {
+        case 1: return launch_bwd_k1(P, dtype, a, s);
+        case 3: return launch_bwd_k3(P, dtype, a, s);
+        case 5: return launch_bwd_k5(P, dtype, a, s);
+        case 7: return launch_bwd_k7(P, dtype, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 size_t workspace_floats(const Plan& P) { return (size_t)P.C * P.parts * P.nv; }
+
+// Workspace both weight-gradient paths accept: the larger of the two plans'.
+size_t workspace_floats_any(const wtconv_desc_t* d) {
+    Plan P;
+    size_t n = 0;
+    if (make_plan(d, kBackwardWeight, &P) == WTCONV_OK) n = workspace_floats(P);
+    if (make_plan(d, kBackward, &P) == WTCONV_OK) n = std::max(n, workspace_floats(P));
+    return n;
+}
 
 }  // namespace
 
@@ -141,9 +160,7 @@ const char* wtconv_status_string(wtconv_status_t s) {
 
 size_t wtconv_workspace_bytes(const wtconv_desc_t* d) {
     if (validate(d) != WTCONV_OK) return 0;
-    Plan P;
-    if (make_plan(d, kBackwardWeight, &P) != WTCONV_OK) return 0;
-    return workspace_floats(P) * sizeof(float);
+    return workspace_floats_any(d) * sizeof(float);
 }
 
 wtconv_status_t wtconv_forward(const wtconv_desc_t* d, const void* x, const float* base_w, const float* base_b,
@@ -194,12 +211,45 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t* d, const void* x, co
     Plan P;
     st = make_plan(d, kBackwardWeight, &P);
     if (st != WTCONV_OK) return st;
-    if (!workspace || workspace_bytes < workspace_floats(P) * sizeof(float)) return WTCONV_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < workspace_floats_any(d) * sizeof(float)) return WTCONV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
     float* part = static_cast<float*>(workspace);
     BwdwArgs a{x, dy, part};
     cudaStream_t s = (cudaStream_t)stream;
     if (launch_bwdw(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    if (launch_bwdw_finish(P, part, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                           d_wt_w, d_wt_scale, s) != cudaSuccess)
+        return WTCONV_ERR_CUDA;
+    return WTCONV_OK;
+}
+
+wtconv_status_t wtconv_backward(const wtconv_desc_t* d, const void* x, const void* dy, const float* base_w,
+                                const float* base_b, const float* base_scale, const float* wt_w,
+                                const float* wt_scale, void* dx, float* d_base_w, float* d_base_b,
+                                float* d_base_scale, float* d_wt_w, float* d_wt_scale, void* workspace,
+                                size_t workspace_bytes, wtconv_stream_t stream) {
+    wtconv_status_t st = validate(d);
+    if (st != WTCONV_OK) return st;
+    if (!x || !dy || !dx || !base_w || !base_b || !base_scale || !d_base_w || !d_base_b || !d_base_scale)
+        return WTCONV_ERR_NULLPTR;
+    if (d->L > 0 && (!wt_w || !wt_scale || !d_wt_w || !d_wt_scale)) return WTCONV_ERR_NULLPTR;
+    if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_MISALIGNED;
+    Plan P;
+    st = make_plan(d, kBackward, &P);
+    if (st == WTCONV_ERR_UNSUPPORTED) {
+        // No one-pass plan (planes split into strips): the two passes.
+        st = wtconv_backward_input(d, dy, base_w, base_scale, wt_w, wt_scale, dx, stream);
+        if (st != WTCONV_OK) return st;
+        return wtconv_backward_weight(d, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b,
+                                      d_base_scale, d_wt_w, d_wt_scale, workspace, workspace_bytes, stream);
+    }
+    if (st != WTCONV_OK) return st;
+    if (!workspace || workspace_bytes < workspace_floats_any(d) * sizeof(float)) return WTCONV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
+    float* part = static_cast<float*>(workspace);
+    cudaStream_t s = (cudaStream_t)stream;
+    BwdArgs a{x, dy, base_w, base_b, base_scale, wt_w, wt_scale, dx, part};
+    if (launch_bwd(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
     if (launch_bwdw_finish(P, part, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
                            d_wt_w, d_wt_scale, s) != cudaSuccess)
         return WTCONV_ERR_CUDA;

@@ -28,6 +28,8 @@
 
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -315,12 +317,6 @@ struct WinRow {
         }
         if constexpr (NW2 % 2 == 1) e[NW2 - 1] = *reinterpret_cast<const float2*>(rp + 2 * (NW2 - 1));
     }
-    // 64-bit loads only: looser register allocation (no 4-register groups)
-    // for the register-heavy correlation tiles.
-    __device__ __forceinline__ void load_pairs(const float* rp) {
-#pragma unroll
-        for (int k = 0; k < NW2; ++k) e[k] = *reinterpret_cast<const float2*>(rp + 2 * k);
-    }
 };
 
 // acc (output columns 2jp, 2jp+1) += w * input columns (2jp+v, 2jp+v+1).
@@ -377,7 +373,10 @@ __device__ __forceinline__ void conv_tile(const float* __restrict__ win, int str
 // column parity (sum the two halves at the end):
 //   acc[u*K+v] += sum_{o<TR, j<TC} D[o][j] * S[o+u][j+v]
 // `swin` is the S window origin (element (r0-p, c0-p)), `dt` the D tile origin.
-template <int K, int TR, int TC>
+// D rows load as 128-bit (DLD = 4) or 64-bit pairs (2; the faster of the two
+// was measured per activation type), or as single floats (1) where the tile
+// sits at an odd float offset (the interior of a padded buffer, p odd).
+template <int K, int TR, int TC, int DLD>
 __device__ __forceinline__ void corr_tile(const float* __restrict__ swin, int sstride,
                                           const float* __restrict__ dt, int dstride, float2 (&acc)[K * K]) {
     constexpr int NP = TC / 2;
@@ -386,11 +385,24 @@ __device__ __forceinline__ void corr_tile(const float* __restrict__ swin, int ss
 #pragma unroll
     for (int r = 0; r < TR + K - 1; ++r) {
         if (r < TR) {
+            if constexpr (DLD == 1) {
 #pragma unroll
-            for (int q = 0; q < NP; ++q) d[r][q] = *reinterpret_cast<const float2*>(dt + r * dstride + 2 * q);
+                for (int q = 0; q < NP; ++q)
+                    d[r][q] = make_float2(dt[r * dstride + 2 * q], dt[r * dstride + 2 * q + 1]);
+            } else if constexpr (DLD == 4) {
+#pragma unroll
+                for (int q = 0; q < NP / 2; ++q) {
+                    const float4 v = *reinterpret_cast<const float4*>(dt + r * dstride + 4 * q);
+                    d[r][2 * q] = make_float2(v.x, v.y);
+                    d[r][2 * q + 1] = make_float2(v.z, v.w);
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < NP; ++q) d[r][q] = *reinterpret_cast<const float2*>(dt + r * dstride + 2 * q);
+            }
         }
         WinRow<NW2> row;
-        row.load_pairs(swin + r * sstride);
+        row.load(swin + r * sstride);
 #pragma unroll
         for (int u = 0; u < K; ++u) {
             const int o = r - u;
@@ -434,14 +446,16 @@ __device__ __forceinline__ float quarter_pow(int l) {
 // those buffers).  `sync()` synchronises the np threads between the levels
 // that run one at a time (levels >= 4, or every level without the pyramid).
 // ---------------------------------------------------------------------------
-template <typename T, int PD, bool SUM, bool TO_Q, class Sync>
+enum : int { kToS = 0, kToQ = 1, kToSS = 2 };
+
+template <typename T, int PD, bool SUM, int DST, class Sync>
 __device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const float* stg, float* dst, int ds, int pad,
                                                int np, int ptid, Sync&& sync) {
     const int H = P.H, W = P.W, L = P.L;
-    // Level l's subbands go to P.Q[l] (TO_Q) or P.S[l]; every index below is
-    // a compile-time constant or goes through the parameter directly, so no
-    // copy of the kernel parameter is made.
-    auto buf = [&](int l) -> const Buf& { return TO_Q ? P.Q[l] : P.S[l]; };
+    // Level l's subbands go to P.S[l], P.Q[l] or P.SS[l] (DST); every index
+    // below is a compile-time constant or goes through the parameter
+    // directly, so no copy of the kernel parameter is made.
+    auto buf = [&](int l) -> const Buf& { return DST == kToQ ? P.Q[l] : (DST == kToSS ? P.SS[l] : P.S[l]); };
     float sum;
     int done;  // levels complete
     if (P.pyr) {
@@ -741,7 +755,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
                 cx.fold(cur_c, nt, tid);
                 folded_c = cur_c;
             }
-            analyse_plane<T, p, false, false>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
+            analyse_plane<T, p, false, kToS>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         }
         if (u > u0 && P.L >= 1) {
             T* yp = y + cx.rows_of(prev_b, prev_c);
@@ -806,6 +820,7 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
     constexpr int p = K / 2, KK = K * K;
+    constexpr int DLD = sizeof(T) == 2 ? 4 : 2;
     const int tid = threadIdx.x, nt = blockDim.x;
     // blockIdx.x = c * nstrips + (strip rank within the cluster).
     const int rank = STRIPS ? (int)cg::this_cluster().block_rank() : 0;
@@ -841,8 +856,8 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
     for (int b = g; b < P.B; b += G) {
         cp_async_wait_all();
         plane_sync<STRIPS>();  // staged pair complete; previous correlations (and halo copies) done
-        analyse_plane<T, p, false, false>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
-        const float s = analyse_plane<T, 0, true, true>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
+        analyse_plane<T, p, false, kToS>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
+        const float s = analyse_plane<T, 0, true, kToQ>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
                                                         P.DY.stride, 0, nt, tid, csync);
         {
             const float yv = s - sdy_c;
@@ -865,13 +880,13 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
             const int local = first + k;
             const int tr = fdiv(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
             if (cl == 0) {
-                corr_tile<K, TR, TC>(sm + P.X.base + tr * TR * P.X.stride + tc * TC, P.X.stride,
+                corr_tile<K, TR, TC, DLD>(sm + P.X.base + tr * TR * P.X.stride + tc * TC, P.X.stride,
                                      sm + P.DY.base + tr * TR * P.DY.stride + tc * TC, P.DY.stride, acc);
             } else {
                 const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
                 const Buf& S = P.S[l];
                 const Buf& Q = P.Q[l];
-                corr_tile<K, TR, TC>(sm + S.base + s2 * S.sub + tr * TR * S.stride + tc * TC, S.stride,
+                corr_tile<K, TR, TC, DLD>(sm + S.base + s2 * S.sub + tr * TR * S.stride + tc * TC, S.stride,
                                      sm + Q.base + s2 * Q.sub + tr * TR * Q.stride + tc * TC, Q.stride, acc);
             }
         }
@@ -900,6 +915,184 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
     if (tid == 0) {
         float s = 0.f;
         for (int w = 0; w < (nt >> 5); ++w) s += red[nt * KK + w];
+        out[ncls * KK] = s;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fused backward: dx and the weight-gradient partials in one pass over x and
+// dy (each read once; dx written once).  Grid (C, groups) of one CTA per SM;
+// the CTA of (c, g) walks the planes b = g, g + groups, ... of channel c.
+// Per plane, phase A: threads [0, an_split) analyse x into XS / SS, the rest
+// analyse dy into X / S (and sum it), then every thread takes synthesis items
+// of the previous plane's dx; phase B: stage the next (x, dy) pair, threads
+// [0, corr0) run one dx conv tile each (the input-gradient pass: dy with
+// every kernel rotated by 180 degrees, no bias) and threads [corr0, ...) run
+// their runs of correlation tiles (x windows against dy tiles) into
+// registers.  After the walk: the last plane's synthesis, then the
+// fixed-order reduction of the correlation sums into one partial vector.
+// ---------------------------------------------------------------------------
+template <int K, int TR, int TC, typename T>
+__global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
+    const T* __restrict__ x, const T* __restrict__ dy, const float* __restrict__ base_w,
+    const float* __restrict__ base_b, const float* __restrict__ base_scale, const float* __restrict__ wt_w,
+    const float* __restrict__ wt_scale, T* __restrict__ dx, float* __restrict__ part, const Plan P) {
+    extern __shared__ float4 smem4[];
+    float* sm = reinterpret_cast<float*>(smem4);
+    constexpr int p = K / 2, KK = K * K, NP = TC / 2;
+    constexpr int DLD = (p % 2 == 0) ? 2 : 1;  // dy tiles sit at the interior of padded buffers
+    static_assert(TC == 4, "4-column tiles");
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int c = blockIdx.x, g = blockIdx.y, G = P.groups;
+    const size_t plane_elems = (size_t)P.H * P.W;
+    auto csync = [&]() { __syncthreads(); };
+    FusedCtx<K, T, true> cx{sm, P, dy, base_w, base_b, base_scale, wt_w, wt_scale, 0, 0, 0, plane_elems, 0};
+
+    zero_smem(sm, P.smem_floats, tid, nt);
+    __syncthreads();
+    cx.fold(c, nt, tid);  // the channel is fixed: dx weights folded once
+    if (g < P.B) {
+        const size_t off = ((size_t)g * P.C + c) * plane_elems;
+        stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
+        stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
+    }
+    cp_async_commit();
+
+    const bool x_side = tid < P.an_split;
+    float* XS0 = sm + P.XS.base + p * P.XS.stride + p;
+    float* X0 = sm + P.X.base + p * P.X.stride + p;
+    const int ct = tid - P.corr0;
+    const int ncorr = P.cls_thr[1 + 4 * P.L];
+    float sdy = 0.f, sdy_c = 0.f;  // compensated running sum of dy over the walk (dy-side threads)
+    float* red = sm + P.red;
+
+    // The plane walk, instantiated once per role (whole warps): CORR = false
+    // runs this thread's dx conv tile, CORR = true its correlation tiles.
+    // Both instantiations meet the same CTA barriers in the same order, and
+    // only the correlation one keeps the K*K accumulators.
+    auto walk = [&](auto corr_tag) {
+        constexpr bool CORR = decltype(corr_tag)::value;
+        TileJob job = TileJob{0, 0, 0, 0, 0, 0, false, false};
+        int cl = -1, first = 0, cnt = 0;
+        if constexpr (!CORR) {
+            job = decode_tile(P, tid, TR, TC);
+        } else if (ct < ncorr) {
+            cl = 0;
+            while (ct >= P.cls_thr[cl + 1]) ++cl;
+            first = (ct - P.cls_thr[cl]) * P.tpt;
+            cnt = min(P.tpt, P.cls_tiles[cl] - first);
+        }
+        const int lvl = cl <= 0 ? kMaxL : ((cl - 1) >> 2);
+        float2 acc[CORR ? KK : 1];
+#pragma unroll
+        for (int t = 0; t < (CORR ? KK : 1); ++t) acc[t] = make_float2(0.f, 0.f);
+
+        int prev_b = -1;
+        for (int b = g;; b += G) {
+            const bool have = b < P.B;
+            cp_async_wait_all();
+            __syncthreads();  // staged pair complete; every tile of the previous plane done
+            // Phase A.
+            if (have) {
+                if (x_side) {
+                    analyse_plane<T, p, false, kToSS>(sm, P, sm + P.stg, XS0, P.XS.stride, p, P.an_split, tid, csync);
+                } else {
+                    const float sv = analyse_plane<T, p, true, kToS>(sm, P, sm + P.stg + P.stg_floats, X0, P.X.stride,
+                                                                     p, nt - P.an_split, tid - P.an_split, csync);
+                    const float yv = sv - sdy_c;
+                    const float tv = sdy + yv;
+                    sdy_c = (tv - sdy) - yv;
+                    sdy = tv;
+                }
+            }
+            if (prev_b >= 0 && P.L >= 1) {
+                T* yp = dx + ((size_t)prev_b * P.C + c) * plane_elems;
+                for (int t = tid; t < P.n_fin; t += nt) synth_item<T>(sm, P, yp, t);
+            }
+            if (!have) break;
+            __syncthreads();  // both analyses complete; the previous plane's Q and Y consumed
+            // Phase B.
+            if (b + G < P.B) {
+                const size_t off = ((size_t)(b + G) * P.C + c) * plane_elems;
+                stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
+                stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
+            }
+            cp_async_commit();
+            if constexpr (!CORR) {
+                if (job.valid) {
+                    float w[KK];
+                    load_weights<K>(sm + job.wts, w);
+                    if (P.L >= 1 || !job.base) {
+                        float* out = sm + job.out;
+                        const int os = job.ostride;
+                        conv_tile<K, TR, TC>(sm + job.win, job.wstride, w, make_float2(0.f, 0.f),
+                                             [&](int o, float2(&a)[NP]) {
+                                                 *reinterpret_cast<float4*>(out + o * os) =
+                                                     make_float4(a[0].x, a[0].y, a[1].x, a[1].y);
+                                             });
+                    } else {
+                        T* yo = dx + ((size_t)b * P.C + c) * plane_elems + job.out;
+                        const int h0 = job.row0;
+                        conv_tile<K, TR, TC>(sm + job.win, job.wstride, w, make_float2(0.f, 0.f),
+                                             [&](int o, float2(&a)[NP]) {
+                                                 if (h0 + o < P.H)
+                                                     gst4<T>(yo + (size_t)o * P.W,
+                                                             make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
+                                             });
+                    }
+                }
+            } else {
+                for (int k = 0; k < cnt; ++k) {
+                    const int local = first + k;
+                    const int tr = fdiv(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
+                    if (cl == 0) {
+                        corr_tile<K, TR, TC, DLD>(sm + P.XS.base + tr * TR * P.XS.stride + tc * TC, P.XS.stride,
+                                                  X0 + tr * TR * P.X.stride + tc * TC, P.X.stride, acc);
+                    } else {
+                        const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
+                        const Buf& SS = P.SS[l];
+                        const Buf& S = P.S[l];
+                        corr_tile<K, TR, TC, DLD>(sm + SS.base + s2 * SS.sub + tr * TR * SS.stride + tc * TC,
+                                                  SS.stride,
+                                                  sm + S.base + s2 * S.sub + (tr * TR + p) * S.stride + tc * TC + p,
+                                                  S.stride, acc);
+                    }
+                }
+            }
+            prev_b = b;
+        }
+        cp_async_wait_all();
+        __syncthreads();  // the last synthesis done: the buffers are free
+        if constexpr (CORR) {
+            if (ct < ncorr) {
+#pragma unroll
+                for (int t = 0; t < KK; ++t) red[ct * KK + t] = acc[t].x + acc[t].y;
+            }
+        }
+    };
+    if (tid < P.corr0) {
+        walk(std::false_type{});
+    } else {
+        walk(std::true_type{});
+    }
+
+    // Fixed-order reduction of every class over its correlation threads.
+    float sw = sdy;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
+    if ((tid & 31) == 0) red[ncorr * KK + (tid >> 5)] = sw;
+    __syncthreads();
+    float* out = part + ((size_t)c * P.parts + g) * P.nv;
+    const int ncls = 1 + 4 * P.L;
+    for (int t = tid; t < ncls * KK; t += nt) {
+        const int k2 = t / KK, tap = t - k2 * KK;
+        float s = 0.f;
+        for (int th = P.cls_thr[k2]; th < P.cls_thr[k2 + 1]; ++th) s += red[th * KK + tap];
+        out[t] = s;
+    }
+    if (tid == 0) {
+        float s = 0.f;
+        for (int w = 0; w < (nt >> 5); ++w) s += red[ncorr * KK + w];
         out[ncls * KK] = s;
     }
 }

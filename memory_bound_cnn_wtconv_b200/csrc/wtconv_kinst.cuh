@@ -115,6 +115,18 @@ cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s)
     return bwd ? fused_typed<TR, T, true, false>(P, a, s) : fused_typed<TR, T, false, false>(P, a, s);
 }
 
+template <int TR, typename T>
+cudaError_t bwd_typed(const Plan& P, const BwdArgs& a, cudaStream_t s) {
+    static bool done[kMaxDevices] = {};
+    auto* fn = wtconv_backward_kernel<WTC_K, TR, 4, T>;
+    cudaError_t e = opt_in_smem(fn, done);
+    if (e != cudaSuccess) return e;
+    fn<<<dim3(P.C, P.groups), P.nthreads, (size_t)P.smem_floats * 4, s>>>(
+        static_cast<const T*>(a.x), static_cast<const T*>(a.dy), a.base_w, a.base_b, a.base_scale, a.wt_w,
+        a.wt_scale, static_cast<T*>(a.dx), a.part, P);
+    return cudaGetLastError();
+}
+
 template <int TR>
 cudaError_t fused_tr(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cudaStream_t s) {
     if (dtype == 0) return fused_t<TR, float>(P, bwd, a, s);
@@ -135,6 +147,14 @@ cudaError_t WTC_CAT(launch_fused_k, WTC_K)(const Plan& P, int dtype, bool bwd, c
     switch (P.TR) {
         case 7: return fused_tr<7>(P, dtype, bwd, a, s);
         case 8: return fused_tr<8>(P, dtype, bwd, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t WTC_CAT(launch_bwd_k, WTC_K)(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s) {
+    switch (P.TR) {
+        case 7: return dtype == 0 ? bwd_typed<7, float>(P, a, s) : bwd_typed<7, __nv_bfloat16>(P, a, s);
+        case 8: return dtype == 0 ? bwd_typed<8, float>(P, a, s) : bwd_typed<8, __nv_bfloat16>(P, a, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -20,9 +20,18 @@ struct BwdwArgs {
     float* part;
 };
 
+struct BwdArgs {
+    const void* x;
+    const void* dy;
+    const float *base_w, *base_b, *base_scale, *wt_w, *wt_scale;
+    void* dx;
+    float* part;
+};
+
 #define WTC_DECLARE_LAUNCHERS(KV)                                                                     \
     cudaError_t launch_fused_k##KV(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cudaStream_t s); \
-    cudaError_t launch_bwdw_k##KV(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s);
+    cudaError_t launch_bwdw_k##KV(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s);           \
+    cudaError_t launch_bwd_k##KV(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s);
 
 WTC_DECLARE_LAUNCHERS(1)
 WTC_DECLARE_LAUNCHERS(3)

@@ -69,9 +69,9 @@ extern "C" wtconv_status_t wtconv_backward_weight_noalloc(
     Plan P;
     st = make_plan(d, kBackwardWeight, &P);
     if (st != WTCONV_OK) return st;
-    // The partials need C * parts * nv floats (wtconv_workspace_bytes / 4);
-    // beyond the fixed array the call is rejected (use wtconv_backward_weight
-    // with a workspace instead).
+    // The partials of this plan need C * parts * nv floats; beyond the fixed
+    // array the call is rejected (use wtconv_backward_weight with a workspace
+    // instead).
     if ((size_t)P.C * P.parts * P.nv > kNoAllocScratchFloats) return WTCONV_ERR_WORKSPACE;
     cudaError_t err = cudaSuccess;
     float* part = scratch_address(&err);

@@ -16,6 +16,10 @@
 //   Y      forward (L >= 1): base-branch outputs (tile-rounded), kept until
 //          the synthesis adds the wavelet terms and stores the plane.
 //   DY     weight gradient: dy plane (tile-rounded).
+//   XS, SS[l]  fused backward: padded x plane and padded x subbands (the
+//          correlation windows); there X and S hold the padded dy plane and
+//          dy subbands (the dx conv windows, and the correlation's dy tiles
+//          at their interior), Q and Y the dx conv outputs.
 //   W      forward: folded weights, one class (K*K floats) per subband and the base.
 //
 // Padded buffers: `base` is the offset of padded element (-p, -p), so a
@@ -57,6 +61,7 @@ inline FastDiv make_fastdiv(uint32_t d) {
 // Thread budgets (also the kernels' __launch_bounds__, two CTAs per SM).
 constexpr int kFusedMaxThreads = 256;
 constexpr int kBwdwMaxThreads = 256;
+constexpr int kBwdMaxThreads = 512;  // fused backward: one CTA per SM
 
 struct Buf {
     int base;    // float offset (see above)
@@ -84,8 +89,8 @@ struct Plan {
     int stg;             // staging buffer offset; one stored plane occupies stg_floats floats
     int stg_floats;
     int plane_chunks;    // 16-byte chunks per stored plane
-    Buf X, Y, DY;
-    Buf S[kMaxL], Q[kMaxL];
+    Buf X, Y, DY, XS;
+    Buf S[kMaxL], Q[kMaxL], SS[kMaxL];
     int ntr[kMaxL + 1], ntc[kMaxL + 1];  // tile grid per level; index kMaxL = full resolution
     // Tile enumeration.  Forward: subband tiles in class order (l, s) first,
     // counted by sub_begin; base tiles separately.  Weight gradient: class cl
@@ -108,6 +113,11 @@ struct Plan {
     // thread t takes items (t - fin_off) mod nthreads + k * nthreads, so the
     // threads that the analysis leaves idle start first.
     int n_fin, fin_off;
+    // Fused backward: threads [0, corr0) run the dx conv tiles (one each),
+    // threads [corr0, corr0 + cls_thr[ncls]) the correlation tiles (class
+    // runs as in the weight gradient); in the analysis threads [0, an_split)
+    // take x and the rest take dy.
+    int corr0, an_split;
     int pyr;             // analysis by the one-pass pyramid (H % 4 == 0 and L >= 1)
     int pyr_levels;      // levels the pyramid computes (min(L, 4)); the rest run level by level
     int pyr_lg;          // pyramid lane groups cover (4 * 2^pyr_lg)^2 pixel regions

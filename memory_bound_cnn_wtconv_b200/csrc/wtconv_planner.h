@@ -17,7 +17,9 @@ constexpr int kSmemLimitFloats = 227 * 1024 / 4;
 constexpr int kSmemPerSM = 228 * 1024;
 constexpr int kNumSMs = 148;  // B200; sizes the persistent grids
 
-enum Kind { kForward = 0, kBackwardInput = 1, kBackwardWeight = 2 };
+// kBackward: the fused backward (dx and the weight-gradient partials in one
+// pass over x and dy).
+enum Kind { kForward = 0, kBackwardInput = 1, kBackwardWeight = 2, kBackward = 3 };
 
 inline int round4(int v) { return (v + 3) & ~3; }
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -77,6 +79,24 @@ inline int pick_groups(int B, int C, int smem_floats) {
     return best;
 }
 
+// Batch groups for the fused backward (one 512-thread CTA per SM).
+inline int pick_groups_one(int B, int C) {
+    const long long slots = kNumSMs;
+    int best = 1;
+    long long best_cost = -1;
+    for (int g = 1; g <= B; ++g) {
+        const int planes = ceil_div(B, g);
+        if (planes > 64 && g != B) continue;
+        const long long waves = (C * (long long)g + slots - 1) / slots;
+        const long long cost = waves * (planes + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = g;
+        }
+    }
+    return best;
+}
+
 inline bool is_supported_k(int k) { return k == 1 || k == 3 || k == 5 || k == 7; }
 
 inline wtconv_status_t validate(const wtconv_desc_t* d) {
@@ -105,6 +125,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, Plan* P) {
     memset(P, 0, sizeof(*P));
     if (nstrips < 1 || nstrips > kMaxStrips || d->H % nstrips) return WTCONV_ERR_UNSUPPORTED;
+    if (kind == kBackward && nstrips != 1) return WTCONV_ERR_UNSUPPORTED;  // whole planes only
     const int Hs = d->H / nstrips;
     if (nstrips > 1 && (Hs % (1 << d->L) != 0 || Hs % 4 != 0)) return WTCONV_ERR_UNSUPPORTED;
     P->B = d->B; P->C = d->C; P->H = Hs; P->W = d->W; P->k = d->k; P->L = d->L;
@@ -134,26 +155,30 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         P->bias = (int)off;
         off += 4;
     }
-    // Padded input plane.
-    {
-        const int ntc = P->ntc[kMaxL];
-        const int rows = P->ntr[kMaxL] * TR + 2 * p;
-        const int need = std::max(W + 2 * p, (ntc - 1) * TC + WV4);
-        P->X.stride = pick_stride(need, TR, ntc);
-        P->X.base = (int)off;
-        off += round4(rows * P->X.stride);
-    }
-    // Padded subbands of every level.
-    for (int l = 0; l < L; ++l) {
-        const int m = W >> (l + 1);
-        const int ntc = P->ntc[l];
-        const int rows = P->ntr[l] * TR + 2 * p;
-        const int need = std::max(m + 2 * p, (ntc - 1) * TC + WV4);
-        P->S[l].stride = pick_stride(need, TR, ntc);
-        P->S[l].sub = round4(rows * P->S[l].stride);
-        P->S[l].base = (int)off;
-        off += 4LL * P->S[l].sub;
-    }
+    // Padded input plane and padded subbands of every level (the fused
+    // backward holds two sets: dy in X / S, x in XS / SS).
+    auto padded = [&](Buf& X, Buf* S) {
+        {
+            const int ntc = P->ntc[kMaxL];
+            const int rows = P->ntr[kMaxL] * TR + 2 * p;
+            const int need = std::max(W + 2 * p, (ntc - 1) * TC + WV4);
+            X.stride = pick_stride(need, TR, ntc);
+            X.base = (int)off;
+            off += round4(rows * X.stride);
+        }
+        for (int l = 0; l < L; ++l) {
+            const int m = W >> (l + 1);
+            const int ntc = P->ntc[l];
+            const int rows = P->ntr[l] * TR + 2 * p;
+            const int need = std::max(m + 2 * p, (ntc - 1) * TC + WV4);
+            S[l].stride = pick_stride(need, TR, ntc);
+            S[l].sub = round4(rows * S[l].stride);
+            S[l].base = (int)off;
+            off += 4LL * S[l].sub;
+        }
+    };
+    padded(P->X, P->S);
+    if (kind == kBackward) padded(P->XS, P->SS);
     // Tile-rounded, unpadded planes: conv outputs (forward) or dy subbands.
     for (int l = 0; l < L; ++l) {
         const int rows = P->ntr[l] * TR;
@@ -181,7 +206,7 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         P->plane_chunks = (int)(bytes / 16);
         P->stg_floats = (int)(bytes / 4);
         P->stg = (int)off;
-        off += (kind == kBackwardWeight ? 2LL : 1LL) * P->stg_floats;
+        off += (kind == kBackwardWeight || kind == kBackward ? 2LL : 1LL) * P->stg_floats;
     }
 
     // Tiles and threads.
@@ -211,7 +236,33 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     for (int l = 0; l < L; ++l) P->div_m[l] = make_fastdiv(W >> (l + 1));
     for (int l = 0; l <= kMaxL; ++l) P->div_ntc[l] = make_fastdiv(std::max(P->ntc[l], 1));
 
-    if (kind == kBackwardWeight) {
+    if (kind == kBackward) {
+        // dx conv tiles one per thread (warps [0, corr0/32)); the correlation
+        // tiles in class runs on the remaining threads.
+        P->base_tid0 = P->n_sub_tiles;
+        P->tile_end = P->base_tid0 + P->n_base_tiles;
+        P->corr0 = ceil_div(P->tile_end, 32) * 32;
+        const int budget = kBwdMaxThreads - P->corr0;
+        if (budget < 32 * ncls / 32 || budget < 32) return WTCONV_ERR_UNSUPPORTED;
+        int tpt = 1, used = 0;
+        for (;; ++tpt) {
+            used = 0;
+            for (int cl = 0; cl < ncls; ++cl) used += ceil_div(P->cls_tiles[cl], tpt);
+            if (used <= budget) break;
+        }
+        P->tpt = tpt;
+        P->cls_thr[0] = 0;
+        for (int cl = 0; cl < ncls; ++cl) P->cls_thr[cl + 1] = P->cls_thr[cl] + ceil_div(P->cls_tiles[cl], tpt);
+        P->nthreads = std::max(64, ceil_div(P->corr0 + used, 32) * 32);
+        P->merged = 1;
+        P->an_split = ceil_div(P->nthreads / 2, 32) * 32;
+        P->n_fin = L >= 1 ? (H / 2) * (W / 4) : 0;
+        P->fin_off = 0;
+        // Reduction scratch (correlation threads' sums, then one sum of dy
+        // per warp) aliases the buffers from offset 0 after the walk.
+        P->red = 0;
+        off = std::max(off, (long long)used * KK + P->nthreads / 32);
+    } else if (kind == kBackwardWeight) {
         // The fewest tiles per thread whose class-pure thread ranges fit.
         int tpt = 1, used = 0;
         for (;; ++tpt) {
@@ -248,8 +299,8 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     off = round4((int)std::min<long long>(off, 1LL << 30));
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;
-    if (kind == kBackwardWeight) {
-        P->groups = pick_groups(P->B, P->C * nstrips, P->smem_floats);
+    if (kind == kBackwardWeight || kind == kBackward) {
+        P->groups = kind == kBackward ? pick_groups_one(P->B, P->C) : pick_groups(P->B, P->C * nstrips, P->smem_floats);
         P->parts = P->groups * nstrips;
     } else {
         const long long units = (long long)P->B * P->C;
@@ -264,8 +315,13 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
 // tile height), times the CTAs of a plane, over the CTAs an SM holds.
 // Cluster strips carry a halo exchange on top (weighted 15%).
 inline double plan_cost(const Plan& P, Kind kind) {
-    const int per_smsp = kind == kBackwardWeight ? P.tpt * ceil_div(ceil_div(P.cls_thr[1 + 4 * P.L], 32), 4)
-                                                 : ceil_div(ceil_div(P.tile_end, 32), 4);
+    int per_smsp;
+    if (kind == kBackward)
+        per_smsp = ceil_div(ceil_div(P.tile_end, 32) + P.tpt * ceil_div(P.cls_thr[1 + 4 * P.L], 32), 4);
+    else if (kind == kBackwardWeight)
+        per_smsp = P.tpt * ceil_div(ceil_div(P.cls_thr[1 + 4 * P.L], 32), 4);
+    else
+        per_smsp = ceil_div(ceil_div(P.tile_end, 32), 4);
     const double c = (double)per_smsp * P.TR * P.nstrips / ctas_per_sm(P.smem_floats);
     if (P.nstrips > kMaxPortableStrips) return 1.3 * c;  // a 16-CTA cluster needs 16 SMs of one GPC
     return P.nstrips > 1 ? 1.15 * c : c;

@@ -29,6 +29,7 @@ namespace {
 enum : int { ZERO = 0, WTS = 1, BIAS = 2, XT = 3, DYT = 4, ZT = 5, YT = 6, RED = 7 };
 int s_tag(int l, int s) { return 100 + 4 * l + s; }
 int q_tag(int l, int s) { return 200 + 4 * l + s; }
+int ss_tag(int l, int s) { return 300 + 4 * l + s; }
 
 struct Shadow {
     std::vector<int> tag;
@@ -230,10 +231,10 @@ void replay_window(Shadow& sh, const Plan& P, long long base, int stride, long l
 
 // Replays the D-tile reads of corr_tile on an unpadded, tile-rounded plane.
 void replay_dtile(Shadow& sh, const Plan& P, long long base, int stride, long long lo, long long hi, int n, int m,
-                  int tr, int tc, int itag) {
+                  int tr, int tc, int itag, int align = 4) {
     const int TR = P.TR, TC = P.TC;
     const long long dt = base + (long long)tr * TR * stride + (long long)tc * TC;
-    if (dt % 4 != 0) sh.fail("D tile not 16-byte aligned", dt);
+    if (dt % align != 0 || stride % align != 0) sh.fail("D tile misaligned for its loads", dt);
     for (int r = 0; r < TR; ++r)
         for (int c = 0; c < TC; ++c) {
             const int i = tr * TR + r, j = tc * TC + c;
@@ -602,6 +603,173 @@ void check_bwdw(const wtconv_desc_t& d) {
                 P.smem_floats * 4, P.nthreads, TR, P.n_all_tiles, P.tpt, P.groups, NS);
 }
 
+// Fused backward: dx conv tiles (the input-gradient pass: dy in X / S, dx
+// in Q / Y) and correlation tiles (x windows in XS / SS against dy tiles at
+// the interior of X / S) in one walk.
+void check_bwd(const wtconv_desc_t& d) {
+    Plan P;
+    const wtconv_status_t st = make_plan(&d, kBackward, &P);
+    if (st == WTCONV_ERR_UNSUPPORTED) {
+        std::printf("bwd: no one-pass plan (two passes)\n");
+        return;
+    }
+    if (st != WTCONV_OK) {
+        std::printf("FAIL bwd plan status %d\n", (int)st);
+        std::exit(1);
+    }
+    const int K = P.k, KK = K * K, p = P.p, L = P.L, H = P.H, W = P.W, TR = P.TR, TC = P.TC;
+    const int ncls = 1 + 4 * L;
+    check_divs(P);
+    Shadow sh(P.smem_floats);
+    const long long all = P.smem_floats;
+    if (P.nstrips != 1) sh.fail("strips in the fused backward", P.nstrips);
+    if (P.nthreads > kBwdMaxThreads || P.nthreads % 32 || P.corr0 % 32 || P.corr0 < P.tile_end) sh.fail("threads", P.nthreads);
+    const int ncorr = P.cls_thr[ncls];
+    if (P.corr0 + ncorr > P.nthreads) sh.fail("correlation threads", ncorr);
+    if (P.an_split % 32 || P.an_split <= 0 || P.an_split >= P.nthreads) sh.fail("analysis split", P.an_split);
+    if (P.parts != P.groups || P.groups < 1 || P.groups > P.B) sh.fail("groups", P.groups);
+    if (P.smem_floats * 4 > 227 * 1024) sh.fail("smem", P.smem_floats);
+    const int xrows = P.ntr[kMaxL] * TR + 2 * p;
+    const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
+    const long long slo = P.XS.base, shi = P.XS.base + (long long)xrows * P.XS.stride;
+    const long long ylo = P.Y.base, yhi = P.Y.base + (long long)P.ntr[kMaxL] * TR * P.Y.stride;
+    const int align = (p % 2 == 0) ? 2 : 1;
+    const long long plane = (long long)P.Hp * W;
+    // Weights folded once (before the first barrier), then the first pair staged.
+    sh.phase = "fold";
+    for (int cl = 0; cl < ncls; ++cl)
+        for (int t = 0; t < KK; ++t)
+            sh.write(P.wbase + (long long)cl * P.wcls + t, P.wbase, P.wbase + (long long)ncls * P.wcls, WTS, "weights");
+    sh.write(P.bias, P.bias, P.bias + 1, BIAS, "bias");
+    sh.phase = "initial staging";
+    replay_stage(sh, P, P.stg, XT + 10, 0);
+    replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10, 0);
+    auto synthesis = [&]() {
+        for (int t = 0; t < P.n_fin; ++t) {
+            const int i = (int)fastdiv_host(t, P.div_q4), q = t - i * (W / 4);
+            const int j0 = 2 * q;
+            for (int l = L - 1; l >= 1; --l) {
+                const Buf& Q = P.Q[l];
+                for (int s2 = 0; s2 < 4; ++s2)
+                    sh.read(Q.base + (long long)s2 * Q.sub + (long long)(i >> l) * Q.stride + (j0 >> l),
+                            Q.base + (long long)s2 * Q.sub, Q.base + (long long)(s2 + 1) * Q.sub, q_tag(l, s2), "coarse Q");
+            }
+            const Buf& Q = P.Q[0];
+            for (int s2 = 0; s2 < 4; ++s2)
+                for (int e = 0; e < 2; ++e)
+                    sh.read(Q.base + (long long)s2 * Q.sub + (long long)i * Q.stride + j0 + e, Q.base + (long long)s2 * Q.sub,
+                            Q.base + (long long)(s2 + 1) * Q.sub, q_tag(0, s2), "level-0 Q");
+            for (int rr = 0; rr < 2; ++rr)
+                for (int e = 0; e < 4; ++e) {
+                    sh.read(P.Y.base + (long long)(2 * i + rr) * P.Y.stride + 4 * q + e, ylo, yhi, YT, "Y");
+                    check_global((long long)(2 * i + rr) * W + 4 * q + e, plane, "dx store");
+                }
+        }
+    };
+    for (int plane_i = 0; plane_i <= 2; ++plane_i) {
+        sh.barrier();
+        if (plane_i < 2) {
+            sh.phase = "A: analysis of x and dy";
+            const int e0 = sh.epoch;
+            replay_analyse(sh, P, P.stg, XT + 10, P.XS.base + (long long)p * P.XS.stride + p, P.XS.stride, slo, shi, XT,
+                           P.SS, p, ss_tag);
+            const int e1 = sh.epoch;
+            sh.epoch = e0;  // both analyses run side by side, meeting the same barriers
+            replay_analyse(sh, P, P.stg + P.stg_floats, DYT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride,
+                           xlo, xhi, DYT, P.S, p, s_tag);
+            if (sh.epoch != e1) sh.fail("the two analyses meet different barriers", e1);
+        }
+        if (plane_i > 0 && L >= 1) {
+            sh.phase = "A: synthesis of the previous dx";
+            synthesis();
+        }
+        if (plane_i == 2) break;
+        sh.barrier();
+        sh.phase = "B: staging";
+        if (plane_i == 0) {
+            replay_stage(sh, P, P.stg, XT + 10, 0);
+            replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10, 0);
+        }
+        sh.phase = "B: dx conv tiles";
+        for (int cl = 1; cl < ncls; ++cl) {
+            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+            const int n = H >> (l + 1), m = W >> (l + 1);
+            for (int local = 0; local < P.sub_begin[cl] - P.sub_begin[cl - 1]; ++local) {
+                const int tr = (int)fastdiv_host(local, P.div_ntc[l]), tc = local - tr * P.ntc[l];
+                for (int t = 0; t < KK; ++t) sh.read(P.wbase + (long long)cl * P.wcls + t, 0, all, WTS, "weights");
+                const Buf& S = P.S[l];
+                replay_window(sh, P, S.base + (long long)s * S.sub, S.stride, S.base + (long long)s * S.sub,
+                              S.base + (long long)(s + 1) * S.sub, n, m, tr, tc, s_tag(l, s), "dy subband window", 0);
+                const Buf& Q = P.Q[l];
+                const long long out = Q.base + (long long)s * Q.sub + (long long)tr * TR * Q.stride + (long long)tc * TC;
+                for (int o = 0; o < TR; ++o)
+                    for (int j = 0; j < TC; ++j)
+                        sh.write(out + (long long)o * Q.stride + j, Q.base + (long long)s * Q.sub,
+                                 Q.base + (long long)(s + 1) * Q.sub, q_tag(l, s), "Q tile");
+            }
+        }
+        for (int t = 0; t < P.n_base_tiles; ++t) {
+            const int tr = (int)fastdiv_host(t, P.div_ntc[kMaxL]), tc = t - tr * P.ntc[kMaxL];
+            for (int q = 0; q < KK; ++q) sh.read(P.wbase + q, 0, all, WTS, "base weights");
+            replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, DYT, "dy window", 0);
+            if (L >= 1) {
+                const long long yo = P.Y.base + (long long)tr * TR * P.Y.stride + (long long)tc * TC;
+                for (int o = 0; o < TR; ++o)
+                    for (int e = 0; e < TC; ++e) sh.write(yo + (long long)o * P.Y.stride + e, ylo, yhi, YT, "Y tile");
+            } else {
+                for (int o = 0; o < TR; ++o)
+                    if (tr * TR + o < H)
+                        for (int e = 0; e < TC; ++e) check_global((long long)(tr * TR + o) * W + tc * TC + e, plane, "dx store");
+            }
+        }
+        sh.phase = "B: correlation tiles";
+        int covered = 0;
+        for (int ct = 0; ct < ncorr; ++ct)
+            for (int k = 0; k < P.tpt; ++k) {
+                int cl = 0;
+                while (ct >= P.cls_thr[cl + 1]) ++cl;
+                const int lvl = (cl == 0) ? kMaxL : ((cl - 1) >> 2);
+                const int first = (ct - P.cls_thr[cl]) * P.tpt;
+                const int cnt = std::min(P.tpt, P.cls_tiles[cl] - first);
+                if (cnt < 1) sh.fail("thread without tiles", ct);
+                if (k >= cnt) continue;
+                const int local = first + k;
+                ++covered;
+                const int tr = (int)fastdiv_host(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
+                if (cl == 0) {
+                    replay_window(sh, P, P.XS.base, P.XS.stride, slo, shi, H, W, tr, tc, XT, "x window", 0);
+                    replay_dtile(sh, P, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, H, W, tr, tc, DYT,
+                                 align);
+                } else {
+                    const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+                    const int n = H >> (l + 1), m = W >> (l + 1);
+                    const Buf& SS = P.SS[l];
+                    const Buf& S = P.S[l];
+                    replay_window(sh, P, SS.base + (long long)s * SS.sub, SS.stride, SS.base + (long long)s * SS.sub,
+                                  SS.base + (long long)(s + 1) * SS.sub, n, m, tr, tc, ss_tag(l, s), "x subband window", 0);
+                    replay_dtile(sh, P, S.base + (long long)s * S.sub + (long long)p * S.stride + p, S.stride,
+                                 S.base + (long long)s * S.sub, S.base + (long long)(s + 1) * S.sub, n, m, tr, tc,
+                                 s_tag(l, s), align);
+                }
+            }
+        if (covered != P.n_all_tiles) sh.fail("correlation tiles covered", covered);
+    }
+    // Reduction scratch after the walk.
+    sh.barrier();
+    sh.phase = "reduction";
+    const long long red_end = (long long)P.red + (long long)ncorr * KK + P.nthreads / 32;
+    if (red_end > P.smem_floats) sh.fail("reduction scratch", red_end);
+    for (int ct = 0; ct < ncorr; ++ct)
+        for (int t = 0; t < KK; ++t) sh.write(P.red + (long long)ct * KK + t, P.red, red_end, RED, "class sums");
+    for (int w = 0; w < P.nthreads / 32; ++w) sh.write(P.red + (long long)ncorr * KK + w, P.red, red_end, RED, "dy sums");
+    sh.barrier();
+    for (int k2 = 0; k2 < ncls; ++k2)
+        for (int th = P.cls_thr[k2]; th < P.cls_thr[k2 + 1]; ++th)
+            for (int t = 0; t < KK; ++t) sh.read(P.red + (long long)th * KK + t, P.red, red_end, RED, "class reduction");
+    std::printf("bwd: smem %d B, threads %d (%d conv + %d correlation), TR %d, groups %d\n", P.smem_floats * 4,
+                P.nthreads, P.corr0, ncorr, TR, P.groups);
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
@@ -619,6 +787,7 @@ int main(int argc, char** argv) {
     check_fused(d, kForward);
     check_fused(d, kBackwardInput);
     check_bwdw(d);
+    check_bwd(d);
     std::printf("OK\n");
     return 0;
 }

@@ -24,13 +24,14 @@ def _oracle_all(oracle, inp, L):
     Case("mod_bf16", 2, 3, 32, 32, 3, 3, "bf16", 41, "uniform", "normal"),
     Case("mod_L0", 1, 2, 8, 8, 5, 0, "f32", 42, "normal", "normal"),
 ], ids=lambda c: c.name)
-def test_autograd_matches_oracle(oracle, case):
+@pytest.mark.parametrize("one_pass", [False, True], ids=["two_pass", "one_pass"])
+def test_autograd_matches_oracle(oracle, case, one_pass):
     inp = make_inputs(case)
     dev = torch.device("cuda", 0)
     dt = torch.bfloat16 if case.dtype == "bf16" else torch.float32
     x = inp["x"].to(dev, dt).requires_grad_(True)
     p = {k: inp[k].to(dev).requires_grad_(True) for k in NAMES}
-    y = wt.wtconv(x, *(p[k] for k in NAMES), case.L)
+    y = wt.wtconv(x, *(p[k] for k in NAMES), case.L, one_pass)
     y.backward(inp["dy"].to(dev, dt))
     torch.cuda.synchronize()
     ry, rdx, rg = _oracle_all(oracle, inp, case.L)

@@ -34,15 +34,20 @@ def gpu_inputs(inp):
     return {k: v.cuda() for k, v in inp.items()}
 
 
-def run_gpu(case: Case, g, calls):
+def run_gpu(case: Case, g, calls, fused_bwd=False):
     out = {}
     if "fwd" in calls:
         out["y"] = wt.forward(g["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], case.L)
-    if "bwd_in" in calls:
-        out["dx"] = wt.backward_input(g["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], case.L)
-    if "bwd_w" in calls:
-        out["grads"] = wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"],
-                                          g["wt_scale"], case.L)
+    if fused_bwd:
+        # dx and the parameter gradients from the one-pass backward.
+        out["dx"], out["grads"] = wt.backward(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"],
+                                              g["wt_scale"], case.L)
+    else:
+        if "bwd_in" in calls:
+            out["dx"] = wt.backward_input(g["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], case.L)
+        if "bwd_w" in calls:
+            out["grads"] = wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"],
+                                              g["wt_scale"], case.L)
     torch.cuda.synchronize()
     return out
 
@@ -55,9 +60,9 @@ def oracle_params(inp, c=None):
     return p
 
 
-def check_full(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w")):
+def check_full(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), fused_bwd=False):
     inp = make_inputs(case)
-    out = run_gpu(case, gpu_inputs(inp), calls)
+    out = run_gpu(case, gpu_inputs(inp), calls, fused_bwd)
     p = oracle_params(inp)
     x, dy = f64(inp["x"]), f64(inp["dy"])
     tol = TOL[case.dtype]
@@ -80,9 +85,10 @@ def check_full(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w")):
     return errs
 
 
-def check_sampled(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), nplanes=6, nchannels=3, seed=0):
+def check_sampled(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), nplanes=6, nchannels=3, seed=0,
+                  fused_bwd=False):
     inp = make_inputs(case)
-    out = run_gpu(case, gpu_inputs(inp), calls)
+    out = run_gpu(case, gpu_inputs(inp), calls, fused_bwd)
     rng = np.random.default_rng(seed)
     planes = {(0, 0), (case.B - 1, case.C - 1)}
     while len(planes) < min(nplanes, case.B * case.C):
@@ -153,6 +159,30 @@ SMALL = [
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: c.name)
 def test_small_case_all_outputs(oracle, case):
     check_full(oracle, case, case.calls)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: c.name)
+def test_small_case_fused_backward(oracle, case):
+    # The one-pass backward (or, for strip planes, its two-pass fallback).
+    check_full(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=True)
+
+
+@pytest.mark.parametrize("case", [STAGE1, STAGE2, TRAIN_BF16], ids=lambda c: c.name)
+def test_full_size_fused_backward_sampled(oracle, case):
+    check_sampled(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=True)
+
+
+def test_fused_backward_is_deterministic():
+    case = STAGE1
+    g = gpu_inputs(make_inputs(case))
+    args = (g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], case.L)
+    dx_a, ga = wt.backward(*args)
+    dx_a, ga = dx_a.clone(), {k: v.clone() for k, v in ga.items()}
+    dx_b, gb = wt.backward(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(dx_a, dx_b)
+    for k in PARAMS:
+        assert torch.equal(ga[k], gb[k]), k
 
 
 def test_tiny_config_forward(oracle):
