@@ -46,95 +46,23 @@ cudaError_t launch_bwd(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t 
     }
 }
 
-size_t workspace_floats(const Plan& P) { return (size_t)P.C * P.parts * P.nv; }
-
 // Workspace both weight-gradient paths accept: the larger of the two plans'.
-size_t workspace_floats_any(const wtconv_desc_t* d) {
+size_t workspace_bytes_any(const wtconv_desc_t* d) {
     Plan P;
     size_t n = 0;
-    if (make_plan(d, kBackwardWeight, &P) == WTCONV_OK) n = workspace_floats(P);
-    if (make_plan(d, kBackward, &P) == WTCONV_OK) n = std::max(n, workspace_floats(P));
+    if (make_plan(d, kBackwardWeight, &P) == WTCONV_OK) n = workspace_bytes_of(P);
+    if (make_plan(d, kBackward, &P) == WTCONV_OK) n = std::max(n, workspace_bytes_of(P));
     return n;
 }
 
+GradArgs grad_args(const float* base_w, const float* base_b, const float* base_scale, const float* wt_w,
+                   const float* wt_scale, float* d_base_w, float* d_base_b, float* d_base_scale, float* d_wt_w,
+                   float* d_wt_scale, unsigned* counters) {
+    return GradArgs{base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                    d_wt_w, d_wt_scale, counters};
+}
+
 }  // namespace
-
-// ---------------------------------------------------------------------------
-// Weight gradient, stage 2: one CTA per channel sums the partials (batch
-// groups x strips) in
-// a fixed order and turns them into the five parameter gradients.  The
-// channel's parameters are staged in shared memory first, and each dot
-// product is one warp's fixed xor-tree.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) wtconv_bwdw_finish_kernel(
-    const float* __restrict__ part, int groups, int nv, int C, int k, int L,
-    const float* __restrict__ base_w, const float* __restrict__ base_b, const float* __restrict__ base_scale,
-    const float* __restrict__ wt_w, const float* __restrict__ wt_scale, float* __restrict__ d_base_w,
-    float* __restrict__ d_base_b, float* __restrict__ d_base_scale, float* __restrict__ d_wt_w,
-    float* __restrict__ d_wt_scale) {
-    extern __shared__ float fsm[];
-    float* gsum = fsm;            // nv: summed partials (un-normalised level sums)
-    float* wts = fsm + nv;        // ncls*KK: this channel's base_w then wt_w[l][c][s]
-    const int c = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
-    const int KK = k * k, ncls = 1 + 4 * L;
-    for (int t = tid; t < nv; t += nt) {
-        float s = 0.f;
-        for (int g = 0; g < groups; ++g) s += part[((size_t)c * groups + g) * nv + t];
-        gsum[t] = s;
-    }
-    for (int t = tid; t < ncls * KK; t += nt) {
-        const int cl = t / KK, tap = t - cl * KK;
-        if (cl == 0) {
-            wts[t] = base_w[c * KK + tap];
-        } else {
-            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-            wts[t] = wt_w[((l * C + c) * 4 + s) * KK + tap];
-        }
-    }
-    __syncthreads();
-    // Level sums were accumulated on un-normalised subbands: scale by 4^-(l+1).
-    for (int t = tid; t < 4 * L * KK; t += nt) {
-        const int l = t / (4 * KK);
-        gsum[KK + t] *= quarter_pow(l);
-    }
-    __syncthreads();
-    const float sdy = gsum[ncls * KK];
-    const float bs = base_scale[c];
-    for (int t = tid; t < KK; t += nt) d_base_w[c * KK + t] = bs * gsum[t];
-    for (int t = tid; t < 4 * L * KK; t += nt) {
-        const int k2 = t / KK, tap = t - k2 * KK;
-        const int l = k2 >> 2, s = k2 & 3;
-        const int pi = (l * C + c) * 4 + s;
-        d_wt_w[pi * KK + tap] = wt_scale[pi] * gsum[KK + t];
-    }
-    // Dot products: class cl -> warp (cl mod warps); lanes stride the taps.
-    const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
-    for (int cl = warp; cl < ncls; cl += nw) {
-        float a = 0.f;
-        for (int tap = lane; tap < KK; tap += 32) a = fmaf(wts[cl * KK + tap], gsum[cl * KK + tap], a);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0) {
-            if (cl == 0) {
-                d_base_b[c] = bs * sdy;
-                d_base_scale[c] = fmaf(base_b[c], sdy, a);
-            } else {
-                const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-                d_wt_scale[(l * C + c) * 4 + s] = a;
-            }
-        }
-    }
-}
-
-cudaError_t launch_bwdw_finish(const Plan& P, const float* part, const float* base_w, const float* base_b,
-                               const float* base_scale, const float* wt_w, const float* wt_scale,
-                               float* d_base_w, float* d_base_b, float* d_base_scale, float* d_wt_w,
-                               float* d_wt_scale, cudaStream_t s) {
-    wtconv_bwdw_finish_kernel<<<P.C, 128, (size_t)(P.nv + (1 + 4 * P.L) * P.k * P.k) * 4, s>>>(part, P.parts, P.nv, P.C, P.k, P.L, base_w,
-                                                                 base_b, base_scale, wt_w, wt_scale, d_base_w,
-                                                                 d_base_b, d_base_scale, d_wt_w, d_wt_scale);
-    return cudaGetLastError();
-}
 
 }  // namespace wtc
 
@@ -160,7 +88,7 @@ const char* wtconv_status_string(wtconv_status_t s) {
 
 size_t wtconv_workspace_bytes(const wtconv_desc_t* d) {
     if (validate(d) != WTCONV_OK) return 0;
-    return workspace_floats_any(d) * sizeof(float);
+    return workspace_bytes_any(d);
 }
 
 wtconv_status_t wtconv_forward(const wtconv_desc_t* d, const void* x, const float* base_w, const float* base_b,
@@ -211,15 +139,16 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t* d, const void* x, co
     Plan P;
     st = make_plan(d, kBackwardWeight, &P);
     if (st != WTCONV_OK) return st;
-    if (!workspace || workspace_bytes < workspace_floats_any(d) * sizeof(float)) return WTCONV_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < workspace_bytes_any(d)) return WTCONV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
     float* part = static_cast<float*>(workspace);
-    BwdwArgs a{x, dy, part};
+    unsigned* counters = reinterpret_cast<unsigned*>(part + counters_offset_floats(P));
     cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(counters, 0, (size_t)P.C * sizeof(unsigned), s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    BwdwArgs a{x, dy, part,
+               grad_args(base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale, d_wt_w,
+                         d_wt_scale, counters)};
     if (launch_bwdw(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
-    if (launch_bwdw_finish(P, part, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
-                           d_wt_w, d_wt_scale, s) != cudaSuccess)
-        return WTCONV_ERR_CUDA;
     return WTCONV_OK;
 }
 
@@ -244,15 +173,16 @@ wtconv_status_t wtconv_backward(const wtconv_desc_t* d, const void* x, const voi
                                       d_base_scale, d_wt_w, d_wt_scale, workspace, workspace_bytes, stream);
     }
     if (st != WTCONV_OK) return st;
-    if (!workspace || workspace_bytes < workspace_floats_any(d) * sizeof(float)) return WTCONV_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < workspace_bytes_any(d)) return WTCONV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
     float* part = static_cast<float*>(workspace);
+    unsigned* counters = reinterpret_cast<unsigned*>(part + counters_offset_floats(P));
     cudaStream_t s = (cudaStream_t)stream;
-    BwdArgs a{x, dy, base_w, base_b, base_scale, wt_w, wt_scale, dx, part};
+    if (cudaMemsetAsync(counters, 0, (size_t)P.C * sizeof(unsigned), s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    BwdArgs a{x, dy, dx, part,
+              grad_args(base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale, d_wt_w,
+                        d_wt_scale, counters)};
     if (launch_bwd(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
-    if (launch_bwdw_finish(P, part, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
-                           d_wt_w, d_wt_scale, s) != cudaSuccess)
-        return WTCONV_ERR_CUDA;
     return WTCONV_OK;
 }
 

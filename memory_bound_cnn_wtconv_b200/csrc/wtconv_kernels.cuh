@@ -805,6 +805,86 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Weight gradient, final step (in the tail of the kernels that write the
+// partial vectors): the last CTA of channel c to publish its partial vector
+// sums the channel's `parts` vectors in a fixed order (so the result does not
+// depend on which CTA is last), scales the level sums by 4^-(l+1) (they were
+// accumulated on un-normalised subbands), and writes the five gradients; each
+// dot product is one warp's fixed xor-tree.  Arrival counters (one per
+// channel) are zero before the launch and reset by the last CTA.
+// ---------------------------------------------------------------------------
+struct GradArgs {
+    const float *base_w, *base_b, *base_scale, *wt_w, *wt_scale;
+    float *d_base_w, *d_base_b, *d_base_scale, *d_wt_w, *d_wt_scale;
+    unsigned* counters;
+};
+
+__device__ __forceinline__ void finish_channel_if_last(float* sm, const Plan& P, const float* part, int c,
+                                                       const GradArgs& ga, int tid, int nt) {
+    const int KK = P.k * P.k, L = P.L, C = P.C, nv = P.nv, ncls = 1 + 4 * L;
+    // Shared scratch from offset 0 (every buffer is dead by now): gsum, wts,
+    // then the "last" flag.
+    int* last = reinterpret_cast<int*>(sm + nv + ncls * KK);
+    __syncthreads();  // this CTA's partial vector is written; the reduction scratch is read
+    if (tid == 0) {
+        __threadfence();  // publish it before counting in
+        *last = atomicAdd(&ga.counters[c], 1u) == (unsigned)(P.parts - 1);
+    }
+    __syncthreads();
+    if (!*last) return;
+    __threadfence();  // every partial vector of the channel is visible
+    float* gsum = sm;       // nv: summed partials
+    float* wts = sm + nv;   // ncls*KK: the channel's base_w then wt_w[l][c][s]
+    const float* pc = part + (size_t)c * P.parts * nv;
+    for (int t = tid; t < nv; t += nt) {
+        float s = 0.f;
+        for (int g = 0; g < P.parts; ++g) s += __ldcg(pc + (size_t)g * nv + t);
+        gsum[t] = s;
+    }
+    for (int t = tid; t < ncls * KK; t += nt) {
+        const int cl = t / KK, tap = t - cl * KK;
+        if (cl == 0) {
+            wts[t] = ga.base_w[c * KK + tap];
+        } else {
+            const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+            wts[t] = ga.wt_w[((l * C + c) * 4 + s) * KK + tap];
+        }
+    }
+    __syncthreads();
+    for (int t = tid; t < 4 * L * KK; t += nt) {
+        const int l = t / (4 * KK);
+        gsum[KK + t] *= quarter_pow(l);
+    }
+    __syncthreads();
+    const float sdy = gsum[ncls * KK];
+    const float bs = ga.base_scale[c];
+    for (int t = tid; t < KK; t += nt) ga.d_base_w[c * KK + t] = bs * gsum[t];
+    for (int t = tid; t < 4 * L * KK; t += nt) {
+        const int k2 = t / KK, tap = t - k2 * KK;
+        const int l = k2 >> 2, s = k2 & 3;
+        const int pi = (l * C + c) * 4 + s;
+        ga.d_wt_w[pi * KK + tap] = ga.wt_scale[pi] * gsum[KK + t];
+    }
+    const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+    for (int cl = warp; cl < ncls; cl += nw) {
+        float a = 0.f;
+        for (int tap = lane; tap < KK; tap += 32) a = fmaf(wts[cl * KK + tap], gsum[cl * KK + tap], a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) {
+            if (cl == 0) {
+                ga.d_base_b[c] = bs * sdy;
+                ga.d_base_scale[c] = fmaf(ga.base_b[c], sdy, a);
+            } else {
+                const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
+                ga.d_wt_scale[(l * C + c) * 4 + s] = a;
+            }
+        }
+    }
+    if (tid == 0) ga.counters[c] = 0u;
+}
+
+// ---------------------------------------------------------------------------
 // Weight gradient, stage 1: grid (C, groups).  The CTA of (c, g) walks the
 // planes b = g, g + groups, ... of channel c, staging the next (x, dy) pair
 // while it computes the current one.  Thread t owns a run of tiles of one
@@ -816,7 +896,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
 // instantiation, so whole-plane walks keep every register for the sums).
 template <int K, int TR, int TC, typename T, bool STRIPS>
 __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel(
-    const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const Plan P) {
+    const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const GradArgs ga, const Plan P) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
     constexpr int p = K / 2, KK = K * K;
@@ -917,6 +997,7 @@ __global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel
         for (int w = 0; w < (nt >> 5); ++w) s += red[nt * KK + w];
         out[ncls * KK] = s;
     }
+    finish_channel_if_last(sm, P, part, c, ga, tid, nt);
 }
 
 // ---------------------------------------------------------------------------
@@ -936,7 +1017,8 @@ template <int K, int TR, int TC, typename T>
 __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
     const T* __restrict__ x, const T* __restrict__ dy, const float* __restrict__ base_w,
     const float* __restrict__ base_b, const float* __restrict__ base_scale, const float* __restrict__ wt_w,
-    const float* __restrict__ wt_scale, T* __restrict__ dx, float* __restrict__ part, const Plan P) {
+    const float* __restrict__ wt_scale, T* __restrict__ dx, float* __restrict__ part, const GradArgs ga,
+    const Plan P) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
     constexpr int p = K / 2, KK = K * K, NP = TC / 2;
@@ -1095,6 +1177,7 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
         for (int w = 0; w < (nt >> 5); ++w) s += red[ncorr * KK + w];
         out[ncls * KK] = s;
     }
+    finish_channel_if_last(sm, P, part, c, ga, tid, nt);
 }
 
 }  // namespace wtc

@@ -104,7 +104,7 @@ cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
         if ((e = cudaOccupancyMaxActiveClusters(&clusters, fn, &L.cfg)) != cudaSuccess) return e;
         if (clusters < 1) return cudaErrorInvalidConfiguration;
     }
-    e = cudaLaunchKernelEx(&L.cfg, fn, static_cast<const T*>(a.x), static_cast<const T*>(a.dy), a.part, P);
+    e = cudaLaunchKernelEx(&L.cfg, fn, static_cast<const T*>(a.x), static_cast<const T*>(a.dy), a.part, a.ga, P);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -121,9 +121,10 @@ cudaError_t bwd_typed(const Plan& P, const BwdArgs& a, cudaStream_t s) {
     auto* fn = wtconv_backward_kernel<WTC_K, TR, 4, T>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
+    const GradArgs& g = a.ga;
     fn<<<dim3(P.C, P.groups), P.nthreads, (size_t)P.smem_floats * 4, s>>>(
-        static_cast<const T*>(a.x), static_cast<const T*>(a.dy), a.base_w, a.base_b, a.base_scale, a.wt_w,
-        a.wt_scale, static_cast<T*>(a.dx), a.part, P);
+        static_cast<const T*>(a.x), static_cast<const T*>(a.dy), g.base_w, g.base_b, g.base_scale, g.wt_w,
+        g.wt_scale, static_cast<T*>(a.dx), a.part, g, P);
     return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 
+#include "wtconv_kernels.cuh"
 #include "wtconv_plan.h"
 
 namespace wtc {
@@ -18,14 +19,15 @@ struct BwdwArgs {
     const void* x;
     const void* dy;
     float* part;
+    GradArgs ga;
 };
 
 struct BwdArgs {
     const void* x;
     const void* dy;
-    const float *base_w, *base_b, *base_scale, *wt_w, *wt_scale;
     void* dx;
     float* part;
+    GradArgs ga;
 };
 
 #define WTC_DECLARE_LAUNCHERS(KV)                                                                     \
@@ -40,9 +42,10 @@ WTC_DECLARE_LAUNCHERS(7)
 
 #undef WTC_DECLARE_LAUNCHERS
 
-cudaError_t launch_bwdw_finish(const Plan& P, const float* part, const float* base_w, const float* base_b,
-                               const float* base_scale, const float* wt_w, const float* wt_scale,
-                               float* d_base_w, float* d_base_b, float* d_base_scale, float* d_wt_w,
-                               float* d_wt_scale, cudaStream_t s);
+// Weight-gradient workspace: the partial vectors, then one arrival counter
+// per channel (16-byte aligned).
+inline size_t partial_floats(const Plan& P) { return (size_t)P.C * P.parts * P.nv; }
+inline size_t counters_offset_floats(const Plan& P) { return (partial_floats(P) + 3) & ~(size_t)3; }
+inline size_t workspace_bytes_of(const Plan& P) { return (counters_offset_floats(P) + (size_t)P.C) * 4; }
 
 }  // namespace wtc

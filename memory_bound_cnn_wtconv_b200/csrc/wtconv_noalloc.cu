@@ -69,20 +69,21 @@ extern "C" wtconv_status_t wtconv_backward_weight_noalloc(
     Plan P;
     st = make_plan(d, kBackwardWeight, &P);
     if (st != WTCONV_OK) return st;
-    // The partials of this plan need C * parts * nv floats; beyond the fixed
-    // array the call is rejected (use wtconv_backward_weight with a workspace
-    // instead).
-    if ((size_t)P.C * P.parts * P.nv > kNoAllocScratchFloats) return WTCONV_ERR_WORKSPACE;
+    // The partials and the per-channel arrival counters of this plan
+    // (workspace_bytes_of); beyond the fixed array the call is rejected (use
+    // wtconv_backward_weight with a workspace instead).
+    if (workspace_bytes_of(P) > kNoAllocScratchFloats * sizeof(float)) return WTCONV_ERR_WORKSPACE;
     cudaError_t err = cudaSuccess;
     float* part = scratch_address(&err);
     if (part == nullptr) return WTCONV_ERR_CUDA;
-    // Every partial slot the finish kernel reads is written by the partial
-    // kernel of the same call, so nothing has to be cleared first.
+    // Every partial slot the final step reads is written by the same launch;
+    // only the counters are cleared.
+    unsigned* counters = reinterpret_cast<unsigned*>(part + counters_offset_floats(P));
     cudaStream_t s = (cudaStream_t)stream;
-    BwdwArgs a{x, dy, part};
+    if (cudaMemsetAsync(counters, 0, (size_t)P.C * sizeof(unsigned), s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    BwdwArgs a{x, dy, part,
+               GradArgs{base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale, d_wt_w,
+                        d_wt_scale, counters}};
     if (launch_partials(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
-    if (launch_bwdw_finish(P, part, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
-                           d_wt_w, d_wt_scale, s) != cudaSuccess)
-        return WTCONV_ERR_CUDA;
     return WTCONV_OK;
 }

@@ -296,6 +296,8 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         const long long busy = ceil_div((int)std::min<long long>(an_items, 1 << 30), 32) * 32LL;
         P->fin_off = busy >= P->nthreads ? 0 : (int)busy;
     }
+    // Weight gradients: the final step's scratch (summed partials, weights, a flag).
+    if (kind == kBackwardWeight || kind == kBackward) off = std::max(off, (long long)P->nv + ncls * KK + 4);
     off = round4((int)std::min<long long>(off, 1LL << 30));
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;

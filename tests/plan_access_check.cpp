@@ -599,6 +599,7 @@ void check_bwdw(const wtconv_desc_t& d) {
     if (P.parts != P.groups * NS) sh.fail("partial vectors", P.parts);
     if ((long long)P.nthreads * KK + P.nthreads / 32 > P.smem_floats) sh.fail("sum-dy scratch", P.nthreads);
     if (P.nv != ncls * KK + 1) sh.fail("partial vector length", P.nv);
+    if ((long long)P.nv + ncls * KK + 1 > P.smem_floats) sh.fail("final-step scratch", P.nv);
     std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d (<= %d per thread), groups %d, strips %d\n",
                 P.smem_floats * 4, P.nthreads, TR, P.n_all_tiles, P.tpt, P.groups, NS);
 }
@@ -766,6 +767,7 @@ void check_bwd(const wtconv_desc_t& d) {
     for (int k2 = 0; k2 < ncls; ++k2)
         for (int th = P.cls_thr[k2]; th < P.cls_thr[k2 + 1]; ++th)
             for (int t = 0; t < KK; ++t) sh.read(P.red + (long long)th * KK + t, P.red, red_end, RED, "class reduction");
+    if ((long long)P.nv + ncls * KK + 1 > P.smem_floats) sh.fail("final-step scratch", P.nv);
     std::printf("bwd: smem %d B, threads %d (%d conv + %d correlation), TR %d, groups %d\n", P.smem_floats * 4,
                 P.nthreads, P.corr0, ncorr, TR, P.groups);
 }
