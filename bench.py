@@ -385,7 +385,7 @@ def run_ours(args, case):
     hbm_achieved = mb[dom] / dom_s / 1e9
     t_alu, t_hbm = flops / (alu_peak * 1e12), mb[dom] / (peak * 1e9)
     kernel_names = {"fwd": "wtconv_fused_kernel (forward)", "bwd_in": "wtconv_fused_kernel (input gradient)",
-                    "bwd_w": "wtconv_bwdw_partial_kernel + wtconv_bwdw_finish_kernel"}
+                    "bwd_w": "wtconv_bwdw_partial_kernel (final step in its tail)"}
     traffic, traffic_src = measured_traffic(case.name, dom)
     if t_alu >= t_hbm:
         roof = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "TFLOP/s",
