@@ -413,7 +413,9 @@ def run_ours(args, case):
         "roofline": roof,
         "alu_frac_per_call": {k: 2.0 * conv_fmas(case) / (per_call[k] * 1e-3) / 1e12 / alu_peak
                               for k in ("fwd", "bwd_in", "bwd_w")},
-        "gpu_launches": K * 4, "wall_s_timed_region": wall,
+        # Our kernels in the timed region: forward, input gradient, weight
+        # gradient (its final step runs in the same launch) per step.
+        "gpu_launches": K * 3, "wall_s_timed_region": wall,
     }
     if clk is not None:
         line["clocks"] = clk

@@ -118,3 +118,17 @@ def test_product_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "wtconv_oracle" not in text and "liboracle" not in text, f
+
+
+def test_backward_validation(cuda_lib):
+    p = ctypes.c_void_p
+    d = _desc()
+    need = cuda_lib.wtconv_workspace_bytes(ctypes.byref(d))
+    args = [p(FAKE)] * 7  # x, dy, base_w, base_b, base_scale, wt_w, wt_scale
+    grads = [p(FAKE)] * 5
+    assert cuda_lib.wtconv_backward(ctypes.byref(d), *args, p(0), *grads, p(FAKE), ctypes.c_size_t(need),
+                                    None) == NULLPTR
+    assert cuda_lib.wtconv_backward(ctypes.byref(d), *args, p(FAKE), *grads, p(FAKE), ctypes.c_size_t(need - 4),
+                                    None) == WORKSPACE
+    assert cuda_lib.wtconv_backward(ctypes.byref(_desc(k=4)), *args, p(FAKE), *grads, p(FAKE),
+                                    ctypes.c_size_t(need), None) == BAD_K
