@@ -651,10 +651,18 @@ def run_compare(args, case):
 
 def main():
     args = parse()
-    from wtconv_inputs import NAMED
-    if args.workload not in NAMED:
-        raise SystemExit(f"unknown workload {args.workload}; choose from {sorted(NAMED)}")
-    case = NAMED[args.workload]
+    from wtconv_inputs import NAMED, sweep_cases
+    sweep = {c.name: c for c in sweep_cases()}
+    if args.workload in NAMED:
+        case = NAMED[args.workload]
+    elif args.workload in sweep or args.workload.startswith("sweep"):
+        # A point of the 128-point shape sweep, by full name or index ("sweep031").
+        by_index = {c.name[:8]: c for c in sweep.values()}
+        case = sweep.get(args.workload) or by_index.get(args.workload[:8])
+        if case is None:
+            raise SystemExit(f"unknown sweep point {args.workload}")
+    else:
+        raise SystemExit(f"unknown workload {args.workload}; choose from {sorted(NAMED)} or sweepNNN")
     if case.name == "tiny":
         case = case.with_(calls=("fwd", "bwd_in", "bwd_w"))
     if args.impl == "reference":

@@ -713,7 +713,7 @@ struct FusedCtx {
 // STRIPS: planes split into strips across a cluster (a separate
 // instantiation, so whole-plane walks carry no cluster code).
 template <int K, int TR, int TC, typename T, bool BWD, bool STRIPS>
-__global__ void __launch_bounds__(kFusedMaxThreads, 2) wtconv_fused_kernel(
+__global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kFusedMaxThreads, STRIPS ? 1 : 2) wtconv_fused_kernel(
     const T* __restrict__ x, const float* __restrict__ base_w, const float* __restrict__ base_b,
     const float* __restrict__ base_scale, const float* __restrict__ wt_w,
     const float* __restrict__ wt_scale, T* __restrict__ y, const Plan P) {
@@ -895,7 +895,7 @@ __device__ __forceinline__ void finish_channel_if_last(float* sm, const Plan& P,
 // STRIPS: the plane is split into strips across a cluster (a separate
 // instantiation, so whole-plane walks keep every register for the sums).
 template <int K, int TR, int TC, typename T, bool STRIPS>
-__global__ void __launch_bounds__(kBwdwMaxThreads, 2) wtconv_bwdw_partial_kernel(
+__global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kBwdwMaxThreads, STRIPS ? 1 : 2) wtconv_bwdw_partial_kernel(
     const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const GradArgs ga, const Plan P) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);

@@ -61,6 +61,10 @@ inline FastDiv make_fastdiv(uint32_t d) {
 // Thread budgets (also the kernels' __launch_bounds__, two CTAs per SM).
 constexpr int kFusedMaxThreads = 256;
 constexpr int kBwdwMaxThreads = 256;
+// Planes split into cluster strips: one CTA per SM at most (their strips'
+// buffers are large), so those instantiations take 512 threads at one CTA
+// per SM (the same 128-register budget).
+constexpr int kStripMaxThreads = 512;
 constexpr int kBwdMaxThreads = 512;  // fused backward: one CTA per SM
 
 struct Buf {

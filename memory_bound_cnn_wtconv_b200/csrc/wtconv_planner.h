@@ -268,12 +268,13 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         for (;; ++tpt) {
             used = 0;
             for (int cl = 0; cl < ncls; ++cl) used += ceil_div(P->cls_tiles[cl], tpt);
-            if (used <= kBwdwMaxThreads) break;
+            if (used <= (nstrips > 1 ? kStripMaxThreads : kBwdwMaxThreads)) break;
         }
         P->tpt = tpt;
         P->cls_thr[0] = 0;
         for (int cl = 0; cl < ncls; ++cl) P->cls_thr[cl + 1] = P->cls_thr[cl] + ceil_div(P->cls_tiles[cl], tpt);
-        P->nthreads = std::max(tile_threads(used, kBwdwMaxThreads), ceil_div(used, 32) * 32);
+        P->nthreads = std::max(tile_threads(used, nstrips > 1 ? kStripMaxThreads : kBwdwMaxThreads),
+                               ceil_div(used, 32) * 32);
         // Reduction scratch aliases the (then dead) buffers from offset 0.
         P->red = 0;
         off = std::max(off, (long long)P->nthreads * (KK + 1));
@@ -281,7 +282,7 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         // Subband and base tiles run the same code, so they share warps.
         P->base_tid0 = P->n_sub_tiles;
         P->tile_end = P->base_tid0 + P->n_base_tiles;
-        P->nthreads = tile_threads(P->tile_end, kFusedMaxThreads);
+        P->nthreads = tile_threads(P->tile_end, nstrips > 1 ? kStripMaxThreads : kFusedMaxThreads);
         P->merged = P->tile_end <= P->nthreads ? 1 : 0;
         P->n_fin = L >= 1 ? (H / 2) * (W / 4) : 0;
         // Threads the analysis keeps busy (whole warps); the synthesis items
@@ -316,6 +317,10 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
 // length of one CTA (its warp-tiles spread over 4 sub-partitions, times the
 // tile height), times the CTAs of a plane, over the CTAs an SM holds.
 // Cluster strips carry a halo exchange on top (weighted 15%).
+inline int plan_ctas_per_sm(const Plan& P) {
+    return P.nthreads > 256 ? 1 : ctas_per_sm(P.smem_floats);
+}
+
 inline double plan_cost(const Plan& P, Kind kind) {
     int per_smsp;
     if (kind == kBackward)
@@ -324,7 +329,7 @@ inline double plan_cost(const Plan& P, Kind kind) {
         per_smsp = P.tpt * ceil_div(ceil_div(P.cls_thr[1 + 4 * P.L], 32), 4);
     else
         per_smsp = ceil_div(ceil_div(P.tile_end, 32), 4);
-    const double c = (double)per_smsp * P.TR * P.nstrips / ctas_per_sm(P.smem_floats);
+    const double c = (double)per_smsp * P.TR * P.nstrips / plan_ctas_per_sm(P);
     if (P.nstrips > kMaxPortableStrips) return 1.3 * c;  // a 16-CTA cluster needs 16 SMs of one GPC
     return P.nstrips > 1 ? 1.15 * c : c;
 }

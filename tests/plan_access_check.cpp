@@ -317,7 +317,7 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
         std::printf("FAIL strips: Hp %d H %d n %d\n", P.Hp, H, NS);
         std::exit(1);
     }
-    if (P.nthreads % 32 || P.nthreads > kFusedMaxThreads || P.nthreads < 32) {
+    if (P.nthreads % 32 || P.nthreads > (P.nstrips > 1 ? kStripMaxThreads : kFusedMaxThreads) || P.nthreads < 32) {
         std::printf("FAIL fused thread count %d\n", P.nthreads);
         std::exit(1);
     }
@@ -590,7 +590,8 @@ void check_bwdw(const wtconv_desc_t& d) {
                 for (int t = 0; t < KK; ++t)
                     shs[r].read(P.red + (long long)th * KK + t, P.red, red_end, RED, "class reduction");
     Shadow& sh = shs[0];
-    if (P.nthreads < P.cls_thr[ncls] || P.nthreads > kBwdwMaxThreads || P.nthreads % 32) sh.fail("thread count", P.nthreads);
+    if (P.nthreads < P.cls_thr[ncls] || P.nthreads > (NS > 1 ? kStripMaxThreads : kBwdwMaxThreads) || P.nthreads % 32)
+        sh.fail("thread count", P.nthreads);
     for (int cl = 0; cl < ncls; ++cl) {
         const int lv = cl == 0 ? kMaxL : (cl - 1) >> 2;
         if (P.cls_tiles[cl] != P.ntr[lv] * P.ntc[lv]) sh.fail("class tiles", cl);
