@@ -11,6 +11,14 @@ conv with per-channel scale and bias, an L-level orthonormal 2-D Haar analysis
 recursing on the raw LL subband, a scaled depthwise conv per subband, and the
 inverse Haar synthesis cascade.  See ``wtconv_oracle.c`` for the formulas and
 the subband convention.
+
+Planes whose H or W is not a multiple of 2^L: the pages fix no rule for them.
+The plainest reading, taken here: zero-pad the plane at the bottom and right
+to the next multiples of 2^L, apply the layer, crop the output back.  Its
+adjoint (input gradient) crops the adjoint applied to the zero-padded dy, and
+the weight gradient is taken on the zero-padded x and dy.  (The same result
+follows from padding each level's LL by one row / column when odd and
+cropping each level's reconstruction; a test checks the two agree.)
 """
 from __future__ import annotations
 
@@ -128,8 +136,24 @@ class Oracle:
             return np.zeros((1,)), np.zeros((1,))
         return _f64(wt_w).reshape(L, C, 4, k, k), _f64(wt_scale).reshape(L, C, 4)
 
+    @staticmethod
+    def _pad(a, L):
+        """a zero-padded at the bottom / right to multiples of 2^L (a itself if already)."""
+        m = 1 << L
+        H, W = a.shape[-2:]
+        Hp, Wp = -(-H // m) * m, -(-W // m) * m
+        if (Hp, Wp) == (H, W):
+            return a
+        out = np.zeros(a.shape[:-2] + (Hp, Wp))
+        out[..., :H, :W] = a
+        return out
+
     def forward(self, x, base_w, base_b, base_scale, wt_w, wt_scale, L):
         x, base_w, base_b, base_scale = map(_f64, (x, base_w, base_b, base_scale))
+        xp = self._pad(x, L)
+        if xp is not x:
+            H, W = x.shape[-2:]
+            return self.forward(xp, base_w, base_b, base_scale, wt_w, wt_scale, L)[..., :H, :W].copy()
         B, C, H, W, k, L = self._dims(x, base_w, L)
         wt_w, wt_scale = self._wt(wt_w, wt_scale, L, C, k)
         y = np.empty_like(x)
@@ -141,6 +165,10 @@ class Oracle:
 
     def backward_input(self, dy, base_w, base_scale, wt_w, wt_scale, L):
         dy, base_w, base_scale = map(_f64, (dy, base_w, base_scale))
+        dyp = self._pad(dy, L)
+        if dyp is not dy:
+            H, W = dy.shape[-2:]
+            return self.backward_input(dyp, base_w, base_scale, wt_w, wt_scale, L)[..., :H, :W].copy()
         B, C, H, W, k, L = self._dims(dy, base_w, L)
         wt_w, wt_scale = self._wt(wt_w, wt_scale, L, C, k)
         dx = np.empty_like(dy)
@@ -152,6 +180,9 @@ class Oracle:
 
     def backward_weight(self, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L):
         x, dy, base_w, base_b, base_scale = map(_f64, (x, dy, base_w, base_b, base_scale))
+        xp = self._pad(x, L)
+        if xp is not x:
+            return self.backward_weight(xp, self._pad(dy, L), base_w, base_b, base_scale, wt_w, wt_scale, L)
         B, C, H, W, k, L = self._dims(x, base_w, L)
         wt_w, wt_scale = self._wt(wt_w, wt_scale, L, C, k)
         d_base_w = np.empty((C, k, k))
