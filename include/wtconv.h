@@ -41,7 +41,12 @@
  *     non-OK status means nothing was enqueued and no output was touched.
  *     A launch failure returns WTCONV_ERR_CUDA.  Faults of an enqueued kernel
  *     surface at the caller's next synchronisation, as for any CUDA call.
- *   - Limits: k in {1, 3, 5, 7}; 0 <= L <= 6; H and W divisible by 2^L.
+ *   - Limits: k in {1, 3, 5, 7}; 0 <= L <= 6.  H and W need not be
+ *     multiples of 2^L: such planes are zero-padded at the bottom and right to
+ *     the next multiples on chip, the layer applied, and only the H x W outputs
+ *     written (the input gradient is the transpose of that cropped map; the
+ *     weight gradients sum over the padded plane, where dy is zero); their rows
+ *     must be whole 16-byte chunks (W a multiple of 4 for fp32, 8 for bf16).
  *     A plane that does not fit on one SM is split into 2, 4 or 8 row strips
  *     held by the CTAs of a thread-block cluster (strip height a multiple of
  *     2^L and of 4); planes that still do not fit return
@@ -65,7 +70,7 @@ typedef struct CUstream_st *wtconv_stream_t; /* same type as cudaStream_t */
 typedef enum {
     WTCONV_OK = 0,
     WTCONV_ERR_NULLPTR = 1,     /* a required pointer is NULL */
-    WTCONV_ERR_BAD_SHAPE = 2,   /* B, C, H or W <= 0, or H, W not divisible by 2^L, or W % 4 != 0 */
+    WTCONV_ERR_BAD_SHAPE = 2,   /* B, C, H or W <= 0, W % 4 != 0, or rows not whole 16-byte chunks where needed */
     WTCONV_ERR_BAD_K = 3,       /* k not in {1, 3, 5, 7} */
     WTCONV_ERR_BAD_L = 4,       /* L < 0 or L > 6 */
     WTCONV_ERR_MISALIGNED = 5,  /* an activation pointer is not 16-byte aligned */

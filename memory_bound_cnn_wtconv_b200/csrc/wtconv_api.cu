@@ -74,7 +74,7 @@ const char* wtconv_status_string(wtconv_status_t s) {
     switch (s) {
         case WTCONV_OK: return "ok";
         case WTCONV_ERR_NULLPTR: return "a required pointer is NULL";
-        case WTCONV_ERR_BAD_SHAPE: return "bad shape (B, C, H, W > 0; H, W divisible by 2^L; W % 4 == 0)";
+        case WTCONV_ERR_BAD_SHAPE: return "bad shape (B, C, H, W > 0; W % 4 == 0; rows of whole 16-byte chunks)";
         case WTCONV_ERR_BAD_K: return "unsupported kernel size (k must be 1, 3, 5 or 7)";
         case WTCONV_ERR_BAD_L: return "unsupported level count (0 <= L <= 6)";
         case WTCONV_ERR_MISALIGNED: return "activation pointer not 16-byte aligned";

@@ -61,6 +61,29 @@ __device__ __forceinline__ void stage_plane(float* stg, const void* src, int chu
     for (int ch = tid; ch < chunks; ch += nt) cp_async16(d + 16 * ch, g + 16 * ch);
 }
 
+// This CTA's rows of a plane into staging: one contiguous copy, or (planes
+// zero-padded on chip) its `rows` real rows, each Wr elements, into staging
+// rows of W elements (the padding was zeroed once and is never written).
+__device__ __forceinline__ void stage_rows(float* stg, const void* src, const Plan& P, int rows, int tid, int nt) {
+    if (!P.padded) {
+        stage_plane(stg, src, P.plane_chunks, tid, nt);
+        return;
+    }
+    const char* g = static_cast<const char*>(src);
+    char* d = reinterpret_cast<char*>(stg);
+    const int rc = P.row_chunks;
+    const size_t sbytes = (size_t)P.Wr * P.esize, dbytes = (size_t)P.W * P.esize;
+    for (int ch = tid; ch < rows * rc; ch += nt) {
+        const int r = fdiv(ch, P.div_rowc), c = ch - r * rc;
+        cp_async16(d + r * dbytes + 16 * c, g + r * sbytes + 16 * c);
+    }
+}
+
+// Real rows of strip `rank` (all H of them unless the plane was padded).
+__device__ __forceinline__ int real_rows(const Plan& P, int rank) {
+    return max(0, min(P.H, P.Hr - rank * P.H));
+}
+
 // 4 consecutive staged elements (element index e, a multiple of 4), as floats.
 template <typename T>
 __device__ __forceinline__ float4 stg_load4(const float* stg, int e);
@@ -493,13 +516,15 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 // Barrier of everything that shares a plane: the CTA, or the whole cluster
 // when the plane is split into strips (then it also orders the shared-memory
 // accesses of the cluster's CTAs to each other's strips).
-template <bool STRIPS>
-__device__ __forceinline__ void plane_sync() {
-    if constexpr (STRIPS) {
-        cg::this_cluster().sync();
-    } else {
-        __syncthreads();
+template <bool GENERAL>
+__device__ __forceinline__ void plane_sync(const Plan& P) {
+    if constexpr (GENERAL) {
+        if (P.nstrips > 1) {
+            cg::this_cluster().sync();
+            return;
+        }
     }
+    __syncthreads();
 }
 
 // Fill the halo rows of one padded buffer of this CTA's strip: nsub planes
@@ -593,7 +618,7 @@ __device__ __forceinline__ TileJob decode_tile(const Plan& P, int t, int TR, int
         j.win = P.X.base + tr * TR * P.X.stride + tc * TC;
         j.row0 = tr * TR;
         // L >= 1: Y in shared memory.  L = 0: the output plane itself.
-        j.out = P.L >= 1 ? P.Y.base + tr * TR * P.Y.stride + tc * TC : (tr * TR) * P.W + tc * TC;
+        j.out = P.L >= 1 ? P.Y.base + tr * TR * P.Y.stride + tc * TC : (tr * TR) * P.Wr + tc * TC;
         j.ostride = P.L >= 1 ? P.Y.stride : P.W;
         j.wts = P.wbase;
         j.wstride = P.X.stride;
@@ -606,15 +631,16 @@ __device__ __forceinline__ TileJob decode_tile(const Plan& P, int t, int TR, int
 
 // Reformulation (2): the synthesis of one work item, output rows 2i, 2i+1 x
 // columns 4q..4q+3 (the level-0 positions (i, 2q) and (i, 2q+1)), added to
-// the base-branch outputs in Y and stored (the only HBM write).
+// the base-branch outputs in Y and stored (the only HBM write; of the
+// planes zero-padded on chip, only the first `rows` rows and Wr columns).
 // Output (h, w) receives, for every level l, the signed sum of the four
 // level-l conv outputs at (h >> (l+1), w >> (l+1)), with LH negated when
 // bit l of h is set, HL when bit l of w is set and HH when exactly one is.
 // The levels >= 1 are gathered Horner-style along the item's path: level l's
 // signed sum for the level-(l-1) position on the path is added to that
 // position's LL term, so the level-0 butterfly carries every coarser level.
-template <typename T>
-__device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp, int t) {
+template <typename T, bool GUARD>
+__device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp, int t, int rows) {
     const int i = fdiv(t, P.div_q4), q = t - i * (P.W >> 2);
     const int j0 = 2 * q;
     float c0 = 0.f, c1 = 0.f;  // coarse terms for LL at (i, j0) and (i, j0 + 1)
@@ -656,9 +682,15 @@ __device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp
         const float a0 = ll.x - lh.x, b0 = hl.x - hh.x, a1 = ll.y - lh.y, b1 = hl.y - hh.y;
         bot.x += a0 + b0; bot.y += a0 - b0; bot.z += a1 + b1; bot.w += a1 - b1;
     }
-    T* yo = yp + (size_t)(2 * i) * P.W + 4 * q;
-    gst4<T>(yo, top);
-    gst4<T>(yo + P.W, bot);
+    // yp: this CTA's rows in y (row stride Wr); only real outputs are stored.
+    T* yo = yp + (size_t)(2 * i) * P.Wr + 4 * q;
+    if (!GUARD) {
+        gst4<T>(yo, top);
+        gst4<T>(yo + P.Wr, bot);
+    } else if (4 * q < P.Wr) {
+        if (2 * i < rows) gst4<T>(yo, top);
+        if (2 * i + 1 < rows) gst4<T>(yo + P.Wr, bot);
+    }
 }
 
 // Shared pieces of the two forward schedules.
@@ -670,7 +702,7 @@ struct FusedCtx {
     const float *base_w, *base_b, *base_scale, *wt_w, *wt_scale;
     long long units;
     int u0, u1;
-    size_t plane_elems;  // Hp * W
+    size_t plane_elems;  // Hr * Wr
     size_t strip_off;    // first element of this CTA's strip within a plane
 
     // Units run channel-major: unit u is plane (b, c) = (u mod B, u / B).
@@ -710,10 +742,11 @@ struct FusedCtx {
 //               subband tiles write Q, base tiles write Y (y itself if L = 0).
 // Within a phase the buffers written (A: X, S, weights; B: staging, Q, Y) and
 // the buffers read (A: staging, Q, Y; B: S, X, weights) are disjoint.
-// STRIPS: planes split into strips across a cluster (a separate
-// instantiation, so whole-plane walks carry no cluster code).
-template <int K, int TR, int TC, typename T, bool BWD, bool STRIPS>
-__global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kFusedMaxThreads, STRIPS ? 1 : 2) wtconv_fused_kernel(
+// GENERAL: planes split into strips across a cluster and / or zero-padded on
+// chip (a separate instantiation, so the common walk of whole planes that
+// are multiples of 2^L carries none of that code).
+template <int K, int TR, int TC, typename T, bool BWD, bool GENERAL>
+__global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads, GENERAL ? 1 : 2) wtconv_fused_kernel(
     const T* __restrict__ x, const float* __restrict__ base_w, const float* __restrict__ base_b,
     const float* __restrict__ base_scale, const float* __restrict__ wt_w,
     const float* __restrict__ wt_scale, T* __restrict__ y, const Plan P) {
@@ -724,12 +757,14 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kFusedMaxThreads, 
     const int tid = threadIdx.x, nt = blockDim.x;
     const long long units = (long long)P.B * P.C;
     // With strips, the nstrips CTAs of a cluster walk the same planes.
-    const int rank = STRIPS ? (int)cg::this_cluster().block_rank() : 0;
-    const long long team = STRIPS ? blockIdx.x / P.nstrips : blockIdx.x;
-    const long long teams = STRIPS ? gridDim.x / P.nstrips : gridDim.x;
+    const bool strips = GENERAL && P.nstrips > 1;
+    const int rank = strips ? (int)cg::this_cluster().block_rank() : 0;
+    const long long team = strips ? blockIdx.x / P.nstrips : blockIdx.x;
+    const long long teams = strips ? gridDim.x / P.nstrips : gridDim.x;
     FusedCtx<K, T, BWD> cx{sm, P, x, base_w, base_b, base_scale, wt_w, wt_scale, units,
                            (int)((team * units) / teams), (int)(((team + 1) * units) / teams),
-                           (size_t)P.Hp * P.W, (size_t)rank * P.H * P.W};
+                           (size_t)P.Hr * P.Wr, (size_t)rank * P.H * P.Wr};
+    const int myrows = real_rows(P, rank);
     const int u0 = cx.u0, u1 = cx.u1;
     auto csync = [&]() { __syncthreads(); };
     float* X0 = sm + P.X.base + p * P.X.stride + p;
@@ -743,12 +778,19 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kFusedMaxThreads, 
     // (b, c) of the plane being analysed / tiled, of the previous plane, and of the next.
     int cur_b = u0 % P.B, cur_c = u0 / P.B;
     int prev_b = 0, prev_c = 0;
-    if (u0 < u1) stage_plane(sm + P.stg, cx.src(cur_b, cur_c), P.plane_chunks, tid, nt);
+    auto stage = [&](const T* src) {
+        if constexpr (GENERAL) {
+            stage_rows(sm + P.stg, src, P, myrows, tid, nt);
+        } else {
+            stage_plane(sm + P.stg, src, P.plane_chunks, tid, nt);
+        }
+    };
+    if (u0 < u1) stage(cx.src(cur_b, cur_c));
     cp_async_commit();
     int folded_c = -1;
     for (int u = u0; u <= u1; ++u) {
         cp_async_wait_all();
-        plane_sync<STRIPS>();  // plane u staged; every tile (and halo copy) of plane u-1 done
+        plane_sync<GENERAL>(P);  // plane u staged; every tile (and halo copy) of plane u-1 done
         // Phase A.
         if (u < u1) {
             if (cur_c != folded_c) {
@@ -759,19 +801,19 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kFusedMaxThreads, 
         }
         if (u > u0 && P.L >= 1) {
             T* yp = y + cx.rows_of(prev_b, prev_c);
-            for (int t = ft; t < P.n_fin; t += nt) synth_item<T>(sm, P, yp, t);
+            for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL>(sm, P, yp, t, myrows);
         }
         if (u == u1) break;
-        plane_sync<STRIPS>();  // X and S of plane u ready (every strip); Q and Y of plane u-1 consumed
+        plane_sync<GENERAL>(P);  // X and S of plane u ready (every strip); Q and Y of plane u-1 consumed
         // Phase B.
         int nb = cur_b + 1, nc = cur_c;
         if (nb == P.B) {
             nb = 0;
             ++nc;
         }
-        if (u + 1 < u1) stage_plane(sm + P.stg, cx.src(nb, nc), P.plane_chunks, tid, nt);
+        if (u + 1 < u1) stage(cx.src(nb, nc));
         cp_async_commit();
-        if (STRIPS) {
+        if (strips) {
             copy_halos(sm, P, rank, tid, nt);
             __syncthreads();  // halo rows in place
         }
@@ -792,7 +834,8 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kFusedMaxThreads, 
                 T* yo = y + cx.rows_of(cur_b, cur_c) + j.out;
                 const int h0 = j.row0;
                 conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
-                    if (h0 + o < P.H) gst4<T>(yo + (size_t)o * P.W, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
+                    if (h0 + o < myrows)
+                        gst4<T>(yo + (size_t)o * P.Wr, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
                 });
             }
         }
@@ -892,10 +935,11 @@ __device__ __forceinline__ void finish_channel_if_last(float* sm, const Plan& P,
 // K*K correlation sums in registers; the CTA then reduces each class over its
 // threads in a fixed order and writes one partial vector (plus sum dy).
 // ---------------------------------------------------------------------------
-// STRIPS: the plane is split into strips across a cluster (a separate
-// instantiation, so whole-plane walks keep every register for the sums).
-template <int K, int TR, int TC, typename T, bool STRIPS>
-__global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kBwdwMaxThreads, STRIPS ? 1 : 2) wtconv_bwdw_partial_kernel(
+// GENERAL: the plane is split into strips across a cluster and / or
+// zero-padded on chip (a separate instantiation, so whole-plane walks keep
+// every register for the sums).
+template <int K, int TR, int TC, typename T, bool GENERAL>
+__global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, GENERAL ? 1 : 2) wtconv_bwdw_partial_kernel(
     const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const GradArgs ga, const Plan P) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
@@ -903,19 +947,26 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kBwdwMaxThreads, S
     constexpr int DLD = sizeof(T) == 2 ? 4 : 2;
     const int tid = threadIdx.x, nt = blockDim.x;
     // blockIdx.x = c * nstrips + (strip rank within the cluster).
-    const int rank = STRIPS ? (int)cg::this_cluster().block_rank() : 0;
-    const int c = STRIPS ? blockIdx.x / P.nstrips : blockIdx.x, g = blockIdx.y, G = P.groups;
-    const size_t plane_elems = (size_t)P.Hp * P.W;
-    const size_t strip_off = (size_t)rank * P.H * P.W;
+    const bool strips = GENERAL && P.nstrips > 1;
+    const int rank = strips ? (int)cg::this_cluster().block_rank() : 0;
+    const int c = strips ? blockIdx.x / P.nstrips : blockIdx.x, g = blockIdx.y, G = P.groups;
+    const size_t plane_elems = (size_t)P.Hr * P.Wr;
+    const size_t strip_off = (size_t)rank * P.H * P.Wr;
+    const int myrows = real_rows(P, rank);
     auto csync = [&]() { __syncthreads(); };
 
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
-    if (g < P.B) {
-        const size_t off = ((size_t)g * P.C + c) * plane_elems + strip_off;
-        stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
-        stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
-    }
+    auto stage = [&](size_t off) {
+        if constexpr (GENERAL) {
+            stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
+            stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
+        } else {
+            stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
+            stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
+        }
+    };
+    if (g < P.B) stage(((size_t)g * P.C + c) * plane_elems + strip_off);
     cp_async_commit();
 
     // This thread's class and its run of that class's tiles.
@@ -935,7 +986,7 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kBwdwMaxThreads, S
     float* X0 = sm + P.X.base + p * P.X.stride + p;
     for (int b = g; b < P.B; b += G) {
         cp_async_wait_all();
-        plane_sync<STRIPS>();  // staged pair complete; previous correlations (and halo copies) done
+        plane_sync<GENERAL>(P);  // staged pair complete; previous correlations (and halo copies) done
         analyse_plane<T, p, false, kToS>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         const float s = analyse_plane<T, 0, true, kToQ>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
                                                         P.DY.stride, 0, nt, tid, csync);
@@ -945,14 +996,10 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kBwdwMaxThreads, S
             sdy_c = (tv - sdy) - yv;
             sdy = tv;
         }
-        plane_sync<STRIPS>();  // both analyses complete (every strip)
-        if (b + G < P.B) {
-            const size_t off = ((size_t)(b + G) * P.C + c) * plane_elems + strip_off;
-            stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
-            stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
-        }
+        plane_sync<GENERAL>(P);  // both analyses complete (every strip)
+        if (b + G < P.B) stage(((size_t)(b + G) * P.C + c) * plane_elems + strip_off);
         cp_async_commit();
-        if (STRIPS) {
+        if (strips) {
             copy_halos(sm, P, rank, tid, nt);
             __syncthreads();  // halo rows in place
         }
@@ -972,7 +1019,7 @@ __global__ void __launch_bounds__(STRIPS ? kStripMaxThreads : kBwdwMaxThreads, S
         }
     }
     cp_async_wait_all();
-    plane_sync<STRIPS>();  // no CTA of the cluster reads this CTA's strip any more
+    plane_sync<GENERAL>(P);  // no CTA of the cluster reads this CTA's strip any more
 
     // Fixed-order reduction of every class over its threads.
     float* red = sm + P.red;
@@ -1026,7 +1073,8 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
     static_assert(TC == 4, "4-column tiles");
     const int tid = threadIdx.x, nt = blockDim.x;
     const int c = blockIdx.x, g = blockIdx.y, G = P.groups;
-    const size_t plane_elems = (size_t)P.H * P.W;
+    const size_t plane_elems = (size_t)P.Hr * P.Wr;
+    const int myrows = real_rows(P, 0);
     auto csync = [&]() { __syncthreads(); };
     FusedCtx<K, T, true> cx{sm, P, dy, base_w, base_b, base_scale, wt_w, wt_scale, 0, 0, 0, plane_elems, 0};
 
@@ -1035,8 +1083,8 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
     cx.fold(c, nt, tid);  // the channel is fixed: dx weights folded once
     if (g < P.B) {
         const size_t off = ((size_t)g * P.C + c) * plane_elems;
-        stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
-        stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
+        stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
+        stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
     }
     cp_async_commit();
 
@@ -1089,15 +1137,15 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
             }
             if (prev_b >= 0 && P.L >= 1) {
                 T* yp = dx + ((size_t)prev_b * P.C + c) * plane_elems;
-                for (int t = tid; t < P.n_fin; t += nt) synth_item<T>(sm, P, yp, t);
+                for (int t = tid; t < P.n_fin; t += nt) synth_item<T, true>(sm, P, yp, t, myrows);
             }
             if (!have) break;
             __syncthreads();  // both analyses complete; the previous plane's Q and Y consumed
             // Phase B.
             if (b + G < P.B) {
                 const size_t off = ((size_t)(b + G) * P.C + c) * plane_elems;
-                stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
-                stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
+                stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
+                stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
             }
             cp_async_commit();
             if constexpr (!CORR) {
@@ -1117,8 +1165,8 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
                         const int h0 = job.row0;
                         conv_tile<K, TR, TC>(sm + job.win, job.wstride, w, make_float2(0.f, 0.f),
                                              [&](int o, float2(&a)[NP]) {
-                                                 if (h0 + o < P.H)
-                                                     gst4<T>(yo + (size_t)o * P.W,
+                                                 if (h0 + o < myrows)
+                                                     gst4<T>(yo + (size_t)o * P.Wr,
                                                              make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
                                              });
                     }

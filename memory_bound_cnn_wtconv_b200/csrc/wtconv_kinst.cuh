@@ -58,10 +58,10 @@ struct Launch {
     }
 };
 
-template <int TR, typename T, bool BWD, bool STRIPS>
+template <int TR, typename T, bool BWD, bool GENERAL>
 cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
     static bool done[kMaxDevices] = {};
-    auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD, STRIPS>;
+    auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD, GENERAL>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
     // Persistent grid: every resident CTA slot (cluster slot, for strips) of
@@ -91,10 +91,10 @@ cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <int TR, typename T, bool STRIPS>
+template <int TR, typename T, bool GENERAL>
 cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
     static bool done[kMaxDevices] = {};
-    auto* fn = wtconv_bwdw_partial_kernel<WTC_K, TR, 4, T, STRIPS>;
+    auto* fn = wtconv_bwdw_partial_kernel<WTC_K, TR, 4, T, GENERAL>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
     Launch L(P, dim3(P.C * P.nstrips, P.groups), s);
@@ -111,7 +111,9 @@ cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
 
 template <int TR, typename T>
 cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s) {
-    if (P.nstrips > 1) return bwd ? fused_typed<TR, T, true, true>(P, a, s) : fused_typed<TR, T, false, true>(P, a, s);
+    // The general instantiation for cluster strips and / or planes padded on chip.
+    if (P.nstrips > 1 || P.padded)
+        return bwd ? fused_typed<TR, T, true, true>(P, a, s) : fused_typed<TR, T, false, true>(P, a, s);
     return bwd ? fused_typed<TR, T, true, false>(P, a, s) : fused_typed<TR, T, false, false>(P, a, s);
 }
 
@@ -136,7 +138,7 @@ cudaError_t fused_tr(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cud
 
 template <int TR>
 cudaError_t bwdw_tr(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
-    const bool strips = P.nstrips > 1;
+    const bool strips = P.nstrips > 1 || P.padded;  // the general instantiation
     if (dtype == 0) return strips ? bwdw_typed<TR, float, true>(P, a, s) : bwdw_typed<TR, float, false>(P, a, s);
     return strips ? bwdw_typed<TR, __nv_bfloat16, true>(P, a, s) : bwdw_typed<TR, __nv_bfloat16, false>(P, a, s);
 }

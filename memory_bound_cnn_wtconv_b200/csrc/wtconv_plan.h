@@ -80,6 +80,12 @@ struct Plan {
     // neighbouring strips' halo rows).  Hp is the plane height.
     int B, C, H, W, k, L, p;
     int Hp, nstrips;
+    // The plane in global memory is Hr x Wr.  When Hr or Wr is not a multiple
+    // of 2^L the CTAs hold it zero-padded to Hp x W (multiples of 2^L; padded
+    // = 1): the real rows are staged row by row (row_chunks 16-byte chunks
+    // each) into staging rows of W elements, and only real outputs are
+    // stored.
+    int Hr, Wr, padded, row_chunks;
     int parts;           // weight gradient: partial vectors per channel (groups * nstrips)
     int TR, TC;          // output tile: TR rows x TC cols per thread (TC = 4: two column pairs)
     int esize;           // bytes per stored activation (4 or 2)
@@ -128,6 +134,7 @@ struct Plan {
     FastDiv div_rw;      // (W >> (pyr_lg + 2)): pyramid regions per row
     FastDiv div_q4;                 // W / 4: 4-column groups per row
     FastDiv div_w;                  // W
+    FastDiv div_rowc;               // row_chunks
     FastDiv div_m[kMaxL];           // W >> (l+1)
     FastDiv div_ntc[kMaxL + 1];     // tile columns per tile row
 };

@@ -105,11 +105,13 @@ inline wtconv_status_t validate(const wtconv_desc_t* d) {
     if (d->B <= 0 || d->C <= 0 || d->H <= 0 || d->W <= 0) return WTCONV_ERR_BAD_SHAPE;
     if (!is_supported_k(d->k)) return WTCONV_ERR_BAD_K;
     if (d->L < 0 || d->L > kMaxL) return WTCONV_ERR_BAD_L;
-    if ((d->H % (1 << d->L)) != 0 || (d->W % (1 << d->L)) != 0) return WTCONV_ERR_BAD_SHAPE;
     if ((d->W % 4) != 0) return WTCONV_ERR_BAD_SHAPE;
-    // Planes are staged in 16-byte chunks.
+    // Planes are staged in 16-byte chunks: whole planes if H and W are
+    // multiples of 2^L, else (zero-padded on chip) row by row.
     const long long esize = d->dtype == WTCONV_BF16 ? 2 : 4;
-    if (((long long)d->H * d->W * esize) % 16 != 0) return WTCONV_ERR_BAD_SHAPE;
+    const bool padded = (d->H % (1 << d->L)) != 0 || (d->W % (1 << d->L)) != 0;
+    if (padded ? ((long long)d->W * esize) % 16 != 0 : ((long long)d->H * d->W * esize) % 16 != 0)
+        return WTCONV_ERR_BAD_SHAPE;
     // Index arithmetic in the kernels is 32-bit within a plane and 64-bit across planes.
     if ((long long)d->H * d->W > (1LL << 30)) return WTCONV_ERR_BAD_SHAPE;
     if ((long long)d->B * d->C > (1LL << 31) - 1) return WTCONV_ERR_BAD_SHAPE;
@@ -124,14 +126,20 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // on-chip rows (H, ntr, buffers, tiles) describes one strip.
 inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, Plan* P) {
     memset(P, 0, sizeof(*P));
-    if (nstrips < 1 || nstrips > kMaxStrips || d->H % nstrips) return WTCONV_ERR_UNSUPPORTED;
+    // The plane the CTAs hold: H and W rounded up to multiples of 2^L.
+    const int m = 1 << d->L;
+    const int Hv = (d->H + m - 1) / m * m, Wv = (d->W + m - 1) / m * m;
+    if (nstrips < 1 || nstrips > kMaxStrips || Hv % nstrips) return WTCONV_ERR_UNSUPPORTED;
     if (kind == kBackward && nstrips != 1) return WTCONV_ERR_UNSUPPORTED;  // whole planes only
-    const int Hs = d->H / nstrips;
-    if (nstrips > 1 && (Hs % (1 << d->L) != 0 || Hs % 4 != 0)) return WTCONV_ERR_UNSUPPORTED;
-    P->B = d->B; P->C = d->C; P->H = Hs; P->W = d->W; P->k = d->k; P->L = d->L;
-    P->Hp = d->H;
+    const int Hs = Hv / nstrips;
+    if (nstrips > 1 && (Hs % m != 0 || Hs % 4 != 0)) return WTCONV_ERR_UNSUPPORTED;
+    P->B = d->B; P->C = d->C; P->H = Hs; P->W = Wv; P->k = d->k; P->L = d->L;
+    P->Hp = Hv;
+    P->Hr = d->H;
+    P->Wr = d->W;
+    P->padded = (Hv != d->H || Wv != d->W) ? 1 : 0;
     P->nstrips = nstrips;
-    const int p = d->k / 2, k = d->k, L = d->L, H = Hs, W = d->W, KK = k * k;
+    const int p = d->k / 2, k = d->k, L = d->L, H = Hs, W = Wv, KK = k * k;
     P->p = p;
     P->esize = d->dtype == WTCONV_BF16 ? 2 : 4;
     P->TC = 4;
@@ -200,11 +208,13 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         P->DY.base = (int)off;
         off += round4(rows * P->DY.stride);
     }
-    // Staging of the next plane(s), stored format.
+    // Staging of the next plane(s), stored format (W elements per row).
     {
         const long long bytes = (long long)H * W * P->esize;
         P->plane_chunks = (int)(bytes / 16);
         P->stg_floats = (int)(bytes / 4);
+        P->row_chunks = (int)((long long)P->Wr * P->esize / 16);
+        P->div_rowc = make_fastdiv(std::max(P->row_chunks, 1));
         P->stg = (int)off;
         off += (kind == kBackwardWeight || kind == kBackward ? 2LL : 1LL) * P->stg_floats;
     }

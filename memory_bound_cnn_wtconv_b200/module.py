@@ -68,7 +68,8 @@ class WTConv2d(torch.nn.Module):
     wt_w [L,C,4,k,k], wt_scale [L,C,4].  Initialisation (the pages give none):
     base_w and wt_w uniform in +-1/k like a depthwise ``nn.Conv2d``, base_b 0,
     base_scale 1, wt_scale 0.1.  Inputs: float32 or bfloat16 CUDA tensors,
-    H and W divisible by 2^levels, W a multiple of 4.
+    W a multiple of 4 (8 for bfloat16 when H or W is not a multiple of
+    2^levels; such planes are zero-padded on chip and cropped).
     """
 
     def __init__(self, channels: int, kernel_size: int = 5, levels: int = 1, device=None):

@@ -27,6 +27,7 @@ using namespace wtc;
 namespace {
 
 enum : int { ZERO = 0, WTS = 1, BIAS = 2, XT = 3, DYT = 4, ZT = 5, YT = 6, RED = 7 };
+int g_rank = 0;  // strip of the CTA being replayed (the analysis replays read it)
 int s_tag(int l, int s) { return 100 + 4 * l + s; }
 int q_tag(int l, int s) { return 200 + 4 * l + s; }
 int ss_tag(int l, int s) { return 300 + 4 * l + s; }
@@ -75,15 +76,38 @@ void check_global(long long idx, long long n, const char* what) {
 
 // Replays stage_plane: 16-byte chunk ch of this CTA's rows (strip `rank`) of
 // the stored plane -> staging floats [stg + 4ch, stg + 4ch + 4).
+int real_rows_host(const Plan& P, int rank) { return std::max(0, std::min(P.H, P.Hr - rank * P.H)); }
+
 void replay_stage(Shadow& sh, const Plan& P, long long stg, int tag, int rank) {
     const long long strip_bytes = (long long)P.H * P.W * P.esize;
-    const long long plane_bytes = (long long)P.Hp * P.W * P.esize;
+    const long long plane_bytes = (long long)P.Hr * P.Wr * P.esize;
     if (P.plane_chunks * 16LL != strip_bytes) sh.fail("strip is not a whole number of 16-byte chunks", strip_bytes);
     if (stg % 4) sh.fail("staging not 16-byte aligned", stg);
-    for (int ch = 0; ch < P.plane_chunks; ++ch) {
-        check_global(rank * strip_bytes + 16LL * ch + 15, plane_bytes, "staging source");
-        for (int e = 0; e < 4; ++e) sh.write(stg + 4LL * ch + e, stg, stg + P.stg_floats, tag, "staging");
+    if (!P.padded) {
+        if (P.Hr != P.Hp || P.Wr != P.W) sh.fail("unpadded plan with padded sizes", P.Hr);
+        for (int ch = 0; ch < P.plane_chunks; ++ch) {
+            check_global(rank * strip_bytes + 16LL * ch + 15, plane_bytes, "staging source");
+            for (int e = 0; e < 4; ++e) sh.write(stg + 4LL * ch + e, stg, stg + P.stg_floats, tag, "staging");
+        }
+        return;
     }
+    // Row by row: the real rows of this strip, Wr elements each, into staging rows of W.
+    const int rows = real_rows_host(P, rank), rc = P.row_chunks;
+    if ((long long)rc * 16 != (long long)P.Wr * P.esize) sh.fail("row chunks", rc);
+    for (int ch = 0; ch < rows * rc; ++ch) {
+        const int r = (int)fastdiv_host(ch, P.div_rowc), c = ch - r * rc;
+        if (r != ch / rc) sh.fail("row-chunk division", ch);
+        const long long src = ((long long)rank * P.H + r) * P.Wr * P.esize + 16LL * c;
+        check_global(src + 15, plane_bytes, "staging source");
+        const long long dst = stg + ((long long)r * P.W * P.esize + 16LL * c) / 4;
+        for (int e = 0; e < 4; ++e) sh.write(dst + e, stg, stg + P.stg_floats, tag, "staging");
+    }
+}
+
+// Tag a staged element (virtual row r, column col of this strip) must carry:
+// the staging tag where the plane has data, zero in the on-chip padding.
+int staged_tag(const Plan& P, int rank, int r, int col, int stag) {
+    return (r < real_rows_host(P, rank) && col < P.Wr) ? stag : ZERO;
 }
 
 // Replays unpack_level0: staged element e (4 at a time) -> dst (element (0,0) at `dst`, row stride ds),
@@ -96,7 +120,8 @@ void replay_unpack(Shadow& sh, const Plan& P, long long stg, int stag, long long
         if (e % 4) sh.fail("staged load not 4-element aligned", e);
         const long long f0 = stg + (long long)e * P.esize / 4;
         const int nf = P.esize;  // 4 elements = esize floats
-        for (int q = 0; q < nf; ++q) sh.read(f0 + q, stg, stg + P.stg_floats, stag, "staging read");
+        const int t = staged_tag(P, g_rank, e / W, e % W, stag);
+        for (int q = 0; q < nf; ++q) sh.read(f0 + q, stg, stg + P.stg_floats, t, "staging read");
     };
     const int rows = level0 ? P.H / 2 : P.H;
     for (int i = 0; i < rows; ++i)
@@ -138,7 +163,8 @@ void replay_pyramid(Shadow& sh, const Plan& P, long long stg, int stag, long lon
         const int r0 = 4 * brow, c0 = 4 * bcol;
         for (int q = 0; q < 4; ++q) {
             const long long f0 = stg + (long long)((r0 + q) * W + c0) * P.esize / 4;
-            for (int e = 0; e < P.esize; ++e) sh.read(f0 + e, stg, stg + P.stg_floats, stag, "pyramid staging read");
+            const int t = staged_tag(P, g_rank, r0 + q, c0, stag);
+            for (int e = 0; e < P.esize; ++e) sh.read(f0 + e, stg, stg + P.stg_floats, t, "pyramid staging read");
             for (int e = 0; e < 4; ++e) sh.write(dst + (long long)(r0 + q) * ds + c0 + e, dlo, dhi, dtag, "pyramid plane store");
         }
         auto lvl_store = [&](int l, int i, int j) {
@@ -344,7 +370,7 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     for (int cl = 0; cl < ncls; ++cl)
         if ((P.wbase + cl * P.wcls) % 4) shs[0].fail("weight class not 16-byte aligned", P.wbase + cl * P.wcls);
     const int ntc = P.ntc[kMaxL];
-    const long long plane = (long long)P.Hp * W;
+    const long long plane = (long long)P.Hr * P.Wr;
 
     // Phase A's synthesis of the previous plane: rows 2i, 2i+1 x columns 4q..4q+3.
     auto synthesis = [&](Shadow& sh, int rank) {
@@ -372,9 +398,10 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
             for (int rr = 0; rr < 2; ++rr) {
                 const long long a = P.Y.base + (long long)(2 * i + rr) * P.Y.stride + 4 * q;
                 if (a % 4) sh.fail("Y load not 16-byte aligned", a);
+                const bool store = 2 * i + rr < real_rows_host(P, rank) && 4 * q < P.Wr;
                 for (int e = 0; e < 4; ++e) {
                     sh.read(a + e, ylo, yhi, YT, "Y read");
-                    check_global((long long)(rank * H + 2 * i + rr) * W + 4 * q + e, plane, "y store");
+                    if (store) check_global((long long)(rank * H + 2 * i + rr) * P.Wr + 4 * q + e, plane, "y store");
                 }
             }
         }
@@ -405,6 +432,7 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
             // at a time); the synthesis runs after its last one.
             for (int r = 0; r < NS; ++r) {
                 shs[r].phase = "A: analysis";
+                g_rank = r;
                 const int e0 = shs[r].epoch;
                 replay_analyse(shs[r], P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi,
                                XT, P.S, p, s_tag);
@@ -471,9 +499,9 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
                 } else {
                     for (int o = 0; o < TR; ++o) {
                         const int h = tr * TR + o;
-                        if (h >= H) continue;
+                        if (h >= real_rows_host(P, r)) continue;
                         for (int e = 0; e < TC; ++e)
-                            check_global((long long)(r * H + h) * W + tc * TC + e, plane, "y store");
+                            check_global((long long)(r * H + h) * P.Wr + tc * TC + e, plane, "y store");
                     }
                 }
             }
@@ -516,6 +544,7 @@ void check_bwdw(const wtconv_desc_t& d) {
         for (int r = 0; r < NS; ++r) {
             Shadow& sh = shs[r];
             sh.phase = "analysis";
+            g_rank = r;
             const int e0 = sh.epoch;
             replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S,
                            p, s_tag);
@@ -636,7 +665,7 @@ void check_bwd(const wtconv_desc_t& d) {
     const long long slo = P.XS.base, shi = P.XS.base + (long long)xrows * P.XS.stride;
     const long long ylo = P.Y.base, yhi = P.Y.base + (long long)P.ntr[kMaxL] * TR * P.Y.stride;
     const int align = (p % 2 == 0) ? 2 : 1;
-    const long long plane = (long long)P.Hp * W;
+    const long long plane = (long long)P.Hr * P.Wr;
     // Weights folded once (before the first barrier), then the first pair staged.
     sh.phase = "fold";
     for (int cl = 0; cl < ncls; ++cl)
@@ -664,7 +693,8 @@ void check_bwd(const wtconv_desc_t& d) {
             for (int rr = 0; rr < 2; ++rr)
                 for (int e = 0; e < 4; ++e) {
                     sh.read(P.Y.base + (long long)(2 * i + rr) * P.Y.stride + 4 * q + e, ylo, yhi, YT, "Y");
-                    check_global((long long)(2 * i + rr) * W + 4 * q + e, plane, "dx store");
+                    if (2 * i + rr < P.Hr && 4 * q < P.Wr)
+                        check_global((long long)(2 * i + rr) * P.Wr + 4 * q + e, plane, "dx store");
                 }
         }
     };
@@ -672,6 +702,7 @@ void check_bwd(const wtconv_desc_t& d) {
         sh.barrier();
         if (plane_i < 2) {
             sh.phase = "A: analysis of x and dy";
+            g_rank = 0;
             const int e0 = sh.epoch;
             replay_analyse(sh, P, P.stg, XT + 10, P.XS.base + (long long)p * P.XS.stride + p, P.XS.stride, slo, shi, XT,
                            P.SS, p, ss_tag);
@@ -720,8 +751,9 @@ void check_bwd(const wtconv_desc_t& d) {
                     for (int e = 0; e < TC; ++e) sh.write(yo + (long long)o * P.Y.stride + e, ylo, yhi, YT, "Y tile");
             } else {
                 for (int o = 0; o < TR; ++o)
-                    if (tr * TR + o < H)
-                        for (int e = 0; e < TC; ++e) check_global((long long)(tr * TR + o) * W + tc * TC + e, plane, "dx store");
+                    if (tr * TR + o < P.Hr)
+                        for (int e = 0; e < TC; ++e)
+                            check_global((long long)(tr * TR + o) * P.Wr + tc * TC + e, plane, "dx store");
             }
         }
         sh.phase = "B: correlation tiles";

@@ -51,11 +51,17 @@ def _fwd(lib, d, x=FAKE, y=FAKE, ww=FAKE, ws=FAKE):
     (dict(B=0), BAD_SHAPE), (dict(C=-1), BAD_SHAPE), (dict(H=0), BAD_SHAPE),
     (dict(k=4), BAD_K), (dict(k=9), BAD_K), (dict(k=0), BAD_K),
     (dict(L=-1), BAD_L), (dict(L=7), BAD_L),
-    (dict(H=12, L=3), BAD_SHAPE), (dict(W=20, L=3), BAD_SHAPE), (dict(W=6, L=1), BAD_SHAPE),
+    (dict(W=6, L=1), BAD_SHAPE), (dict(H=12, W=12, L=3, dtype=1), BAD_SHAPE),
     (dict(dtype=2), DTYPE),
 ])
 def test_forward_validation(cuda_lib, kw, code):
     assert _fwd(cuda_lib, _desc(**kw)) == code
+
+
+@pytest.mark.parametrize("kw", [dict(H=12, L=3), dict(W=20, L=3), dict(H=13, W=12, L=2), dict(H=9, W=16, L=4, dtype=1)])
+def test_sizes_not_multiples_of_2L_are_planned(cuda_lib, kw):
+    # Zero-padded on chip (host planning only; nothing is launched here).
+    assert cuda_lib.wtconv_workspace_bytes(ctypes.byref(_desc(**kw))) > 0
 
 
 def test_null_and_alignment(cuda_lib):

@@ -153,6 +153,13 @@ SMALL = [
     Case("strips_256_L4", 1, 1, 256, 256, 5, 4, "f32", 28, "normal", "normal"),
     Case("strips_256_L3_k3", 2, 1, 256, 256, 3, 3, "f32", 29, "normal", "normal"),
     Case("strips_256_L2_bf16", 1, 2, 256, 256, 5, 2, "bf16", 30, "normal", "normal"),
+    # H or W not a multiple of 2^L: zero-padded on chip, real outputs only.
+    Case("pad_13x12_L2", 2, 3, 13, 12, 5, 2, "f32", 31, "normal", "normal"),
+    Case("pad_20x16_k3_L3", 2, 3, 20, 16, 3, 3, "f32", 32, "normal", "normal"),
+    Case("pad_9x8_k7_L4", 1, 2, 9, 8, 7, 4, "f32", 33, "normal", "normal"),
+    Case("pad_17x8_k3_L1", 2, 3, 17, 8, 3, 1, "f32", 34, "normal", "normal"),
+    Case("pad_bf16_13x16", 2, 3, 13, 16, 5, 2, "bf16", 35, "uniform", "normal"),
+    Case("pad_strips_250x248", 1, 1, 250, 248, 5, 4, "f32", 36, "normal", "normal"),
 ]
 
 

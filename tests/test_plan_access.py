@@ -19,6 +19,9 @@ EDGE = [
     (1, 2, 32, 32, 3, 4, 0), (1, 2, 64, 64, 5, 4, 0), (1, 2, 12, 8, 1, 0, 0), (1, 2, 4, 4, 7, 2, 0),
     (2, 2, 8, 4, 3, 2, 1), (1, 1, 64, 4, 7, 2, 0), (5, 3, 20, 12, 5, 2, 1), (1, 1, 2, 4, 3, 1, 0),
     (1, 1, 64, 64, 7, 6, 0), (1, 1, 4, 4, 1, 1, 1),
+    # not multiples of 2^L (zero-padded on chip), incl. strips
+    (2, 3, 13, 12, 5, 2, 0), (2, 3, 20, 16, 3, 3, 0), (1, 2, 9, 8, 7, 4, 0), (2, 3, 17, 8, 3, 1, 0),
+    (2, 3, 13, 16, 5, 2, 1), (1, 1, 250, 248, 5, 4, 0), (3, 2, 30, 28, 5, 3, 0), (1, 1, 100, 40, 5, 3, 1),
 ]
 
 
