@@ -16,14 +16,21 @@
 // term  2^-(l+1) * Shat_{l,s}  that the closed-form synthesis adds.
 //
 // Depthwise convolution is not a dense contraction, so the convs run on the
-// FP32 pipes.  They are issue-bound, so every conv uses the packed f32x2 FMA
-// (64 multiply-adds per warp instruction): a thread owns a TR x 4 output tile
-// as TR x 2 column pairs, streams its window's TR+K-1 input rows from shared
-// memory once with 128-bit loads, and keeps the K*K folded weights in
-// registers.
+// FP32 pipes, with the packed f32x2 FMA (64 multiply-adds per warp
+// instruction, half the issue slots of scalar FMAs): a thread owns a TR x 4
+// output tile as TR x 2 column pairs, streams its window's TR+K-1 input rows
+// from shared memory once with 128-bit loads, and keeps the K*K folded
+// weights in registers.
 //
 // CTAs are persistent: each walks a run of planes; while it computes one
-// plane, cp.async copies the next one from HBM into a staging buffer.
+// plane, cp.async copies the next one from HBM into a staging buffer.  Per
+// plane, a phase of on-chip analysis (and of the previous plane's synthesis)
+// and a phase of conv tiles, separated by CTA barriers (cluster barriers when
+// a plane is split into strips across a thread-block cluster).
+//
+// Kernels: wtconv_fused_kernel (forward; input gradient with BWD),
+// wtconv_bwdw_partial_kernel (weight gradient, with its final step in the
+// tail) and wtconv_backward_kernel (input and weight gradients in one pass).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -504,10 +511,6 @@ __device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const f
                    sm + s1.base + pad * s1.stride + pad, s1.stride, s1.sub, ptid, np);
     }
     return sum;
-}
-
-__device__ __forceinline__ void named_barrier(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------------------
