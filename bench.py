@@ -421,7 +421,7 @@ def run_ours(args, case):
         line["clocks"] = clk
 
     if not args.no_e2e:
-        line["e2e"] = e2e(args, case, g, y, dx, grads, ws, dev, stream, world, calls)
+        line["e2e"] = e2e(args, case, g, grads, ws, dev, world)
     if world > 1:
         dist.barrier()
     # The one-pass backward (wtconv_backward), timed after the step with the
@@ -461,40 +461,78 @@ def run_ours(args, case):
     return 0
 
 
-def e2e(args, case, g, y, dx, grads, ws, dev, stream, world, calls):
-    """Same metric through the public API with host buffers: pinned host ->
-    device copies of x and dy, the three calls, device -> host copies of y,
-    dx and the gradients, every step."""
+def e2e(args, case, g, grads, ws, dev, world):
+    """Same metric through the public API with host buffers: every step copies
+    x and dy from pinned host memory to the device, runs the three calls (and,
+    with several ranks, the gradient all-reduce), and copies y, dx and the
+    gradients back.  Steps are pipelined over three streams (inputs, compute,
+    results) with two device buffer sets, so one step's copies in and out
+    overlap the neighbouring steps' compute; events keep every buffer from
+    being overwritten before its last reader is done."""
     import torch
     import torch.distributed as dist
 
+    import memory_bound_cnn_wtconv_b200 as wt
+
+    L = case.L
     xh = g["x"].cpu().pin_memory()
     dyh = g["dy"].cpu().pin_memory()
     yh = torch.empty_like(xh).pin_memory()
     dxh = torch.empty_like(dyh).pin_memory()
     gh = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()}
-    K = args.e2e_steps
+    bufs = [dict(x=torch.empty_like(g["x"]), dy=torch.empty_like(g["dy"]), y=torch.empty_like(g["x"]),
+                 dx=torch.empty_like(g["dy"]), grads={k: torch.empty_like(v) for k, v in grads.items()})
+            for _ in range(2)]
+    flat = torch.empty(sum(v.numel() for v in grads.values()), device=dev)
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    done = {"in": [None, None], "comp": [None, None], "out": [None, None]}
 
-    def step():
-        g["x"].copy_(xh, non_blocking=True)
-        g["dy"].copy_(dyh, non_blocking=True)
-        for name, f in calls:
-            f()
-        yh.copy_(y, non_blocking=True)
-        dxh.copy_(dx, non_blocking=True)
-        for k in grads:
-            gh[k].copy_(grads[k], non_blocking=True)
+    def mark(kind, b, strm):
+        e = torch.cuda.Event()
+        e.record(strm)
+        done[kind][b] = e
 
-    for _ in range(3):
-        step()
+    def step(i):
+        b = i % 2
+        d = bufs[b]
+        with torch.cuda.stream(s_in):
+            if done["comp"][b] is not None:
+                s_in.wait_event(done["comp"][b])  # step i-2 no longer reads x, dy of this set
+            d["x"].copy_(xh, non_blocking=True)
+            d["dy"].copy_(dyh, non_blocking=True)
+            mark("in", b, s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(done["in"][b])
+            if done["out"][b] is not None:
+                s_comp.wait_event(done["out"][b])  # step i-2's results are on the host
+            wt.forward(d["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L, y=d["y"],
+                       stream=s_comp)
+            wt.backward_input(d["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], L, dx=d["dx"],
+                              stream=s_comp)
+            wt.backward_weight(d["x"], d["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"],
+                               L, grads=d["grads"], workspace=ws, stream=s_comp)
+            if world > 1:
+                allreduce_weight_grads(d["grads"], flat, dist)
+            mark("comp", b, s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done["comp"][b])
+            yh.copy_(d["y"], non_blocking=True)
+            dxh.copy_(d["dx"], non_blocking=True)
+            for k in gh:
+                gh[k].copy_(d["grads"][k], non_blocking=True)
+            mark("out", b, s_out)
+
+    for i in range(3):
+        step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    K = args.e2e_steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(K):
+        step(i)
+    e1.record(s_out)
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / K
     if world > 1:
@@ -502,9 +540,10 @@ def e2e(args, case, g, y, dx, grads, ws, dev, stream, world, calls):
     step_bytes = sum(modeled_bytes(case).values())
     h2d = xh.numel() * xh.element_size() + dyh.numel() * dyh.element_size()
     d2h = yh.numel() * yh.element_size() + dxh.numel() * dxh.element_size() + sum(
-        v.numel() * 4 for v in gh.values())
+        v.numel() * v.element_size() for v in gh.values())
     return {"value": step_bytes * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "pipelined": "3 streams (copy in / compute / copy out), 2 device buffer sets"}
 
 
 # --------------------------------------------------------------------------
