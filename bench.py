@@ -93,8 +93,8 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
                   "wtconv_launch.h", "wtconv_api.cu", "wtconv_k1.cu", "wtconv_k3.cu", "wtconv_k5.cu", "wtconv_k7.cu")
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
-    ("stage1", "bwd_w"): (79.02336e6, "wtconv_bwdw_partial_kernel",
-                          "2ccd58ca3c396b12ccc0a389bc4b2ab8aa26480c11a07f8c6e62ab514febab89",
+    ("stage1", "bwd_w"): (79720448.0, "wtconv_bwdw_partial_kernel",
+                          "37f0608c88cbbd9daef299e2012956c733c14b5f2d7fcd3da6a4456b44e1a362",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 
