@@ -58,30 +58,21 @@ inline int ctas_per_sm(int smem_floats) {
     return std::max(1, std::min(2, kSmemPerSM / (smem_floats * 4 + 1024)));
 }
 
+// CTAs of `nthreads` threads one SM holds: the least of what its shared
+// memory, its 64K registers at the kernels' register cap (every launch bound
+// allows at most 128 registers a thread) and its 64 warps allow.
+inline int resident_ctas(int nthreads, int smem_floats) {
+    const int by_smem = kSmemPerSM / (smem_floats * 4 + 1024);
+    const int by_regs = 65536 / (std::max(nthreads, 32) * 128);
+    const int by_warps = 64 / std::max(ceil_div(nthreads, 32), 1);
+    return std::max(1, std::min(std::min(by_smem, by_regs), std::min(by_warps, 32)));
+}
+
 // Weight-gradient batch groups (grid.y): the CTA of group g walks planes
 // b = g, g + groups, ...  Chosen to minimise waves x planes-per-CTA over the
 // resident CTA slots, with at most 64 planes per CTA so every per-thread
 // running sum stays short.
-inline int pick_groups(int B, int C, int smem_floats) {
-    const long long slots = (long long)kNumSMs * ctas_per_sm(smem_floats);
-    int best = 1;
-    long long best_cost = -1;
-    for (int g = 1; g <= B; ++g) {
-        const int planes = ceil_div(B, g);
-        if (planes > 64 && g != B) continue;
-        const long long waves = (C * (long long)g + slots - 1) / slots;
-        const long long cost = waves * (planes + 1);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = g;
-        }
-    }
-    return best;
-}
-
-// Batch groups for the fused backward (one 512-thread CTA per SM).
-inline int pick_groups_one(int B, int C) {
-    const long long slots = kNumSMs;
+inline int pick_groups(int B, int C, long long slots) {
     int best = 1;
     long long best_cost = -1;
     for (int g = 1; g <= B; ++g) {
@@ -313,7 +304,8 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;
     if (kind == kBackwardWeight || kind == kBackward) {
-        P->groups = kind == kBackward ? pick_groups_one(P->B, P->C) : pick_groups(P->B, P->C * nstrips, P->smem_floats);
+        const long long slots = (long long)kNumSMs * resident_ctas(P->nthreads, P->smem_floats);
+        P->groups = pick_groups(P->B, P->C * nstrips, slots);
         P->parts = P->groups * nstrips;
     } else {
         const long long units = (long long)P->B * P->C;
