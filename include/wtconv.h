@@ -76,7 +76,7 @@ typedef enum {
     WTCONV_ERR_MISALIGNED = 5,  /* an activation pointer is not 16-byte aligned */
     WTCONV_ERR_DTYPE = 6,       /* unknown activation dtype */
     WTCONV_ERR_WORKSPACE = 7,   /* workspace missing or smaller than wtconv_workspace_bytes() */
-    WTCONV_ERR_UNSUPPORTED = 8, /* valid shape that this build cannot stage on chip */
+    WTCONV_ERR_UNSUPPORTED = 8, /* valid shape whose plane (or strip) does not fit on chip */
     WTCONV_ERR_CUDA = 9         /* a CUDA runtime call or kernel launch failed */
 } wtconv_status_t;
 

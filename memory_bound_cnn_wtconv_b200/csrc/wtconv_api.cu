@@ -80,7 +80,7 @@ const char* wtconv_status_string(wtconv_status_t s) {
         case WTCONV_ERR_MISALIGNED: return "activation pointer not 16-byte aligned";
         case WTCONV_ERR_DTYPE: return "unknown activation dtype";
         case WTCONV_ERR_WORKSPACE: return "workspace missing or too small";
-        case WTCONV_ERR_UNSUPPORTED: return "plane too large to stage on chip for this build";
+        case WTCONV_ERR_UNSUPPORTED: return "plane too large to stage on chip";
         case WTCONV_ERR_CUDA: return "CUDA runtime error";
     }
     return "unknown status";
