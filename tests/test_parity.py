@@ -160,6 +160,12 @@ SMALL = [
     Case("pad_17x8_k3_L1", 2, 3, 17, 8, 3, 1, "f32", 34, "normal", "normal"),
     Case("pad_bf16_13x16", 2, 3, 13, 16, 5, 2, "bf16", 35, "uniform", "normal"),
     Case("pad_strips_250x248", 1, 1, 250, 248, 5, 4, "f32", 36, "normal", "normal"),
+    # deepest levels, bf16 with k = 7, and one channel over many batch elements
+    Case("L5_32_k3", 1, 2, 32, 32, 3, 5, "f32", 37, "normal", "normal"),
+    Case("bf16_k7_L3", 2, 2, 24, 24, 7, 3, "bf16", 38, "uniform", "normal"),
+    Case("one_channel_130_planes", 130, 1, 16, 16, 5, 2, "f32", 39, "normal", "normal"),
+    Case("pad_40x36_L6", 1, 2, 40, 36, 5, 6, "f32", 40, "normal", "normal"),
+    Case("pad_60x64_k3_L6", 2, 1, 60, 64, 3, 6, "f32", 41, "normal", "normal"),
 ]
 
 

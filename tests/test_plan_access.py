@@ -22,6 +22,9 @@ EDGE = [
     # not multiples of 2^L (zero-padded on chip), incl. strips
     (2, 3, 13, 12, 5, 2, 0), (2, 3, 20, 16, 3, 3, 0), (1, 2, 9, 8, 7, 4, 0), (2, 3, 17, 8, 3, 1, 0),
     (2, 3, 13, 16, 5, 2, 1), (1, 1, 250, 248, 5, 4, 0), (3, 2, 30, 28, 5, 3, 0), (1, 1, 100, 40, 5, 3, 1),
+    # deepest levels, bf16 with k = 7, one channel over many batch elements, padded L = 6
+    (1, 2, 32, 32, 3, 5, 0), (2, 2, 24, 24, 7, 3, 1), (130, 1, 16, 16, 5, 2, 0), (1, 2, 40, 36, 5, 6, 0),
+    (2, 1, 60, 64, 3, 6, 0), (1, 1, 70, 68, 5, 6, 0),
 ]
 
 
