@@ -94,7 +94,7 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
     ("stage1", "bwd_w"): (78782720.0, "wtconv_bwdw_partial_kernel",
-                          "73d18c1dd579293705f061ef8a57186658709e956126d1c39873e42250e0dd00",
+                          "2cf8626a8eee8fd44321918112b9e6e3f36b0a38360dc6c752e6816ca2159883",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 

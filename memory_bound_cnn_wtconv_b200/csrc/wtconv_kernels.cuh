@@ -399,8 +399,26 @@ __device__ __forceinline__ void conv_tile(const float* __restrict__ win, int str
     }
 }
 
-// Correlation of one TR x TC tile of D with the K x K shifts of S, split by
-// column parity (sum the two halves at the end):
+// Correlation sums of one thread: split by column parity (float2, the even
+// taps as packed FMAs) for K <= 5; one float per tap for K = 7, whose 49
+// float2 sums would not fit the register budget beside the D tile.
+template <int K>
+struct CorrAcc {
+    using type = float2;
+};
+template <>
+struct CorrAcc<7> {
+    using type = float;
+};
+__device__ __forceinline__ float acc_total(float2 a) { return a.x + a.y; }
+__device__ __forceinline__ float acc_total(float a) { return a; }
+template <class A>
+__device__ __forceinline__ A acc_zero() {
+    if constexpr (std::is_same_v<A, float2>) return make_float2(0.f, 0.f); else return 0.f;
+}
+
+// Correlation of one TR x TC tile of D with the K x K shifts of S (float2
+// sums split by column parity: sum the two halves at the end):
 //   acc[u*K+v] += sum_{o<TR, j<TC} D[o][j] * S[o+u][j+v]
 // `swin` is the S window origin (element (r0-p, c0-p)), `dt` the D tile origin.
 // D rows load as 128-bit (DLD = 4) or 64-bit pairs (2; the faster of the two
@@ -408,7 +426,8 @@ __device__ __forceinline__ void conv_tile(const float* __restrict__ win, int str
 // sits at an odd float offset (the interior of a padded buffer, p odd).
 template <int K, int TR, int TC, int DLD>
 __device__ __forceinline__ void corr_tile(const float* __restrict__ swin, int sstride,
-                                          const float* __restrict__ dt, int dstride, float2 (&acc)[K * K]) {
+                                          const float* __restrict__ dt, int dstride,
+                                          typename CorrAcc<K>::type (&acc)[K * K]) {
     constexpr int NP = TC / 2;
     constexpr int NW2 = (TC + K - 1) / 2;
     float2 d[TR][NP];
@@ -439,10 +458,24 @@ __device__ __forceinline__ void corr_tile(const float* __restrict__ swin, int ss
             if (o >= 0 && o < TR) {
 #pragma unroll
                 for (int v = 0; v < K; ++v) {
-                    float2 a = acc[u * K + v];
+                    if constexpr (std::is_same_v<typename CorrAcc<K>::type, float2>) {
+                        float2 a = acc[u * K + v];
 #pragma unroll
-                    for (int jp = 0; jp < NP; ++jp) a = ctap<NW2>(a, d[o][jp], row, jp, v);
-                    acc[u * K + v] = a;
+                        for (int jp = 0; jp < NP; ++jp) a = ctap<NW2>(a, d[o][jp], row, jp, v);
+                        acc[u * K + v] = a;
+                    } else {
+                        float a = acc[u * K + v];
+#pragma unroll
+                        for (int jp = 0; jp < NP; ++jp) {
+                            // input columns 2jp+v and 2jp+v+1 of the window row
+                            const int c = 2 * jp + v;
+                            const float s0 = (c & 1) ? row.e[c >> 1].y : row.e[c >> 1].x;
+                            const float s1 = (c & 1) ? row.e[(c + 1) >> 1].x : row.e[(c + 1) >> 1].y;
+                            a = fmaf(d[o][jp].x, s0, a);
+                            a = fmaf(d[o][jp].y, s1, a);
+                        }
+                        acc[u * K + v] = a;
+                    }
                 }
             }
         }
@@ -981,9 +1014,10 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
         cnt = min(P.tpt, P.cls_tiles[cl] - first);
     }
     const int lvl = cl <= 0 ? kMaxL : ((cl - 1) >> 2);
-    float2 acc[KK];
+    using Acc = typename CorrAcc<K>::type;
+    Acc acc[KK];
 #pragma unroll
-    for (int t = 0; t < KK; ++t) acc[t] = make_float2(0.f, 0.f);
+    for (int t = 0; t < KK; ++t) acc[t] = acc_zero<Acc>();
     float sdy = 0.f, sdy_c = 0.f;  // compensated running sum of dy over the walk
 
     float* X0 = sm + P.X.base + p * P.X.stride + p;
@@ -1027,7 +1061,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
     // Fixed-order reduction of every class over its threads.
     float* red = sm + P.red;
 #pragma unroll
-    for (int t = 0; t < KK; ++t) red[tid * KK + t] = acc[t].x + acc[t].y;
+    for (int t = 0; t < KK; ++t) red[tid * KK + t] = acc_total(acc[t]);
     // sum dy: a fixed xor-tree inside each warp, then the warps in order.
     float sw = sdy;
 #pragma unroll
@@ -1116,9 +1150,10 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
             cnt = min(P.tpt, P.cls_tiles[cl] - first);
         }
         const int lvl = cl <= 0 ? kMaxL : ((cl - 1) >> 2);
-        float2 acc[CORR ? KK : 1];
+        using Acc = typename CorrAcc<K>::type;
+        Acc acc[CORR ? KK : 1];
 #pragma unroll
-        for (int t = 0; t < (CORR ? KK : 1); ++t) acc[t] = make_float2(0.f, 0.f);
+        for (int t = 0; t < (CORR ? KK : 1); ++t) acc[t] = acc_zero<Acc>();
 
         int prev_b = -1;
         for (int b = g;; b += G) {
@@ -1199,7 +1234,7 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
         if constexpr (CORR) {
             if (ct < ncorr) {
 #pragma unroll
-                for (int t = 0; t < KK; ++t) red[ct * KK + t] = acc[t].x + acc[t].y;
+                for (int t = 0; t < KK; ++t) red[ct * KK + t] = acc_total(acc[t]);
             }
         }
     };
