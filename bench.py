@@ -59,6 +59,10 @@ def parse():
     ap.add_argument("--compare-only", default="", help="with --compare: only the implementation named so")
     ap.add_argument("--profile-one-forward", action="store_true",
                     help="with --compare: run one forward per implementation between profiler start/stop")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the three calls at every point of the 128-point shape sweep (one JSON line each)")
+    ap.add_argument("--sweep-steps", type=int, default=20, help="with --sweep: timed calls per point")
+    ap.add_argument("--sweep-points", default="", help="with --sweep: a range of point indices, e.g. 0:32")
     return ap.parse_args()
 
 
@@ -688,8 +692,78 @@ def run_compare(args, case):
     return 0
 
 
+def run_sweep(args):
+    """Per-call device time (CUDA events, L2 flushed before every call) of the
+    forward, input gradient and weight gradient at each sweep point; one JSON
+    line per point, then a summary line.  One GPU."""
+    import torch
+
+    import memory_bound_cnn_wtconv_b200 as wt
+    from wtconv_inputs import make_inputs, sweep_cases
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wt.load_library()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cases = sweep_cases()
+    if args.sweep_points:
+        a, b = (int(v) if v else None for v in args.sweep_points.split(":"))
+        cases = cases[a:b]
+    peak, peak_kind = hbm_peak()
+    alu_peak = 148 * 128 * 2 * 1965e6
+    rows = []
+    for case in cases:
+        g = {k: v.to(dev) for k, v in make_inputs(case).items()}
+        L = case.L
+        y, dx = torch.empty_like(g["x"]), torch.empty_like(g["dy"])
+        grads = {k: torch.empty_like(g[k]) for k in ("base_w", "base_b", "base_scale", "wt_w", "wt_scale")}
+        ws = torch.empty(max(16, wt.workspace_bytes(g["x"].shape, case.k, L, g["x"].dtype)), dtype=torch.uint8,
+                         device=dev)
+        calls = {
+            "fwd": lambda: wt.forward(g["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
+                                      y=y, stream=stream),
+            "bwd_in": lambda: wt.backward_input(g["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
+                                                dx=dx, stream=stream),
+            "bwd_w": lambda: wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"],
+                                                g["wt_scale"], L, grads=grads, workspace=ws, stream=stream),
+        }
+        us = {}
+        for name, f in calls.items():
+            for _ in range(3):
+                f()
+            ev = []
+            for _ in range(args.sweep_steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                f()
+                e1.record(stream)
+                ev.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            us[name] = sorted(a.elapsed_time(b) for a, b in ev)[len(ev) // 2] * 1e3
+        mb = modeled_bytes(case)
+        step_us = sum(us.values())
+        gbs = sum(mb.values()) / (step_us * 1e-6) / 1e9
+        alu = 3 * 2 * conv_fmas(case) / (step_us * 1e-6) / alu_peak
+        row = {"sweep_point": case.name, "B": case.B, "C": case.C, "H": case.H, "k": case.k, "L": case.L,
+               "us": {k: round(v, 1) for k, v in us.items()}, "step_us": round(step_us, 1),
+               "gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4), "alu_frac": round(alu, 4)}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        del g, y, dx, grads, ws
+        torch.cuda.empty_cache()
+    gb = sorted(r["gbs"] for r in rows)
+    print(json.dumps({"sweep_points": len(rows), "gbs_median": gb[len(gb) // 2], "gbs_min": gb[0], "gbs_max": gb[-1],
+                      "hbm_peak_gbs": peak, "hbm_peak_source": peak_kind, "timing": "median of per-call CUDA events, "
+                      "L2 flushed before every call", "data": "synthetic"}))
+    return 0
+
+
 def main():
     args = parse()
+    if args.sweep:
+        return run_sweep(args)
     from wtconv_inputs import NAMED, sweep_cases
     sweep = {c.name: c for c in sweep_cases()}
     if args.workload in NAMED:
