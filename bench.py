@@ -62,7 +62,7 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="time the three calls at every point of the 128-point shape sweep (one JSON line each)")
     ap.add_argument("--sweep-steps", type=int, default=20, help="with --sweep: timed calls per point")
-    ap.add_argument("--sweep-points", default="", help="with --sweep: a range of point indices, e.g. 0:32")
+    ap.add_argument("--sweep-points", default="", help="with --sweep: one point index or a range, e.g. 5 or 0:32")
     return ap.parse_args()
 
 
@@ -708,8 +708,11 @@ def run_sweep(args):
     stream = torch.cuda.current_stream(dev)
     cases = sweep_cases()
     if args.sweep_points:
-        a, b = (int(v) if v else None for v in args.sweep_points.split(":"))
-        cases = cases[a:b]
+        if ":" in args.sweep_points:
+            a, b = (int(v) if v else None for v in args.sweep_points.split(":"))
+            cases = cases[a:b]
+        else:
+            cases = [cases[int(args.sweep_points)]]
     peak, peak_kind = hbm_peak()
     alu_peak = 148 * 128 * 2 * 1965e6
     rows = []
