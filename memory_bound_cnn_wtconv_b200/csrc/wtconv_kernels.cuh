@@ -161,8 +161,9 @@ __device__ __forceinline__ void zero_smem(float* sm, int nfloats, int tid, int n
 // un-normalised butterflies into the 4 subband planes at `sb` (element (0,0),
 // congruent to PD mod 2).  One work item = rows 2i, 2i+1 x columns 4q..4q+3,
 // i.e. two 2x2 blocks.  Returns the thread's sum of the unpacked values if SUM.
+// COPY = false: the plane buffer is not written (its reader uses the staging).
 // ---------------------------------------------------------------------------
-template <typename T, int PD, bool SUM>
+template <typename T, int PD, bool SUM, bool COPY = true>
 __device__ __forceinline__ float unpack_level0(const float* stg, int H, int W, FastDiv dq4, float* dst, int ds,
                                                float* sb, int sbs, int sbsub, bool level0, int tid, int nt) {
     const int W4 = W >> 2;
@@ -174,8 +175,10 @@ __device__ __forceinline__ float unpack_level0(const float* stg, int H, int W, F
             const int r0 = 2 * i, c0 = 4 * q;
             const float4 a = stg_load4<T>(stg, r0 * W + c0);
             const float4 b = stg_load4<T>(stg, (r0 + 1) * W + c0);
-            sts4<PD>(dst + r0 * ds + c0, a);
-            sts4<PD>(dst + (r0 + 1) * ds + c0, b);
+            if (COPY) {
+                sts4<PD>(dst + r0 * ds + c0, a);
+                sts4<PD>(dst + (r0 + 1) * ds + c0, b);
+            }
             if (SUM) sum += ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
             const float apb0 = a.x + a.y, amb0 = a.x - a.y, cpd0 = b.x + b.y, cmd0 = b.x - b.y;
             const float apb1 = a.z + a.w, amb1 = a.z - a.w, cpd1 = b.z + b.w, cmd1 = b.z - b.w;
@@ -190,7 +193,7 @@ __device__ __forceinline__ float unpack_level0(const float* stg, int H, int W, F
         for (int t = tid; t < n; t += nt) {
             const int i = fdiv(t, dq4), q = t - i * W4;
             const float4 a = stg_load4<T>(stg, i * W + 4 * q);
-            sts4<PD>(dst + i * ds + 4 * q, a);
+            if (COPY) sts4<PD>(dst + i * ds + 4 * q, a);
             if (SUM) sum += (a.x + a.y) + (a.z + a.w);
         }
     }
@@ -243,8 +246,8 @@ __device__ __forceinline__ void butterfly(float a, float b, float c, float d, fl
 // that cover one 2^(l+1) x 2^(l+1) region.  Lane groups: a region of
 // (4G)^2 pixels, G = 2^lg, occupies G*G consecutive lanes (block (by, bx) of
 // the region at lane offset by*G + bx).  Returns the thread's sum of the
-// unpacked values if SUM.
-template <typename T, int PD, bool SUM>
+// unpacked values if SUM; COPY = false leaves the plane buffer unwritten.
+template <typename T, int PD, bool SUM, bool COPY = true>
 __device__ __forceinline__ float analysis_pyramid(const float* stg, int H, int W, int levels, int lg, FastDiv drw,
                                                   float* dst, int ds, const Levels& levs, int np, int ptid) {
     const LevelDst* lev = levs.d;
@@ -267,7 +270,8 @@ __device__ __forceinline__ float analysis_pyramid(const float* stg, int H, int W
         for (int q = 0; q < 4; ++q) v[q] = stg_load4<T>(stg, (r0 + q) * W + c0);
         if (valid) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) sts4<PD>(dst + (r0 + q) * ds + c0, v[q]);
+            if (COPY)
+                for (int q = 0; q < 4; ++q) sts4<PD>(dst + (r0 + q) * ds + c0, v[q]);
             if (SUM) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) sum += (v[q].x + v[q].y) + (v[q].z + v[q].w);
@@ -511,7 +515,7 @@ __device__ __forceinline__ float quarter_pow(int l) {
 // ---------------------------------------------------------------------------
 enum : int { kToS = 0, kToQ = 1, kToSS = 2 };
 
-template <typename T, int PD, bool SUM, int DST, class Sync>
+template <typename T, int PD, bool SUM, int DST, bool COPY = true, class Sync>
 __device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const float* stg, float* dst, int ds, int pad,
                                                int np, int ptid, Sync&& sync) {
     const int H = P.H, W = P.W, L = P.L;
@@ -528,11 +532,11 @@ __device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const f
             const Buf& b = buf(l < L ? l : 0);
             lev.d[l] = LevelDst{sm + b.base + pad * b.stride + pad, b.stride, b.sub};
         }
-        sum = analysis_pyramid<T, PD, SUM>(stg, H, W, P.pyr_levels, P.pyr_lg, P.div_rw, dst, ds, lev, np, ptid);
+        sum = analysis_pyramid<T, PD, SUM, COPY>(stg, H, W, P.pyr_levels, P.pyr_lg, P.div_rw, dst, ds, lev, np, ptid);
         done = P.pyr_levels;
     } else {
         const Buf& b = buf(0);
-        sum = unpack_level0<T, PD, SUM>(stg, H, W, P.div_q4, dst, ds, sm + b.base + pad * b.stride + pad, b.stride,
+        sum = unpack_level0<T, PD, SUM, COPY>(stg, H, W, P.div_q4, dst, ds, sm + b.base + pad * b.stride + pad, b.stride,
                                         b.sub, L >= 1, ptid, np);
         done = L >= 1 ? 1 : 0;
     }
@@ -991,18 +995,22 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
     const int myrows = real_rows(P, rank);
     auto csync = [&]() { __syncthreads(); };
 
+    // dys: the correlation tiles read dy straight from its staging buffer
+    // (P.DY aliases it; strips of fp32 planes whose height is whole tiles),
+    // so the next dy strip is staged only after them.
+    const bool dys = GENERAL && P.dy_stg;
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
-    auto stage = [&](size_t off) {
+    auto stage = [&](size_t off, bool with_dy) {
         if constexpr (GENERAL) {
             stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
-            stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
+            if (with_dy) stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
         } else {
             stage_plane(sm + P.stg, x + off, P.plane_chunks, tid, nt);
             stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
         }
     };
-    if (g < P.B) stage(((size_t)g * P.C + c) * plane_elems + strip_off);
+    if (g < P.B) stage(((size_t)g * P.C + c) * plane_elems + strip_off, true);
     cp_async_commit();
 
     // This thread's class and its run of that class's tiles.
@@ -1025,8 +1033,10 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
         cp_async_wait_all();
         plane_sync<GENERAL>(P);  // staged pair complete; previous correlations (and halo copies) done
         analyse_plane<T, p, false, kToS>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
-        const float s = analyse_plane<T, 0, true, kToQ>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
-                                                        P.DY.stride, 0, nt, tid, csync);
+        const float s = dys ? analyse_plane<T, 0, true, kToQ, false>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
+                                                                     P.DY.stride, 0, nt, tid, csync)
+                            : analyse_plane<T, 0, true, kToQ>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
+                                                              P.DY.stride, 0, nt, tid, csync);
         {
             const float yv = s - sdy_c;
             const float tv = sdy + yv;
@@ -1034,7 +1044,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
             sdy = tv;
         }
         plane_sync<GENERAL>(P);  // both analyses complete (every strip)
-        if (b + G < P.B) stage(((size_t)(b + G) * P.C + c) * plane_elems + strip_off);
+        if (b + G < P.B) stage(((size_t)(b + G) * P.C + c) * plane_elems + strip_off, !dys);
         cp_async_commit();
         if (strips) {
             copy_halos(sm, P, rank, tid, nt);
@@ -1053,6 +1063,13 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
                 corr_tile<K, TR, TC, DLD>(sm + S.base + s2 * S.sub + tr * TR * S.stride + tc * TC, S.stride,
                                      sm + Q.base + s2 * Q.sub + tr * TR * Q.stride + tc * TC, Q.stride, acc);
             }
+        }
+        if (dys) {
+            __syncthreads();  // every dy tile read (dy is this CTA's own; no other CTA reads it)
+            if (b + G < P.B)
+                stage_rows(sm + P.stg + P.stg_floats, dy + ((size_t)(b + G) * P.C + c) * plane_elems + strip_off, P,
+                           myrows, tid, nt);
+            cp_async_commit();
         }
     }
     cp_async_wait_all();

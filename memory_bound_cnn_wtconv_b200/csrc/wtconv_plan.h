@@ -98,6 +98,7 @@ struct Plan {
     int red;             // weight gradient: reduction scratch (aliases the plane buffers)
     int stg;             // staging buffer offset; one stored plane occupies stg_floats floats
     int stg_floats;
+    int dy_stg;          // weight gradient (strips): DY aliases the dy staging (see the kernel)
     int plane_chunks;    // 16-byte chunks per stored plane
     Buf X, Y, DY, XS;
     Buf S[kMaxL], Q[kMaxL], SS[kMaxL];

@@ -115,13 +115,18 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // horizontal strips of H / nstrips rows (one CTA of a thread-block cluster
 // per strip; 1 = whole planes, no cluster).  Every field that describes
 // on-chip rows (H, ntr, buffers, tiles) describes one strip.
-inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, Plan* P) {
+// dy_stg (weight gradient on strips of fp32 planes whose height is whole
+// tiles): no DY buffer; the correlation tiles read dy from its staging.
+inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, Plan* P,
+                                     bool dy_stg = false) {
     memset(P, 0, sizeof(*P));
     // The plane the CTAs hold: H and W rounded up to multiples of 2^L.
     const int m = 1 << d->L;
     const int Hv = (d->H + m - 1) / m * m, Wv = (d->W + m - 1) / m * m;
     if (nstrips < 1 || nstrips > kMaxStrips || Hv % nstrips) return WTCONV_ERR_UNSUPPORTED;
     if (kind == kBackward && nstrips != 1) return WTCONV_ERR_UNSUPPORTED;  // whole planes only
+    if (dy_stg && (kind != kBackwardWeight || nstrips == 1 || d->dtype != WTCONV_F32 || Hv != d->H || Wv != d->W))
+        return WTCONV_ERR_UNSUPPORTED;
     const int Hs = Hv / nstrips;
     if (nstrips > 1 && (Hs % m != 0 || Hs % 4 != 0)) return WTCONV_ERR_UNSUPPORTED;
     P->B = d->B; P->C = d->C; P->H = Hs; P->W = Wv; P->k = d->k; P->L = d->L;
@@ -193,7 +198,7 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         P->Y.base = (int)off;
         off += round4(P->ntr[kMaxL] * TR * P->Y.stride);
     }
-    if (kind == kBackwardWeight) {
+    if (kind == kBackwardWeight && !dy_stg) {
         const int rows = P->ntr[kMaxL] * TR;
         P->DY.stride = round4(P->ntc[kMaxL] * TC);
         P->DY.base = (int)off;
@@ -208,6 +213,15 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         P->div_rowc = make_fastdiv(std::max(P->row_chunks, 1));
         P->stg = (int)off;
         off += (kind == kBackwardWeight || kind == kBackward ? 2LL : 1LL) * P->stg_floats;
+    }
+    if (dy_stg) {
+        // The dy staging holds the strip as H rows of W floats: the DY layout
+        // exactly when H is whole tiles and W is whole tile columns.
+        if (H % TR != 0 || W % TC != 0) return WTCONV_ERR_UNSUPPORTED;
+        P->DY.base = P->stg + P->stg_floats;
+        P->DY.stride = W;
+        P->DY.sub = 0;
+        P->dy_stg = 1;
     }
 
     // Tiles and threads.
@@ -347,13 +361,18 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
     double best = 0.0;
     Plan cand;
     for (int n = 1; n <= kMaxStrips && !have; n *= 2) {
-        for (int TR = 7; TR <= 8; ++TR) {
-            if (make_plan_for(d, kind, TR, n, &cand) != WTCONV_OK) continue;
-            const double c = plan_cost(cand, kind);
-            if (!have || c < best) {
-                best = c;
-                *P = cand;
-                have = true;
+        // The weight gradient on strips may read dy from its staging (no DY
+        // buffer) when that is what lets this strip count fit.
+        for (int alias = 0; alias < 2 && !have; ++alias) {
+            if (alias && (kind != kBackwardWeight || n == 1)) break;
+            for (int TR = 7; TR <= 8; ++TR) {
+                if (make_plan_for(d, kind, TR, n, &cand, alias == 1) != WTCONV_OK) continue;
+                const double c = plan_cost(cand, kind);
+                if (!have || c < best) {
+                    best = c;
+                    *P = cand;
+                    have = true;
+                }
             }
         }
     }

@@ -76,6 +76,10 @@ void check_global(long long idx, long long n, const char* what) {
 
 // Replays stage_plane: 16-byte chunk ch of this CTA's rows (strip `rank`) of
 // the stored plane -> staging floats [stg + 4ch, stg + 4ch + 4).
+// False while replaying an analysis whose plane copy the kernel skips (the
+// weight gradient's dy when its tiles read the staging; COPY = false).
+bool g_copy_plane = true;
+
 int real_rows_host(const Plan& P, int rank) { return std::max(0, std::min(P.H, P.Hr - rank * P.H)); }
 
 void replay_stage(Shadow& sh, const Plan& P, long long stg, int tag, int rank) {
@@ -130,7 +134,8 @@ void replay_unpack(Shadow& sh, const Plan& P, long long stg, int stag, long long
             for (int rr = 0; rr < nr; ++rr) {
                 const int r = level0 ? 2 * i + rr : i;
                 stage_read(r * W + 4 * q);
-                for (int e = 0; e < 4; ++e) sh.write(dst + (long long)r * ds + 4 * q + e, dlo, dhi, dtag, "unpack store");
+                if (g_copy_plane)
+                    for (int e = 0; e < 4; ++e) sh.write(dst + (long long)r * ds + 4 * q + e, dlo, dhi, dtag, "unpack store");
             }
             if (level0)
                 for (int s = 0; s < 4; ++s)
@@ -165,7 +170,8 @@ void replay_pyramid(Shadow& sh, const Plan& P, long long stg, int stag, long lon
             const long long f0 = stg + (long long)((r0 + q) * W + c0) * P.esize / 4;
             const int t = staged_tag(P, g_rank, r0 + q, c0, stag);
             for (int e = 0; e < P.esize; ++e) sh.read(f0 + e, stg, stg + P.stg_floats, t, "pyramid staging read");
-            for (int e = 0; e < 4; ++e) sh.write(dst + (long long)(r0 + q) * ds + c0 + e, dlo, dhi, dtag, "pyramid plane store");
+            if (g_copy_plane)
+                for (int e = 0; e < 4; ++e) sh.write(dst + (long long)(r0 + q) * ds + c0 + e, dlo, dhi, dtag, "pyramid plane store");
         }
         auto lvl_store = [&](int l, int i, int j) {
             const Buf& b = bufs[l];
@@ -529,7 +535,16 @@ void check_bwdw(const wtconv_desc_t& d) {
     std::vector<Shadow> shs(NS, Shadow(P.smem_floats));
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
-    const long long dlo = P.DY.base, dhi = P.DY.base + (long long)P.ntr[kMaxL] * TR * P.DY.stride;
+    // dys: DY is the dy staging itself (strips of fp32 planes of whole tile
+    // rows); the dy analysis writes no plane copy and the next dy strip is
+    // staged after the correlation tiles, behind a CTA barrier.
+    const bool dys = P.dy_stg != 0;
+    const long long dlo = dys ? (long long)P.stg + P.stg_floats : P.DY.base;
+    const long long dhi = dys ? dlo + P.stg_floats : P.DY.base + (long long)P.ntr[kMaxL] * TR * P.DY.stride;
+    const int dtile_tag = dys ? DYT + 10 : DYT;
+    if (dys && (P.DY.base != dlo || P.DY.stride != W || P.ntr[kMaxL] * TR != H || P.esize != 4 || P.padded || NS < 2 ||
+                (long long)H * W != P.stg_floats))
+        shs[0].fail("dy read from staging needs fp32 strips of whole tile rows", P.DY.base);
     if (P.stg % 4 || P.stg_floats % 4) shs[0].fail("staging alignment", P.stg);
     // Two planes in a row (the second must see the same zero padding), with
     // the kernel's barriers (cluster-wide with strips) as phase boundaries:
@@ -548,7 +563,9 @@ void check_bwdw(const wtconv_desc_t& d) {
             const int e0 = sh.epoch;
             replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S,
                            p, s_tag);
+            g_copy_plane = !dys;
             replay_analyse(sh, P, P.stg + P.stg_floats, DYT + 10, P.DY.base, P.DY.stride, dlo, dhi, DYT, P.Q, 0, q_tag);
+            g_copy_plane = true;
             if (r + 1 < NS) sh.epoch = e0;
             else for (int q = 0; q + 1 < NS; ++q) shs[q].epoch = sh.epoch;
         }
@@ -557,7 +574,7 @@ void check_bwdw(const wtconv_desc_t& d) {
             shs[r].phase = "staging";
             if (plane == 0) {
                 replay_stage(shs[r], P, P.stg, XT + 10, r);
-                replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
+                if (!dys) replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
             }
         }
         if (NS > 1) {
@@ -586,7 +603,7 @@ void check_bwdw(const wtconv_desc_t& d) {
                 if (tr >= P.ntr[lvl]) sh.fail("tile row out of grid", tid);
                 if (cl == 0) {
                     replay_window(sh, P, P.X.base, P.X.stride, xlo, xhi, H, W, tr, tc, XT, "base S window", r);
-                    replay_dtile(sh, P, P.DY.base, P.DY.stride, dlo, dhi, H, W, tr, tc, DYT);
+                    replay_dtile(sh, P, P.DY.base, P.DY.stride, dlo, dhi, H, W, tr, tc, dtile_tag);
                 } else {
                     const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
                     const int n = H >> (l + 1), m = W >> (l + 1);
@@ -599,6 +616,11 @@ void check_bwdw(const wtconv_desc_t& d) {
                 }
               }
             if (covered != P.n_all_tiles) sh.fail("tiles covered", covered);
+            if (dys) {
+                sh.barrier();  // the CTA's dy tiles are all read
+                sh.phase = "dy staging";
+                if (plane == 0) replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10, r);
+            }
         }
     }
     const long long red_end = (long long)P.red + (long long)P.nthreads * KK + P.nthreads;
@@ -630,8 +652,8 @@ void check_bwdw(const wtconv_desc_t& d) {
     if ((long long)P.nthreads * KK + P.nthreads / 32 > P.smem_floats) sh.fail("sum-dy scratch", P.nthreads);
     if (P.nv != ncls * KK + 1) sh.fail("partial vector length", P.nv);
     if ((long long)P.nv + ncls * KK + 1 > P.smem_floats) sh.fail("final-step scratch", P.nv);
-    std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d (<= %d per thread), groups %d, strips %d\n",
-                P.smem_floats * 4, P.nthreads, TR, P.n_all_tiles, P.tpt, P.groups, NS);
+    std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d (<= %d per thread), groups %d, strips %d%s\n",
+                P.smem_floats * 4, P.nthreads, TR, P.n_all_tiles, P.tpt, P.groups, NS, dys ? ", dy read from staging" : "");
 }
 
 // Fused backward: dx conv tiles (the input-gradient pass: dy in X / S, dx
