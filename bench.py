@@ -98,7 +98,7 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
     ("stage1", "bwd_w"): (78782720.0, "wtconv_bwdw_partial_kernel",
-                          "dca0d68918792fcfcdde0b25c08f0b5c1d85a1c6247e271c5c131c7ef9a7bb62",
+                          "9ccf711d142033688489bc1d6c6d162588cc9b5612f6e69a579991495fc16b33",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 
