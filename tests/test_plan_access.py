@@ -52,3 +52,17 @@ def _cases():
 def test_every_access_in_bounds(checker, case):
     r = subprocess.run([checker, *map(str, case)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout + r.stderr
+
+
+@pytest.mark.parametrize("case,strips,alias", [
+    ((1, 1, 256, 256, 5, 4, 0), 8, True),    # DY would not fit beside two staged strips at 8 strips
+    ((2, 2, 128, 128, 5, 4, 0), 2, True),
+    ((2, 2, 128, 128, 5, 3, 0), 2, False),   # fits with its own DY buffer
+    ((3, 5, 56, 56, 5, 3, 0), 1, False),     # whole planes never alias
+])
+def test_weight_gradient_strip_choice(checker, case, strips, alias):
+    # The fewest strips that fit; dy read from its staging only when that is what makes them fit.
+    out = subprocess.run([checker, *map(str, case)], capture_output=True, text=True).stdout
+    line = next(l for l in out.splitlines() if l.startswith("bwdw:"))
+    assert f"strips {strips}" in line, line
+    assert ("dy read from staging" in line) == alias, line
