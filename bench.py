@@ -5,6 +5,9 @@ input gradient + weight gradient over one synthetic batch.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload stage1|stage2|train_bf16|tiny]
 
+With --gpus N > 1 and no torch.distributed environment, the script launches
+itself as N ranks (torch.distributed.run, one rank per GPU, 127.0.0.1).
+
 Prints one JSON line (rank 0).  Metric: modeled minimum HBM bytes of the three
 calls divided by their device time (GB/s), the achieved fraction of the
 measured HBM peak, and microseconds per call.  Modeled bytes per step:
@@ -53,6 +56,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="time only the named workload (by default the other WTConvNeXt stage shapes are timed too)")
+    ap.add_argument("--dist-check", action="store_true",
+                    help="CPU check of the multi-rank launch path (gloo): each rank all-reduces synthetic weight "
+                         "gradients and the slowest rank's time is reported; no kernels run")
     ap.add_argument("--compare", action="store_true",
                     help="time the unfused PyTorch layer and the plain depthwise conv beside this library "
                          "(context lines, not the bench line)")
@@ -293,12 +301,110 @@ def run_reference(args, case):
 # --------------------------------------------------------------------------
 # The CUDA path.
 # --------------------------------------------------------------------------
+class Workload:
+    """Device buffers of one workload and its three calls (plus, with several
+    ranks, the all-reduce of the weight gradients)."""
+
+    def __init__(self, case, dev, stream, rank: int, world: int):
+        import torch
+
+        import memory_bound_cnn_wtconv_b200 as wt
+        from wtconv_inputs import make_inputs
+
+        self.case, self.dev, self.stream, self.world = case, dev, stream, world
+        inp = make_inputs(case.with_(seed=case.seed + 7919 * rank))
+        self.g = g = {k: v.to(dev) for k, v in inp.items()}
+        L = case.L
+        self.y = torch.empty_like(g["x"])
+        self.dx = torch.empty_like(g["dy"])
+        self.grads = grads = {k: torch.empty_like(g[k]) for k in ("base_w", "base_b", "base_scale", "wt_w", "wt_scale")}
+        self.flat = torch.empty(sum(v.numel() for v in grads.values()), device=dev)
+        self.ws = torch.empty(max(16, wt.workspace_bytes(g["x"].shape, case.k, L, g["x"].dtype)), dtype=torch.uint8,
+                              device=dev)
+
+        def fwd():
+            wt.forward(g["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L, y=self.y,
+                       stream=stream)
+
+        def bwd_in():
+            wt.backward_input(g["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], L, dx=self.dx,
+                              stream=stream)
+
+        def bwd_w():
+            wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
+                               grads=grads, workspace=self.ws, stream=stream)
+
+        def bwd_fused():
+            wt.backward(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
+                        dx=self.dx, grads=grads, workspace=self.ws, stream=stream)
+
+        self.calls = [("fwd", fwd), ("bwd_in", bwd_in), ("bwd_w", bwd_w)]
+        if world > 1:
+            import torch.distributed as dist
+            self.calls.append(("allreduce", lambda: allreduce_weight_grads(grads, self.flat, dist)))
+        self.bwd_fused = bwd_fused
+
+    def time_calls(self, calls, steps: int, warmup: int, flush, clocks=None):
+        """Per-call device times (ms) of `steps` timed steps after `warmup`
+        untimed ones: CUDA events on the launching stream around every call,
+        L2 flushed (a 256 MiB write) before every call.  Returns the lists of
+        per-call times and the wall time of the timed region."""
+        import torch
+        for _ in range(warmup):
+            for _, f in calls:
+                flush.zero_()
+                f()
+        torch.cuda.synchronize(self.dev)
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+              for _ in range(steps)]
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(self.dev)
+        wall0 = time.perf_counter()
+        for s in range(steps):
+            for i, (_, f) in enumerate(calls):
+                flush.zero_()
+                ev[s][i][0].record(self.stream)
+                f()
+                ev[s][i][1].record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        wall = time.perf_counter() - wall0
+        clk = clocks.stop() if clocks is not None else None
+        times = {name: [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)] for i, (name, _) in enumerate(calls)}
+        return times, wall, clk
+
+
+def call_record(case, per_call_ms: dict, peak: float) -> dict:
+    """GB/s, HBM fraction and FP32-pipe fraction of each call and of the step."""
+    mb = modeled_bytes(case)
+    alu_peak = SMS * FP32_LANES * 2 * MAX_SM_MHZ * 1e6 / 1e12
+    step_ms = sum(per_call_ms[k] for k in mb)
+    gbs = sum(mb.values()) / (step_ms * 1e-3) / 1e9
+    return {
+        "workload": workload_name(case),
+        "us_per_call": {k: per_call_ms[k] * 1e3 for k in mb},
+        "gbs_per_call": {k: mb[k] / (per_call_ms[k] * 1e-3) / 1e9 for k in mb},
+        "hbm_frac_per_call": {k: mb[k] / (per_call_ms[k] * 1e-3) / 1e9 / peak for k in mb},
+        "alu_frac_per_call": {k: 2.0 * conv_fmas(case) / (per_call_ms[k] * 1e-3) / 1e12 / alu_peak for k in mb},
+        "step_us": step_ms * 1e3, "step_gbs": gbs, "step_hbm_frac": gbs / peak,
+        "modeled_bytes_per_step": sum(mb.values()),
+    }
+
+
+def median(v):
+    return statistics.median(v)
+
+
 def run_ours(args, case):
     import torch
     import torch.distributed as dist
 
     import memory_bound_cnn_wtconv_b200 as wt
-    from wtconv_inputs import make_inputs
+    from wtconv_inputs import NAMED
 
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -306,71 +412,15 @@ def run_ours(args, case):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     wt.load_library()
-
-    my_case = case.with_(seed=case.seed + 7919 * rank)
-    inp = make_inputs(my_case)
-    g = {k: v.to(dev) for k, v in inp.items()}
-    L = case.L
-    y = torch.empty_like(g["x"])
-    dx = torch.empty_like(g["dy"])
-    grads = dict(base_w=torch.empty_like(g["base_w"]), base_b=torch.empty_like(g["base_b"]),
-                 base_scale=torch.empty_like(g["base_scale"]), wt_w=torch.empty_like(g["wt_w"]),
-                 wt_scale=torch.empty_like(g["wt_scale"]))
-    flat = torch.empty(sum(v.numel() for v in grads.values()), device=dev)
-    ws = torch.empty(max(16, wt.workspace_bytes(g["x"].shape, case.k, L, g["x"].dtype)), dtype=torch.uint8,
-                     device=dev)
+    wt.wait_timeouts(reset=True)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-
-    def fwd():
-        wt.forward(g["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L, y=y, stream=stream)
-
-    def bwd_in():
-        wt.backward_input(g["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], L, dx=dx, stream=stream)
-
-    def bwd_w():
-        wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
-                           grads=grads, workspace=ws, stream=stream)
-
-    def allreduce():
-        allreduce_weight_grads(grads, flat, dist)
-
-    def bwd_fused():
-        wt.backward(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L, dx=dx,
-                    grads=grads, workspace=ws, stream=stream)
-
-    calls = [("fwd", fwd), ("bwd_in", bwd_in), ("bwd_w", bwd_w)]
-    if world > 1:
-        calls.append(("allreduce", allreduce))
-
-    for _ in range(args.warmup):
-        for _, f in calls:
-            flush.zero_()
-            f()
-    torch.cuda.synchronize(dev)
-
+    wl = Workload(case, dev, stream, rank, world)
     K = args.steps
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
-          for _ in range(K)]
     clocks = Clocks(not args.no_clocks, physical_gpu_index(local))
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    wall0 = time.perf_counter()
-    for s in range(K):
-        for i, (_, f) in enumerate(calls):
-            flush.zero_()
-            ev[s][i][0].record(stream)
-            f()
-            ev[s][i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    wall = time.perf_counter() - wall0
-    clk = clocks.stop()
-
-    per_call = {name: sum(ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(K)) / K
-                for i, (name, _) in enumerate(calls)}
+    times, wall, clk = wl.time_calls(wl.calls, K, args.warmup, flush, clocks)
+    # Per-call medians over the K timed steps; the step is their sum.
+    per_call = {name: median(v) for name, v in times.items()}
     step_ms = sum(per_call.values())
     if world > 1:
         step_ms = max_over_ranks(step_ms, dist, dev)
@@ -388,7 +438,7 @@ def run_ours(args, case):
     alu_achieved = flops / dom_s / 1e12
     hbm_achieved = mb[dom] / dom_s / 1e9
     t_alu, t_hbm = flops / (alu_peak * 1e12), mb[dom] / (peak * 1e9)
-    kernel_names = {"fwd": "wtconv_fused_kernel (forward)", "bwd_in": "wtconv_fused_kernel (input gradient)",
+    kernel_names = {"fwd": "wtconv_ws_kernel (forward)", "bwd_in": "wtconv_ws_kernel (input gradient)",
                     "bwd_w": "wtconv_bwdw_partial_kernel (final step in its tail)"}
     traffic, traffic_src = measured_traffic(case.name, dom)
     if t_alu >= t_hbm:
@@ -396,27 +446,28 @@ def run_ours(args, case):
                 "frac": alu_achieved / alu_peak, "traffic": traffic, "traffic_source": traffic_src,
                 "kernel": kernel_names[dom],
                 "peak_source": "148 SMs x 128 FP32 FMA lanes x 2 x 1965 MHz (unit counts x max clock)",
-                "flops_per_launch": flops}
+                "flops_per_launch": flops, "hbm_frac": hbm_achieved / peak, "bytes_per_launch": mb[dom]}
     else:
         roof = {"bound": "hbm", "achieved": hbm_achieved, "peak": peak, "unit": "GB/s", "frac": hbm_achieved / peak,
                 "traffic": traffic, "traffic_source": traffic_src, "kernel": kernel_names[dom],
                 "peak_source": peak_kind,
                 "bytes_per_launch": mb[dom]}
 
+    rec = call_record(case, per_call, peak)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if case.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": workload_name(case), "global_batch": case.B * world,
                    "parallelism": f"dp{world}", "l2": "flushed before every call (256 MiB write)",
+                   "timing": f"median over the {K} timed steps of each call's CUDA-event time; step = their sum",
                    "modeled_bytes_per_step": step_bytes},
         "hbm_frac_of_peak": value / world / peak, "hbm_peak_gbs": peak, "hbm_peak_source": peak_kind,
         "frac_of_8tbs": value / world / 8000.0,
         "us_per_call": {k: v * 1e3 for k, v in per_call.items()},
-        "gbs_per_call": {k: mb[k] / (per_call[k] * 1e-3) / 1e9 for k in mb},
+        "gbs_per_call": rec["gbs_per_call"],
         "roofline": roof,
-        "alu_frac_per_call": {k: 2.0 * conv_fmas(case) / (per_call[k] * 1e-3) / 1e12 / alu_peak
-                              for k in ("fwd", "bwd_in", "bwd_w")},
+        "alu_frac_per_call": rec["alu_frac_per_call"],
         # Our kernels in the timed region: forward, input gradient, weight
         # gradient (its final step runs in the same launch) per step.
         "gpu_launches": K * 3, "wall_s_timed_region": wall,
@@ -425,35 +476,42 @@ def run_ours(args, case):
         line["clocks"] = clk
 
     if not args.no_e2e:
-        line["e2e"] = e2e(args, case, g, grads, ws, dev, world)
+        line["e2e"] = e2e(args, case, wl.g, wl.grads, wl.ws, dev, world)
     if world > 1:
         dist.barrier()
     # The one-pass backward (wtconv_backward), timed after the step with the
     # same protocol; reported beside the three-call step, not in it.
     KF = min(K, 500)
-    for _ in range(3):
-        flush.zero_()
-        bwd_fused()
-    evf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(KF)]
-    for s in range(KF):
-        flush.zero_()
-        evf[s][0].record(stream)
-        bwd_fused()
-        evf[s][1].record(stream)
-    torch.cuda.synchronize(dev)
-    fb_ms = sum(a.elapsed_time(b) for a, b in evf) / KF
+    ft, _, _ = wl.time_calls([("bwd_fused", wl.bwd_fused)], KF, 3, flush)
+    fb_ms = median(ft["bwd_fused"])
     if world > 1:
         fb_ms = max_over_ranks(fb_ms, dist, dev)
     fb_bytes = 3 * case.numel * case.esize + 2 * 4 * param_floats(case)
     fstep_bytes = mb["fwd"] + fb_bytes
     fstep_ms = per_call["fwd"] + fb_ms
     line["fused_backward"] = {
-        "call": "wtconv_backward (dx and all parameter gradients in one pass)",
+        "call": "wtconv_backward (dx and all parameter gradients; one pass or the two passes, as the library picks)",
         "us_per_call": fb_ms * 1e3, "modeled_bytes": fb_bytes, "gbs": fb_bytes / (fb_ms * 1e-3) / 1e9,
         "step_forward_plus_fused_backward_us": fstep_ms * 1e3,
         "step_modeled_bytes": fstep_bytes,
         "step_gbs": fstep_bytes * world / (fstep_ms * 1e-3) / 1e9,
     }
+    # The other WTConvNeXt stage shapes, same protocol, one GPU.
+    if world == 1 and not args.no_other_workloads:
+        other = {}
+        for name in ("stage1", "stage2", "train_bf16"):
+            if name == case.name:
+                other[name] = rec
+                continue
+            del_wl = Workload(NAMED[name], dev, stream, 0, 1)
+            t2, _, _ = del_wl.time_calls(del_wl.calls, K, args.warmup, flush)
+            other[name] = call_record(NAMED[name], {n: median(v) for n, v in t2.items()}, peak)
+            line["gpu_launches"] += K * 3
+            del del_wl
+            torch.cuda.empty_cache()
+        line["workloads"] = other
+    timeouts = wt.wait_timeouts()
+    line["kernel_wait_timeouts"] = timeouts
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nb, t, planes, cores, desc = oracle_sample(case, args.cpu_seconds, wrap=True)
         line["cpu_baseline"] = {"value": nb / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
@@ -462,7 +520,7 @@ def run_ours(args, case):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
-    return 0
+    return 0 if timeouts == 0 else 3
 
 
 def e2e(args, case, g, grads, ws, dev, world):
@@ -763,8 +821,76 @@ def run_sweep(args):
     return 0
 
 
+def relaunch(args) -> int:
+    """`--gpus N` (N > 1) outside a torch.distributed launch: run this script
+    again as N ranks on this node (one per GPU) through torch.distributed.run,
+    rendezvous on 127.0.0.1, and return its exit status."""
+    import signal
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=1800)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGTERM)
+        try:
+            proc.wait(timeout=60)
+        except subprocess.TimeoutExpired:
+            os.killpg(proc.pid, signal.SIGKILL)
+        return 124
+
+
+def run_dist_check(args) -> int:
+    """The multi-rank path without kernels (gloo on the CPU): each rank fills
+    its weight gradients with rank-dependent values, sums them over the ranks
+    with the bench's all-reduce, checks the sums, and reports the slowest
+    rank's time.  Rank 0 prints one JSON line."""
+    import torch
+    import torch.distributed as dist
+
+    world, rank, _ = dist_env()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    case = __import__("wtconv_inputs").TINY
+    shapes = {"base_w": (case.C, case.k, case.k), "base_b": (case.C,), "base_scale": (case.C,),
+              "wt_w": (case.L, case.C, 4, case.k, case.k), "wt_scale": (case.L, case.C, 4)}
+    grads = {k: torch.full(v, float(rank + 1)) for k, v in shapes.items()}
+    flat = torch.empty(sum(v.numel() for v in grads.values()))
+    t0 = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        for v in grads.values():
+            v.fill_(float(rank + 1))
+        if world > 1:
+            allreduce_weight_grads(grads, flat, dist)
+    t = time.perf_counter() - t0
+    ok = all(bool(torch.all(v == world * (world + 1) / 2)) for v in grads.values())
+    if world > 1:
+        t = max_over_ranks(t, dist, torch.device("cpu"))
+        okt = torch.tensor([1 if ok else 0])
+        dist.all_reduce(okt, op=dist.ReduceOp.MIN)
+        ok = bool(okt.item())
+    if rank == 0:
+        print(json.dumps({"impl": "dist-check", "n_gpus": world, "steps": args.steps, "backend": "gloo",
+                          "allreduce_sum_ok": ok, "s_max_over_ranks": t}), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0 if ok else 1
+
+
 def main():
     args = parse()
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        return relaunch(args)
+    if env_world is not None and int(env_world) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={env_world}; launch one rank per GPU", file=sys.stderr)
+        return 2
+    if args.dist_check:
+        return run_dist_check(args)
     if args.sweep:
         return run_sweep(args)
     from wtconv_inputs import NAMED, sweep_cases
