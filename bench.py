@@ -412,7 +412,6 @@ def run_ours(args, case):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     wt.load_library()
-    wt.wait_timeouts(reset=True)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     wl = Workload(case, dev, stream, rank, world)
@@ -438,7 +437,7 @@ def run_ours(args, case):
     alu_achieved = flops / dom_s / 1e12
     hbm_achieved = mb[dom] / dom_s / 1e9
     t_alu, t_hbm = flops / (alu_peak * 1e12), mb[dom] / (peak * 1e9)
-    kernel_names = {"fwd": "wtconv_ws_kernel (forward)", "bwd_in": "wtconv_ws_kernel (input gradient)",
+    kernel_names = {"fwd": "wtconv_fused_kernel (forward)", "bwd_in": "wtconv_fused_kernel (input gradient)",
                     "bwd_w": "wtconv_bwdw_partial_kernel (final step in its tail)"}
     traffic, traffic_src = measured_traffic(case.name, dom)
     if t_alu >= t_hbm:
@@ -510,8 +509,6 @@ def run_ours(args, case):
             del del_wl
             torch.cuda.empty_cache()
         line["workloads"] = other
-    timeouts = wt.wait_timeouts()
-    line["kernel_wait_timeouts"] = timeouts
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nb, t, planes, cores, desc = oracle_sample(case, args.cpu_seconds, wrap=True)
         line["cpu_baseline"] = {"value": nb / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
@@ -520,7 +517,7 @@ def run_ours(args, case):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
-    return 0 if timeouts == 0 else 3
+    return 0
 
 
 def e2e(args, case, g, grads, ws, dev, world):

@@ -92,15 +92,6 @@ typedef struct {
 /* Human-readable name of a status code (static string, never NULL). */
 const char *wtconv_status_string(wtconv_status_t s);
 
-/* Number of times a wait inside a kernel of this library (on an mbarrier
- * that hands a shared-memory buffer from one group of warps to another) gave
- * up after its one-second limit, on the current device, since the last reset.
- * Such a wait ends its warp's work early, so the results of that launch are
- * incomplete; 0 is the only value a correct run produces.  Synchronous: it
- * reads device memory (and, if `reset` is non-zero, sets the count to 0).
- * Returns 0xffffffff if the CUDA runtime reports an error. */
-unsigned wtconv_wait_timeouts(int reset);
-
 /* Bytes of device workspace wtconv_backward_weight and wtconv_backward need
  * for `d` (0 if `d` is invalid); one size serves both.  The forward and
  * input-gradient calls need none. */

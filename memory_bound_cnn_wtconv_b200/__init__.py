@@ -21,7 +21,6 @@ import os
 import torch
 
 __all__ = [
-    "wait_timeouts",
     "forward", "backward_input", "backward_weight", "backward", "workspace_bytes", "WTConvError",
     "WTConvLibraryMissing", "library_path", "load_library", "Desc", "STATUS",
 ]
@@ -80,20 +79,8 @@ def load_library():
     lib.wtconv_backward_weight.restype = ctypes.c_int
     lib.wtconv_backward.argtypes = [dp, vp, vp, fp, fp, fp, fp, fp, vp, fp, fp, fp, fp, fp, vp, sz, vp]
     lib.wtconv_backward.restype = ctypes.c_int
-    lib.wtconv_wait_timeouts.argtypes = [ctypes.c_int]
-    lib.wtconv_wait_timeouts.restype = ctypes.c_uint
     _lib = lib
     return lib
-
-
-def wait_timeouts(reset: bool = False) -> int:
-    """Waits inside this library's kernels that gave up after their limit on
-    the current device (``wtconv_wait_timeouts``; 0 in every correct run).
-    Synchronous."""
-    v = int(load_library().wtconv_wait_timeouts(1 if reset else 0))
-    if v == 0xFFFFFFFF:
-        raise WTConvError(9, "wtconv_wait_timeouts")
-    return v
 
 
 def status_string(code: int) -> str:

@@ -86,17 +86,6 @@ const char* wtconv_status_string(wtconv_status_t s) {
     return "unknown status";
 }
 
-unsigned wtconv_wait_timeouts(int reset) {
-    const unsigned v[4] = {read_wait_timeouts_k1(reset != 0), read_wait_timeouts_k3(reset != 0),
-                           read_wait_timeouts_k5(reset != 0), read_wait_timeouts_k7(reset != 0)};
-    unsigned sum = 0;
-    for (unsigned t : v) {
-        if (t == ~0u) return ~0u;
-        sum += t;
-    }
-    return sum;
-}
-
 size_t wtconv_workspace_bytes(const wtconv_desc_t* d) {
     if (validate(d) != WTCONV_OK) return 0;
     return workspace_bytes_any(d);

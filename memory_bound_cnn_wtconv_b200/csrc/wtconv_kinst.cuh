@@ -6,8 +6,6 @@
 
 #include "wtconv_kernels.cuh"
 #include "wtconv_launch.h"
-#include "wtconv_duo.cuh"
-#include "wtconv_ws.cuh"
 
 #ifndef WTC_K
 #error "define WTC_K before including wtconv_kinst.cuh"
@@ -111,45 +109,8 @@ cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-// Warp-specialised forward / input gradient: one CTA per SM (at most one
-// per plane).
-template <typename T, bool BWD>
-cudaError_t ws_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
-    static bool done[kMaxDevices] = {};
-    auto* fn = wtconv_ws_kernel<WTC_K, T, BWD>;
-    cudaError_t e = opt_in_smem(fn, done);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const long long units = (long long)P.B * P.C;
-    const unsigned grid = (unsigned)std::min<long long>(units, std::max(sms, 1));
-    fn<<<grid, P.nthreads, (size_t)P.smem_floats * 4, s>>>(static_cast<const T*>(a.x), a.base_w, a.base_b,
-                                                           a.base_scale, a.wt_w, a.wt_scale, static_cast<T*>(a.y), P);
-    return cudaGetLastError();
-}
-
-// Two alternating warp groups: one CTA per SM (at most one per plane).
-template <typename T, bool BWD>
-cudaError_t duo_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
-    static bool done[kMaxDevices] = {};
-    auto* fn = wtconv_duo_kernel<WTC_K, T, BWD>;
-    cudaError_t e = opt_in_smem(fn, done);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const long long units = (long long)P.B * P.C;
-    const unsigned grid = (unsigned)std::min<long long>(units, std::max(sms, 1));
-    fn<<<grid, kDuoThreads, (size_t)P.smem_floats * 4, s>>>(static_cast<const T*>(a.x), a.base_w, a.base_b,
-                                                            a.base_scale, a.wt_w, a.wt_scale, static_cast<T*>(a.y), P);
-    return cudaGetLastError();
-}
-
 template <int TR, typename T>
 cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s) {
-    if (P.duo) return bwd ? duo_typed<T, true>(P, a, s) : duo_typed<T, false>(P, a, s);
-    if (P.ws) return bwd ? ws_typed<T, true>(P, a, s) : ws_typed<T, false>(P, a, s);
     // The general instantiation for cluster strips and / or planes padded on chip.
     if (P.nstrips > 1 || P.padded)
         return bwd ? fused_typed<TR, T, true, true>(P, a, s) : fused_typed<TR, T, false, true>(P, a, s);
@@ -183,16 +144,6 @@ cudaError_t bwdw_tr(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s)
 }
 
 }  // namespace
-
-unsigned WTC_CAT(read_wait_timeouts_k, WTC_K)(bool reset) {
-    unsigned v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_wait_timeouts, sizeof(v)) != cudaSuccess) return ~0u;
-    if (reset) {
-        const unsigned z = 0;
-        if (cudaMemcpyToSymbol(g_wait_timeouts, &z, sizeof(z)) != cudaSuccess) return ~0u;
-    }
-    return v;
-}
 
 cudaError_t WTC_CAT(launch_fused_k, WTC_K)(const Plan& P, int dtype, bool bwd, const FusedArgs& a,
                                            cudaStream_t s) {

@@ -33,8 +33,7 @@ struct BwdArgs {
 #define WTC_DECLARE_LAUNCHERS(KV)                                                                     \
     cudaError_t launch_fused_k##KV(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cudaStream_t s); \
     cudaError_t launch_bwdw_k##KV(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s);           \
-    cudaError_t launch_bwd_k##KV(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s);           \
-    unsigned read_wait_timeouts_k##KV(bool reset);
+    cudaError_t launch_bwd_k##KV(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s);
 
 WTC_DECLARE_LAUNCHERS(1)
 WTC_DECLARE_LAUNCHERS(3)

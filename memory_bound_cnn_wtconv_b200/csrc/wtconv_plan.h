@@ -66,35 +66,6 @@ constexpr int kBwdwMaxThreads = 256;
 // per SM (the same 128-register budget).
 constexpr int kStripMaxThreads = 512;
 constexpr int kBwdMaxThreads = 512;  // fused backward: one CTA per SM
-// Two alternating warp groups (forward / input gradient): one CTA per SM.
-constexpr int kDuoThreads = 512;
-// Warp-specialised forward: one CTA per SM of conv warps + producer warps.
-constexpr int kWsMaxThreads = 512;  // conv warps + producer warps + the copy warp
-constexpr int kWsMaxStg = 4;         // staging slots at most
-// mbarriers of the warp-specialised kernels (indices into the array at mbar).
-enum : int {
-    // Slots of the ana and sub barrier rings (plane j uses j % 16).  Conv
-    // warps take tasks in order and hold one each, so a task of plane j is
-    // only taken once fewer than kWsMaxConvWarps tasks of the planes before
-    // it are unfinished; with 16 slots that means the phase of plane j - 16
-    // in its slot has completed, which a parity wait needs.
-    kWsBarRing = 16,
-    kWsMaxConvWarps = 8,
-    kBarStgFull = 0,                          // [kWsMaxStg] plane landed in staging slot (bulk copy, tx bytes)
-    kBarStgEmpty = kWsMaxStg,                 // [kWsMaxStg] every producer warp has read the staging slot
-    kBarAna = 2 * kWsMaxStg,                  // [16] X, S and weights of a plane written (producer warps)
-    kBarSub = 2 * kWsMaxStg + kWsBarRing,     // [16] every sub tile of a plane done: S slot free, Q slot full
-    kBarBase = 2 * kWsMaxStg + 2 * kWsBarRing,  // [3] every base tile of a plane done: X, weight and Q slots free
-    kNumBars = 2 * kWsMaxStg + 2 * kWsBarRing + 3
-};
-// Ring depths of the warp-specialised kernels (plane j uses slot j % depth).
-enum : int {
-    kWsMaxXSlots = 3,  // X and weights (Plan::x_slots of them, = kWsQSlots): written by the analysis of j,
-                       // read by the base tiles of j; the analysis of j waits for the base tiles of
-                       // plane j-3, which also frees the Q slot of plane j
-    kWsMaxSSlots = 3,  // S (Plan::s_slots): written by the analysis of j, read by the sub tiles of j (step j)
-    kWsQSlots = 3      // Q: written by the sub tiles of j (step j), read by the base tiles of j (step j + 1)
-};
 
 struct Buf {
     int base;    // float offset (see above)
@@ -167,26 +138,6 @@ struct Plan {
     FastDiv div_rowc;               // row_chunks
     FastDiv div_m[kMaxL];           // W >> (l+1)
     FastDiv div_ntc[kMaxL + 1];     // tile columns per tile row
-    // Warp-specialised forward / input gradient (ws = 1; wtconv_ws.cuh).
-    // One CTA per SM: a copy warp stages planes by bulk copy, npw producer
-    // warps analyse them, ncw conv warps run every conv tile.  Ring buffers, one plane each:
-    // nstg staging slots (stg + i*stg_floats), x_slots slots of X and of the
-    // folded weights (X.base + i*x_slot, wbase + i*w_slot; the bias of slot
-    // i at wbase + i*w_slot + ncls*wcls), s_slots slots of S (S[l].base +
-    // i*s_slot) and 3 of Q (Q[l].base + i*q_slot).  Base tiles add the synthesis in their
-    // epilogue and store y; there is no Y buffer.  desc: one int4 per conv
-    // tile of a step (sub tiles, padding to whole warp-tiles, then base
-    // tiles); mbar: the mbarriers.
-    int ws, ncw, npw, nstg, x_slots, s_slots;
-    int x_slot, s_slot, q_slot, w_slot;
-    int desc, mbar;
-    int n_step_tiles, nwt;  // conv tiles per step (incl. padding), warp-tiles (of 32) per step
-    // Two alternating warp groups (duo = 1; wtconv_duo.cuh): each group's
-    // buffers at gbase + g*gsize; every buffer offset above (wbase, stg, X,
-    // S, Q) is then relative to the group's base; two slots of the weights,
-    // X and Q (w_slot, x_slot, q_slot apart), one of S and of the staging.
-    int duo, gbase, gsize;
-    int sub_pad;            // sub tiles rounded up to whole warp-tiles: base tiles start there
 };
 
 }  // namespace wtc

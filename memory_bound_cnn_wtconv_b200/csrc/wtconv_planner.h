@@ -329,167 +329,6 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     return WTCONV_OK;
 }
 
-// Two alternating warp groups (wtconv_duo.cuh) on whole planes that are
-// multiples of 2^L: 512 threads in one CTA per SM, 8-row tiles (the base
-// tiles' synthesis epilogue covers whole 2x2 level-0 blocks).  The strides,
-// tile grid and analysis fields are those of the single-buffer plan; the
-// buffers are laid out again, once per group.
-inline wtconv_status_t make_duo_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
-    if (kind != kForward && kind != kBackwardInput) return WTCONV_ERR_UNSUPPORTED;
-    const wtconv_status_t st = make_plan_for(d, kind, 8, 1, P);
-    if (st != WTCONV_OK) return st;
-    if (P->padded) {
-        memset(P, 0, sizeof(*P));
-        return WTCONV_ERR_UNSUPPORTED;
-    }
-    const int L = P->L, p = P->p, KK = P->k * P->k, ncls = 1 + 4 * L;
-    P->sub_pad = P->n_sub_tiles;  // no padding: a step's tiles have no order among them
-    P->n_step_tiles = P->n_sub_tiles + P->n_base_tiles;
-    P->nwt = ceil_div(P->n_step_tiles, 32);
-    P->desc = 0;
-    long long off = 4LL * P->n_step_tiles;
-    P->gbase = round4((int)off);
-    long long g = 0;  // offsets within a group
-    P->wcls = round4(KK);
-    P->w_slot = round4(ncls * P->wcls + 4);
-    P->wbase = 0;
-    P->bias = ncls * P->wcls;  // within a weight slot
-    g += 2LL * P->w_slot;
-    P->stg = (int)g;
-    g += P->stg_floats;
-    P->x_slot = round4((P->ntr[kMaxL] * 8 + 2 * p) * P->X.stride);
-    P->X.base = (int)g;
-    g += 2LL * P->x_slot;
-    for (int l = 0; l < L; ++l) {
-        P->S[l].base = (int)g;
-        g += 4LL * P->S[l].sub;
-    }
-    {
-        const long long q0 = g;
-        for (int l = 0; l < L; ++l) {
-            P->Q[l].base = (int)g;
-            g += 4LL * P->Q[l].sub;
-        }
-        P->q_slot = (int)(g - q0);
-        g += P->q_slot;
-    }
-    P->Y = Buf{0, 0, 0};
-    P->gsize = round4((int)std::min<long long>(g, 1LL << 30));
-    off = (long long)P->gbase + 2LL * P->gsize;
-    if (off > kSmemLimitFloats) {
-        memset(P, 0, sizeof(*P));
-        return WTCONV_ERR_UNSUPPORTED;
-    }
-    P->smem_floats = (int)off;
-    P->duo = 1;
-    P->nthreads = kDuoThreads;
-    P->merged = 0;
-    P->n_fin = 0;
-    P->fin_off = 0;
-    P->red = 0;
-    P->grid = (int)std::min<long long>((long long)P->B * P->C, kNumSMs);
-    P->groups = 1;
-    return WTCONV_OK;
-}
-
-// Warp-specialised forward / input gradient (wtconv_ws.cuh) on whole planes
-// that are multiples of 2^L and whose analysis is one pass (no level computed
-// on its own behind a barrier): ncw conv warps, npw producer warps and one
-// copy warp in one CTA per SM, 8-row tiles (the base tiles' synthesis
-// epilogue covers whole 2x2 level-0 blocks), nstg staging slots, xslots X /
-// weight slots and sslots S slots.  The strides, tile grid and analysis
-// fields are those of the single-buffer plan; the buffers are laid out again
-// as rings (wtconv_plan.h).
-constexpr int kWsConvWarps = 8;
-constexpr int kWsProducerWarps = 7;
-
-inline wtconv_status_t make_ws_plan_for(const wtconv_desc_t* d, Kind kind, int ncw, int npw, int nstg, int xslots,
-                                        int sslots, Plan* P) {
-    if (kind != kForward && kind != kBackwardInput) return WTCONV_ERR_UNSUPPORTED;
-    if (ncw < 1 || ncw > kWsMaxConvWarps || npw < 1 || (ncw + npw + 1) * 32 > kWsMaxThreads || nstg < 2 ||
-        nstg > kWsMaxStg || xslots < 3 ||
-        xslots > kWsMaxXSlots || sslots < 2 || sslots > kWsMaxSSlots)
-        return WTCONV_ERR_UNSUPPORTED;
-    const wtconv_status_t st = make_plan_for(d, kind, 8, 1, P);
-    if (st != WTCONV_OK) return st;
-    const bool one_pass = P->L == 0 || (P->pyr && P->L <= 4) || (!P->pyr && P->L == 1);
-    if (P->padded || !one_pass) {
-        memset(P, 0, sizeof(*P));
-        return WTCONV_ERR_UNSUPPORTED;
-    }
-    const int L = P->L, p = P->p, KK = P->k * P->k, ncls = 1 + 4 * L;
-    long long off = 0;
-    P->mbar = 0;
-    off += round4(2 * kNumBars + 2);  // 8 bytes per mbarrier, then the conv warps' task counter
-    P->sub_pad = ceil_div(P->n_sub_tiles, 32) * 32;
-    P->n_step_tiles = P->sub_pad + P->n_base_tiles;
-    P->nwt = ceil_div(P->n_step_tiles, 32);
-    P->desc = (int)off;
-    off += 4LL * P->n_step_tiles;
-    P->wcls = round4(KK);
-    P->w_slot = round4(ncls * P->wcls + 4);
-    P->wbase = (int)off;
-    P->bias = ncls * P->wcls;  // within a weight slot
-    off += (long long)xslots * P->w_slot;
-    P->stg = (int)off;
-    off += (long long)nstg * P->stg_floats;
-    P->x_slot = round4((P->ntr[kMaxL] * 8 + 2 * p) * P->X.stride);
-    P->X.base = (int)off;
-    off += (long long)xslots * P->x_slot;
-    {
-        const long long s0 = off;
-        for (int l = 0; l < L; ++l) {
-            P->S[l].base = (int)off;
-            off += 4LL * P->S[l].sub;
-        }
-        P->s_slot = (int)(off - s0);
-        off += (long long)(sslots - 1) * P->s_slot;
-    }
-    {
-        const long long q0 = off;
-        for (int l = 0; l < L; ++l) {
-            P->Q[l].base = (int)off;
-            off += 4LL * P->Q[l].sub;
-        }
-        P->q_slot = (int)(off - q0);
-        off += (long long)(kWsQSlots - 1) * P->q_slot;
-    }
-    P->Y = Buf{0, 0, 0};
-    P->red = 0;
-    off = round4((int)std::min<long long>(off, 1LL << 30));
-    if (off > kSmemLimitFloats) {
-        memset(P, 0, sizeof(*P));
-        return WTCONV_ERR_UNSUPPORTED;
-    }
-    P->smem_floats = (int)off;
-    P->ws = 1;
-    P->ncw = ncw;
-    P->npw = npw;
-    P->nstg = nstg;
-    P->x_slots = xslots;
-    P->s_slots = sslots;
-    P->nthreads = (ncw + npw + 1) * 32;
-    P->merged = 0;
-    P->n_fin = 0;
-    P->fin_off = 0;
-    P->grid = (int)std::min<long long>((long long)P->B * P->C, kNumSMs);
-    P->groups = 1;
-    return WTCONV_OK;
-}
-
-// The warp-specialised plan with the deepest rings that fit: the S ring first
-// (it bounds how far the analysis may run ahead of the sub tiles), then the X
-// ring (ahead of the base tiles), then the staging ring.
-inline wtconv_status_t make_ws_plan(const wtconv_desc_t* d, Kind kind, Plan* P, int ncw = kWsConvWarps,
-                                    int npw = kWsProducerWarps) {
-    for (int ss = kWsMaxSSlots; ss >= 2; --ss)
-        for (int xs = kWsMaxXSlots; xs >= 3; --xs)
-            for (int nstg = 3; nstg >= 2; --nstg)
-                if (make_ws_plan_for(d, kind, ncw, npw, nstg, xs, ss, P) == WTCONV_OK) return WTCONV_OK;
-    memset(P, 0, sizeof(*P));
-    return WTCONV_ERR_UNSUPPORTED;
-}
-
 // Tile rows on the busiest SM sub-partition per plane and SM: the tile-phase
 // length of one CTA (its warp-tiles spread over 4 sub-partitions, times the
 // tile height), times the CTAs of a plane, over the CTAs an SM holds.
@@ -518,7 +357,6 @@ inline double plan_cost(const Plan& P, Kind kind) {
 // strips measured 1.7-1.9x faster than eight, and at every shape measured
 // fewer strips were faster.
 inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
-    if ((kind == kForward || kind == kBackwardInput) && make_duo_plan(d, kind, P) == WTCONV_OK) return WTCONV_OK;
     bool have = false;
     double best = 0.0;
     Plan cand;

@@ -74,12 +74,6 @@ void check_global(long long idx, long long n, const char* what) {
     }
 }
 
-// Warp-specialised kernels: the analysis of a plane is shared by the
-// producer warps; the replay of one warp's share visits only the work items
-// of that warp (item t belongs to producer thread t mod np).
-int g_share = -1, g_share_np = 1;
-bool mine(long long idx) { return g_share < 0 || (int)((idx % g_share_np) / 32) == g_share; }
-
 // Replays stage_plane: 16-byte chunk ch of this CTA's rows (strip `rank`) of
 // the stored plane -> staging floats [stg + 4ch, stg + 4ch + 4).
 // False while replaying an analysis whose plane copy the kernel skips (the
@@ -136,7 +130,6 @@ void replay_unpack(Shadow& sh, const Plan& P, long long stg, int stag, long long
     const int rows = level0 ? P.H / 2 : P.H;
     for (int i = 0; i < rows; ++i)
         for (int q = 0; q < W / 4; ++q) {
-            if (!mine((long long)i * (W / 4) + q)) continue;
             const int nr = level0 ? 2 : 1;
             for (int rr = 0; rr < nr; ++rr) {
                 const int r = level0 ? 2 * i + rr : i;
@@ -167,7 +160,6 @@ void replay_pyramid(Shadow& sh, const Plan& P, long long stg, int stag, long lon
     const int nreg_w = W >> (lg + 2);
     const int items = (H >> (lg + 2)) * nreg_w * G2;
     for (int item = 0; item < items; ++item) {
-        if (!mine(item)) continue;
         const int r = item >> (2 * lg), o = item & (G2 - 1);
         const int by = o >> lg, bx = o & (G - 1);
         const int rrow = (int)fastdiv_host(r, P.div_rw), rcol = r - rrow * nreg_w;
@@ -227,7 +219,6 @@ void replay_haar(Shadow& sh, long long src, int ss, long long slo, long long shi
                  long long dst, int ds, int dsub, long long dlo, long long dhi, int (*dtag)(int, int), int l) {
     for (int i = 0; i < n; ++i)
         for (int j = 0; j < m; ++j) {
-            if (!mine((long long)i * m + j)) continue;
             const long long s0 = src + 2LL * i * ss + 2LL * j;
             sh.read(s0, slo, shi, stag, "haar src");
             sh.read(s0 + 1, slo, shi, stag, "haar src");
@@ -237,7 +228,6 @@ void replay_haar(Shadow& sh, long long src, int ss, long long slo, long long shi
     for (int i = 0; i < n; ++i)
         for (int j = 0; j < m; ++j)
             for (int s = 0; s < 4; ++s) {
-                if (!mine((long long)i * m + j)) continue;
                 const long long d = dst + (long long)i * ds + j + (long long)s * dsub;
                 sh.write(d, dlo + (long long)s * dsub, dlo + (long long)(s + 1) * dsub, dtag(l, s), "haar dst");
             }
@@ -340,20 +330,9 @@ void barrier_all(std::vector<Shadow>& shs) {
     for (auto& sh : shs) sh.barrier();
 }
 
-void check_ws_all(const Plan& P, Kind kind);
-void check_duo_all(const Plan& P, Kind kind);
-
 void check_fused(const wtconv_desc_t& d, Kind kind) {
     Plan P;
     const wtconv_status_t st = make_plan(&d, kind, &P);
-    if (st == WTCONV_OK && P.duo) {
-        check_duo_all(P, kind);
-        return;
-    }
-    if (st == WTCONV_OK && P.ws) {
-        check_ws_all(P, kind);
-        return;
-    }
     if (st == WTCONV_ERR_UNSUPPORTED) {
         std::printf("fused: unsupported (plane too large)\n");
         return;
@@ -846,636 +825,6 @@ void check_bwd(const wtconv_desc_t& d) {
     if ((long long)P.nv + ncls * KK + 1 > P.smem_floats) sh.fail("final-step scratch", P.nv);
     std::printf("bwd: smem %d B, threads %d (%d conv + %d correlation), TR %d, groups %d\n", P.smem_floats * 4,
                 P.nthreads, P.corr0, ncorr, TR, P.groups);
-}
-
-
-
-// ---------------------------------------------------------------------------
-// Warp-specialised forward / input gradient (wtconv_ws.cuh).  Every role's
-// sequence of mbarrier waits and arrivals is written out below exactly as
-// the kernel executes it; a scheduler then runs the roles (and the landing
-// of every bulk copy) in random orders, one action at a time, and
-//   - fails if no role can move (deadlock) or a wait would see its barrier
-//     two phases ahead (the parity test would then be wrong),
-//   - replays every shared-memory access of each action with tags that carry
-//     the plane (and, for the weights, the channel) they belong to, so a
-//     buffer overwritten before its last reader, or read before its writer,
-//     fails the tag check; and checks every output is stored exactly once.
-// ---------------------------------------------------------------------------
-int g_tag_off = 0;
-int s_tag_ws(int l, int s) { return s_tag(l, s) + g_tag_off; }
-int plane_off(int j) { return 1000 * (j + 1); }
-int chan_off(int c) { return 1000 * (c + 1); }
-
-struct MBar {
-    int expected = 0, pending = 0, phase = 0;
-    long long tx = 0;
-    void init(int n) { expected = pending = n; phase = 0; tx = 0; }
-    void maybe_complete() {
-        if (pending == 0 && tx == 0) {
-            ++phase;
-            pending = expected;
-        }
-    }
-    void arrive(int for_phase = -1) {
-        if (pending <= 0) { std::printf("FAIL mbarrier arrival beyond its count\n"); std::exit(1); }
-        if (for_phase >= 0 && for_phase != phase) {
-            std::printf("FAIL ws: arrival meant for phase %d lands in phase %d\n", for_phase, phase);
-            std::exit(1);
-        }
-        --pending;
-        maybe_complete();
-    }
-};
-
-enum WsOp { OP_WAIT, OP_ARRIVE, OP_ISSUE, OP_ANALYSE, OP_TILES };
-struct Op {
-    WsOp k;
-    int bar, a, b;  // WAIT: bar, phase a | ARRIVE: bar, phase a | ISSUE: plane a | ANALYSE: plane a, warp b | TILES: step a, warp-tile b
-};
-
-// Host copy of ws_describe.
-void ws_desc_host(const Plan& P, int t, int& win, int& out, int& wcl, int& level, int& r0, int& c0, bool& base) {
-    const int TR = 8, TC = 4;
-    if (t < P.n_sub_tiles) {
-        int cl = 1;
-        while (t >= P.sub_begin[cl]) ++cl;
-        const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
-        const int local = t - P.sub_begin[cl - 1];
-        const int tr = local / P.ntc[l], tc = local - tr * P.ntc[l];
-        win = P.S[l].base + s * P.S[l].sub + tr * TR * P.S[l].stride + tc * TC;
-        out = P.Q[l].base + s * P.Q[l].sub + tr * TR * P.Q[l].stride + tc * TC;
-        wcl = cl;
-        level = l;
-        r0 = tr;  // tile row / column of the subband
-        c0 = tc;
-        base = false;
-    } else {
-        const int bt = t - P.sub_pad;
-        const int tr = bt / P.ntc[kMaxL], tc = bt - tr * P.ntc[kMaxL];
-        win = P.X.base + tr * TR * P.X.stride + tc * TC;
-        out = 0;
-        wcl = 0;
-        level = kMaxL;
-        r0 = tr * TR;
-        c0 = tc * TC;
-        base = true;
-    }
-}
-
-void check_ws(const Plan& P, int u0, int n, unsigned seed, bool verbose) {
-    const int K = P.k, KK = K * K, p = P.p, L = P.L, H = P.H, W = P.W, ncls = 1 + 4 * L;
-    const int NSTG = P.nstg, np = P.npw * 32, nsub = P.n_sub_tiles, ntiles = P.n_step_tiles, nwt = P.nwt;
-    const int ncw = P.ncw, npw = P.npw;
-    Shadow sh(P.smem_floats);
-    sh.phase = "ws layout";
-    if (P.TR != 8 || P.TC != 4 || P.padded || P.nstrips != 1) sh.fail("ws plan shape", P.TR);
-    if (!(L == 0 || (P.pyr && L <= P.pyr_levels) || (!P.pyr && L == 1))) sh.fail("ws analysis is not one pass", L);
-    if (P.nthreads != (ncw + npw + 1) * 32 || P.nthreads > kWsMaxThreads || NSTG < 2 || NSTG > kWsMaxStg || npw < 1 ||
-        P.s_slots < 2 || P.s_slots > kWsMaxSSlots || P.x_slots != kWsQSlots)
-        sh.fail("ws threads / staging slots", P.nthreads);
-    if (nwt != (ntiles + 31) / 32 || P.sub_pad != (nsub + 31) / 32 * 32 || ntiles != P.sub_pad + P.n_base_tiles)
-        sh.fail("ws tile counts", ntiles);
-    if (P.smem_floats % 4 || P.smem_floats * 4LL > 227 * 1024) sh.fail("ws smem size", P.smem_floats);
-    // Regions: disjoint, in bounds, aligned.
-    struct R { long long lo, hi; const char* what; };
-    std::vector<R> regs;
-    regs.push_back({P.mbar, P.mbar + 2LL * kNumBars, "mbarriers"});
-    regs.push_back({P.desc, P.desc + 4LL * ntiles, "tile descriptors"});
-    for (int i = 0; i < P.x_slots; ++i)
-        regs.push_back({P.wbase + (long long)i * P.w_slot, P.wbase + (long long)i * P.w_slot + ncls * P.wcls + 1, "weights"});
-    for (int i = 0; i < NSTG; ++i)
-        regs.push_back({P.stg + (long long)i * P.stg_floats, P.stg + (long long)(i + 1) * P.stg_floats, "staging"});
-    const long long xsize = (long long)(P.ntr[kMaxL] * 8 + 2 * p) * P.X.stride;
-    if (xsize > P.x_slot) sh.fail("X slot too small", P.x_slot);
-    for (int i = 0; i < P.x_slots; ++i) regs.push_back({P.X.base + (long long)i * P.x_slot, P.X.base + (long long)i * P.x_slot + xsize, "X"});
-    for (int l = 0; l < L; ++l) {
-        for (int i = 0; i < P.s_slots; ++i)
-            regs.push_back({P.S[l].base + (long long)i * P.s_slot, P.S[l].base + (long long)i * P.s_slot + 4LL * P.S[l].sub, "S"});
-        for (int i = 0; i < kWsQSlots; ++i)
-            regs.push_back({P.Q[l].base + (long long)i * P.q_slot, P.Q[l].base + (long long)i * P.q_slot + 4LL * P.Q[l].sub, "Q"});
-    }
-    for (size_t a = 0; a < regs.size(); ++a) {
-        if (regs[a].lo < 0 || regs[a].hi > P.smem_floats) sh.fail(std::string(regs[a].what) + " outside shared memory", regs[a].lo);
-        for (size_t b = a + 1; b < regs.size(); ++b)
-            if (regs[a].lo < regs[b].hi && regs[b].lo < regs[a].hi)
-                sh.fail(std::string(regs[a].what) + " overlaps " + regs[b].what, regs[a].lo);
-    }
-    if (P.mbar % 2 || P.desc % 4 || P.stg % 4 || P.stg_floats % 4 || P.wbase % 4 || P.w_slot % 4 || P.x_slot % 4 ||
-        P.s_slot % 4 || P.q_slot % 4)
-        sh.fail("ws alignment", 0);
-    const long long plane_bytes = (long long)H * W * P.esize;
-    if (plane_bytes % 16 || plane_bytes != 4LL * P.stg_floats || plane_bytes >= (1LL << 20))
-        sh.fail("bulk copy size", plane_bytes);
-    if (P.X.stride >= 4096) sh.fail("window stride field", P.X.stride);
-    for (int l = 0; l < L; ++l)
-        if (P.S[l].stride >= 4096 || P.Q[l].stride >= 4096) sh.fail("stride field", l);
-
-    // Role programs.
-    // Roles: producer warps [0, npw), the copy warp npw, conv warps after it.
-    const int NS = P.s_slots, NX = P.x_slots, R = kWsBarRing;
-    std::vector<std::vector<Op>> prog(npw + 1 + ncw);
-    for (int pw = 0; pw < npw; ++pw) {
-        auto& g = prog[pw];
-        for (int j = 0; j < n; ++j) {
-            g.push_back({OP_WAIT, kBarStgFull + j % NSTG, j / NSTG, 0});
-            if (j >= NS && P.sub_pad > 0) g.push_back({OP_WAIT, kBarSub + (j - NS) % R, (j - NS) / R, 0});
-            if (j >= NX) g.push_back({OP_WAIT, kBarBase + (j - NX) % 3, (j - NX) / 3, 0});
-            g.push_back({OP_ANALYSE, 0, j, pw});
-            g.push_back({OP_ARRIVE, kBarStgEmpty + j % NSTG, j / NSTG, 0});
-            g.push_back({OP_ARRIVE, kBarAna + j % R, j / R, 0});
-        }
-    }
-    {
-        auto& g = prog[npw];
-        for (int q = 0; q < n; ++q) {
-            if (q >= NSTG) g.push_back({OP_WAIT, kBarStgEmpty + q % NSTG, (q - NSTG) / NSTG, 0});
-            g.push_back({OP_ISSUE, 0, q, 0});
-        }
-        for (int q = std::max(0, n - NSTG); q < n; ++q) g.push_back({OP_WAIT, kBarStgFull + q % NSTG, q / NSTG, 0});
-    }
-    // Conv warps take tasks from a shared counter (see the kernel): their
-    // programs are appended one task at a time when the role asks for work.
-    const int nsub_pad = P.sub_pad, nsub_wt = nsub_pad / 32, nbase_wt = nwt - nsub_wt, per_step = nsub_wt + nbase_wt;
-    const int ntasks = n * per_step;
-    int next_task = 0;
-    auto grab = [&](std::vector<Op>& g) {
-        const int t = next_task++;
-        int j, wt;
-        if (t < nsub_wt) {
-            j = 0;
-            wt = t;
-        } else {
-            const int h = t - nsub_wt;
-            j = 1 + h / per_step;
-            wt = h - (j - 1) * per_step;
-            if (j == n) wt += nsub_wt;
-        }
-        const bool is_sub = wt < nsub_wt;
-        const int jj = is_sub ? j : j - 1;
-        if (is_sub) {
-            g.push_back({OP_WAIT, kBarAna + jj % R, jj / R, 0});
-        } else if (nsub_wt > 0) {
-            g.push_back({OP_WAIT, kBarSub + jj % R, jj / R, 0});
-        } else {
-            g.push_back({OP_WAIT, kBarAna + jj % R, jj / R, 0});
-        }
-        g.push_back({OP_TILES, 0, j, wt});
-        g.push_back({OP_ARRIVE, is_sub ? kBarSub + jj % R : kBarBase + jj % 3, is_sub ? jj / R : jj / 3, 0});
-    };
-
-    MBar bars[kNumBars];
-    for (int i = 0; i < NSTG; ++i) {
-        bars[kBarStgFull + i].init(1);
-        bars[kBarStgEmpty + i].init(npw);
-    }
-    for (int i = 0; i < kWsBarRing; ++i) {
-        bars[kBarAna + i].init(npw);
-        bars[kBarSub + i].init(nsub_wt > 0 ? nsub_wt : 1);
-    }
-    for (int i = 0; i < 3; ++i) bars[kBarBase + i].init(nbase_wt);
-
-    std::vector<size_t> pc(prog.size(), 0);
-    std::vector<int> landing;  // planes whose bulk copy is in flight
-    const long long plane_elems = (long long)H * W;
-    std::vector<std::vector<int>> stored(n, std::vector<int>(plane_elems, 0));
-    const long long units = (long long)P.B * P.C;
-    auto chan = [&](int j) { return (u0 + j) / P.B; };
-    unsigned rng = seed * 2654435761u + 12345u;
-    auto rnd = [&]() { rng = rng * 1664525u + 1013904223u; return rng >> 8; };
-
-    // The hardware tests parity only: try_wait.parity(k & 1) passes whenever
-    // the current phase's parity differs from k's.  So a wait is only
-    // meaningful while the barrier is in phase k (blocks) or k + 1 (passes);
-    // two phases ahead it would block for good, and one phase behind (the
-    // phase before k still open) it would pass at once with k not complete.
-    auto wait_ok = [&](const Op& o, int role) {
-        const MBar& m = bars[o.bar];
-        if (m.phase < o.a) {
-            std::printf("FAIL ws: role %d (%s) waits on barrier %d for phase %d while phase %d is still open "
-                        "(parity would pass it at once; seed %u)\n", role,
-                        role < npw ? "producer" : role == npw ? "copy" : "conv", o.bar, o.a, m.phase, seed);
-            std::exit(1);
-        }
-        if (m.phase > o.a + 1) {
-            std::printf("FAIL ws: role %d (%s) wait on barrier %d for phase %d sees phase %d (two ahead; seed %u)\n", role,
-                        role < npw ? "producer" : role == npw ? "copy" : "conv", o.bar, o.a, m.phase, seed);
-            std::exit(1);
-        }
-        return ((m.phase ^ o.a) & 1) != 0;  // the hardware's test; equals m.phase == o.a + 1 here
-    };
-    auto land = [&](int j) {
-        sh.barrier();
-        sh.phase = "ws: bulk copy lands";
-        const long long stg = P.stg + (long long)(j % NSTG) * P.stg_floats;
-        const long long u = u0 + j;
-        const long long b = u % P.B, c = u / P.B;
-        check_global(((b * P.C + c) * plane_elems * P.esize + plane_bytes) - 1, units * plane_elems * P.esize,
-                     "bulk copy source");
-        for (long long f = 0; f < P.stg_floats; ++f) sh.write(stg + f, stg, stg + P.stg_floats, XT + 10 + plane_off(j), "staging");
-        MBar& m = bars[kBarStgFull + j % NSTG];
-        m.tx -= plane_bytes;
-        if (m.tx < 0) sh.fail("bulk copy transaction count", m.tx);
-        m.maybe_complete();
-    };
-    auto analyse = [&](int j, int pw, int seg) {
-        sh.barrier();
-        sh.phase = "ws: analysis share";
-        g_share = pw;
-        g_share_np = np;
-        g_tag_off = plane_off(j);
-        g_rank = 0;
-        const long long stg = P.stg + (long long)(j % NSTG) * P.stg_floats;
-        const long long xs = P.X.base + (long long)(j % P.x_slots) * P.x_slot;
-        Buf sb[kMaxL];
-        for (int l = 0; l < kMaxL; ++l) {
-            sb[l] = P.S[l];
-            sb[l].base += (j % P.s_slots) * P.s_slot;
-        }
-        const int stag = XT + 10 + plane_off(j), xt = XT + plane_off(j);
-        const long long xlo = xs, xhi = xs + xsize;
-        if (seg == 0) {
-            const int c = chan(j);
-            if (j < P.x_slots || c != chan(j - P.x_slots)) {
-                const long long ws = P.wbase + (long long)(j % P.x_slots) * P.w_slot;
-                for (int t = 0; t < ncls * KK; ++t) {
-                    if (!mine(t)) continue;
-                    const int cl = t / KK, tap = t - cl * KK;
-                    sh.write(ws + (long long)cl * P.wcls + tap, ws, ws + ncls * P.wcls, WTS + chan_off(c), "ws weights");
-                }
-                if (pw == 0) sh.write(ws + P.bias, ws + P.bias, ws + P.bias + 1, BIAS + chan_off(c), "ws bias");
-            }
-            if (P.pyr) {
-                replay_pyramid(sh, P, stg, stag, xs + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, xt, sb, p, s_tag_ws);
-            } else {
-                const Buf& b0 = sb[0];
-                replay_unpack(sh, P, stg, stag, xs + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, xt,
-                              L >= 1 ? b0.base + (long long)p * b0.stride + p : 0, b0.stride, b0.sub, b0.base, s_tag_ws, L >= 1);
-            }
-        } else {
-            const int done = P.pyr ? P.pyr_levels : (L >= 1 ? 1 : 0);
-            const int l = done + seg - 1;
-            const int nn = H >> (l + 1), m = W >> (l + 1);
-            const Buf& s0 = sb[l - 1];
-            const Buf& s1 = sb[l];
-            replay_haar(sh, s0.base + (long long)p * s0.stride + p, s0.stride, s0.base, s0.base + s0.sub, s_tag_ws(l - 1, 0), nn,
-                        m, s1.base + (long long)p * s1.stride + p, s1.stride, s1.sub, s1.base, s1.base + 4LL * s1.sub, s_tag_ws,
-                        l);
-        }
-        g_share = -1;
-    };
-    auto tiles = [&](int j, int wt) {
-        sh.barrier();
-        for (int lane = 0; lane < 32; ++lane) {
-            const int t = 32 * wt + lane;
-            if (t >= ntiles) continue;
-            if (t >= nsub && t < P.sub_pad) continue;  // padding
-            int win, out, wcl, level, r0, c0;
-            bool base;
-            ws_desc_host(P, t, win, out, wcl, level, r0, c0, base);
-            if (base ? j < 1 : j >= n) continue;
-            const int jj = base ? j - 1 : j;
-            const int c = chan(jj);
-            const long long ws = P.wbase + (long long)(jj % P.x_slots) * P.w_slot;
-            sh.phase = base ? "ws: base tile" : "ws: sub tile";
-            if ((ws + (long long)wcl * P.wcls) % 4) sh.fail("weight class alignment", ws);
-            for (int q = 0; q < KK; ++q)
-                sh.read(ws + (long long)wcl * P.wcls + q, ws, ws + ncls * P.wcls, WTS + chan_off(c), "ws weights read");
-            if (base) {
-                sh.read(ws + P.bias, ws + P.bias, ws + P.bias + 1, BIAS + chan_off(c), "ws bias read");
-                const long long xs = P.X.base + (long long)(jj % P.x_slots) * P.x_slot;
-                if (win != P.X.base + (r0 / 8) * 8 * P.X.stride + c0) sh.fail("base descriptor", t);
-                replay_window(sh, P, xs, P.X.stride, xs, xs + xsize, H, W, r0 / 8, c0 / 4, XT + plane_off(jj), "ws base window", 0);
-                // Synthesis epilogue reads (synth_tile).
-                const long long qs = (long long)(jj % kWsQSlots) * P.q_slot;
-                auto qread = [&](int l, int s2, int pr, int pc, bool need) {
-                    const Buf& Q = P.Q[l];
-                    const long long lo = qs + Q.base + (long long)s2 * Q.sub, hi = lo + Q.sub;
-                    const long long a = lo + (long long)pr * Q.stride + pc;
-                    if (need) {
-                        if (pr >= (H >> (l + 1)) || pc >= (W >> (l + 1))) sh.fail("synthesis position outside the subband", l);
-                        sh.read(a, lo, hi, q_tag(l, s2) + plane_off(jj), "ws synthesis Q read");
-                    } else {
-                        sh.touch(a, lo, hi, "ws synthesis Q read (unused)");
-                    }
-                };
-                // A level-l position (pr, pc) feeds outputs of rows
-                // [pr << (l+1), (pr+1) << (l+1)); it is needed when one of them
-                // lies in this tile and in the plane.
-                auto need = [&](int l, int pr) {
-                    const int lo = std::max(pr << (l + 1), r0), hi = std::min((pr + 1) << (l + 1), std::min(r0 + 8, H));
-                    return lo < hi;
-                };
-                for (int l = kMaxL - 1; l >= 3; --l) {
-                    if (l >= L) continue;
-                    const int pr = r0 >> (l + 1), pcc = c0 >> (l + 1);
-                    for (int s2 = 0; s2 < 4; ++s2) qread(l, s2, pr, pcc, need(l, pr));
-                }
-                if (L >= 3)
-                    for (int s2 = 0; s2 < 4; ++s2) qread(2, s2, r0 >> 3, c0 >> 3, need(2, r0 >> 3));
-                if (L >= 2)
-                    for (int ah = 0; ah < 2; ++ah)
-                        for (int s2 = 0; s2 < 4; ++s2) qread(1, s2, (r0 >> 2) + ah, c0 >> 2, need(1, (r0 >> 2) + ah));
-                if (L >= 1)
-                    for (int a = 0; a < 4; ++a)
-                        for (int s2 = 0; s2 < 4; ++s2) {
-                            const long long addr = qs + P.Q[0].base + (long long)s2 * P.Q[0].sub +
-                                                   (long long)((r0 >> 1) + a) * P.Q[0].stride + (c0 >> 1);
-                            if (addr % 2) sh.fail("level-0 pair load not 8-byte aligned", addr);
-                            for (int e = 0; e < 2; ++e) qread(0, s2, (r0 >> 1) + a, (c0 >> 1) + e, need(0, (r0 >> 1) + a));
-                        }
-                for (int o = 0; o < 8; ++o) {
-                    if (r0 + o >= H) continue;
-                    if (c0 + 4 > W) sh.fail("base tile column", c0);
-                    for (int e = 0; e < 4; ++e) ++stored[jj][(long long)(r0 + o) * W + c0 + e];
-                }
-            } else {
-                const int s2 = (wcl - 1) & 3;
-                const Buf& S = P.S[level];
-                const Buf& Q = P.Q[level];
-                const long long ss = (long long)(jj % P.s_slots) * P.s_slot, qq = (long long)(jj % kWsQSlots) * P.q_slot;
-                const long long slo = ss + S.base + (long long)s2 * S.sub;
-                replay_window(sh, P, slo, S.stride, slo, slo + S.sub, H >> (level + 1), W >> (level + 1), r0, c0,
-                              s_tag(level, s2) + plane_off(jj), "ws subband window", 0);
-                const long long o0 = qq + out;
-                if (o0 % 4) sh.fail("Q tile not 16-byte aligned", o0);
-                const long long qlo = qq + Q.base + (long long)s2 * Q.sub;
-                for (int o = 0; o < 8; ++o)
-                    for (int e = 0; e < 4; ++e)
-                        sh.write(o0 + (long long)o * Q.stride + e, qlo, qlo + Q.sub, q_tag(level, s2) + plane_off(jj), "ws Q tile");
-            }
-        }
-    };
-
-    const int nroles = (int)prog.size();
-    long long steps = 0;
-    // seed 0: producers first where possible; 1: conv warps first; others random.
-    auto runnable = [&](int r) -> bool {
-        if (pc[r] >= prog[r].size()) return r > npw && next_task < ntasks;  // a conv warp can take a task
-        const Op& o = prog[r][pc[r]];
-        if (o.k == OP_WAIT) return wait_ok(o, r);
-        return true;
-    };
-    for (;;) {
-        std::vector<int> ready;
-        for (int r = 0; r < nroles; ++r)
-            if (runnable(r)) ready.push_back(r);
-        const bool all_done = [&] {
-            for (int r = 0; r < nroles; ++r)
-                if (pc[r] < prog[r].size()) return false;
-            return next_task >= ntasks;
-        }();
-        if (all_done && landing.empty()) break;
-        if (ready.empty() && landing.empty()) {
-            std::printf("FAIL ws: deadlock after %lld actions (seed %u); next ops:", steps, seed);
-            for (int r = 0; r < nroles; ++r)
-                if (pc[r] < prog[r].size())
-                    std::printf(" [role %d op %d bar %d a %d]", r, (int)prog[r][pc[r]].k, prog[r][pc[r]].bar, prog[r][pc[r]].a);
-            std::printf("\n");
-            std::exit(1);
-        }
-        ++steps;
-        // Choose: a landing or a role.
-        const size_t nchoice = ready.size() + landing.size();
-        size_t pick;
-        if (seed == 0) pick = !ready.empty() ? 0 : ready.size();          // lowest role first (producers)
-        else if (seed == 1) pick = !ready.empty() ? ready.size() - 1 : ready.size();  // conv warps first
-        else pick = rnd() % nchoice;
-        if (pick >= ready.size()) {
-            const size_t li = pick - ready.size();
-            const int j = landing[li];
-            landing.erase(landing.begin() + li);
-            land(j);
-            continue;
-        }
-        const int r = ready[pick];
-        if (pc[r] >= prog[r].size()) {  // a conv warp takes the next task
-            grab(prog[r]);
-            continue;
-        }
-        const Op o = prog[r][pc[r]];
-        switch (o.k) {
-            case OP_WAIT: ++pc[r]; break;
-            case OP_ARRIVE: bars[o.bar].arrive(o.a); ++pc[r]; break;
-            case OP_ISSUE: {
-                MBar& m = bars[kBarStgFull + o.a % NSTG];
-                m.tx += plane_bytes;  // arrive.expect_tx: expect, then arrive
-                m.arrive();
-                landing.push_back(o.a);
-                ++pc[r];
-                break;
-            }
-            case OP_ANALYSE: analyse(o.a, o.b, 0); ++pc[r]; break;
-            case OP_TILES: tiles(o.a, o.b); ++pc[r]; break;
-        }
-    }
-    for (int j = 0; j < n; ++j)
-        for (long long e = 0; e < plane_elems; ++e)
-            if (stored[j][e] != 1) {
-                std::printf("FAIL ws: plane %d output %lld stored %d times\n", j, e, stored[j][e]);
-                std::exit(1);
-            }
-    for (int i = 0; i < kNumBars; ++i)
-        if (bars[i].expected && bars[i].pending != bars[i].expected) {
-            std::printf("FAIL ws: barrier %d left with %d of %d arrivals pending\n", i, bars[i].pending, bars[i].expected);
-            std::exit(1);
-        }
-    if (verbose)
-        std::printf("ws: smem %d B, threads %d (%d conv + %d producer warps + 1 copy warp), rings stg %d X %d S %d, tiles %d+%d, planes %d from %d\n",
-                    P.smem_floats * 4, P.nthreads, ncw, npw, NSTG, P.x_slots, P.s_slots, nsub, P.n_base_tiles, n, u0);
-}
-
-void check_ws_all(const Plan& P, Kind kind) {
-    const long long units = (long long)P.B * P.C;
-    const int n = (int)std::min<long long>(units, 9);
-    // From the first unit, and across a channel boundary.
-    const int u_alt = (int)std::min<long long>(std::max(0, P.B - 4), units - n);
-    for (unsigned seed = 0; seed < 40; ++seed) check_ws(P, seed % 2 ? u_alt : 0, n, seed, seed == 0);
-    // A short run (fewer planes than staging slots) and a single plane.
-    check_ws(P, 0, std::min(n, 2), 3, false);
-    check_ws(P, 0, 1, 4, false);
-    std::printf("fused(kind %d): warp-specialised\n", (int)kind);
-}
-
-// ---------------------------------------------------------------------------
-// Two alternating warp groups (wtconv_duo.cuh): the kernel's half-cycle
-// schedule replayed with its barriers as phase boundaries (a CTA barrier
-// ends every half-cycle; inside A the group barrier splits the analysis from
-// the staging of the next plane), every access checked against tags that
-// carry the plane (and, for the weights, the channel).
-// ---------------------------------------------------------------------------
-void check_duo(const Plan& P, int u0, int n) {
-    const int K = P.k, KK = K * K, p = P.p, L = P.L, H = P.H, W = P.W, ncls = 1 + 4 * L;
-    const int nsub = P.n_sub_tiles, ntiles = P.n_step_tiles;
-    Shadow sh(P.smem_floats);
-    sh.phase = "duo layout";
-    if (P.TR != 8 || P.TC != 4 || P.padded || P.nstrips != 1 || P.nthreads != kDuoThreads || P.sub_pad != nsub ||
-        ntiles != nsub + P.n_base_tiles)
-        sh.fail("duo plan", P.nthreads);
-    if (P.smem_floats % 4 || P.smem_floats * 4LL > 227 * 1024 || P.gbase % 4 || P.gsize % 4) sh.fail("duo smem", 0);
-    if (P.gbase < 4LL * ntiles || P.gbase + 2LL * P.gsize > P.smem_floats) sh.fail("duo groups", P.gbase);
-    const long long xsize = (long long)(P.ntr[kMaxL] * 8 + 2 * p) * P.X.stride;
-    struct R { long long lo, hi; const char* what; };
-    std::vector<R> regs;
-    for (int i = 0; i < 2; ++i) {
-        regs.push_back({P.wbase + (long long)i * P.w_slot, P.wbase + (long long)i * P.w_slot + ncls * P.wcls + 1, "weights"});
-        regs.push_back({P.X.base + (long long)i * P.x_slot, P.X.base + (long long)i * P.x_slot + xsize, "X"});
-        for (int l = 0; l < L; ++l)
-            regs.push_back({P.Q[l].base + (long long)i * P.q_slot, P.Q[l].base + (long long)i * P.q_slot + 4LL * P.Q[l].sub, "Q"});
-    }
-    regs.push_back({P.stg, P.stg + (long long)P.stg_floats, "staging"});
-    for (int l = 0; l < L; ++l) regs.push_back({P.S[l].base, P.S[l].base + 4LL * P.S[l].sub, "S"});
-    for (size_t a = 0; a < regs.size(); ++a) {
-        if (regs[a].lo < 0 || regs[a].hi > P.gsize) sh.fail(std::string(regs[a].what) + " outside its group", regs[a].lo);
-        for (size_t b = a + 1; b < regs.size(); ++b)
-            if (regs[a].lo < regs[b].hi && regs[b].lo < regs[a].hi)
-                sh.fail(std::string(regs[a].what) + " overlaps " + regs[b].what, regs[a].lo);
-    }
-    if (P.stg % 4 || P.w_slot % 4 || P.x_slot % 4 || P.q_slot % 4 || (P.gbase + P.stg) % 4 || (P.gbase + P.gsize) % 4)
-        sh.fail("duo alignment", 0);
-    const long long plane_elems = (long long)H * W, units = (long long)P.B * P.C;
-    std::vector<std::vector<int>> stored(n, std::vector<int>(plane_elems, 0));
-    auto chan = [&](int j) { return (u0 + j) / P.B; };
-    // Local plane j of group g = g + 2k.
-    auto stage = [&](int g, int k) {
-        const long long gb = P.gbase + (long long)g * P.gsize;
-        const int j = g + 2 * k;
-        const long long u = u0 + j;
-        check_global(((u % P.B) * P.C + u / P.B) * plane_elems * P.esize + (long long)P.plane_chunks * 16 - 1,
-                     units * plane_elems * P.esize, "staging source");
-        for (long long f = 0; f < P.stg_floats; ++f)
-            sh.write(gb + P.stg + f, gb + P.stg, gb + P.stg + P.stg_floats, XT + 10 + plane_off(j), "duo staging");
-    };
-    auto analyse = [&](int g, int k) {
-        const long long gb = P.gbase + (long long)g * P.gsize;
-        const int j = g + 2 * k;
-        g_share = -1;
-        g_tag_off = plane_off(j);
-        g_rank = 0;
-        const int c = chan(j);
-        const long long ws = gb + P.wbase + (long long)(k & 1) * P.w_slot;
-        if (k < 2 || c != chan(j - 4)) {
-            for (int t = 0; t < ncls * KK; ++t) {
-                const int cl = t / KK, tap = t - cl * KK;
-                sh.write(ws + (long long)cl * P.wcls + tap, ws, ws + ncls * P.wcls, WTS + chan_off(c), "duo weights");
-            }
-            sh.write(ws + P.bias, ws + P.bias, ws + P.bias + 1, BIAS + chan_off(c), "duo bias");
-        }
-        Buf sb[kMaxL];
-        for (int l = 0; l < kMaxL; ++l) {
-            sb[l] = P.S[l];
-            sb[l].base += gb;
-        }
-        const long long xs = gb + P.X.base + (long long)(k & 1) * P.x_slot;
-        replay_analyse(sh, P, gb + P.stg, XT + 10 + plane_off(j), xs + (long long)p * P.X.stride + p, P.X.stride, xs,
-                       xs + xsize, XT + plane_off(j), sb, p, s_tag_ws);
-    };
-    auto tiles = [&](int g, int k, int m) {
-        const long long gb = P.gbase + (long long)g * P.gsize;
-        for (int t = 0; t < ntiles; ++t) {
-            const bool base = t >= nsub;
-            if (base ? k < 1 : k >= m) continue;
-            const int kk = base ? k - 1 : k, j = g + 2 * kk;
-            int win, out, wcl, level, r0, c0;
-            bool b2;
-            ws_desc_host(P, t, win, out, wcl, level, r0, c0, b2);
-            const long long ws = gb + P.wbase + (long long)(kk & 1) * P.w_slot;
-            sh.phase = base ? "duo: base tile" : "duo: sub tile";
-            for (int q = 0; q < KK; ++q)
-                sh.read(ws + (long long)wcl * P.wcls + q, ws, ws + ncls * P.wcls, WTS + chan_off(chan(j)), "duo weights read");
-            if (base) {
-                sh.read(ws + P.bias, ws + P.bias, ws + P.bias + 1, BIAS + chan_off(chan(j)), "duo bias read");
-                const long long xs = gb + P.X.base + (long long)(kk & 1) * P.x_slot;
-                replay_window(sh, P, xs, P.X.stride, xs, xs + xsize, H, W, r0 / 8, c0 / 4, XT + plane_off(j), "duo base window", 0);
-                const long long qs = gb + (long long)(kk & 1) * P.q_slot;
-                auto need = [&](int l, int pr) {
-                    const int lo = std::max(pr << (l + 1), r0), hi = std::min((pr + 1) << (l + 1), std::min(r0 + 8, H));
-                    return lo < hi;
-                };
-                auto qread = [&](int l, int s2, int pr, int pc, bool nd) {
-                    const Buf& Q = P.Q[l];
-                    const long long lo = qs + Q.base + (long long)s2 * Q.sub, hi = lo + Q.sub;
-                    const long long a = lo + (long long)pr * Q.stride + pc;
-                    if (nd) sh.read(a, lo, hi, q_tag(l, s2) + plane_off(j), "duo synthesis Q read");
-                    else sh.touch(a, lo, hi, "duo synthesis Q read (unused)");
-                };
-                for (int l = kMaxL - 1; l >= 3; --l) {
-                    if (l >= L) continue;
-                    for (int s2 = 0; s2 < 4; ++s2) qread(l, s2, r0 >> (l + 1), c0 >> (l + 1), need(l, r0 >> (l + 1)));
-                }
-                if (L >= 3)
-                    for (int s2 = 0; s2 < 4; ++s2) qread(2, s2, r0 >> 3, c0 >> 3, need(2, r0 >> 3));
-                if (L >= 2)
-                    for (int ah = 0; ah < 2; ++ah)
-                        for (int s2 = 0; s2 < 4; ++s2) qread(1, s2, (r0 >> 2) + ah, c0 >> 2, need(1, (r0 >> 2) + ah));
-                if (L >= 1)
-                    for (int a = 0; a < 4; ++a)
-                        for (int s2 = 0; s2 < 4; ++s2)
-                            for (int e = 0; e < 2; ++e) qread(0, s2, (r0 >> 1) + a, (c0 >> 1) + e, need(0, (r0 >> 1) + a));
-                for (int o = 0; o < 8; ++o) {
-                    if (r0 + o >= H) continue;
-                    for (int e = 0; e < 4; ++e) ++stored[j][(long long)(r0 + o) * W + c0 + e];
-                }
-            } else {
-                const int s2 = (wcl - 1) & 3;
-                const Buf& S = P.S[level];
-                const Buf& Q = P.Q[level];
-                const long long slo = gb + S.base + (long long)s2 * S.sub;
-                replay_window(sh, P, slo, S.stride, slo, slo + S.sub, H >> (level + 1), W >> (level + 1), r0, c0,
-                              s_tag(level, s2) + plane_off(j), "duo subband window", 0);
-                const long long qq = gb + (long long)(kk & 1) * P.q_slot;
-                const long long qlo = qq + Q.base + (long long)s2 * Q.sub;
-                for (int o = 0; o < 8; ++o)
-                    for (int e = 0; e < 4; ++e)
-                        sh.write(qq + out + (long long)o * Q.stride + e, qlo, qlo + Q.sub, q_tag(level, s2) + plane_off(j), "duo Q tile");
-            }
-        }
-    };
-    const int mg[2] = {(n + 1) / 2, n / 2};
-    for (int g = 0; g < 2; ++g)
-        if (mg[g] > 0) stage(g, 0);
-    const int Hh = std::max(2 * mg[0] + 2, 2 * mg[1] + 3);
-    for (int h = 0; h < Hh; ++h) {
-        sh.barrier();
-        int a_grp = -1, a_k = -1;
-        for (int g = 0; g < 2; ++g) {
-            const bool runs_a = ((h + g) & 1) == 0;
-            if (runs_a) {
-                const int k = (h - g) >> 1;
-                if (k >= 0 && k < mg[g]) {
-                    sh.phase = "duo: analysis";
-                    analyse(g, k);
-                    a_grp = g;
-                    a_k = k;
-                }
-            } else {
-                const int k = (h - 1 - g) >> 1;
-                if (k >= 0 && k <= mg[g]) tiles(g, k, mg[g]);
-            }
-        }
-        if (a_grp >= 0 && a_k + 1 < mg[a_grp]) {
-            sh.barrier();  // the group barrier after the analysis
-            sh.phase = "duo: staging";
-            stage(a_grp, a_k + 1);
-        }
-    }
-    for (int j = 0; j < n; ++j)
-        for (long long e = 0; e < plane_elems; ++e)
-            if (stored[j][e] != 1) {
-                std::printf("FAIL duo: plane %d output %lld stored %d times\n", j, e, stored[j][e]);
-                std::exit(1);
-            }
-}
-
-void check_duo_all(const Plan& P, Kind kind) {
-    const long long units = (long long)P.B * P.C;
-    const int n = (int)std::min<long long>(units, 9);
-    const int u_alt = (int)std::min<long long>(std::max(0, P.B - 4), units - n);
-    check_duo(P, 0, n);
-    check_duo(P, u_alt, n);
-    check_duo(P, 0, std::min(n, 2));
-    check_duo(P, 0, 1);
-    std::printf("fused(kind %d): two alternating warp groups, smem %d B\n", (int)kind, P.smem_floats * 4);
 }
 
 }  // namespace
