@@ -338,11 +338,23 @@ class Workload:
             wt.backward(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
                         dx=self.dx, grads=grads, workspace=self.ws, stream=stream)
 
+        def bwd_one_pass():
+            wt.backward(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
+                        dx=self.dx, grads=grads, workspace=self.ws, stream=stream, one_pass=True)
+
         self.calls = [("fwd", fwd), ("bwd_in", bwd_in), ("bwd_w", bwd_w)]
         if world > 1:
             import torch.distributed as dist
             self.calls.append(("allreduce", lambda: allreduce_weight_grads(grads, self.flat, dist)))
         self.bwd_fused = bwd_fused
+        # The one-pass kernel, where the shape has a one-pass plan.
+        try:
+            bwd_one_pass()
+            self.bwd_one_pass = bwd_one_pass
+        except wt.WTConvError as e:
+            if e.code != 8:  # WTCONV_ERR_UNSUPPORTED: planes split into cluster strips
+                raise
+            self.bwd_one_pass = None
 
     def time_calls(self, calls, steps: int, warmup: int, flush, clocks=None):
         """Per-call device times (ms) of `steps` timed steps after `warmup`
@@ -397,6 +409,32 @@ def call_record(case, per_call_ms: dict, peak: float) -> dict:
 
 def median(v):
     return statistics.median(v)
+
+
+def backward_record(wl, case, per_call_ms: dict, steps: int, flush, dist=None, dev=None) -> tuple:
+    """The whole-backward calls beside the two passes, same protocol: the
+    library's pick (wtconv_backward) and the one-pass kernel
+    (wtconv_backward_one_pass).  Returns (record, kernel launches timed)."""
+    calls = [("library_pick", wl.bwd_fused)]
+    if wl.bwd_one_pass is not None:
+        calls.append(("one_pass", wl.bwd_one_pass))
+    t, _, _ = wl.time_calls(calls, steps, 3, flush)
+    ms = {n: median(v) for n, v in t.items()}
+    if dist is not None:
+        ms = {n: max_over_ranks(v, dist, dev) for n, v in ms.items()}
+    two = per_call_ms["bwd_in"] + per_call_ms["bwd_w"]
+    fb_bytes = 3 * case.numel * case.esize + 2 * 4 * param_floats(case)
+    rec = {
+        "call": "wtconv_backward: dx and all parameter gradients (the library picks the one-pass kernel or the "
+                "two passes by the planner's cost); wtconv_backward_one_pass: the one-pass kernel",
+        "two_pass_us": two * 1e3,
+        "library_pick_us": ms["library_pick"] * 1e3,
+        "one_pass_us": ms["one_pass"] * 1e3 if "one_pass" in ms else None,
+        "one_pass_modeled_bytes": fb_bytes,
+        "one_pass_gbs": fb_bytes / (ms["one_pass"] * 1e-3) / 1e9 if "one_pass" in ms else None,
+        "step_forward_plus_library_pick_us": (per_call_ms["fwd"] + ms["library_pick"]) * 1e3,
+    }
+    return rec, steps * (2 + (1 if "one_pass" in ms else 0))
 
 
 def run_ours(args, case):
@@ -478,34 +516,26 @@ def run_ours(args, case):
         line["e2e"] = e2e(args, case, wl.g, wl.grads, wl.ws, dev, world)
     if world > 1:
         dist.barrier()
-    # The one-pass backward (wtconv_backward), timed after the step with the
-    # same protocol; reported beside the three-call step, not in it.
+    # The whole-backward calls (library pick, one-pass kernel), timed after
+    # the step with the same protocol; reported beside the three-call step,
+    # not in it.
     KF = min(K, 500)
-    ft, _, _ = wl.time_calls([("bwd_fused", wl.bwd_fused)], KF, 3, flush)
-    fb_ms = median(ft["bwd_fused"])
-    if world > 1:
-        fb_ms = max_over_ranks(fb_ms, dist, dev)
-    fb_bytes = 3 * case.numel * case.esize + 2 * 4 * param_floats(case)
-    fstep_bytes = mb["fwd"] + fb_bytes
-    fstep_ms = per_call["fwd"] + fb_ms
-    line["fused_backward"] = {
-        "call": "wtconv_backward (dx and all parameter gradients; one pass or the two passes, as the library picks)",
-        "us_per_call": fb_ms * 1e3, "modeled_bytes": fb_bytes, "gbs": fb_bytes / (fb_ms * 1e-3) / 1e9,
-        "step_forward_plus_fused_backward_us": fstep_ms * 1e3,
-        "step_modeled_bytes": fstep_bytes,
-        "step_gbs": fstep_bytes * world / (fstep_ms * 1e-3) / 1e9,
-    }
+    line["fused_backward"], n_launch = backward_record(wl, case, per_call, KF, flush,
+                                                       dist if world > 1 else None, dev)
+    line["gpu_launches"] += n_launch
     # The other WTConvNeXt stage shapes, same protocol, one GPU.
     if world == 1 and not args.no_other_workloads:
         other = {}
         for name in ("stage1", "stage2", "train_bf16"):
             if name == case.name:
-                other[name] = rec
+                other[name] = dict(rec, fused_backward=line["fused_backward"])
                 continue
             del_wl = Workload(NAMED[name], dev, stream, 0, 1)
             t2, _, _ = del_wl.time_calls(del_wl.calls, K, args.warmup, flush)
-            other[name] = call_record(NAMED[name], {n: median(v) for n, v in t2.items()}, peak)
-            line["gpu_launches"] += K * 3
+            pc2 = {n: median(v) for n, v in t2.items()}
+            other[name] = call_record(NAMED[name], pc2, peak)
+            other[name]["fused_backward"], n_launch = backward_record(del_wl, NAMED[name], pc2, KF, flush)
+            line["gpu_launches"] += K * 3 + n_launch
             del del_wl
             torch.cuda.empty_cache()
         line["workloads"] = other
@@ -786,6 +816,15 @@ def run_sweep(args):
             "bwd_w": lambda: wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"],
                                                 g["wt_scale"], L, grads=grads, workspace=ws, stream=stream),
         }
+        def one_pass():
+            wt.backward(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L,
+                        dx=dx, grads=grads, workspace=ws, stream=stream, one_pass=True)
+        try:  # the one-pass backward kernel, timed beside the step where the shape has a plan for it
+            one_pass()
+            calls["one_pass_bwd"] = one_pass
+        except wt.WTConvError as e:
+            if e.code != 8:
+                raise
         us = {}
         for name, f in calls.items():
             for _ in range(3):
@@ -801,12 +840,14 @@ def run_sweep(args):
             torch.cuda.synchronize(dev)
             us[name] = sorted(a.elapsed_time(b) for a, b in ev)[len(ev) // 2] * 1e3
         mb = modeled_bytes(case)
+        one_pass_us = us.pop("one_pass_bwd", None)
         step_us = sum(us.values())
         gbs = sum(mb.values()) / (step_us * 1e-6) / 1e9
         alu = 3 * 2 * conv_fmas(case) / (step_us * 1e-6) / alu_peak
         row = {"sweep_point": case.name, "B": case.B, "C": case.C, "H": case.H, "k": case.k, "L": case.L,
                "us": {k: round(v, 1) for k, v in us.items()}, "step_us": round(step_us, 1),
-               "gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4), "alu_frac": round(alu, 4)}
+               "gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4), "alu_frac": round(alu, 4),
+               "one_pass_bwd_us": None if one_pass_us is None else round(one_pass_us, 1)}
         rows.append(row)
         print(json.dumps(row), flush=True)
         del g, y, dx, grads, ws

@@ -47,10 +47,14 @@
  *     written (the input gradient is the transpose of that cropped map; the
  *     weight gradients sum over the padded plane, where dy is zero); their rows
  *     must be whole 16-byte chunks (W a multiple of 4 for fp32, 8 for bf16).
- *     A plane that does not fit on one SM is split into 2, 4 or 8 row strips
- *     held by the CTAs of a thread-block cluster (strip height a multiple of
- *     2^L and of 4); planes that still do not fit return
- *     WTCONV_ERR_UNSUPPORTED.
+ *     A plane that does not fit on one SM is split into 2, 4, 8 or 16 row
+ *     strips held by the CTAs of a thread-block cluster (strip height a
+ *     multiple of 2^L and of 4; 16-CTA clusters use the non-portable cluster
+ *     size); planes that still do not fit return WTCONV_ERR_UNSUPPORTED.
+ *   - Plans (grid sizes, the weight gradient's batch groups and so its
+ *     workspace size) are made for the SM count of the device current at the
+ *     call; make the wtconv_workspace_bytes call and the call that uses the
+ *     workspace with the same device current.
  *   - L = 0 is the base branch only; wt_w and wt_scale may then be NULL.
  *   - Calls are reentrant; apart from the fixed scratch array of
  *     wtconv_backward_weight_noalloc (see there), the library holds no
@@ -92,13 +96,17 @@ typedef struct {
 /* Human-readable name of a status code (static string, never NULL). */
 const char *wtconv_status_string(wtconv_status_t s);
 
-/* Bytes of device workspace wtconv_backward_weight and wtconv_backward need
- * for `d` (0 if `d` is invalid); one size serves both.  The forward and
- * input-gradient calls need none. */
+/* Bytes of device workspace wtconv_backward_weight, wtconv_backward and
+ * wtconv_backward_one_pass need for `d` on the current device (0 if `d` is
+ * invalid); one size serves all three.  Planned for 148 SMs (a B200) when no
+ * CUDA device can be queried.  The forward and input-gradient calls need
+ * none: every intermediate stays on chip. */
 size_t wtconv_workspace_bytes(const wtconv_desc_t *d);
 
-/* Forward pass: y = WTConv(x).  x, y: [B][C][H][W] in desc->dtype; x and y
- * must not overlap.  Reads x once and writes y once. */
+/* Forward pass: y = WTConv(x), the fused layer of the Abstract with its three
+ * reformulations (on-chip Haar analysis, closed-form synthesis, scales folded
+ * into the weights).  x, y: [B][C][H][W] in desc->dtype; x and y must not
+ * overlap.  Reads x once and writes y once. */
 wtconv_status_t wtconv_forward(const wtconv_desc_t *d, const void *x,
                                const float *base_w, const float *base_b, const float *base_scale,
                                const float *wt_w, const float *wt_scale,
@@ -106,7 +114,9 @@ wtconv_status_t wtconv_forward(const wtconv_desc_t *d, const void *x,
 
 /* Gradient with respect to the input: dx = J^T dy, the transpose of the
  * forward map (the same pass run on dy with every kernel rotated by 180
- * degrees and no bias).  dy, dx: [B][C][H][W] in desc->dtype; must not
+ * degrees and no bias), one of the backward passes of the training step
+ * whose speedup the Abstract reports; the same three reformulations apply
+ * to the transposed map.  dy, dx: [B][C][H][W] in desc->dtype; must not
  * overlap. */
 wtconv_status_t wtconv_backward_input(const wtconv_desc_t *d, const void *dy,
                                       const float *base_w, const float *base_scale,
@@ -114,7 +124,10 @@ wtconv_status_t wtconv_backward_input(const wtconv_desc_t *d, const void *dy,
                                       void *dx, wtconv_stream_t stream);
 
 /* Gradients with respect to every parameter, summed over the batch and all
- * positions (overwritten):
+ * positions (overwritten); the other backward pass of the Abstract's
+ * training step, with the subbands of x and dy recomputed on chip
+ * (reformulation (1)) and the folded scales' gradients recovered from the
+ * unscaled correlations (reformulation (3)):
  *   d_base_w[c][u][v]   = base_scale[c] * sum dy[h][w] x[h+u-p][w+v-p]
  *   d_base_b[c]         = base_scale[c] * sum dy
  *   d_base_scale[c]     = sum dy * (dwconv(x, base_w[c]) + base_b[c])
@@ -131,19 +144,35 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, co
                                        void *workspace, size_t workspace_bytes,
                                        wtconv_stream_t stream);
 
-/* Fused backward: dx (as wtconv_backward_input) and every parameter gradient
- * (as wtconv_backward_weight, bitwise-repeatable) in one pass that reads x
- * and dy once and writes dx once -- the backward half of the training step
- * the Abstract's speedup refers to.  dx: [B][C][H][W] in desc->dtype, not
- * overlapping x or dy.  Workspace as for wtconv_backward_weight.  Planes too
- * large for one SM (split into cluster strips) are done in the two separate
- * passes instead, with the same results. */
+/* Whole backward of the layer (the backward half of the Abstract's training
+ * step): dx (as wtconv_backward_input) and every parameter gradient (as
+ * wtconv_backward_weight, bitwise-repeatable).  The library picks the path:
+ * the one-pass kernel of wtconv_backward_one_pass where its plan exists and
+ * the planner's cost (conv-tile rows on the busiest SM sub-partition) is
+ * below that of the two passes together, else wtconv_backward_input then
+ * wtconv_backward_weight.  Both paths give the same results.  dx:
+ * [B][C][H][W] in desc->dtype, not overlapping x or dy.  Workspace as for
+ * wtconv_backward_weight.  Every argument is checked before either pass is
+ * enqueued. */
 wtconv_status_t wtconv_backward(const wtconv_desc_t *d, const void *x, const void *dy,
                                 const float *base_w, const float *base_b, const float *base_scale,
                                 const float *wt_w, const float *wt_scale, void *dx,
                                 float *d_base_w, float *d_base_b, float *d_base_scale,
                                 float *d_wt_w, float *d_wt_scale,
                                 void *workspace, size_t workspace_bytes, wtconv_stream_t stream);
+
+/* The one-pass backward: the results of wtconv_backward from one kernel that
+ * reads x and dy once and writes dx once (the fewest HBM bytes of any
+ * backward, per the Abstract's I/O model), at the cost of an on-chip
+ * footprint that holds one CTA per SM.  Only whole planes: a plane split
+ * into cluster strips returns WTCONV_ERR_UNSUPPORTED.  Arguments as for
+ * wtconv_backward. */
+wtconv_status_t wtconv_backward_one_pass(const wtconv_desc_t *d, const void *x, const void *dy,
+                                         const float *base_w, const float *base_b, const float *base_scale,
+                                         const float *wt_w, const float *wt_scale, void *dx,
+                                         float *d_base_w, float *d_base_b, float *d_base_scale,
+                                         float *d_wt_w, float *d_wt_scale,
+                                         void *workspace, size_t workspace_bytes, wtconv_stream_t stream);
 
 /* The paper has no counterpart to this entry point.
  *
@@ -157,12 +186,17 @@ wtconv_status_t wtconv_backward(const wtconv_desc_t *d, const void *x, const voi
  *   - Size limit: its partial sums (at most wtconv_workspace_bytes(d) bytes)
  *     must fit in 2^20 floats; larger problems return WTCONV_ERR_WORKSPACE (use
  *     wtconv_backward_weight).
- *   - The first call on each device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *   - Every call looks up the array's address in the current context (a
+ *     host-side lookup), so a context created after cudaDeviceReset, or a
+ *     non-primary context, gets its own copy of the array.  Under lazy module
+ *     loading the first call in a context may load the library's device code;
+ *     make one call before any stream capture.
  *   - Every call shares the one array: calls whose kernels overlap on the GPU
  *     (different streams, no ordering between them) race and corrupt each
- *     other's results.  Calls ordered on one stream are safe; each call
- *     overwrites every partial it later reads, so nothing is cleared.
+ *     other's results.  Calls ordered on one stream are safe.  Each call
+ *     enqueues, on `stream`, one memset of its per-channel arrival counters
+ *     (C unsigned ints) and then the kernel; the partial sums are never
+ *     cleared, since each call overwrites every partial it later reads.
  * Arguments, layouts and gradients as for wtconv_backward_weight. */
 wtconv_status_t wtconv_backward_weight_noalloc(const wtconv_desc_t *d, const void *x, const void *dy,
                                                const float *base_w, const float *base_b, const float *base_scale,

@@ -79,6 +79,8 @@ def load_library():
     lib.wtconv_backward_weight.restype = ctypes.c_int
     lib.wtconv_backward.argtypes = [dp, vp, vp, fp, fp, fp, fp, fp, vp, fp, fp, fp, fp, fp, vp, sz, vp]
     lib.wtconv_backward.restype = ctypes.c_int
+    lib.wtconv_backward_one_pass.argtypes = lib.wtconv_backward.argtypes
+    lib.wtconv_backward_one_pass.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -220,8 +222,11 @@ def backward_weight(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, g
 
 
 def backward(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, dx=None, grads=None, workspace=None,
-             stream=None):
-    """dx and the parameter gradients in one pass via ``wtconv_backward``.
+             stream=None, one_pass: bool = False):
+    """dx and the parameter gradients via ``wtconv_backward`` (the library
+    picks the one-pass kernel or the two passes), or with ``one_pass`` via
+    ``wtconv_backward_one_pass`` (raises WTConvError WTCONV_ERR_UNSUPPORTED
+    for planes split into cluster strips).
 
     Returns (dx, grads) with grads as for ``backward_weight``.
     """
@@ -244,13 +249,15 @@ def backward(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, dx=None,
     nbytes = int(lib.wtconv_workspace_bytes(ctypes.byref(d)))
     if workspace is None:
         workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=dev)
-    _check(lib.wtconv_backward(
+    fn, name = ((lib.wtconv_backward_one_pass, "wtconv_backward_one_pass") if one_pass
+                else (lib.wtconv_backward, "wtconv_backward"))
+    _check(fn(
         ctypes.byref(d), _ptr(x), _ptr(dy), _ptr(base_w), _ptr(base_b), _ptr(base_scale),
         _ptr(wt_w if L > 0 else None), _ptr(wt_scale if L > 0 else None), _ptr(dx),
         _ptr(grads["base_w"]), _ptr(grads["base_b"]), _ptr(grads["base_scale"]),
         _ptr(grads["wt_w"] if L > 0 else None), _ptr(grads["wt_scale"] if L > 0 else None),
         _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
-        _stream(dev, stream)), "wtconv_backward")
+        _stream(dev, stream)), name)
     return dx, grads
 
 

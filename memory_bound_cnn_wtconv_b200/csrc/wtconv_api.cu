@@ -16,50 +16,43 @@ namespace wtc {
 
 namespace {
 
-cudaError_t launch_fused(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cudaStream_t s) {
-    switch (P.k) {
-        case 1: return launch_fused_k1(P, dtype, bwd, a, s);
-        case 3: return launch_fused_k3(P, dtype, bwd, a, s);
-        case 5: return launch_fused_k5(P, dtype, bwd, a, s);
-        case 7: return launch_fused_k7(P, dtype, bwd, a, s);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
-cudaError_t launch_bwdw(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
-    switch (P.k) {
-        case 1: return launch_bwdw_k1(P, dtype, a, s);
-        case 3: return launch_bwdw_k3(P, dtype, a, s);
-        case 5: return launch_bwdw_k5(P, dtype, a, s);
-        case 7: return launch_bwdw_k7(P, dtype, a, s);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
-cudaError_t launch_bwd(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s) {
-    switch (P.k) {
-        case 1: return launch_bwd_k1(P, dtype, a, s);
-        case 3: return launch_bwd_k3(P, dtype, a, s);
-        case 5: return launch_bwd_k5(P, dtype, a, s);
-        case 7: return launch_bwd_k7(P, dtype, a, s);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 // Workspace both weight-gradient paths accept: the larger of the two plans'.
-size_t workspace_bytes_any(const wtconv_desc_t* d) {
+size_t workspace_bytes_any(const wtconv_desc_t* d, int sms) {
     Plan P;
     size_t n = 0;
-    if (make_plan(d, kBackwardWeight, &P) == WTCONV_OK) n = workspace_bytes_of(P);
-    if (make_plan(d, kBackward, &P) == WTCONV_OK) n = std::max(n, workspace_bytes_of(P));
+    if (make_plan(d, kBackwardWeight, sms, &P) == WTCONV_OK) n = workspace_bytes_of(P);
+    if (make_plan(d, kBackward, sms, &P) == WTCONV_OK) n = std::max(n, workspace_bytes_of(P));
     return n;
 }
 
-GradArgs grad_args(const float* base_w, const float* base_b, const float* base_scale, const float* wt_w,
-                   const float* wt_scale, float* d_base_w, float* d_base_b, float* d_base_scale, float* d_wt_w,
-                   float* d_wt_scale, unsigned* counters) {
-    return GradArgs{base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
-                    d_wt_w, d_wt_scale, counters};
+// Shared checks of the calls that write parameter gradients.
+wtconv_status_t check_grad_args(const wtconv_desc_t* d, const void* x, const void* dy, const float* base_w,
+                                const float* base_b, const float* base_scale, const float* wt_w,
+                                const float* wt_scale, const float* d_base_w, const float* d_base_b,
+                                const float* d_base_scale, const float* d_wt_w, const float* d_wt_scale) {
+    if (!x || !dy || !base_w || !base_b || !base_scale || !d_base_w || !d_base_b || !d_base_scale)
+        return WTCONV_ERR_NULLPTR;
+    if (d->L > 0 && (!wt_w || !wt_scale || !d_wt_w || !d_wt_scale)) return WTCONV_ERR_NULLPTR;
+    if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_MISALIGNED;
+    return WTCONV_OK;
+}
+
+// The one-pass kernel on plan P (validated arguments).
+wtconv_status_t run_one_pass(const wtconv_desc_t* d, const Plan& P, int sms, const void* x, const void* dy,
+                             const float* base_w, const float* base_b, const float* base_scale, const float* wt_w,
+                             const float* wt_scale, void* dx, float* d_base_w, float* d_base_b,
+                             float* d_base_scale, float* d_wt_w, float* d_wt_scale, void* workspace,
+                             size_t workspace_bytes, cudaStream_t s) {
+    if (!workspace || workspace_bytes < workspace_bytes_any(d, sms)) return WTCONV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
+    float* part = static_cast<float*>(workspace);
+    unsigned* counters = reinterpret_cast<unsigned*>(part + counters_offset_floats(P));
+    if (cudaMemsetAsync(counters, 0, (size_t)P.C * sizeof(unsigned), s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    BwdArgs a{x, dy, dx, part,
+              grad_args(base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale, d_wt_w,
+                        d_wt_scale, counters)};
+    if (launch_bwd(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
+    return WTCONV_OK;
 }
 
 }  // namespace
@@ -88,7 +81,7 @@ const char* wtconv_status_string(wtconv_status_t s) {
 
 size_t wtconv_workspace_bytes(const wtconv_desc_t* d) {
     if (validate(d) != WTCONV_OK) return 0;
-    return workspace_bytes_any(d);
+    return workspace_bytes_any(d, planning_sm_count());
 }
 
 wtconv_status_t wtconv_forward(const wtconv_desc_t* d, const void* x, const float* base_w, const float* base_b,
@@ -100,7 +93,7 @@ wtconv_status_t wtconv_forward(const wtconv_desc_t* d, const void* x, const floa
     if (d->L > 0 && (!wt_w || !wt_scale)) return WTCONV_ERR_NULLPTR;
     if (!aligned16(x) || !aligned16(y)) return WTCONV_ERR_MISALIGNED;
     Plan P;
-    st = make_plan(d, kForward, &P);
+    st = make_plan(d, kForward, planning_sm_count(), &P);
     if (st != WTCONV_OK) return st;
     FusedArgs a{x, base_w, base_b, base_scale, wt_w, wt_scale, y};
     return launch_fused(P, d->dtype, false, a, (cudaStream_t)stream) == cudaSuccess ? WTCONV_OK
@@ -116,7 +109,7 @@ wtconv_status_t wtconv_backward_input(const wtconv_desc_t* d, const void* dy, co
     if (d->L > 0 && (!wt_w || !wt_scale)) return WTCONV_ERR_NULLPTR;
     if (!aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_MISALIGNED;
     Plan P;
-    st = make_plan(d, kBackwardInput, &P);
+    st = make_plan(d, kBackwardInput, planning_sm_count(), &P);
     if (st != WTCONV_OK) return st;
     // base_b is unused by the transpose; pass base_scale as a valid pointer.
     FusedArgs a{dy, base_w, base_scale, base_scale, wt_w, wt_scale, dx};
@@ -132,14 +125,14 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t* d, const void* x, co
                                        wtconv_stream_t stream) {
     wtconv_status_t st = validate(d);
     if (st != WTCONV_OK) return st;
-    if (!x || !dy || !base_w || !base_b || !base_scale || !d_base_w || !d_base_b || !d_base_scale)
-        return WTCONV_ERR_NULLPTR;
-    if (d->L > 0 && (!wt_w || !wt_scale || !d_wt_w || !d_wt_scale)) return WTCONV_ERR_NULLPTR;
-    if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_MISALIGNED;
-    Plan P;
-    st = make_plan(d, kBackwardWeight, &P);
+    st = check_grad_args(d, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                         d_wt_w, d_wt_scale);
     if (st != WTCONV_OK) return st;
-    if (!workspace || workspace_bytes < workspace_bytes_any(d)) return WTCONV_ERR_WORKSPACE;
+    const int sms = planning_sm_count();
+    Plan P;
+    st = make_plan(d, kBackwardWeight, sms, &P);
+    if (st != WTCONV_OK) return st;
+    if (!workspace || workspace_bytes < workspace_bytes_any(d, sms)) return WTCONV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
     float* part = static_cast<float*>(workspace);
     unsigned* counters = reinterpret_cast<unsigned*>(part + counters_offset_floats(P));
@@ -159,31 +152,54 @@ wtconv_status_t wtconv_backward(const wtconv_desc_t* d, const void* x, const voi
                                 size_t workspace_bytes, wtconv_stream_t stream) {
     wtconv_status_t st = validate(d);
     if (st != WTCONV_OK) return st;
-    if (!x || !dy || !dx || !base_w || !base_b || !base_scale || !d_base_w || !d_base_b || !d_base_scale)
-        return WTCONV_ERR_NULLPTR;
-    if (d->L > 0 && (!wt_w || !wt_scale || !d_wt_w || !d_wt_scale)) return WTCONV_ERR_NULLPTR;
-    if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return WTCONV_ERR_MISALIGNED;
-    Plan P;
-    st = make_plan(d, kBackward, &P);
-    if (st == WTCONV_ERR_UNSUPPORTED) {
-        // No one-pass plan (planes split into strips): the two passes.
-        st = wtconv_backward_input(d, dy, base_w, base_scale, wt_w, wt_scale, dx, stream);
-        if (st != WTCONV_OK) return st;
-        return wtconv_backward_weight(d, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b,
-                                      d_base_scale, d_wt_w, d_wt_scale, workspace, workspace_bytes, stream);
-    }
+    if (!dx) return WTCONV_ERR_NULLPTR;
+    st = check_grad_args(d, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                         d_wt_w, d_wt_scale);
     if (st != WTCONV_OK) return st;
-    if (!workspace || workspace_bytes < workspace_bytes_any(d)) return WTCONV_ERR_WORKSPACE;
+    if (!aligned16(dx)) return WTCONV_ERR_MISALIGNED;
+    const int sms = planning_sm_count();
+    // The one pass where its plan exists and costs less than the two passes'
+    // plans together (plan_cost: tile rows on the busiest SM sub-partition);
+    // else the input- and weight-gradient passes, with the same results.
+    Plan P, Pin, Pw;
+    st = make_plan(d, kBackward, sms, &P);
+    if (st != WTCONV_OK && st != WTCONV_ERR_UNSUPPORTED) return st;
+    bool one_pass = st == WTCONV_OK;
+    if (one_pass && make_plan(d, kBackwardInput, sms, &Pin) == WTCONV_OK &&
+        make_plan(d, kBackwardWeight, sms, &Pw) == WTCONV_OK)
+        one_pass = plan_cost(P, kBackward) < plan_cost(Pin, kBackwardInput) + plan_cost(Pw, kBackwardWeight);
+    if (one_pass)
+        return run_one_pass(d, P, sms, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, dx, d_base_w, d_base_b,
+                            d_base_scale, d_wt_w, d_wt_scale, workspace, workspace_bytes, (cudaStream_t)stream);
+    // Check everything the weight pass checks before the input pass writes dx.
+    st = make_plan(d, kBackwardWeight, sms, &Pw);
+    if (st != WTCONV_OK) return st;
+    if (!workspace || workspace_bytes < workspace_bytes_any(d, sms)) return WTCONV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return WTCONV_ERR_MISALIGNED;
-    float* part = static_cast<float*>(workspace);
-    unsigned* counters = reinterpret_cast<unsigned*>(part + counters_offset_floats(P));
-    cudaStream_t s = (cudaStream_t)stream;
-    if (cudaMemsetAsync(counters, 0, (size_t)P.C * sizeof(unsigned), s) != cudaSuccess) return WTCONV_ERR_CUDA;
-    BwdArgs a{x, dy, dx, part,
-              grad_args(base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale, d_wt_w,
-                        d_wt_scale, counters)};
-    if (launch_bwd(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
-    return WTCONV_OK;
+    st = wtconv_backward_input(d, dy, base_w, base_scale, wt_w, wt_scale, dx, stream);
+    if (st != WTCONV_OK) return st;
+    return wtconv_backward_weight(d, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b,
+                                  d_base_scale, d_wt_w, d_wt_scale, workspace, workspace_bytes, stream);
+}
+
+wtconv_status_t wtconv_backward_one_pass(const wtconv_desc_t* d, const void* x, const void* dy,
+                                         const float* base_w, const float* base_b, const float* base_scale,
+                                         const float* wt_w, const float* wt_scale, void* dx, float* d_base_w,
+                                         float* d_base_b, float* d_base_scale, float* d_wt_w, float* d_wt_scale,
+                                         void* workspace, size_t workspace_bytes, wtconv_stream_t stream) {
+    wtconv_status_t st = validate(d);
+    if (st != WTCONV_OK) return st;
+    if (!dx) return WTCONV_ERR_NULLPTR;
+    st = check_grad_args(d, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                         d_wt_w, d_wt_scale);
+    if (st != WTCONV_OK) return st;
+    if (!aligned16(dx)) return WTCONV_ERR_MISALIGNED;
+    const int sms = planning_sm_count();
+    Plan P;
+    st = make_plan(d, kBackward, sms, &P);
+    if (st != WTCONV_OK) return st;
+    return run_one_pass(d, P, sms, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, dx, d_base_w, d_base_b,
+                        d_base_scale, d_wt_w, d_wt_scale, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 }  // extern "C"

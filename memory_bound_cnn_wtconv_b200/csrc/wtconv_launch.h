@@ -6,6 +6,7 @@
 
 #include "wtconv_kernels.cuh"
 #include "wtconv_plan.h"
+#include "wtconv_planner.h"
 
 namespace wtc {
 
@@ -41,6 +42,57 @@ WTC_DECLARE_LAUNCHERS(5)
 WTC_DECLARE_LAUNCHERS(7)
 
 #undef WTC_DECLARE_LAUNCHERS
+
+// Dispatch on the kernel size (every entry point launches through these).
+inline cudaError_t launch_fused(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cudaStream_t s) {
+    switch (P.k) {
+        case 1: return launch_fused_k1(P, dtype, bwd, a, s);
+        case 3: return launch_fused_k3(P, dtype, bwd, a, s);
+        case 5: return launch_fused_k5(P, dtype, bwd, a, s);
+        case 7: return launch_fused_k7(P, dtype, bwd, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+inline cudaError_t launch_bwdw(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
+    switch (P.k) {
+        case 1: return launch_bwdw_k1(P, dtype, a, s);
+        case 3: return launch_bwdw_k3(P, dtype, a, s);
+        case 5: return launch_bwdw_k5(P, dtype, a, s);
+        case 7: return launch_bwdw_k7(P, dtype, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+inline cudaError_t launch_bwd(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s) {
+    switch (P.k) {
+        case 1: return launch_bwd_k1(P, dtype, a, s);
+        case 3: return launch_bwd_k3(P, dtype, a, s);
+        case 5: return launch_bwd_k5(P, dtype, a, s);
+        case 7: return launch_bwd_k7(P, dtype, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+inline GradArgs grad_args(const float* base_w, const float* base_b, const float* base_scale, const float* wt_w,
+                          const float* wt_scale, float* d_base_w, float* d_base_b, float* d_base_scale,
+                          float* d_wt_w, float* d_wt_scale, unsigned* counters) {
+    return GradArgs{base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale,
+                    d_wt_w, d_wt_scale, counters};
+}
+
+// SM count of the current device, which the plans size their grids for; a
+// B200's 148 when no device can be queried (then nothing can launch, and
+// only host-side planning, such as a workspace size, is asked for).
+inline int planning_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();  // clear the (non-sticky) query error
+        return kB200SMs;
+    }
+    return n;
+}
 
 // Weight-gradient workspace: the partial vectors, then one arrival counter
 // per channel (16-byte aligned).

@@ -18,37 +18,15 @@ constexpr size_t kNoAllocScratchFloats = (size_t)1 << 20;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
-constexpr int kMaxScratchDevices = 64;
-
-// Device address of g_noalloc_scratch, resolved once per device with that
-// device current.  The host-side name is only a stand-in for the device
-// array and must never be passed to a kernel.
+// Device address of g_noalloc_scratch in the current context.  Looked up on
+// every call (a host-side lookup, no device work), so that a new context on
+// the device (after cudaDeviceReset, or a context other than the primary one)
+// gets its own module's address.  The host-side name is only a stand-in for
+// the device array and must never be passed to a kernel.
 float* scratch_address(cudaError_t* err) {
-    static float* addr[kMaxScratchDevices] = {};
-    int dev = 0;
-    *err = cudaGetDevice(&dev);
-    if (*err != cudaSuccess) return nullptr;
-    if (dev < 0 || dev >= kMaxScratchDevices) {
-        *err = cudaErrorInvalidDevice;
-        return nullptr;
-    }
-    if (addr[dev] == nullptr) {
-        void* p = nullptr;
-        *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (*err != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<float*>(p);
-    }
-    return addr[dev];
-}
-
-cudaError_t launch_partials(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
-    switch (P.k) {
-        case 1: return launch_bwdw_k1(P, dtype, a, s);
-        case 3: return launch_bwdw_k3(P, dtype, a, s);
-        case 5: return launch_bwdw_k5(P, dtype, a, s);
-        case 7: return launch_bwdw_k7(P, dtype, a, s);
-        default: return cudaErrorInvalidValue;
-    }
+    void* p = nullptr;
+    *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    return *err == cudaSuccess ? static_cast<float*>(p) : nullptr;
 }
 
 }  // namespace
@@ -67,7 +45,7 @@ extern "C" wtconv_status_t wtconv_backward_weight_noalloc(
     if (d->L > 0 && (!wt_w || !wt_scale || !d_wt_w || !d_wt_scale)) return WTCONV_ERR_NULLPTR;
     if (!aligned16(x) || !aligned16(dy)) return WTCONV_ERR_MISALIGNED;
     Plan P;
-    st = make_plan(d, kBackwardWeight, &P);
+    st = make_plan(d, kBackwardWeight, planning_sm_count(), &P);
     if (st != WTCONV_OK) return st;
     // The partials and the per-channel arrival counters of this plan
     // (workspace_bytes_of); beyond the fixed array the call is rejected (use
@@ -82,8 +60,8 @@ extern "C" wtconv_status_t wtconv_backward_weight_noalloc(
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaMemsetAsync(counters, 0, (size_t)P.C * sizeof(unsigned), s) != cudaSuccess) return WTCONV_ERR_CUDA;
     BwdwArgs a{x, dy, part,
-               GradArgs{base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale, d_wt_w,
-                        d_wt_scale, counters}};
-    if (launch_partials(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
+               grad_args(base_w, base_b, base_scale, wt_w, wt_scale, d_base_w, d_base_b, d_base_scale, d_wt_w,
+                         d_wt_scale, counters)};
+    if (launch_bwdw(P, d->dtype, a, s) != cudaSuccess) return WTCONV_ERR_CUDA;
     return WTCONV_OK;
 }

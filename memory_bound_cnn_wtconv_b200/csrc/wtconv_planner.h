@@ -15,7 +15,9 @@ namespace wtc {
 
 constexpr int kSmemLimitFloats = 227 * 1024 / 4;
 constexpr int kSmemPerSM = 228 * 1024;
-constexpr int kNumSMs = 148;  // B200; sizes the persistent grids
+// SMs of a B200: the SM count planned for when no CUDA device can be
+// queried (host-only planning; nothing can launch then).
+constexpr int kB200SMs = 148;
 
 // kBackward: the fused backward (dx and the weight-gradient partials in one
 // pass over x and dy).
@@ -117,9 +119,12 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // on-chip rows (H, ntr, buffers, tiles) describes one strip.
 // dy_stg (weight gradient on strips of fp32 planes whose height is whole
 // tiles): no DY buffer; the correlation tiles read dy from its staging.
-inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, Plan* P,
+// num_sms (the device's SM count) sizes the persistent forward grid and the
+// weight gradient's batch groups.
+inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, int num_sms, Plan* P,
                                      bool dy_stg = false) {
     memset(P, 0, sizeof(*P));
+    if (num_sms < 1) return WTCONV_ERR_UNSUPPORTED;
     // The plane the CTAs hold: H and W rounded up to multiples of 2^L.
     const int m = 1 << d->L;
     const int Hv = (d->H + m - 1) / m * m, Wv = (d->W + m - 1) / m * m;
@@ -318,12 +323,12 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;
     if (kind == kBackwardWeight || kind == kBackward) {
-        const long long slots = (long long)kNumSMs * resident_ctas(P->nthreads, P->smem_floats);
+        const long long slots = (long long)num_sms * resident_ctas(P->nthreads, P->smem_floats);
         P->groups = pick_groups(P->B, P->C * nstrips, slots);
         P->parts = P->groups * nstrips;
     } else {
         const long long units = (long long)P->B * P->C;
-        P->grid = (int)std::min<long long>(units, (long long)kNumSMs * ctas_per_sm(P->smem_floats));
+        P->grid = (int)std::min<long long>(units, (long long)num_sms * ctas_per_sm(P->smem_floats));
         P->groups = 1;
     }
     return WTCONV_OK;
@@ -356,7 +361,7 @@ inline double plan_cost(const Plan& P, Kind kind) {
 // plane that the tile count does not show: at 128 x 128 (L = 2..4) two
 // strips measured 1.7-1.9x faster than eight, and at every shape measured
 // fewer strips were faster.
-inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
+inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, int num_sms, Plan* P) {
     bool have = false;
     double best = 0.0;
     Plan cand;
@@ -366,7 +371,7 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, Plan* P) {
         for (int alias = 0; alias < 2 && !have; ++alias) {
             if (alias && (kind != kBackwardWeight || n == 1)) break;
             for (int TR = 7; TR <= 8; ++TR) {
-                if (make_plan_for(d, kind, TR, n, &cand, alias == 1) != WTCONV_OK) continue;
+                if (make_plan_for(d, kind, TR, n, num_sms, &cand, alias == 1) != WTCONV_OK) continue;
                 const double c = plan_cost(cand, kind);
                 if (!have || c < best) {
                     best = c;

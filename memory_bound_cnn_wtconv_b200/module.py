@@ -22,9 +22,10 @@ _PARAMS = ("base_w", "base_b", "base_scale", "wt_w", "wt_scale")
 
 class WTConvFunction(torch.autograd.Function):
     """y = WTConv(x).  Backward: the input- and weight-gradient passes, or
-    with ``one_pass`` the single ``wtconv_backward`` pass (same results; it
-    moves a quarter fewer bytes but was measured no faster on B200, its
-    larger on-chip footprint allowing one CTA per SM instead of two)."""
+    with ``one_pass`` the one-pass kernel ``wtconv_backward_one_pass`` (same
+    results; it moves a quarter fewer bytes but was measured no faster on
+    B200, its larger on-chip footprint allowing one CTA per SM instead of
+    two; planes split into cluster strips have no one-pass plan and raise)."""
 
     @staticmethod
     def forward(ctx, x, base_w, base_b, base_scale, wt_w, wt_scale, L: int, one_pass: bool = False):
@@ -43,7 +44,7 @@ class WTConvFunction(torch.autograd.Function):
         need = ctx.needs_input_grad
         dx, g = None, {}
         if ctx.one_pass and need[0] and any(need[1:6]):
-            dx, g = backward(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L)
+            dx, g = backward(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L, one_pass=True)
         else:
             if need[0]:
                 dx = backward_input(dy, base_w, base_scale, wt_w, wt_scale, L)

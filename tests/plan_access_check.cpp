@@ -332,7 +332,7 @@ void barrier_all(std::vector<Shadow>& shs) {
 
 void check_fused(const wtconv_desc_t& d, Kind kind) {
     Plan P;
-    const wtconv_status_t st = make_plan(&d, kind, &P);
+    const wtconv_status_t st = make_plan(&d, kind, kB200SMs, &P);
     if (st == WTCONV_ERR_UNSUPPORTED) {
         std::printf("fused: unsupported (plane too large)\n");
         return;
@@ -519,7 +519,7 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
 
 void check_bwdw(const wtconv_desc_t& d) {
     Plan P;
-    const wtconv_status_t st = make_plan(&d, kBackwardWeight, &P);
+    const wtconv_status_t st = make_plan(&d, kBackwardWeight, kB200SMs, &P);
     if (st == WTCONV_ERR_UNSUPPORTED) {
         std::printf("bwdw: unsupported (plane too large)\n");
         return;
@@ -661,7 +661,7 @@ void check_bwdw(const wtconv_desc_t& d) {
 // the interior of X / S) in one walk.
 void check_bwd(const wtconv_desc_t& d) {
     Plan P;
-    const wtconv_status_t st = make_plan(&d, kBackward, &P);
+    const wtconv_status_t st = make_plan(&d, kBackward, kB200SMs, &P);
     if (st == WTCONV_ERR_UNSUPPORTED) {
         std::printf("bwd: no one-pass plan (two passes)\n");
         return;

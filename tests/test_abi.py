@@ -138,3 +138,47 @@ def test_backward_validation(cuda_lib):
                                     None) == WORKSPACE
     assert cuda_lib.wtconv_backward(ctypes.byref(_desc(k=4)), *args, p(FAKE), *grads, p(FAKE),
                                     ctypes.c_size_t(need), None) == BAD_K
+
+
+def test_backward_one_pass_validation(cuda_lib):
+    p = ctypes.c_void_p
+    args = [p(FAKE)] * 7
+    grads = [p(FAKE)] * 5
+    d = _desc(H=32, W=32, L=2)
+    need = cuda_lib.wtconv_workspace_bytes(ctypes.byref(d))
+    fn = cuda_lib.wtconv_backward_one_pass
+    assert fn(ctypes.byref(d), *args, p(0), *grads, p(FAKE), ctypes.c_size_t(need), None) == NULLPTR
+    assert fn(ctypes.byref(d), *args, p(FAKE + 4), *grads, p(FAKE), ctypes.c_size_t(need), None) == MISALIGNED
+    assert fn(ctypes.byref(d), *args, p(FAKE), *grads, p(FAKE), ctypes.c_size_t(need - 4), None) == WORKSPACE
+    # A 256 x 256 plane is held as cluster strips: no one-pass plan.  The
+    # library-picked backward still plans it (as the two passes).
+    big = _desc(H=256, W=256, L=4)
+    need_big = cuda_lib.wtconv_workspace_bytes(ctypes.byref(big))
+    assert need_big > 0
+    assert fn(ctypes.byref(big), *args, p(FAKE), *grads, p(FAKE), ctypes.c_size_t(need_big), None) == UNSUPPORTED
+    assert cuda_lib.wtconv_backward(ctypes.byref(big), *args, p(FAKE), *grads, p(FAKE),
+                                    ctypes.c_size_t(need_big - 4), None) == WORKSPACE
+
+
+def test_backward_checks_the_workspace_before_any_pass(cuda_lib):
+    # Whichever path the library picks, a short workspace is refused before
+    # the input-gradient pass could write dx (dx is a never-dereferenced fake).
+    p = ctypes.c_void_p
+    for kw in (dict(), dict(B=32, C=96, H=56, W=56, k=5, L=3), dict(H=128, W=128, L=3)):
+        d = _desc(**kw)
+        need = cuda_lib.wtconv_workspace_bytes(ctypes.byref(d))
+        assert need > 0
+        rc = cuda_lib.wtconv_backward(ctypes.byref(d), *([p(FAKE)] * 14), ctypes.c_size_t(need - 4), None)
+        assert rc == WORKSPACE, kw
+
+
+def test_noalloc_rejects_plans_beyond_its_array(cuda_lib):
+    # The fixed array holds 2^20 floats of partial sums and counters; a plan
+    # that needs more is refused after planning, before any CUDA call.
+    p = ctypes.c_void_p
+    d = _desc(B=4, C=4096, H=16, W=16, k=7, L=2)
+    assert cuda_lib.wtconv_workspace_bytes(ctypes.byref(d)) > 4 << 20
+    fn = cuda_lib.wtconv_backward_weight_noalloc
+    fn.argtypes = [ctypes.POINTER(w.Desc)] + [p] * 13
+    fn.restype = ctypes.c_int
+    assert fn(ctypes.byref(d), *([p(FAKE)] * 12), None) == WORKSPACE

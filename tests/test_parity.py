@@ -39,9 +39,10 @@ def run_gpu(case: Case, g, calls, fused_bwd=False):
     if "fwd" in calls:
         out["y"] = wt.forward(g["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], case.L)
     if fused_bwd:
-        # dx and the parameter gradients from the one-pass backward.
+        # dx and the parameter gradients from one backward call: the path
+        # the library picks ("auto") or the one-pass kernel ("one_pass").
         out["dx"], out["grads"] = wt.backward(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"],
-                                              g["wt_scale"], case.L)
+                                              g["wt_scale"], case.L, one_pass=fused_bwd == "one_pass")
     else:
         if "bwd_in" in calls:
             out["dx"] = wt.backward_input(g["dy"], g["base_w"], g["base_scale"], g["wt_w"], g["wt_scale"], case.L)
@@ -174,24 +175,41 @@ def test_small_case_all_outputs(oracle, case):
     check_full(oracle, case, case.calls)
 
 
+def _one_pass_plan_exists(case: Case) -> bool:
+    """Whether wtconv_backward_one_pass plans this case (whole planes only);
+    asked through the call itself with an empty workspace, which returns
+    WTCONV_ERR_WORKSPACE (7) after planning and before any launch."""
+    import ctypes
+    lib = wt.load_library()
+    d = wt.Desc(case.B, case.C, case.H, case.W, case.k, case.L, 1 if case.dtype == "bf16" else 0)
+    fake = ctypes.c_void_p(0x10000)
+    rc = lib.wtconv_backward_one_pass(ctypes.byref(d), *([fake] * 13), ctypes.c_void_p(0), ctypes.c_size_t(0), None)
+    assert rc in (7, 8), rc
+    return rc == 7
+
+
+@pytest.mark.parametrize("mode", ["auto", "one_pass"])
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: c.name)
-def test_small_case_fused_backward(oracle, case):
-    # The one-pass backward (or, for strip planes, its two-pass fallback).
-    check_full(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=True)
+def test_small_case_fused_backward(oracle, case, mode):
+    if mode == "one_pass" and not _one_pass_plan_exists(case):
+        pytest.skip("planes split into cluster strips have no one-pass plan")
+    check_full(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=mode)
 
 
+@pytest.mark.parametrize("mode", ["auto", "one_pass"])
 @pytest.mark.parametrize("case", [STAGE1, STAGE2, TRAIN_BF16], ids=lambda c: c.name)
-def test_full_size_fused_backward_sampled(oracle, case):
-    check_sampled(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=True)
+def test_full_size_fused_backward_sampled(oracle, case, mode):
+    check_sampled(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=mode)
 
 
-def test_fused_backward_is_deterministic():
+@pytest.mark.parametrize("one_pass", [False, True], ids=["auto", "one_pass"])
+def test_fused_backward_is_deterministic(one_pass):
     case = STAGE1
     g = gpu_inputs(make_inputs(case))
     args = (g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], case.L)
-    dx_a, ga = wt.backward(*args)
+    dx_a, ga = wt.backward(*args, one_pass=one_pass)
     dx_a, ga = dx_a.clone(), {k: v.clone() for k, v in ga.items()}
-    dx_b, gb = wt.backward(*args)
+    dx_b, gb = wt.backward(*args, one_pass=one_pass)
     torch.cuda.synchronize()
     assert torch.equal(dx_a, dx_b)
     for k in PARAMS:
@@ -213,12 +231,57 @@ def _supported(case: Case) -> bool:
     return wt.load_library().wtconv_workspace_bytes(ctypes.byref(d)) > 0
 
 
-SWEEP_PICK = [0, 7, 9, 14, 17, 31, 40, 63, 66, 95, 105, 127]
+def _one_point_per_geometry() -> list:
+    """One sweep point for each of the sweep's 32 plane geometries (H, L, k),
+    the channel count rotating through all four values.  The plan (strip
+    count, tile height, dy read from its staging, threads) depends on the
+    geometry only, so these points run every plan the sweep uses."""
+    cases = sweep_cases()
+    picks = []
+    for hi in range(4):
+        for li in range(4):
+            for ki in range(2):
+                ci = (hi + li + ki) % 4
+                picks.append(((ci * 4 + hi) * 4 + li) * 2 + ki)
+    assert len({(cases[i].H, cases[i].L, cases[i].k) for i in picks}) == 32
+    return sorted(picks)
+
+
+SWEEP_PICK = _one_point_per_geometry()
 
 
 @pytest.mark.parametrize("idx", SWEEP_PICK)
 def test_sweep_points_sampled(oracle, idx):
     case = sweep_cases()[idx]
+    assert _supported(case), f"{case.name}: no on-chip plan"
+    check_sampled(oracle, case, nplanes=4, nchannels=2)
+
+
+@pytest.mark.parametrize("idx", [i for i in SWEEP_PICK if sweep_cases()[i].H <= 64])
+def test_sweep_points_one_pass_backward_sampled(oracle, idx):
+    # Whole planes (H <= 64) have a one-pass plan; larger ones are strips.
+    case = sweep_cases()[idx]
+    check_sampled(oracle, case, ("bwd_in", "bwd_w"), nplanes=4, nchannels=2, fused_bwd="one_pass")
+
+
+def _sweep_batch(C: int, H: int) -> int:
+    return max(1, round(2 ** 28 / (4 * C * H * H)))
+
+
+# Plans the sweep's shapes never pick, at the sweep's channel counts and
+# batch rule (x of about 256 Mi elements): clusters of 4 and 16 strips, the
+# weight gradient reading dy from its staging at 4 strips, and bf16 strips.
+PLAN_VARIANTS = [
+    Case("strips4_dy_from_staging_H192_L1_k5", _sweep_batch(128, 192), 128, 192, 192, 5, 1, "f32", 2001),
+    Case("strips4_dy_from_staging_H192_L4_k3", _sweep_batch(256, 192), 256, 192, 192, 3, 4, "f32", 2002),
+    Case("strips4_bf16_H192_L1_k7", _sweep_batch(64, 192), 64, 192, 192, 7, 1, "bf16", 2003, "uniform"),
+    Case("strips16_H320_L1_k3", _sweep_batch(64, 320), 64, 320, 320, 3, 1, "f32", 2004),
+    Case("strips16_bf16_H320_L1_k5", _sweep_batch(512, 320), 512, 320, 320, 5, 1, "bf16", 2005, "uniform"),
+]
+
+
+@pytest.mark.parametrize("case", PLAN_VARIANTS, ids=lambda c: c.name)
+def test_plan_variants_at_sweep_sizes_sampled(oracle, case):
     assert _supported(case), f"{case.name}: no on-chip plan"
     check_sampled(oracle, case, nplanes=4, nchannels=2)
 

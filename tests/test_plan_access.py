@@ -25,6 +25,9 @@ EDGE = [
     # deepest levels, bf16 with k = 7, one channel over many batch elements, padded L = 6
     (1, 2, 32, 32, 3, 5, 0), (2, 2, 24, 24, 7, 3, 1), (130, 1, 16, 16, 5, 2, 0), (1, 2, 40, 36, 5, 6, 0),
     (2, 1, 60, 64, 3, 6, 0), (1, 1, 70, 68, 5, 6, 0),
+    # clusters of 4 and 16 strips at the sweep's channel counts and batch rule
+    (14, 128, 192, 192, 5, 1, 0), (7, 256, 192, 192, 3, 4, 0), (28, 64, 192, 192, 7, 1, 1),
+    (10, 64, 320, 320, 3, 1, 0), (1, 512, 320, 320, 5, 1, 1),
 ]
 
 
