@@ -112,6 +112,9 @@ def check_sampled(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), nplanes=
             r_all.append(r[0, 0])
         errs[name] = relerr(np.stack(g_all), np.stack(r_all))
     if "bwd_w" in calls:
+        # Normwise per gradient tensor over its sampled channels, as the
+        # outputs above are over their sampled planes.
+        got, want = {}, {}
         for c in chans:
             p = oracle_params(inp, c)
             ref = oracle.backward_weight(f64(inp["x"][:, c:c + 1]), f64(inp["dy"][:, c:c + 1]), p["base_w"],
@@ -123,7 +126,10 @@ def check_sampled(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), nplanes=
                 pairs["wt_w"] = (g["wt_w"][:, c], ref["wt_w"][:, 0])
                 pairs["wt_scale"] = (g["wt_scale"][:, c], ref["wt_scale"][:, 0])
             for k, (gv, rv) in pairs.items():
-                errs[f"d_{k}[c={c}]"] = relerr(f64(gv), rv)
+                got.setdefault(k, []).append(f64(gv))
+                want.setdefault(k, []).append(np.asarray(rv))
+        for k in got:
+            errs[f"d_{k}[c in {chans}]"] = relerr(np.stack(got[k]), np.stack(want[k]))
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, f"{case}: {errs}"
     return errs
