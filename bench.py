@@ -305,7 +305,7 @@ class Workload:
     """Device buffers of one workload and its three calls (plus, with several
     ranks, the all-reduce of the weight gradients)."""
 
-    def __init__(self, case, dev, stream, rank: int, world: int):
+    def __init__(self, case, dev, stream, rank: int, world: int, nhwc: bool = False):
         import torch
 
         import memory_bound_cnn_wtconv_b200 as wt
@@ -314,6 +314,9 @@ class Workload:
         self.case, self.dev, self.stream, self.world = case, dev, stream, world
         inp = make_inputs(case.with_(seed=case.seed + 7919 * rank))
         self.g = g = {k: v.to(dev) for k, v in inp.items()}
+        if nhwc:  # channels-last activations (same values, NHWC storage)
+            for k in ("x", "dy"):
+                g[k] = g[k].contiguous(memory_format=torch.channels_last)
         L = case.L
         self.y = torch.empty_like(g["x"])
         self.dx = torch.empty_like(g["dy"])
@@ -526,15 +529,19 @@ def run_ours(args, case):
     # The other WTConvNeXt stage shapes, same protocol, one GPU.
     if world == 1 and not args.no_other_workloads:
         other = {}
-        for name in ("stage1", "stage2", "train_bf16"):
+        for name in ("stage1", "stage2", "train_bf16", "stage1_nhwc"):
             if name == case.name:
                 other[name] = dict(rec, fused_backward=line["fused_backward"])
                 continue
-            del_wl = Workload(NAMED[name], dev, stream, 0, 1)
+            nhwc = name.endswith("_nhwc")
+            wcase = NAMED[name[:-len("_nhwc")] if nhwc else name]
+            del_wl = Workload(wcase, dev, stream, 0, 1, nhwc=nhwc)
             t2, _, _ = del_wl.time_calls(del_wl.calls, K, args.warmup, flush)
             pc2 = {n: median(v) for n, v in t2.items()}
-            other[name] = call_record(NAMED[name], pc2, peak)
-            other[name]["fused_backward"], n_launch = backward_record(del_wl, NAMED[name], pc2, KF, flush)
+            other[name] = call_record(wcase, pc2, peak)
+            if nhwc:
+                other[name]["workload"] += " (NHWC activations)"
+            other[name]["fused_backward"], n_launch = backward_record(del_wl, wcase, pc2, KF, flush)
             line["gpu_launches"] += K * 3 + n_launch
             del del_wl
             torch.cuda.empty_cache()

@@ -27,8 +27,9 @@
  * per-subband scales are folded into the conv weights before the convs run.
  *
  * Conventions for every entry point:
- *   - Layouts.  Activations are NCHW, contiguous, stored as float32 or bf16
- *     (desc->dtype); arithmetic is float32.  Parameters and gradients are
+ *   - Layouts.  Activations are NCHW or NHWC (desc->layout), contiguous,
+ *     stored as float32 or bf16 (desc->dtype); arithmetic is float32; x, dy,
+ *     y and dx of one call share the layout.  Parameters and gradients are
  *     float32, contiguous:  base_w [C][k][k], base_b [C], base_scale [C],
  *     wt_w [L][C][4][k][k], wt_scale [L][C][4].
  *   - Pointers are DEVICE pointers on the current device; activation pointers
@@ -81,16 +82,24 @@ typedef enum {
     WTCONV_ERR_DTYPE = 6,       /* unknown activation dtype */
     WTCONV_ERR_WORKSPACE = 7,   /* workspace missing or smaller than wtconv_workspace_bytes() */
     WTCONV_ERR_UNSUPPORTED = 8, /* valid shape whose plane (or strip) does not fit on chip */
-    WTCONV_ERR_CUDA = 9         /* a CUDA runtime call or kernel launch failed */
+    WTCONV_ERR_CUDA = 9,        /* a CUDA runtime call or kernel launch failed */
+    WTCONV_ERR_LAYOUT = 10      /* unknown activation layout */
 } wtconv_status_t;
 
 typedef enum { WTCONV_F32 = 0, WTCONV_BF16 = 1 } wtconv_dtype_t; /* activation storage */
+
+/* Activation layout: NCHW, or NHWC (channels last: element (b, c, h, w) at
+ * ((b*H + h)*W + w)*C + c).  NHWC planes are gathered and scattered
+ * element by element (C elements apart) by the same on-chip pass; the
+ * parameters' layouts do not change. */
+typedef enum { WTCONV_NCHW = 0, WTCONV_NHWC = 1 } wtconv_layout_t;
 
 typedef struct {
     int B, C, H, W; /* batch, channels, height, width */
     int k;          /* odd depthwise kernel size, shared by the base and subband convs */
     int L;          /* number of wavelet decomposition levels */
     int dtype;      /* a wtconv_dtype_t value */
+    int layout;     /* a wtconv_layout_t value (0 = NCHW) */
 } wtconv_desc_t;
 
 /* Human-readable name of a status code (static string, never NULL). */

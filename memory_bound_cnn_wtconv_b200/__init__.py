@@ -10,8 +10,9 @@ Reformulation", arXiv 2608.10805, Abstract): a depthwise k x k base conv with
 per-channel scale and bias, plus an L-level orthonormal Haar wavelet branch
 with one scaled depthwise conv per subband, recombined by the inverse Haar
 synthesis.  Parameter layouts: base_w [C,k,k], base_b [C], base_scale [C],
-wt_w [L,C,4,k,k], wt_scale [L,C,4] (float32); activations NCHW float32 or
-bfloat16, contiguous, on one CUDA device.
+wt_w [L,C,4,k,k], wt_scale [L,C,4] (float32); activations float32 or bfloat16
+on one CUDA device, either contiguous (NCHW) or channels-last contiguous
+(NHWC, ``torch.channels_last``); a call's activations share the layout.
 """
 from __future__ import annotations
 
@@ -32,9 +33,10 @@ _lib = None
 STATUS = {
     0: "WTCONV_OK", 1: "WTCONV_ERR_NULLPTR", 2: "WTCONV_ERR_BAD_SHAPE", 3: "WTCONV_ERR_BAD_K",
     4: "WTCONV_ERR_BAD_L", 5: "WTCONV_ERR_MISALIGNED", 6: "WTCONV_ERR_DTYPE", 7: "WTCONV_ERR_WORKSPACE",
-    8: "WTCONV_ERR_UNSUPPORTED", 9: "WTCONV_ERR_CUDA",
+    8: "WTCONV_ERR_UNSUPPORTED", 9: "WTCONV_ERR_CUDA", 10: "WTCONV_ERR_LAYOUT",
 }
 F32, BF16 = 0, 1
+NCHW, NHWC = 0, 1
 
 
 class WTConvError(RuntimeError):
@@ -49,7 +51,7 @@ class WTConvLibraryMissing(RuntimeError):
 
 class Desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("C", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
-                ("k", ctypes.c_int), ("L", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("k", ctypes.c_int), ("L", ctypes.c_int), ("dtype", ctypes.c_int), ("layout", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -105,11 +107,23 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
 
 
-def _act(t: torch.Tensor, name: str) -> torch.Tensor:
+def layout_of(t: torch.Tensor) -> int:
+    """NCHW (0) for a contiguous tensor, NHWC (1) for a channels-last
+    contiguous one (a tensor that is both reads the same either way)."""
+    if t.dim() == 4 and t.is_contiguous():
+        return NCHW
+    if t.dim() == 4 and t.is_contiguous(memory_format=torch.channels_last):
+        return NHWC
+    raise ValueError("activations must be 4-D and contiguous (NCHW) or channels-last contiguous (NHWC)")
+
+
+def _act(t: torch.Tensor, name: str, layout=None) -> torch.Tensor:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous (NCHW)")
+    if layout is None:
+        layout_of(t)
+    elif not t.is_contiguous(memory_format=torch.channels_last if layout == NHWC else torch.contiguous_format):
+        raise ValueError(f"{name} must have the layout of the input ({'NHWC' if layout == NHWC else 'NCHW'})")
     return t
 
 
@@ -134,7 +148,7 @@ def _stream(device, stream):
 
 def make_desc(x: torch.Tensor, k: int, L: int) -> Desc:
     B, C, H, W = x.shape
-    return Desc(B, C, H, W, int(k), int(L), _dtype_code(x))
+    return Desc(B, C, H, W, int(k), int(L), _dtype_code(x), layout_of(x))
 
 
 def _params(x, base_w, base_b, base_scale, wt_w, wt_scale, L):
@@ -164,7 +178,7 @@ def forward(x, base_w, base_b, base_scale, wt_w, wt_scale, L: int, y=None, strea
     k = _params(x, base_w, base_b, base_scale, wt_w, wt_scale, L)
     if y is None:
         y = torch.empty_like(x)
-    _act(y, "y")
+    _act(y, "y", layout_of(x))
     d = make_desc(x, k, L)
     _check(lib.wtconv_forward(ctypes.byref(d), _ptr(x), _ptr(base_w), _ptr(base_b), _ptr(base_scale),
                               _ptr(wt_w if L > 0 else None), _ptr(wt_scale if L > 0 else None), _ptr(y),
@@ -179,7 +193,7 @@ def backward_input(dy, base_w, base_scale, wt_w, wt_scale, L: int, dx=None, stre
     k = _params(dy, base_w, None, base_scale, wt_w, wt_scale, L)
     if dx is None:
         dx = torch.empty_like(dy)
-    _act(dx, "dx")
+    _act(dx, "dx", layout_of(dy))
     d = make_desc(dy, k, L)
     _check(lib.wtconv_backward_input(ctypes.byref(d), _ptr(dy), _ptr(base_w), _ptr(base_scale),
                                      _ptr(wt_w if L > 0 else None), _ptr(wt_scale if L > 0 else None), _ptr(dx),
@@ -197,7 +211,7 @@ def backward_weight(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, g
     """
     lib = load_library()
     _act(x, "x")
-    _act(dy, "dy")
+    _act(dy, "dy", layout_of(x))
     if dy.shape != x.shape or dy.dtype != x.dtype or dy.device != x.device:
         raise ValueError("x and dy must have the same shape, dtype and device")
     k = _params(x, base_w, base_b, base_scale, wt_w, wt_scale, L)
@@ -232,7 +246,7 @@ def backward(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, dx=None,
     """
     lib = load_library()
     _act(x, "x")
-    _act(dy, "dy")
+    _act(dy, "dy", layout_of(x))
     if dy.shape != x.shape or dy.dtype != x.dtype or dy.device != x.device:
         raise ValueError("x and dy must have the same shape, dtype and device")
     k = _params(x, base_w, base_b, base_scale, wt_w, wt_scale, L)
@@ -240,7 +254,7 @@ def backward(x, dy, base_w, base_b, base_scale, wt_w, wt_scale, L: int, dx=None,
     dev = x.device
     if dx is None:
         dx = torch.empty_like(dy)
-    _act(dx, "dx")
+    _act(dx, "dx", layout_of(dy))
     if grads is None:
         grads = dict(base_w=torch.empty((C, k, k), device=dev), base_b=torch.empty((C,), device=dev),
                      base_scale=torch.empty((C,), device=dev),

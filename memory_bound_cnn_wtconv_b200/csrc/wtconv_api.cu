@@ -75,6 +75,7 @@ const char* wtconv_status_string(wtconv_status_t s) {
         case WTCONV_ERR_WORKSPACE: return "workspace missing or too small";
         case WTCONV_ERR_UNSUPPORTED: return "plane too large to stage on chip";
         case WTCONV_ERR_CUDA: return "CUDA runtime error";
+        case WTCONV_ERR_LAYOUT: return "unknown activation layout (0 = NCHW, 1 = NHWC)";
     }
     return "unknown status";
 }

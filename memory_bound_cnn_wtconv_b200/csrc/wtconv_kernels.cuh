@@ -59,6 +59,10 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gsrc) : "memory");
 }
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gsrc) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
@@ -68,10 +72,55 @@ __device__ __forceinline__ void stage_plane(float* stg, const void* src, int chu
     for (int ch = tid; ch < chunks; ch += nt) cp_async16(d + 16 * ch, g + 16 * ch);
 }
 
+// Activations in global memory.  NCHW: plane (b, c) is Hr x Wr contiguous
+// elements.  NHWC: the C channels of a pixel are adjacent, so plane (b, c)
+// starts at element b*Hr*Wr*C + c and its elements are C apart.  `act_es`
+// is that element stride; an offset within a plane is (h*Wr + w) * act_es.
+// NHWC is a runtime layout of the general instantiations and the one-pass
+// backward only (NHW = false compiles the plain NCHW walk).
+template <bool NHW>
+__device__ __forceinline__ size_t act_es(const Plan& P) {
+    return (NHW && P.nhwc) ? (size_t)P.C : (size_t)1;
+}
+template <bool NHW>
+__device__ __forceinline__ size_t plane_origin(const Plan& P, int b, int c) {
+    const size_t hw = (size_t)P.Hr * P.Wr;
+    return (NHW && P.nhwc) ? (size_t)b * hw * P.C + c : ((size_t)b * P.C + c) * hw;
+}
+
+// NHWC staging: this CTA's `rows` real rows of Wr elements, each element C
+// elements from the next, into staging rows of W elements.  fp32 elements
+// go by 4-byte cp.async; bf16 elements (2 bytes, below the smallest
+// cp.async) by plain loads and shared stores.
+__device__ __forceinline__ void stage_nhwc(float* stg, const void* src, const Plan& P, int rows, int tid, int nt) {
+    const int n = rows * P.Wr;
+    const size_t es = (size_t)P.C;
+    if (P.esize == 4) {
+        const float* g = static_cast<const float*>(src);
+        for (int e = tid; e < n; e += nt) {
+            const int r = fdiv(e, P.div_wr), col = e - r * P.Wr;
+            cp_async4(stg + r * P.W + col, g + (size_t)e * es);
+        }
+    } else {
+        const unsigned short* g = static_cast<const unsigned short*>(src);
+        unsigned short* d = reinterpret_cast<unsigned short*>(stg);
+#pragma unroll 4
+        for (int e = tid; e < n; e += nt) {
+            const int r = fdiv(e, P.div_wr), col = e - r * P.Wr;
+            d[r * P.W + col] = __ldg(g + (size_t)e * es);
+        }
+    }
+}
+
 // This CTA's rows of a plane into staging: one contiguous copy, or (planes
 // zero-padded on chip) its `rows` real rows, each Wr elements, into staging
-// rows of W elements (the padding was zeroed once and is never written).
+// rows of W elements (the padding was zeroed once and is never written), or
+// the NHWC gather above.
 __device__ __forceinline__ void stage_rows(float* stg, const void* src, const Plan& P, int rows, int tid, int nt) {
+    if (P.nhwc) {
+        stage_nhwc(stg, src, P, rows, tid, nt);
+        return;
+    }
     if (!P.padded) {
         stage_plane(stg, src, P.plane_chunks, tid, nt);
         return;
@@ -125,6 +174,29 @@ __device__ __forceinline__ void gst4<__nv_bfloat16>(__nv_bfloat16* p, float4 v) 
     r.x = *reinterpret_cast<uint32_t*>(&a);
     r.y = *reinterpret_cast<uint32_t*>(&b);
     *reinterpret_cast<uint2*>(p) = r;
+}
+
+// Store 4 activations that are `es` elements apart (es = 1: gst4).
+template <typename T>
+__device__ __forceinline__ void gst1(T* p, float v);
+template <>
+__device__ __forceinline__ void gst1<float>(float* p, float v) {
+    *p = v;
+}
+template <>
+__device__ __forceinline__ void gst1<__nv_bfloat16>(__nv_bfloat16* p, float v) {
+    *p = __float2bfloat16_rn(v);
+}
+template <typename T>
+__device__ __forceinline__ void gst4s(T* p, float4 v, size_t es) {
+    if (es == 1) {
+        gst4<T>(p, v);
+    } else {
+        gst1<T>(p, v.x);
+        gst1<T>(p + es, v.y);
+        gst1<T>(p + 2 * es, v.z);
+        gst1<T>(p + 3 * es, v.w);
+    }
 }
 
 // Store 4 / 2 floats to a shared address congruent to P (mod 4) floats.
@@ -722,19 +794,22 @@ __device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp
         const float a0 = ll.x - lh.x, b0 = hl.x - hh.x, a1 = ll.y - lh.y, b1 = hl.y - hh.y;
         bot.x += a0 + b0; bot.y += a0 - b0; bot.z += a1 + b1; bot.w += a1 - b1;
     }
-    // yp: this CTA's rows in y (row stride Wr); only real outputs are stored.
-    T* yo = yp + (size_t)(2 * i) * P.Wr + 4 * q;
+    // yp: this CTA's rows in y (row stride Wr elements, each act_es apart);
+    // only real outputs are stored.
     if (!GUARD) {
+        T* yo = yp + (size_t)(2 * i) * P.Wr + 4 * q;
         gst4<T>(yo, top);
         gst4<T>(yo + P.Wr, bot);
     } else if (4 * q < P.Wr) {
-        if (2 * i < rows) gst4<T>(yo, top);
-        if (2 * i + 1 < rows) gst4<T>(yo + P.Wr, bot);
+        const size_t es = act_es<true>(P);
+        T* yo = yp + ((size_t)(2 * i) * P.Wr + 4 * q) * es;
+        if (2 * i < rows) gst4s<T>(yo, top, es);
+        if (2 * i + 1 < rows) gst4s<T>(yo + (size_t)P.Wr * es, bot, es);
     }
 }
 
-// Shared pieces of the two forward schedules.
-template <int K, typename T, bool BWD>
+// Shared pieces of the two forward schedules (NHW: the NHWC layout may occur).
+template <int K, typename T, bool BWD, bool NHW>
 struct FusedCtx {
     float* sm;
     const Plan& P;
@@ -743,12 +818,12 @@ struct FusedCtx {
     long long units;
     int u0, u1;
     size_t plane_elems;  // Hr * Wr
-    size_t strip_off;    // first element of this CTA's strip within a plane
+    size_t strip_off;    // first element of this CTA's strip within a plane (plane-relative index)
 
     // Units run channel-major: unit u is plane (b, c) = (u mod B, u / B).
     // Offset of this CTA's rows of plane (b, c).
     __device__ __forceinline__ size_t rows_of(int b, int c) const {
-        return ((size_t)b * P.C + c) * plane_elems + strip_off;
+        return plane_origin<NHW>(P, b, c) + strip_off * act_es<NHW>(P);
     }
     __device__ __forceinline__ const T* src(int b, int c) const { return x + rows_of(b, c); }
     // Reformulation (3): fold the scales (and the Haar factors) into the
@@ -801,7 +876,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
     const int rank = strips ? (int)cg::this_cluster().block_rank() : 0;
     const long long team = strips ? blockIdx.x / P.nstrips : blockIdx.x;
     const long long teams = strips ? gridDim.x / P.nstrips : gridDim.x;
-    FusedCtx<K, T, BWD> cx{sm, P, x, base_w, base_b, base_scale, wt_w, wt_scale, units,
+    FusedCtx<K, T, BWD, GENERAL> cx{sm, P, x, base_w, base_b, base_scale, wt_w, wt_scale, units,
                            (int)((team * units) / teams), (int)(((team + 1) * units) / teams),
                            (size_t)P.Hr * P.Wr, (size_t)rank * P.H * P.Wr};
     const int myrows = real_rows(P, rank);
@@ -871,11 +946,12 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
                 });
             } else {
                 // L = 0: the base branch is the whole output.
-                T* yo = y + cx.rows_of(cur_b, cur_c) + j.out;
+                const size_t es = act_es<GENERAL>(P);
+                T* yo = y + cx.rows_of(cur_b, cur_c) + (size_t)j.out * es;
                 const int h0 = j.row0;
                 conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
                     if (h0 + o < myrows)
-                        gst4<T>(yo + (size_t)o * P.Wr, make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
+                        gst4s<T>(yo + (size_t)o * P.Wr * es, make_float4(a[0].x, a[0].y, a[1].x, a[1].y), es);
                 });
             }
         }
@@ -990,8 +1066,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
     const bool strips = GENERAL && P.nstrips > 1;
     const int rank = strips ? (int)cg::this_cluster().block_rank() : 0;
     const int c = strips ? blockIdx.x / P.nstrips : blockIdx.x, g = blockIdx.y, G = P.groups;
-    const size_t plane_elems = (size_t)P.Hr * P.Wr;
-    const size_t strip_off = (size_t)rank * P.H * P.Wr;
+    const size_t strip_off = (size_t)rank * P.H * P.Wr * act_es<GENERAL>(P);
     const int myrows = real_rows(P, rank);
     auto csync = [&]() { __syncthreads(); };
 
@@ -1010,7 +1085,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
             stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
         }
     };
-    if (g < P.B) stage(((size_t)g * P.C + c) * plane_elems + strip_off, true);
+    if (g < P.B) stage(plane_origin<GENERAL>(P, g, c) + strip_off, true);
     cp_async_commit();
 
     // This thread's class and its run of that class's tiles.
@@ -1044,7 +1119,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
             sdy = tv;
         }
         plane_sync<GENERAL>(P);  // both analyses complete (every strip)
-        if (b + G < P.B) stage(((size_t)(b + G) * P.C + c) * plane_elems + strip_off, !dys);
+        if (b + G < P.B) stage(plane_origin<GENERAL>(P, b + G, c) + strip_off, !dys);
         cp_async_commit();
         if (strips) {
             copy_halos(sm, P, rank, tid, nt);
@@ -1067,7 +1142,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
         if (dys) {
             __syncthreads();  // every dy tile read (dy is this CTA's own; no other CTA reads it)
             if (b + G < P.B)
-                stage_rows(sm + P.stg + P.stg_floats, dy + ((size_t)(b + G) * P.C + c) * plane_elems + strip_off, P,
+                stage_rows(sm + P.stg + P.stg_floats, dy + plane_origin<GENERAL>(P, b + G, c) + strip_off, P,
                            myrows, tid, nt);
             cp_async_commit();
         }
@@ -1130,13 +1205,14 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
     const size_t plane_elems = (size_t)P.Hr * P.Wr;
     const int myrows = real_rows(P, 0);
     auto csync = [&]() { __syncthreads(); };
-    FusedCtx<K, T, true> cx{sm, P, dy, base_w, base_b, base_scale, wt_w, wt_scale, 0, 0, 0, plane_elems, 0};
+    FusedCtx<K, T, true, true> cx{sm, P, dy, base_w, base_b, base_scale, wt_w, wt_scale, 0, 0, 0, plane_elems, 0};
+    const size_t es = act_es<true>(P);
 
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
     cx.fold(c, nt, tid);  // the channel is fixed: dx weights folded once
     if (g < P.B) {
-        const size_t off = ((size_t)g * P.C + c) * plane_elems;
+        const size_t off = plane_origin<true>(P, g, c);
         stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
         stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
     }
@@ -1191,14 +1267,14 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
                 }
             }
             if (prev_b >= 0 && P.L >= 1) {
-                T* yp = dx + ((size_t)prev_b * P.C + c) * plane_elems;
+                T* yp = dx + plane_origin<true>(P, prev_b, c);
                 for (int t = tid; t < P.n_fin; t += nt) synth_item<T, true>(sm, P, yp, t, myrows);
             }
             if (!have) break;
             __syncthreads();  // both analyses complete; the previous plane's Q and Y consumed
             // Phase B.
             if (b + G < P.B) {
-                const size_t off = ((size_t)(b + G) * P.C + c) * plane_elems;
+                const size_t off = plane_origin<true>(P, b + G, c);
                 stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
                 stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
             }
@@ -1216,13 +1292,13 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
                                                      make_float4(a[0].x, a[0].y, a[1].x, a[1].y);
                                              });
                     } else {
-                        T* yo = dx + ((size_t)b * P.C + c) * plane_elems + job.out;
+                        T* yo = dx + plane_origin<true>(P, b, c) + (size_t)job.out * es;
                         const int h0 = job.row0;
                         conv_tile<K, TR, TC>(sm + job.win, job.wstride, w, make_float2(0.f, 0.f),
                                              [&](int o, float2(&a)[NP]) {
                                                  if (h0 + o < myrows)
-                                                     gst4<T>(yo + (size_t)o * P.Wr,
-                                                             make_float4(a[0].x, a[0].y, a[1].x, a[1].y));
+                                                     gst4s<T>(yo + (size_t)o * P.Wr * es,
+                                                              make_float4(a[0].x, a[0].y, a[1].x, a[1].y), es);
                                              });
                     }
                 }

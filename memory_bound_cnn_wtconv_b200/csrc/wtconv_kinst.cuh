@@ -111,8 +111,9 @@ cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
 
 template <int TR, typename T>
 cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s) {
-    // The general instantiation for cluster strips and / or planes padded on chip.
-    if (P.nstrips > 1 || P.padded)
+    // The general instantiation for cluster strips, planes padded on chip
+    // and / or NHWC activations.
+    if (P.nstrips > 1 || P.padded || P.nhwc)
         return bwd ? fused_typed<TR, T, true, true>(P, a, s) : fused_typed<TR, T, false, true>(P, a, s);
     return bwd ? fused_typed<TR, T, true, false>(P, a, s) : fused_typed<TR, T, false, false>(P, a, s);
 }
@@ -138,7 +139,7 @@ cudaError_t fused_tr(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cud
 
 template <int TR>
 cudaError_t bwdw_tr(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
-    const bool strips = P.nstrips > 1 || P.padded;  // the general instantiation
+    const bool strips = P.nstrips > 1 || P.padded || P.nhwc;  // the general instantiation
     if (dtype == 0) return strips ? bwdw_typed<TR, float, true>(P, a, s) : bwdw_typed<TR, float, false>(P, a, s);
     return strips ? bwdw_typed<TR, __nv_bfloat16, true>(P, a, s) : bwdw_typed<TR, __nv_bfloat16, false>(P, a, s);
 }

@@ -86,6 +86,10 @@ struct Plan {
     // each) into staging rows of W elements, and only real outputs are
     // stored.
     int Hr, Wr, padded, row_chunks;
+    // Activation layout in global memory: 0 = NCHW, 1 = NHWC (planes
+    // gathered element by element, C elements apart; the general
+    // instantiations and the one-pass backward only).
+    int nhwc;
     int parts;           // weight gradient: partial vectors per channel (groups * nstrips)
     int TR, TC;          // output tile: TR rows x TC cols per thread (TC = 4: two column pairs)
     int esize;           // bytes per stored activation (4 or 2)
@@ -136,6 +140,7 @@ struct Plan {
     FastDiv div_q4;                 // W / 4: 4-column groups per row
     FastDiv div_w;                  // W
     FastDiv div_rowc;               // row_chunks
+    FastDiv div_wr;                 // Wr (NHWC staging)
     FastDiv div_m[kMaxL];           // W >> (l+1)
     FastDiv div_ntc[kMaxL + 1];     // tile columns per tile row
 };

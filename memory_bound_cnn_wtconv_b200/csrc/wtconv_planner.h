@@ -98,12 +98,15 @@ inline wtconv_status_t validate(const wtconv_desc_t* d) {
     if (d->B <= 0 || d->C <= 0 || d->H <= 0 || d->W <= 0) return WTCONV_ERR_BAD_SHAPE;
     if (!is_supported_k(d->k)) return WTCONV_ERR_BAD_K;
     if (d->L < 0 || d->L > kMaxL) return WTCONV_ERR_BAD_L;
+    if (d->layout != WTCONV_NCHW && d->layout != WTCONV_NHWC) return WTCONV_ERR_LAYOUT;
     if ((d->W % 4) != 0) return WTCONV_ERR_BAD_SHAPE;
-    // Planes are staged in 16-byte chunks: whole planes if H and W are
-    // multiples of 2^L, else (zero-padded on chip) row by row.
+    // NCHW planes are staged in 16-byte chunks: whole planes if H and W are
+    // multiples of 2^L, else (zero-padded on chip) row by row.  NHWC planes
+    // are gathered element by element.
     const long long esize = d->dtype == WTCONV_BF16 ? 2 : 4;
     const bool padded = (d->H % (1 << d->L)) != 0 || (d->W % (1 << d->L)) != 0;
-    if (padded ? ((long long)d->W * esize) % 16 != 0 : ((long long)d->H * d->W * esize) % 16 != 0)
+    if (d->layout == WTCONV_NCHW &&
+        (padded ? ((long long)d->W * esize) % 16 != 0 : ((long long)d->H * d->W * esize) % 16 != 0))
         return WTCONV_ERR_BAD_SHAPE;
     // Index arithmetic in the kernels is 32-bit within a plane and 64-bit across planes.
     if ((long long)d->H * d->W > (1LL << 30)) return WTCONV_ERR_BAD_SHAPE;
@@ -140,6 +143,8 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     P->Wr = d->W;
     P->padded = (Hv != d->H || Wv != d->W) ? 1 : 0;
     P->nstrips = nstrips;
+    P->nhwc = d->layout == WTCONV_NHWC ? 1 : 0;
+    P->div_wr = make_fastdiv(P->Wr);
     const int p = d->k / 2, k = d->k, L = d->L, H = Hs, W = Wv, KK = k * k;
     P->p = p;
     P->esize = d->dtype == WTCONV_BF16 ? 2 : 4;

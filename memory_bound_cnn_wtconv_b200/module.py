@@ -29,7 +29,8 @@ class WTConvFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, x, base_w, base_b, base_scale, wt_w, wt_scale, L: int, one_pass: bool = False):
-        x = x.contiguous()
+        # Channels-last inputs stay NHWC (the kernels read either layout).
+        x = x if x.dim() == 4 and x.is_contiguous(memory_format=torch.channels_last) else x.contiguous()
         y = forward(x, base_w, base_b, base_scale, wt_w, wt_scale, L)
         ctx.save_for_backward(x, base_w, base_b, base_scale, wt_w, wt_scale)
         ctx.L = L
@@ -40,7 +41,8 @@ class WTConvFunction(torch.autograd.Function):
     def backward(ctx, dy):
         x, base_w, base_b, base_scale, wt_w, wt_scale = ctx.saved_tensors
         L = ctx.L
-        dy = dy.to(x.dtype).contiguous()
+        fmt = torch.contiguous_format if x.is_contiguous() else torch.channels_last
+        dy = dy.to(x.dtype).contiguous(memory_format=fmt)
         need = ctx.needs_input_grad
         dx, g = None, {}
         if ctx.one_pass and need[0] and any(need[1:6]):

@@ -85,6 +85,27 @@ int real_rows_host(const Plan& P, int rank) { return std::max(0, std::min(P.H, P
 void replay_stage(Shadow& sh, const Plan& P, long long stg, int tag, int rank) {
     const long long strip_bytes = (long long)P.H * P.W * P.esize;
     const long long plane_bytes = (long long)P.Hr * P.Wr * P.esize;
+    if (P.nhwc) {
+        // Element by element: strip element e = r*Wr + col (plane element
+        // rank*H*Wr + e) -> staging element r*W + col; a staging float holds
+        // 4 / esize elements and is written once.
+        if (stg % 4) sh.fail("staging not 16-byte aligned", stg);
+        const int rows = real_rows_host(P, rank);
+        const int per = 4 / P.esize;
+        std::vector<char> hit((size_t)P.stg_floats, 0);
+        for (long long e = 0; e < (long long)rows * P.Wr; ++e) {
+            const int r = (int)fastdiv_host((uint32_t)e, P.div_wr), col = (int)e - r * P.Wr;
+            if (r != e / P.Wr) sh.fail("element-row division", e);
+            check_global((long long)rank * P.H * P.Wr + e, (long long)P.Hr * P.Wr, "staging source element");
+            const long long f = ((long long)r * P.W + col) / per;
+            if (f < 0 || f >= P.stg_floats) sh.fail("staging element outside the staging buffer", f);
+            if (!hit[f]) {
+                hit[f] = 1;
+                sh.write(stg + f, stg, stg + P.stg_floats, tag, "staging");
+            }
+        }
+        return;
+    }
     if (P.plane_chunks * 16LL != strip_bytes) sh.fail("strip is not a whole number of 16-byte chunks", strip_bytes);
     if (stg % 4) sh.fail("staging not 16-byte aligned", stg);
     if (!P.padded) {
@@ -827,16 +848,50 @@ void check_bwd(const wtconv_desc_t& d) {
                 P.nthreads, P.corr0, ncorr, TR, P.groups);
 }
 
+// NHWC: the kernels address element e (plane-relative, row-major over the
+// real Hr x Wr plane) of plane (b, c), strip `rank`, at
+//   b*Hr*Wr*C + c  +  rank*H*Wr*C  +  e*C     (e < real rows of the strip x Wr).
+// Every (b, c, rank, e) must land on a distinct element of the B*C*Hr*Wr
+// tensor, and every element must be reached.
+void check_nhwc_map(const wtconv_desc_t& d) {
+    Plan P;
+    if (make_plan(&d, kForward, kB200SMs, &P) != WTCONV_OK) return;
+    const long long hw = (long long)P.Hr * P.Wr, n = (long long)P.B * P.C * hw;
+    if (n > (1LL << 26)) return;
+    std::vector<unsigned char> seen(n, 0);
+    for (int b = 0; b < P.B; ++b)
+        for (int c = 0; c < P.C; ++c)
+            for (int rank = 0; rank < P.nstrips; ++rank) {
+                const int rows = std::max(0, std::min(P.H, P.Hr - rank * P.H));
+                const long long base = (long long)b * hw * P.C + c + (long long)rank * P.H * P.Wr * P.C;
+                for (long long e = 0; e < (long long)rows * P.Wr; ++e) {
+                    const long long off = base + e * P.C;
+                    if (off < 0 || off >= n || seen[off]) {
+                        std::printf("FAIL nhwc element map b %d c %d strip %d e %lld -> %lld\n", b, c, rank, e, off);
+                        std::exit(1);
+                    }
+                    seen[off] = 1;
+                }
+            }
+    for (long long i = 0; i < n; ++i)
+        if (!seen[i]) {
+            std::printf("FAIL nhwc element %lld never addressed\n", i);
+            std::exit(1);
+        }
+    std::printf("nhwc: %lld elements, each addressed once\n", n);
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
-    if (argc != 8) {
-        std::printf("usage: plan_access_check B C H W k L dtype\n");
+    if (argc != 8 && argc != 9) {
+        std::printf("usage: plan_access_check B C H W k L dtype [layout]\n");
         return 2;
     }
-    wtconv_desc_t d;
+    wtconv_desc_t d{};
     d.B = std::atoi(argv[1]); d.C = std::atoi(argv[2]); d.H = std::atoi(argv[3]); d.W = std::atoi(argv[4]);
     d.k = std::atoi(argv[5]); d.L = std::atoi(argv[6]); d.dtype = std::atoi(argv[7]);
+    d.layout = argc == 9 ? std::atoi(argv[8]) : WTCONV_NCHW;
     if (validate(&d) != WTCONV_OK) {
         std::printf("invalid (status %d)\n", (int)validate(&d));
         return 3;
@@ -845,6 +900,7 @@ int main(int argc, char** argv) {
     check_fused(d, kBackwardInput);
     check_bwdw(d);
     check_bwd(d);
+    if (d.layout == WTCONV_NHWC) check_nhwc_map(d);
     std::printf("OK\n");
     return 0;
 }

@@ -16,7 +16,7 @@ import memory_bound_cnn_wtconv_b200 as w
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "wtconv.h")
 
-OK, NULLPTR, BAD_SHAPE, BAD_K, BAD_L, MISALIGNED, DTYPE, WORKSPACE, UNSUPPORTED, CUDA = range(10)
+OK, NULLPTR, BAD_SHAPE, BAD_K, BAD_L, MISALIGNED, DTYPE, WORKSPACE, UNSUPPORTED, CUDA, LAYOUT = range(11)
 FAKE = 0x10000  # 16-byte aligned, never dereferenced
 
 
@@ -37,8 +37,8 @@ def test_library_exports_every_declared_symbol(cuda_lib):
         assert hasattr(cuda_lib, name), name
 
 
-def _desc(B=2, C=3, H=16, W=16, k=5, L=2, dtype=0):
-    return w.Desc(B, C, H, W, k, L, dtype)
+def _desc(B=2, C=3, H=16, W=16, k=5, L=2, dtype=0, layout=0):
+    return w.Desc(B, C, H, W, k, L, dtype, layout)
 
 
 def _fwd(lib, d, x=FAKE, y=FAKE, ww=FAKE, ws=FAKE):
@@ -52,9 +52,14 @@ def _fwd(lib, d, x=FAKE, y=FAKE, ww=FAKE, ws=FAKE):
     (dict(k=4), BAD_K), (dict(k=9), BAD_K), (dict(k=0), BAD_K),
     (dict(L=-1), BAD_L), (dict(L=7), BAD_L),
     (dict(W=6, L=1), BAD_SHAPE), (dict(H=12, W=12, L=3, dtype=1), BAD_SHAPE),
-    (dict(dtype=2), DTYPE),
+    (dict(dtype=2), DTYPE), (dict(layout=2), LAYOUT), (dict(layout=-1), LAYOUT),
+    # NHWC gathers element by element, so bf16 rows need not be whole 16-byte chunks
+    (dict(H=12, W=12, L=3, dtype=1, layout=1), OK),
 ])
 def test_forward_validation(cuda_lib, kw, code):
+    if code == OK:  # valid: planned without launching (the workspace query plans every pass)
+        assert cuda_lib.wtconv_workspace_bytes(ctypes.byref(_desc(**kw))) > 0
+        return
     assert _fwd(cuda_lib, _desc(**kw)) == code
 
 
@@ -103,7 +108,7 @@ def test_backward_weight_workspace(cuda_lib):
 
 
 def test_status_strings(cuda_lib):
-    for code in range(10):
+    for code in range(11):
         s = cuda_lib.wtconv_status_string(code)
         assert s and len(s) > 1
     assert cuda_lib.wtconv_status_string(999) == b"unknown status"

@@ -30,8 +30,14 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def gpu_inputs(inp):
-    return {k: v.cuda() for k, v in inp.items()}
+def gpu_inputs(inp, nhwc=False):
+    """The case's tensors on the GPU; with nhwc the activations channels-last
+    (the same logical NCHW values, stored NHWC)."""
+    g = {k: v.cuda() for k, v in inp.items()}
+    if nhwc:
+        for k in ("x", "dy"):
+            g[k] = g[k].contiguous(memory_format=torch.channels_last)
+    return g
 
 
 def run_gpu(case: Case, g, calls, fused_bwd=False):
@@ -50,6 +56,11 @@ def run_gpu(case: Case, g, calls, fused_bwd=False):
             out["grads"] = wt.backward_weight(g["x"], g["dy"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"],
                                               g["wt_scale"], case.L)
     torch.cuda.synchronize()
+    for k in ("y", "dx"):
+        if k in out:
+            assert out[k].is_contiguous(memory_format=torch.channels_last) == g["x"].is_contiguous(
+                memory_format=torch.channels_last), f"{k} does not keep the input's layout"
+            out[k] = out[k].contiguous()
     return out
 
 
@@ -61,9 +72,9 @@ def oracle_params(inp, c=None):
     return p
 
 
-def check_full(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), fused_bwd=False):
+def check_full(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), fused_bwd=False, nhwc=False):
     inp = make_inputs(case)
-    out = run_gpu(case, gpu_inputs(inp), calls, fused_bwd)
+    out = run_gpu(case, gpu_inputs(inp, nhwc), calls, fused_bwd)
     p = oracle_params(inp)
     x, dy = f64(inp["x"]), f64(inp["dy"])
     tol = TOL[case.dtype]
@@ -87,9 +98,9 @@ def check_full(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), fused_bwd=F
 
 
 def check_sampled(oracle, case: Case, calls=("fwd", "bwd_in", "bwd_w"), nplanes=6, nchannels=3, seed=0,
-                  fused_bwd=False):
+                  fused_bwd=False, nhwc=False):
     inp = make_inputs(case)
-    out = run_gpu(case, gpu_inputs(inp), calls, fused_bwd)
+    out = run_gpu(case, gpu_inputs(inp, nhwc), calls, fused_bwd)
     rng = np.random.default_rng(seed)
     planes = {(0, 0), (case.B - 1, case.C - 1)}
     while len(planes) < min(nplanes, case.B * case.C):
@@ -181,13 +192,13 @@ def test_small_case_all_outputs(oracle, case):
     check_full(oracle, case, case.calls)
 
 
-def _one_pass_plan_exists(case: Case) -> bool:
+def _one_pass_plan_exists(case: Case, nhwc: bool = False) -> bool:
     """Whether wtconv_backward_one_pass plans this case (whole planes only);
     asked through the call itself with an empty workspace, which returns
     WTCONV_ERR_WORKSPACE (7) after planning and before any launch."""
     import ctypes
     lib = wt.load_library()
-    d = wt.Desc(case.B, case.C, case.H, case.W, case.k, case.L, 1 if case.dtype == "bf16" else 0)
+    d = wt.Desc(case.B, case.C, case.H, case.W, case.k, case.L, 1 if case.dtype == "bf16" else 0, int(nhwc))
     fake = ctypes.c_void_p(0x10000)
     rc = lib.wtconv_backward_one_pass(ctypes.byref(d), *([fake] * 13), ctypes.c_void_p(0), ctypes.c_size_t(0), None)
     assert rc in (7, 8), rc
@@ -319,3 +330,51 @@ def test_outputs_do_not_depend_on_stale_memory(oracle):
     assert torch.isfinite(y).all()
     for k in PARAMS:
         assert torch.isfinite(grads[k]).all(), k
+
+
+# NHWC (channels-last) activations: the same layer on the same logical
+# values, gathered and scattered element by element.  Shapes cover whole
+# planes, strips (2, 8 and 16 CTAs), planes padded on chip, L = 0, k = 1 and
+# 7, bf16, and rows that are not whole 16-byte chunks (allowed in NHWC only).
+NHWC_SMALL = [
+    Case("nhwc_odd_batch_stage1_plane", 3, 5, 56, 56, 5, 3, "f32", 51, "normal", "normal"),
+    Case("nhwc_rect_24x40", 2, 3, 24, 40, 3, 3, "f32", 52, "normal", "normal"),
+    Case("nhwc_L0", 2, 3, 12, 8, 5, 0, "f32", 53, "normal", "normal"),
+    Case("nhwc_k1", 1, 2, 16, 16, 1, 2, "f32", 54, "normal", "normal"),
+    Case("nhwc_k7_L4", 2, 3, 32, 32, 7, 4, "f32", 55, "normal", "normal"),
+    Case("nhwc_bf16_stage1_plane", 3, 4, 56, 56, 5, 3, "bf16", 56, "uniform", "normal"),
+    Case("nhwc_bf16_pad_13x12", 2, 3, 13, 12, 5, 2, "bf16", 57, "normal", "normal"),
+    Case("nhwc_pad_30x28_L3", 3, 2, 30, 28, 5, 3, "f32", 58, "normal", "normal"),
+    Case("nhwc_strips_128_L2", 1, 3, 128, 128, 5, 2, "f32", 59, "normal", "normal"),
+    Case("nhwc_strips_256_L3_bf16", 1, 2, 256, 256, 3, 3, "bf16", 60, "normal", "normal"),
+    Case("nhwc_pad_strips_250x248", 1, 1, 250, 248, 5, 4, "f32", 61, "normal", "normal"),
+]
+
+
+@pytest.mark.parametrize("case", NHWC_SMALL, ids=lambda c: c.name)
+def test_nhwc_small_case_all_outputs(oracle, case):
+    check_full(oracle, case, case.calls, nhwc=True)
+
+
+@pytest.mark.parametrize("mode", ["auto", "one_pass"])
+@pytest.mark.parametrize("case", NHWC_SMALL[:8], ids=lambda c: c.name)
+def test_nhwc_small_case_fused_backward(oracle, case, mode):
+    if mode == "one_pass" and not _one_pass_plan_exists(case, nhwc=True):
+        pytest.skip("planes split into cluster strips have no one-pass plan")
+    check_full(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=mode, nhwc=True)
+
+
+@pytest.mark.parametrize("case", [STAGE1, TRAIN_BF16], ids=lambda c: c.name)
+def test_nhwc_full_size_workloads_sampled(oracle, case):
+    check_sampled(oracle, case, nhwc=True)
+
+
+def test_nhwc_matches_nchw_bitwise():
+    # Same on-chip arithmetic in the same order: the layouts must agree bit for bit.
+    case = Case("nhwc_vs_nchw", 4, 6, 40, 36, 5, 3, "f32", 62, "normal", "normal")
+    inp = make_inputs(case)
+    a = run_gpu(case, gpu_inputs(inp), ("fwd", "bwd_in", "bwd_w"))
+    b = run_gpu(case, gpu_inputs(inp, nhwc=True), ("fwd", "bwd_in", "bwd_w"))
+    assert torch.equal(a["y"], b["y"]) and torch.equal(a["dx"], b["dx"])
+    for k in PARAMS:
+        assert torch.equal(a["grads"][k], b["grads"][k]), k

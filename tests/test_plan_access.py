@@ -57,6 +57,24 @@ def test_every_access_in_bounds(checker, case):
     assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout + r.stderr
 
 
+# NHWC activations (layout 1): element-by-element staging and stores; the
+# checker also verifies that the kernels' NHWC element map covers the tensor
+# exactly once.  Includes shapes whose rows are not whole 16-byte chunks
+# (allowed in NHWC only), strips and padded planes.
+NHWC = [
+    (3, 5, 56, 56, 5, 3, 0), (2, 4, 56, 56, 5, 3, 1), (2, 3, 13, 12, 5, 2, 1), (1, 2, 12, 8, 1, 0, 0),
+    (2, 3, 24, 40, 3, 3, 1), (1, 2, 128, 128, 5, 2, 0), (1, 1, 250, 248, 5, 4, 1), (3, 2, 30, 28, 5, 3, 0),
+    (2, 2, 64, 64, 7, 4, 0), (5, 3, 20, 12, 5, 2, 1),
+]
+
+
+@pytest.mark.parametrize("case", NHWC, ids=lambda c: "x".join(map(str, c)) + "_nhwc")
+def test_every_access_in_bounds_nhwc(checker, case):
+    r = subprocess.run([checker, *map(str, case), "1"], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip().endswith("OK") and "each addressed once" in r.stdout, \
+        r.stdout + r.stderr
+
+
 @pytest.mark.parametrize("case,strips,alias", [
     ((1, 1, 256, 256, 5, 4, 0), 8, True),    # DY would not fit beside two staged strips at 8 strips
     ((2, 2, 128, 128, 5, 4, 0), 2, True),
