@@ -3,6 +3,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "wtconv_kernels.cuh"
 #include "wtconv_launch.h"
@@ -20,18 +21,19 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-// cudaFuncSetAttribute for the dynamic shared-memory opt-in, once per kernel
-// and device (idempotent; a repeated call is harmless).
-// (and the non-portable cluster-size opt-in for 16-CTA clusters).
+// cudaFuncSetAttribute for the dynamic shared-memory opt-in (and the
+// non-portable cluster-size opt-in for 16-CTA clusters), once per kernel and
+// device.  The attributes are idempotent, so host threads racing on the first
+// call both set them; the flags are atomic so that the race is benign.
 template <class F>
-cudaError_t opt_in_smem(F* fn, bool (&done)[kMaxDevices]) {
+cudaError_t opt_in_smem(F* fn, std::atomic<bool> (&done)[kMaxDevices]) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && done[dev]) return cudaSuccess;
+    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev] = true;
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
     return e;
 }
 
@@ -60,7 +62,7 @@ struct Launch {
 
 template <int TR, typename T, bool BWD, bool GENERAL>
 cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
-    static bool done[kMaxDevices] = {};
+    static std::atomic<bool> done[kMaxDevices] = {};
     auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD, GENERAL>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
@@ -93,7 +95,7 @@ cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
 
 template <int TR, typename T, bool GENERAL>
 cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
-    static bool done[kMaxDevices] = {};
+    static std::atomic<bool> done[kMaxDevices] = {};
     auto* fn = wtconv_bwdw_partial_kernel<WTC_K, TR, 4, T, GENERAL>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
@@ -120,7 +122,7 @@ cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s)
 
 template <int TR, typename T>
 cudaError_t bwd_typed(const Plan& P, const BwdArgs& a, cudaStream_t s) {
-    static bool done[kMaxDevices] = {};
+    static std::atomic<bool> done[kMaxDevices] = {};
     auto* fn = wtconv_backward_kernel<WTC_K, TR, 4, T>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;

@@ -54,3 +54,15 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_lib):
             r, o = ref[k].double(), out[k].double()
             err = float((o - r).abs().max() / r.abs().max().clamp_min(1e-30))
             assert err <= 1e-5, (case.name, k, err)
+
+
+def test_noalloc_refuses_oversize_plans_and_leaves_outputs_untouched(cuda_lib):
+    # Partials beyond the fixed 4 MiB array: WTCONV_ERR_WORKSPACE, nothing enqueued.
+    case = Case("noalloc_oversize", 2, 4096, 16, 16, 7, 2, "f32", 43, "normal", "normal")
+    g = {k: v.cuda() for k, v in make_inputs(case).items()}
+    out = {k: torch.full_like(g[k], float("nan")) for k in PARAMS}
+    rc = _noalloc(cuda_lib, case, g, out, torch.cuda.current_stream())
+    assert rc == 7, wt.STATUS.get(rc, rc)
+    torch.cuda.synchronize()
+    for k in PARAMS:
+        assert torch.isnan(out[k]).all(), k
