@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="stage1")
+    ap.add_argument("--nhwc", action="store_true", help="channels-last (NHWC) activations for the named workload")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -91,8 +92,8 @@ def conv_fmas(c) -> float:
     return c.numel * c.k * c.k * (1.0 + sum(4.0 ** -l for l in range(c.L)))
 
 
-def workload_name(c) -> str:
-    return (f"{c.name}: B={c.B} C={c.C} H={c.H} W={c.W} k={c.k} L={c.L} {c.dtype} NCHW, "
+def workload_name(c, nhwc: bool = False) -> str:
+    return (f"{c.name}: B={c.B} C={c.C} H={c.H} W={c.W} k={c.k} L={c.L} {c.dtype} {'NHWC' if nhwc else 'NCHW'}, "
             f"forward + backward_input + backward_weight")
 
 
@@ -455,7 +456,7 @@ def run_ours(args, case):
     wt.load_library()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    wl = Workload(case, dev, stream, rank, world)
+    wl = Workload(case, dev, stream, rank, world, nhwc=args.nhwc)
     K = args.steps
     clocks = Clocks(not args.no_clocks, physical_gpu_index(local))
     times, wall, clk = wl.time_calls(wl.calls, K, args.warmup, flush, clocks)
@@ -498,7 +499,7 @@ def run_ours(args, case):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if case.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": workload_name(case), "global_batch": case.B * world,
+        "config": {"workload": workload_name(case, args.nhwc), "global_batch": case.B * world,
                    "parallelism": f"dp{world}", "l2": "flushed before every call (256 MiB write)",
                    "timing": f"median over the {K} timed steps of each call's CUDA-event time; step = their sum",
                    "modeled_bytes_per_step": step_bytes},
@@ -527,7 +528,7 @@ def run_ours(args, case):
                                                        dist if world > 1 else None, dev)
     line["gpu_launches"] += n_launch
     # The other WTConvNeXt stage shapes, same protocol, one GPU.
-    if world == 1 and not args.no_other_workloads:
+    if world == 1 and not args.no_other_workloads and not args.nhwc:
         other = {}
         for name in ("stage1", "stage2", "train_bf16", "stage1_nhwc"):
             if name == case.name:
