@@ -107,7 +107,7 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
     ("stage1", "bwd_w"): (79317760.0, "wtconv_bwdw_partial_kernel",
-                          "160b4f780c8cb07ac62697156f6668309e7bbc20b3822c0fdac9962833e88a5e",
+                          "5305f420c9afa45d0db6cb11c892f7249c20b9df55dfdeafe55dc62b18cf2b45",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 

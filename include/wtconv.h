@@ -155,11 +155,13 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, co
 
 /* Whole backward of the layer (the backward half of the Abstract's training
  * step): dx (as wtconv_backward_input) and every parameter gradient (as
- * wtconv_backward_weight, bitwise-repeatable).  The library picks the path:
- * the one-pass kernel of wtconv_backward_one_pass where its plan exists and
- * the planner's cost (conv-tile rows on the busiest SM sub-partition) is
- * below that of the two passes together, else wtconv_backward_input then
- * wtconv_backward_weight.  Both paths give the same results.  dx:
+ * wtconv_backward_weight, bitwise-repeatable).  The library picks the path
+ * from the plans, not by timing: the one-pass kernel of
+ * wtconv_backward_one_pass where its plan exists and the planner's cost
+ * (conv-tile rows on the busiest SM sub-partition) is below that of the two
+ * passes together, or equal to it while one of the two passes runs one CTA
+ * per SM; else wtconv_backward_input then wtconv_backward_weight.  Both
+ * paths give the same results.  dx:
  * [B][C][H][W] in desc->dtype, not overlapping x or dy.  Workspace as for
  * wtconv_backward_weight.  Every argument is checked before either pass is
  * enqueued. */

@@ -159,16 +159,17 @@ wtconv_status_t wtconv_backward(const wtconv_desc_t* d, const void* x, const voi
     if (st != WTCONV_OK) return st;
     if (!aligned16(dx)) return WTCONV_ERR_MISALIGNED;
     const int sms = planning_sm_count();
-    // The one pass where its plan exists and costs less than the two passes'
-    // plans together (plan_cost: tile rows on the busiest SM sub-partition);
-    // else the input- and weight-gradient passes, with the same results.
+    // The one pass where its plan exists and the planner prefers it to the
+    // two passes' plans (prefer_one_pass: tile rows on the busiest SM
+    // sub-partition, then CTAs per SM); else the input- and weight-gradient
+    // passes, with the same results.
     Plan P, Pin, Pw;
     st = make_plan(d, kBackward, sms, &P);
     if (st != WTCONV_OK && st != WTCONV_ERR_UNSUPPORTED) return st;
     bool one_pass = st == WTCONV_OK;
     if (one_pass && make_plan(d, kBackwardInput, sms, &Pin) == WTCONV_OK &&
         make_plan(d, kBackwardWeight, sms, &Pw) == WTCONV_OK)
-        one_pass = plan_cost(P, kBackward) < plan_cost(Pin, kBackwardInput) + plan_cost(Pw, kBackwardWeight);
+        one_pass = prefer_one_pass(P, Pin, Pw);
     if (one_pass)
         return run_one_pass(d, P, sms, x, dy, base_w, base_b, base_scale, wt_w, wt_scale, dx, d_base_w, d_base_b,
                             d_base_scale, d_wt_w, d_wt_scale, workspace, workspace_bytes, (cudaStream_t)stream);

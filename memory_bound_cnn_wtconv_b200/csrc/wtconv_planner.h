@@ -360,6 +360,23 @@ inline double plan_cost(const Plan& P, Kind kind) {
     return P.nstrips > 1 ? 1.15 * c : c;
 }
 
+// The whole backward: the one-pass plan P against the input- and
+// weight-gradient plans Pin and Pw.  The one pass when its tile-row cost is
+// lower; on equal costs, when one of the two passes also runs one CTA per SM
+// (then neither path hides an analysis phase behind a second CTA's tiles, and
+// the one pass saves a pass over dy and one analysis of it).  Measured on the
+// 64 whole-plane points of the shape sweep: the one pass is faster exactly at
+// 32x32, L = 1 (cost 4 vs 7) and at 64x64, L = 3 and 4 (cost 40 vs 12 + 28, the
+// weight pass at one CTA per SM), by 5-20%, and slower by 8-30% everywhere else
+// (32x32 at L = 4, k = 3 is within 1% either way).
+inline bool prefer_one_pass(const Plan& P, const Plan& Pin, const Plan& Pw) {
+    const double c1 = plan_cost(P, kBackward);
+    const double c2 = plan_cost(Pin, kBackwardInput) + plan_cost(Pw, kBackwardWeight);
+    if (c1 < c2 * (1.0 - 1e-9)) return true;
+    if (c1 > c2 * (1.0 + 1e-9)) return false;
+    return plan_ctas_per_sm(Pin) == 1 || plan_ctas_per_sm(Pw) == 1;
+}
+
 // Chooses the fewest strips that fit (whole planes, else clusters of 2, 4,
 // 8, 16 strips), and for that count the tile height (7 or 8 rows) with the
 // lowest plan_cost.  Every cluster strip adds barriers and halo copies per

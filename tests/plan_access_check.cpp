@@ -844,8 +844,11 @@ void check_bwd(const wtconv_desc_t& d) {
         for (int th = P.cls_thr[k2]; th < P.cls_thr[k2 + 1]; ++th)
             for (int t = 0; t < KK; ++t) sh.read(P.red + (long long)th * KK + t, P.red, red_end, RED, "class reduction");
     if ((long long)P.nv + ncls * KK + 1 > P.smem_floats) sh.fail("final-step scratch", P.nv);
-    std::printf("bwd: smem %d B, threads %d (%d conv + %d correlation), TR %d, groups %d\n", P.smem_floats * 4,
-                P.nthreads, P.corr0, ncorr, TR, P.groups);
+    Plan Pin, Pw;
+    const bool one = make_plan(&d, kBackwardInput, kB200SMs, &Pin) == WTCONV_OK &&
+                     make_plan(&d, kBackwardWeight, kB200SMs, &Pw) == WTCONV_OK && prefer_one_pass(P, Pin, Pw);
+    std::printf("bwd: smem %d B, threads %d (%d conv + %d correlation), TR %d, groups %d, library picks %s\n",
+                P.smem_floats * 4, P.nthreads, P.corr0, ncorr, TR, P.groups, one ? "one pass" : "two passes");
 }
 
 // NHWC: the kernels address element e (plane-relative, row-major over the

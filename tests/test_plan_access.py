@@ -87,3 +87,18 @@ def test_weight_gradient_strip_choice(checker, case, strips, alias):
     line = next(l for l in out.splitlines() if l.startswith("bwdw:"))
     assert f"strips {strips}" in line, line
     assert ("dy read from staging" in line) == alias, line
+
+
+@pytest.mark.parametrize("case,one_pass", [
+    # Measured on B200 (the shape sweep and the stage shapes): the one pass is
+    # faster at 32x32, L = 1 and at 64x64, L >= 3, slower elsewhere.
+    ((4, 64, 32, 32, 5, 1, 0), True), ((4, 64, 32, 32, 3, 1, 0), True),
+    ((4, 64, 64, 64, 5, 3, 0), True), ((4, 64, 64, 64, 5, 4, 0), True), ((4, 64, 64, 64, 3, 4, 0), True),
+    ((4, 64, 32, 32, 5, 2, 0), False), ((4, 64, 32, 32, 5, 3, 0), False), ((4, 64, 64, 64, 5, 1, 0), False),
+    ((4, 64, 64, 64, 3, 2, 0), False),
+    ((32, 96, 56, 56, 5, 3, 0), False), ((32, 192, 28, 28, 5, 2, 0), False), ((64, 96, 56, 56, 5, 3, 1), False),
+])
+def test_backward_path_choice(checker, case, one_pass):
+    out = subprocess.run([checker, *map(str, case)], capture_output=True, text=True).stdout
+    line = next(l for l in out.splitlines() if l.startswith("bwd:"))
+    assert ("library picks one pass" in line) == one_pass, line
