@@ -341,9 +341,10 @@ __device__ __forceinline__ float analysis_pyramid(const float* stg, int H, int W
 #pragma unroll
         for (int q = 0; q < 4; ++q) v[q] = stg_load4<T>(stg, (r0 + q) * W + c0);
         if (valid) {
+            if (COPY) {
 #pragma unroll
-            if (COPY)
                 for (int q = 0; q < 4; ++q) sts4<PD>(dst + (r0 + q) * ds + c0, v[q]);
+            }
             if (SUM) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) sum += (v[q].x + v[q].y) + (v[q].z + v[q].w);
@@ -639,54 +640,71 @@ __device__ __forceinline__ void plane_sync(const Plan& P) {
     __syncthreads();
 }
 
-// Fill the halo rows of one padded buffer of this CTA's strip: nsub planes
-// (1 or 4) of `rows` x `cols` interior elements behind `pad` border rows and
-// columns.  Halo row i (i in [-pad, 0) or [rows, rows + pad)) is plane row
-// rank*rows + i, read from the shared memory of the cluster CTA that owns it
-// (same offsets: every CTA of the cluster runs the same plan); rows outside
-// the plane are left as they are (zero).  Loads are issued in batches of 4
-// before the stores.
-__device__ __forceinline__ void copy_halo_rows(float* sm, const Buf& b, int nsub_lg, int rows, int cols, FastDiv dcols,
-                                               int pad, int rank, int nstrips, int tid, int nt) {
-    cg::cluster_group cl = cg::this_cluster();
-    const int n = (2 * pad << nsub_lg) * cols;
-    constexpr int U = 4;
-    for (int t0 = tid; t0 < n; t0 += U * nt) {
-        float v[U];
-        int dst[U];
-#pragma unroll
-        for (int q = 0; q < U; ++q) {
-            const int t = t0 + q * nt;
-            dst[q] = -1;
-            if (t < n) {
-                const int rest = fdiv(t, dcols), c = t - rest * cols;
-                const int hr = rest >> nsub_lg, s = rest - (hr << nsub_lg);
-                const int i = hr < pad ? hr - pad : rows + hr - pad;
-                const int g = rank * rows + i;
-                if (g >= 0 && g < nstrips * rows) {
-                    const int owner = g / rows, lr = g - owner * rows;
-                    const int col = b.base + s * b.sub + c + pad;
-                    const float* src = cl.map_shared_rank(sm + col + (lr + pad) * b.stride, owner);
-                    v[q] = *src;
-                    dst[q] = col + (i + pad) * b.stride;
-                }
-            }
+// The two halves of a cluster barrier, for work that can run between this
+// CTA's arrival and the others': arrive (release: this CTA's earlier shared
+// and distributed-shared stores become visible to the cluster) and wait
+// (acquire).  Every thread of every CTA of the cluster executes them in the
+// same order, alternating.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
+
+// Send this CTA's rows that other strips hold as halo rows, for one padded
+// buffer: nsub planes (1 or 4) of `rows` x `cols` interior elements behind
+// `pad` border rows and columns.  Halo row i (i in [-pad, 0) or
+// [rows, rows + pad)) of strip t = rank + d is plane row t*rows + i, i.e. row
+// d*rows + i of this strip; the CTA that owns the row stores it straight into
+// strip t's shared memory (same offsets: every CTA of the cluster runs the
+// same plan).  Strip t below (d > 0) takes rows into its top halo, strip t
+// above (d < 0) into its bottom halo, each a contiguous run of rows; only
+// strips within ceil(pad / rows) can need this strip's rows (coarse levels may
+// have fewer rows than pad).  Halo rows outside the plane are never written
+// and stay zero.  A row goes whole, padding columns included (zero on both
+// sides), as 16-byte stores from its 16-byte aligned start (the row stride
+// covers the rounding).  The stores need no reply; the cluster barrier after
+// them (release / acquire) makes them visible.
+__device__ __forceinline__ void push_halo_rows(float* sm, const Buf& b, int nsub_lg, int rows, int cols, int pad,
+                                               int rank, int nstrips, int tid, int nt) {
+    const int reach = (pad + rows - 1) / rows;
+    const int nq = (cols + 2 * pad + 3) >> 2;  // 16-byte chunks of a padded row
+    const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm));
+    for (int d = -reach; d <= reach; ++d) {
+        const int t = rank + d;
+        if (d == 0 || t < 0 || t >= nstrips) continue;
+        // Halo rows i0 .. i0 + n - 1 of strip t, from rows i0 + d*rows .. of this one.
+        int i0, n;
+        if (d > 0) {
+            i0 = max(-pad, -d * rows);
+            n = min(0, (1 - d) * rows) - i0;
+        } else {
+            i0 = max(rows, -d * rows);
+            n = min(rows + pad, (1 - d) * rows) - i0;
         }
-#pragma unroll
-        for (int q = 0; q < U; ++q)
-            if (dst[q] >= 0) sm[dst[q]] = v[q];
+        if (n <= 0) continue;
+        unsigned tsm;  // strip t's copy of this shared memory in the cluster window
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(tsm) : "r"(local), "r"(t));
+        const int total = (n << nsub_lg) * nq;
+        for (int e = tid; e < total; e += nt) {
+            const int rest = e / nq, q = e - rest * nq;
+            const int j = rest >> nsub_lg, s = rest - (j << nsub_lg);
+            const int i = i0 + j;
+            const int at = b.base + s * b.sub + 4 * q;
+            const float4 v = *reinterpret_cast<const float4*>(sm + at + (d * rows + i + pad) * b.stride);
+            asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                             tsm + 4u * (unsigned)(at + (i + pad) * b.stride)),
+                         "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                         : "memory");
+        }
     }
 }
 
 // Halo rows of the padded input strip (X) and, for the subband convs, of
-// every level's padded subbands (S).
-__device__ __forceinline__ void copy_halos(float* sm, const Plan& P, int rank, int tid, int nt) {
+// every level's padded subbands (S), sent to the strips that hold them.
+__device__ __forceinline__ void push_halos(float* sm, const Plan& P, int rank, int tid, int nt) {
     const int p = P.p;
-    copy_halo_rows(sm, P.X, 0, P.H, P.W, P.div_w, p, rank, P.nstrips, tid, nt);
+    push_halo_rows(sm, P.X, 0, P.H, P.W, p, rank, P.nstrips, tid, nt);
 #pragma unroll
     for (int l = 0; l < kMaxL; ++l)
-        if (l < P.L)
-            copy_halo_rows(sm, P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), P.div_m[l], p, rank, P.nstrips, tid, nt);
+        if (l < P.L) push_halo_rows(sm, P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), p, rank, P.nstrips, tid, nt);
 }
 
 // ---------------------------------------------------------------------------
@@ -905,7 +923,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
     int folded_c = -1;
     for (int u = u0; u <= u1; ++u) {
         cp_async_wait_all();
-        plane_sync<GENERAL>(P);  // plane u staged; every tile (and halo copy) of plane u-1 done
+        plane_sync<GENERAL>(P);  // plane u staged; every tile of plane u-1 done (its halo rows are free)
         // Phase A.
         if (u < u1) {
             if (cur_c != folded_c) {
@@ -919,7 +937,11 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
             for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL>(sm, P, yp, t, myrows);
         }
         if (u == u1) break;
-        plane_sync<GENERAL>(P);  // X and S of plane u ready (every strip); Q and Y of plane u-1 consumed
+        if (strips) {
+            __syncthreads();  // this strip's X and S of plane u complete
+            push_halos(sm, P, rank, tid, nt);
+        }
+        plane_sync<GENERAL>(P);  // X, S and halo rows of plane u ready (every strip); Q and Y of plane u-1 consumed
         // Phase B.
         int nb = cur_b + 1, nc = cur_c;
         if (nb == P.B) {
@@ -928,10 +950,6 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
         }
         if (u + 1 < u1) stage(cx.src(nb, nc));
         cp_async_commit();
-        if (strips) {
-            copy_halos(sm, P, rank, tid, nt);
-            __syncthreads();  // halo rows in place
-        }
         for (int t = tid; t < P.tile_end; t += nt) {
             const TileJob j = P.merged ? fixed : decode_tile(P, t, TR, TC);
             if (!j.valid) continue;
@@ -1106,7 +1124,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
     float* X0 = sm + P.X.base + p * P.X.stride + p;
     for (int b = g; b < P.B; b += G) {
         cp_async_wait_all();
-        plane_sync<GENERAL>(P);  // staged pair complete; previous correlations (and halo copies) done
+        plane_sync<GENERAL>(P);  // staged pair complete; previous correlations done (halo rows free)
         analyse_plane<T, p, false, kToS>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         const float s = dys ? analyse_plane<T, 0, true, kToQ, false>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
                                                                      P.DY.stride, 0, nt, tid, csync)
@@ -1118,12 +1136,17 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
             sdy_c = (tv - sdy) - yv;
             sdy = tv;
         }
-        plane_sync<GENERAL>(P);  // both analyses complete (every strip)
-        if (b + G < P.B) stage(plane_origin<GENERAL>(P, b + G, c) + strip_off, !dys);
-        cp_async_commit();
         if (strips) {
-            copy_halos(sm, P, rank, tid, nt);
-            __syncthreads();  // halo rows in place
+            __syncthreads();  // this strip's analyses complete (staging consumed)
+            push_halos(sm, P, rank, tid, nt);
+            cluster_arrive();  // this strip's halo stores released
+            if (b + G < P.B) stage(plane_origin<GENERAL>(P, b + G, c) + strip_off, !dys);
+            cp_async_commit();
+            cluster_wait();  // every strip's X, S and halo rows ready
+        } else {
+            plane_sync<GENERAL>(P);  // both analyses complete
+            if (b + G < P.B) stage(plane_origin<GENERAL>(P, b + G, c) + strip_off, !dys);
+            cp_async_commit();
         }
         for (int k = 0; k < cnt; ++k) {
             const int local = first + k;
@@ -1148,7 +1171,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
         }
     }
     cp_async_wait_all();
-    plane_sync<GENERAL>(P);  // no CTA of the cluster reads this CTA's strip any more
+    plane_sync<GENERAL>(P);  // the cluster leaves together
 
     // Fixed-order reduction of every class over its threads.
     float* red = sm + P.red;

@@ -316,35 +316,67 @@ void check_divs(const Plan& P) {
     }
 }
 
-// Replays copy_halos for strip `rank`: every halo row of X and of every
-// level's subbands is read from the CTA that owns the row (its own tag) and
-// written into this CTA's padding rows.
-void replay_halos(std::vector<Shadow>& shs, const Plan& P, int rank) {
-    Shadow& me = shs[rank];
-    auto one = [&](const Buf& b, int nsub_lg, int rows, int cols, FastDiv dcols, int tagbase, bool per_sub_tag) {
+// Replays push_halos of every strip (all strips in the phase after their own
+// CTA barrier that follows the analysis): strip r sends each of its rows that
+// strip t = r + d holds as a halo row, whole (padding columns and the 16-byte
+// rounding included), into t's padding row.  t may still be in its analysis
+// phase when the store lands (no cluster barrier in between), so each float
+// written must also be untouched in t's previous phase.
+void replay_push(std::vector<Shadow>& shs, const Plan& P) {
+    const int NS = (int)shs.size();
+    auto one = [&](int rank, const Buf& b, int nsub_lg, int rows, int cols, int tagbase, bool per_sub_tag) {
+        Shadow& me = shs[rank];
         const int pad = P.p;
-        const int n = (2 * pad << nsub_lg) * cols;
+        const int reach = (pad + rows - 1) / rows;
+        const int nq = (cols + 2 * pad + 3) >> 2;
         const long long span = (long long)(1 << nsub_lg) * (b.sub ? b.sub : 0);
         const long long lo = b.base, hi = nsub_lg ? b.base + span : b.base + (long long)(rows + 2 * pad) * b.stride;
-        for (int t = 0; t < n; ++t) {
-            const int rest = (int)fastdiv_host(t, dcols), c = t - rest * cols;
-            if (rest != t / cols) me.fail("halo column division", t);
-            const int hr = rest >> nsub_lg, s = rest - (hr << nsub_lg);
-            const int i = hr < pad ? hr - pad : rows + hr - pad;
-            const int g = rank * rows + i;
-            if (g < 0 || g >= P.nstrips * rows) continue;
-            const int owner = g / rows, lr = g - owner * rows;
-            if (owner == rank) me.fail("halo row owned by the copying strip", g);
-            const long long col = b.base + (long long)s * b.sub + c + pad;
-            const int tag = per_sub_tag ? tagbase + s : tagbase;
-            const long long slo = nsub_lg ? b.base + (long long)s * b.sub : lo;
-            const long long shi = nsub_lg ? b.base + (long long)(s + 1) * b.sub : hi;
-            shs[owner].read(col + (long long)(lr + pad) * b.stride, slo, shi, tag, "halo source");
-            me.write(col + (long long)(i + pad) * b.stride, slo, shi, tag, "halo row");
+        if (b.base % 4 || b.stride % 4 || b.sub % 4) me.fail("halo rows not 16-byte aligned", b.base);
+        if (4 * nq > b.stride) me.fail("padded row rounded to 16 bytes exceeds the stride", nq);
+        for (int d = -reach; d <= reach; ++d) {
+            const int t = rank + d;
+            if (d == 0 || t < 0 || t >= NS) continue;
+            int i0, n;
+            if (d > 0) {
+                i0 = std::max(-pad, -d * rows);
+                n = std::min(0, (1 - d) * rows) - i0;
+            } else {
+                i0 = std::max(rows, -d * rows);
+                n = std::min(rows + pad, (1 - d) * rows) - i0;
+            }
+            if (n <= 0) continue;
+            const int total = (n << nsub_lg) * nq;
+            for (int e = 0; e < total; ++e) {
+                const int rest = e / nq, q = e - rest * nq;
+                const int j = rest >> nsub_lg, s = rest - (j << nsub_lg);
+                const int i = i0 + j;
+                const int lr = d * rows + i;
+                if (lr < 0 || lr >= rows) me.fail("halo source row outside the strip", lr);
+                if (!(i < 0 || i >= rows)) me.fail("halo destination row inside the strip", i);
+                const long long slo = nsub_lg ? b.base + (long long)s * b.sub : lo;
+                const long long shi = nsub_lg ? b.base + (long long)(s + 1) * b.sub : hi;
+                const int tag = per_sub_tag ? tagbase + s : tagbase;
+                Shadow& tg = shs[t];
+                for (int f = 0; f < 4; ++f) {
+                    const int c = 4 * q + f - pad;  // interior column (negative or >= cols: padding, zero)
+                    const long long at = b.base + (long long)s * b.sub + 4LL * q + f;
+                    const long long src = at + (long long)(lr + pad) * b.stride;
+                    const long long dst = at + (long long)(i + pad) * b.stride;
+                    const int expect = (c >= 0 && c < cols) ? tag : ZERO;
+                    me.read(src, slo, shi, expect, "halo source row");
+                    tg.in_bounds(dst, slo, shi, "halo row");
+                    if (tg.rd[dst] >= tg.epoch - 1 || tg.wr[dst] >= tg.epoch - 1)
+                        tg.fail("halo row touched by its strip while the owner's store may land", dst);
+                    tg.write(dst, slo, shi, expect, "halo row");
+                }
+            }
         }
     };
-    one(P.X, 0, P.H, P.W, P.div_w, XT, false);
-    for (int l = 0; l < P.L; ++l) one(P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), P.div_m[l], s_tag(l, 0), true);
+    for (int r = 0; r < NS; ++r) {
+        shs[r].phase = "halo push";
+        one(r, P.X, 0, P.H, P.W, XT, false);
+        for (int l = 0; l < P.L; ++l) one(r, P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), s_tag(l, 0), true);
+    }
 }
 
 void barrier_all(std::vector<Shadow>& shs) {
@@ -436,7 +468,7 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
 
     // The persistent walk over two planes and the final synthesis, with the
     // kernel's barriers (cluster-wide with strips) as phase boundaries:
-    //   stage(0) | A(0) | B(0): stage(1), halos(0), | tiles(0) | A(1) | B(1) ... | A(end)
+    //   stage(0) | A(0) | [strips: halo push(0)] | B(0): stage(1), tiles(0) | A(1) | ... | A(end)
     for (int r = 0; r < NS; ++r) {
         shs[r].phase = "initial staging";
         replay_stage(shs[r], P, P.stg, XT + 10, r);
@@ -473,21 +505,15 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
                 synthesis(shs[r], r);
             }
         if (unit == 2) break;
+        // Strips: CTA barrier, halo push, then the cluster barrier.
+        if (NS > 1) {
+            barrier_all(shs);
+            replay_push(shs, P);
+        }
         barrier_all(shs);
         for (int r = 0; r < NS; ++r) {
             shs[r].phase = "B: staging";
             if (unit + 1 < 2) replay_stage(shs[r], P, P.stg, XT + 10, r);
-        }
-        if (NS > 1) {
-            for (int r = 0; r < NS; ++r) {
-                shs[r].phase = "B: halo copy";
-                replay_halos(shs, P, r);
-            }
-            // Local barrier after the copy: a new phase for each CTA (the other
-            // CTAs' phase is unchanged, so remote reads still conflict with
-            // their later writes only through this CTA's epoch -- the replay
-            // keeps the cluster in lockstep, which is the stricter check).
-            barrier_all(shs);
         }
         for (int r = 0; r < NS; ++r) {
             Shadow& sh = shs[r];
@@ -569,7 +595,7 @@ void check_bwdw(const wtconv_desc_t& d) {
     if (P.stg % 4 || P.stg_floats % 4) shs[0].fail("staging alignment", P.stg);
     // Two planes in a row (the second must see the same zero padding), with
     // the kernel's barriers (cluster-wide with strips) as phase boundaries:
-    //   stage(0) | analysis(0) | stage(1), halos(0) | correlation(0) | analysis(1) | ... | reduction
+    //   stage(0) | analysis(0) | [strips: halo push(0), stage(1)] | [whole planes: stage(1)], correlation(0) | analysis(1) | ... | reduction
     for (int r = 0; r < NS; ++r) {
         shs[r].phase = "initial staging";
         replay_stage(shs[r], P, P.stg, XT + 10, r);
@@ -590,7 +616,12 @@ void check_bwdw(const wtconv_desc_t& d) {
             if (r + 1 < NS) sh.epoch = e0;
             else for (int q = 0; q + 1 < NS; ++q) shs[q].epoch = sh.epoch;
         }
-        barrier_all(shs);
+        if (NS > 1) {
+            barrier_all(shs);
+            replay_push(shs, P);
+        } else {
+            barrier_all(shs);
+        }
         for (int r = 0; r < NS; ++r) {
             shs[r].phase = "staging";
             if (plane == 0) {
@@ -598,13 +629,7 @@ void check_bwdw(const wtconv_desc_t& d) {
                 if (!dys) replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
             }
         }
-        if (NS > 1) {
-            for (int r = 0; r < NS; ++r) {
-                shs[r].phase = "halo copy";
-                replay_halos(shs, P, r);
-            }
-            barrier_all(shs);
-        }
+        if (NS > 1) barrier_all(shs);
         for (int r = 0; r < NS; ++r) {
             Shadow& sh = shs[r];
             sh.phase = "correlation";
