@@ -662,15 +662,30 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // sides), as 16-byte stores from its 16-byte aligned start (the row stride
 // covers the rounding).  The stores need no reply; the cluster barrier after
 // them (release / acquire) makes them visible.
-__device__ __forceinline__ void push_halo_rows(float* sm, const Buf& b, int nsub_lg, int rows, int cols, int pad,
-                                               int rank, int nstrips, int tid, int nt) {
+__device__ __forceinline__ void st_cluster4(unsigned addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+
+// One buffer's halo rows (see above), as row groups: for every direction d
+// and subband s, the run of halo rows i0 .. i0 + n - 1 of strip t = rank + d.
+// Warp w takes the groups gbase + w, gbase + w + nw, ... (gbase: groups of the
+// buffers before this one); its lanes copy a row's 16-byte chunks, loading up
+// to two per lane before storing them.
+__device__ __forceinline__ void push_halo_rows(float* sm, unsigned local, const Buf& b, int nsub_lg, int rows, int cols,
+                                               int pad, int rank, int nstrips, int warp, int lane, int nw, int& gbase) {
     const int reach = (pad + rows - 1) / rows;
     const int nq = (cols + 2 * pad + 3) >> 2;  // 16-byte chunks of a padded row
-    const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm));
-    for (int d = -reach; d <= reach; ++d) {
+    const int ngroups = (2 * reach) << nsub_lg;
+    int g = warp - gbase % nw;
+    if (g < 0) g += nw;
+    gbase += ngroups;
+    for (; g < ngroups; g += nw) {
+        const int di = g >> nsub_lg, s = g - (di << nsub_lg);
+        const int d = di < reach ? di - reach : di - reach + 1;
         const int t = rank + d;
-        if (d == 0 || t < 0 || t >= nstrips) continue;
-        // Halo rows i0 .. i0 + n - 1 of strip t, from rows i0 + d*rows .. of this one.
+        if (t < 0 || t >= nstrips) continue;
         int i0, n;
         if (d > 0) {
             i0 = max(-pad, -d * rows);
@@ -682,17 +697,24 @@ __device__ __forceinline__ void push_halo_rows(float* sm, const Buf& b, int nsub
         if (n <= 0) continue;
         unsigned tsm;  // strip t's copy of this shared memory in the cluster window
         asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(tsm) : "r"(local), "r"(t));
-        const int total = (n << nsub_lg) * nq;
-        for (int e = tid; e < total; e += nt) {
-            const int rest = e / nq, q = e - rest * nq;
-            const int j = rest >> nsub_lg, s = rest - (j << nsub_lg);
+        for (int j = 0; j < n; ++j) {
             const int i = i0 + j;
-            const int at = b.base + s * b.sub + 4 * q;
-            const float4 v = *reinterpret_cast<const float4*>(sm + at + (d * rows + i + pad) * b.stride);
-            asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(
-                             tsm + 4u * (unsigned)(at + (i + pad) * b.stride)),
-                         "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
-                         : "memory");
+            const int row = b.base + s * b.sub;
+            const float* src = sm + row + (d * rows + i + pad) * b.stride;
+            const unsigned dst = tsm + 4u * (unsigned)(row + (i + pad) * b.stride);
+            for (int q0 = 0; q0 < nq; q0 += 64) {
+                float4 v[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int q = q0 + lane + 32 * k;
+                    if (q < nq) v[k] = *reinterpret_cast<const float4*>(src + 4 * q);
+                }
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int q = q0 + lane + 32 * k;
+                    if (q < nq) st_cluster4(dst + 16u * (unsigned)q, v[k]);
+                }
+            }
         }
     }
 }
@@ -700,11 +722,15 @@ __device__ __forceinline__ void push_halo_rows(float* sm, const Buf& b, int nsub
 // Halo rows of the padded input strip (X) and, for the subband convs, of
 // every level's padded subbands (S), sent to the strips that hold them.
 __device__ __forceinline__ void push_halos(float* sm, const Plan& P, int rank, int tid, int nt) {
-    const int p = P.p;
-    push_halo_rows(sm, P.X, 0, P.H, P.W, p, rank, P.nstrips, tid, nt);
+    const int p = P.p, warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+    const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm));
+    int gbase = 0;
+    push_halo_rows(sm, local, P.X, 0, P.H, P.W, p, rank, P.nstrips, warp, lane, nw, gbase);
 #pragma unroll
     for (int l = 0; l < kMaxL; ++l)
-        if (l < P.L) push_halo_rows(sm, P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), p, rank, P.nstrips, tid, nt);
+        if (l < P.L)
+            push_halo_rows(sm, local, P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), p, rank, P.nstrips, warp, lane, nw,
+                           gbase);
 }
 
 // ---------------------------------------------------------------------------
