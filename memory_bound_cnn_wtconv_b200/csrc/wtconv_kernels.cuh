@@ -670,17 +670,17 @@ __device__ __forceinline__ void st_cluster4(unsigned addr, float4 v) {
 
 // One buffer's halo rows (see above), as row groups: for every direction d
 // and subband s, the run of halo rows i0 .. i0 + n - 1 of strip t = rank + d.
-// Warp w takes the groups gbase + w, gbase + w + nw, ... (gbase: groups of the
-// buffers before this one); its lanes copy a row's 16-byte chunks, loading up
-// to two per lane before storing them.
-__device__ __forceinline__ void push_halo_rows(float* sm, unsigned local, const Buf& b, int nsub_lg, int rows, int cols,
-                                               int pad, int rank, int nstrips, int warp, int lane, int nw, int& gbase) {
-    const int reach = (pad + rows - 1) / rows;
-    const int nq = (cols + 2 * pad + 3) >> 2;  // 16-byte chunks of a padded row
+// The groups of all buffers are numbered in order; warp w takes every nw-th
+// from w (the planner gives the buffer's chunks per row nq, its reach and g0,
+// the offset of this buffer's first group that warp 0 takes, so no index is
+// divided here).  A warp's lanes copy a row's 16-byte chunks, loading up to
+// two per lane before storing them.
+__device__ __forceinline__ void push_halo_rows(float* sm, unsigned local, const Buf& b, int nsub_lg, int rows, int nq,
+                                               int reach, int g0, int pad, int rank, int nstrips, int warp, int lane,
+                                               int nw) {
     const int ngroups = (2 * reach) << nsub_lg;
-    int g = warp - gbase % nw;
+    int g = warp - g0;
     if (g < 0) g += nw;
-    gbase += ngroups;
     for (; g < ngroups; g += nw) {
         const int di = g >> nsub_lg, s = g - (di << nsub_lg);
         const int d = di < reach ? di - reach : di - reach + 1;
@@ -724,13 +724,12 @@ __device__ __forceinline__ void push_halo_rows(float* sm, unsigned local, const 
 __device__ __forceinline__ void push_halos(float* sm, const Plan& P, int rank, int tid, int nt) {
     const int p = P.p, warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
     const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm));
-    int gbase = 0;
-    push_halo_rows(sm, local, P.X, 0, P.H, P.W, p, rank, P.nstrips, warp, lane, nw, gbase);
+    push_halo_rows(sm, local, P.X, 0, P.H, P.hal_nq[0], P.hal_reach[0], P.hal_g0[0], p, rank, P.nstrips, warp, lane, nw);
 #pragma unroll
     for (int l = 0; l < kMaxL; ++l)
         if (l < P.L)
-            push_halo_rows(sm, local, P.S[l], 2, P.H >> (l + 1), P.W >> (l + 1), p, rank, P.nstrips, warp, lane, nw,
-                           gbase);
+            push_halo_rows(sm, local, P.S[l], 2, P.H >> (l + 1), P.hal_nq[l + 1], P.hal_reach[l + 1], P.hal_g0[l + 1], p,
+                           rank, P.nstrips, warp, lane, nw);
 }
 
 // ---------------------------------------------------------------------------

@@ -133,6 +133,10 @@ struct Plan {
     // runs as in the weight gradient); in the analysis threads [0, an_split)
     // take x and the rest take dy.
     int corr0, an_split;
+    // Strips: halo push constants of buffer b (0 = X, 1 + l = S[l]): 16-byte
+    // chunks of a padded row, strips reached, and the first of its row groups
+    // that warp 0 takes (the groups of buffers < b, modulo the warps).
+    int hal_nq[kMaxL + 1], hal_reach[kMaxL + 1], hal_g0[kMaxL + 1];
     int pyr;             // analysis by the one-pass pyramid (H % 4 == 0 and L >= 1)
     int pyr_levels;      // levels the pyramid computes (min(L, 4)); the rest run level by level
     int pyr_lg;          // pyramid lane groups cover (4 * 2^pyr_lg)^2 pixel regions

@@ -322,6 +322,19 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         const long long busy = ceil_div((int)std::min<long long>(an_items, 1 << 30), 32) * 32LL;
         P->fin_off = busy >= P->nthreads ? 0 : (int)busy;
     }
+    // Halo push constants (strips; see wtconv_plan.h): per buffer the row
+    // chunks, the reach and the warp-0 offset of its row groups.
+    if (nstrips > 1) {
+        const int nw = P->nthreads / 32;
+        int gbase = 0;
+        for (int bi = 0; bi <= L; ++bi) {
+            const int rows = bi == 0 ? H : H >> bi, cols = bi == 0 ? W : W >> bi, nsub_lg = bi == 0 ? 0 : 2;
+            P->hal_nq[bi] = (cols + 2 * p + 3) >> 2;
+            P->hal_reach[bi] = (p + rows - 1) / rows;
+            P->hal_g0[bi] = gbase % nw;
+            gbase += (2 * P->hal_reach[bi]) << nsub_lg;
+        }
+    }
     // Weight gradients: the final step's scratch (summed partials, weights, a flag).
     if (kind == kBackwardWeight || kind == kBackward) off = std::max(off, (long long)P->nv + ncls * KK + 4);
     off = round4((int)std::min<long long>(off, 1LL << 30));

@@ -372,6 +372,18 @@ void replay_push(std::vector<Shadow>& shs, const Plan& P) {
             }
         }
     };
+    // The planner's push constants against the kernel's formulas.
+    {
+        const int nw = P.nthreads / 32;
+        int gbase = 0;
+        for (int bi = 0; bi <= P.L; ++bi) {
+            const int rows = bi == 0 ? P.H : P.H >> bi, cols = bi == 0 ? P.W : P.W >> bi;
+            const int reach = (P.p + rows - 1) / rows;
+            if (P.hal_nq[bi] != ((cols + 2 * P.p + 3) >> 2) || P.hal_reach[bi] != reach || P.hal_g0[bi] != gbase % nw)
+                shs[0].fail("halo push constants", bi);
+            gbase += (2 * reach) << (bi == 0 ? 0 : 2);
+        }
+    }
     for (int r = 0; r < NS; ++r) {
         shs[r].phase = "halo push";
         one(r, P.X, 0, P.H, P.W, XT, false);
