@@ -794,16 +794,19 @@ __device__ __forceinline__ TileJob decode_tile(const Plan& P, int t, int TR, int
 // The levels >= 1 are gathered Horner-style along the item's path: level l's
 // signed sum for the level-(l-1) position on the path is added to that
 // position's LL term, so the level-0 butterfly carries every coarser level.
-template <typename T, bool GUARD>
+// LL: the level count when the caller has dispatched on it (the Horner walk
+// then has no per-level tests), or 0 for any L (P.L).
+template <typename T, bool GUARD, int LL = 0>
 __device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp, int t, int rows) {
     const int i = fdiv(t, P.div_q4), q = t - i * (P.W >> 2);
     const int j0 = 2 * q;
+    const int L = LL > 0 ? LL : P.L;
     float c0 = 0.f, c1 = 0.f;  // coarse terms for LL at (i, j0) and (i, j0 + 1)
-    if (P.L >= 2) {
+    if (L >= 2) {
         float v = 0.f;
 #pragma unroll
-        for (int l = kMaxL - 1; l >= 1; --l) {
-            if (l >= P.L) continue;
+        for (int l = (LL > 0 ? LL : kMaxL) - 1; l >= 1; --l) {
+            if (LL == 0 && l >= P.L) continue;
             const Buf& Q = P.Q[l];
             const float* r = sm + Q.base + (i >> l) * Q.stride + (j0 >> l);
             const float q0 = r[0] + v, q1 = r[Q.sub], q2 = r[2 * Q.sub], q3 = r[3 * Q.sub];
@@ -959,7 +962,15 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
         }
         if (u > u0 && P.L >= 1) {
             T* yp = y + cx.rows_of(prev_b, prev_c);
-            for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL>(sm, P, yp, t, myrows);
+            // One synthesis loop per level count (uniform dispatch), so that
+            // the items' level walk is unrolled with no per-level tests.
+            switch (P.L) {
+                case 1: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 1>(sm, P, yp, t, myrows); break;
+                case 2: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 2>(sm, P, yp, t, myrows); break;
+                case 3: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 3>(sm, P, yp, t, myrows); break;
+                case 4: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 4>(sm, P, yp, t, myrows); break;
+                default: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL>(sm, P, yp, t, myrows); break;
+            }
         }
         if (u == u1) break;
         if (strips) {
