@@ -1151,6 +1151,17 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
         cnt = min(P.tpt, P.cls_tiles[cl] - first);
     }
     const int lvl = cl <= 0 ? kMaxL : ((cl - 1) >> 2);
+    // The class's window buffer (padded X or subband S) and dy buffer (DY or
+    // its subband Q), the same for every plane: one tile call site, no
+    // per-plane buffer selection.
+    int wb = 0, ws = 0, db = 0, dsd = 0;
+    if (cl == 0) {
+        wb = P.X.base; ws = P.X.stride; db = P.DY.base; dsd = P.DY.stride;
+    } else if (cl > 0) {
+        const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
+        wb = P.S[l].base + s2 * P.S[l].sub; ws = P.S[l].stride;
+        db = P.Q[l].base + s2 * P.Q[l].sub; dsd = P.Q[l].stride;
+    }
     using Acc = typename CorrAcc<K>::type;
     Acc acc[KK];
 #pragma unroll
@@ -1187,16 +1198,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
         for (int k = 0; k < cnt; ++k) {
             const int local = first + k;
             const int tr = fdiv(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
-            if (cl == 0) {
-                corr_tile<K, TR, TC, DLD>(sm + P.X.base + tr * TR * P.X.stride + tc * TC, P.X.stride,
-                                     sm + P.DY.base + tr * TR * P.DY.stride + tc * TC, P.DY.stride, acc);
-            } else {
-                const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
-                const Buf& S = P.S[l];
-                const Buf& Q = P.Q[l];
-                corr_tile<K, TR, TC, DLD>(sm + S.base + s2 * S.sub + tr * TR * S.stride + tc * TC, S.stride,
-                                     sm + Q.base + s2 * Q.sub + tr * TR * Q.stride + tc * TC, Q.stride, acc);
-            }
+            corr_tile<K, TR, TC, DLD>(sm + wb + tr * TR * ws + tc * TC, ws, sm + db + tr * TR * dsd + tc * TC, dsd, acc);
         }
         if (dys) {
             __syncthreads();  // every dy tile read (dy is this CTA's own; no other CTA reads it)
