@@ -986,21 +986,32 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
         }
         if (u + 1 < u1) stage(cx.src(nb, nc));
         cp_async_commit();
-        for (int t = tid; t < P.tile_end; t += nt) {
-            const TileJob j = P.merged ? fixed : decode_tile(P, t, TR, TC);
-            if (!j.valid) continue;
-            float w[KK];
-            load_weights<K>(sm + j.wts, w);
-            const float b0 = j.base ? sm[P.bias] : 0.f;
-            if (P.L >= 1 || !j.base) {
+        // One tile loop per output kind (a uniform branch), each with a
+        // single conv-tile call site.
+        if (P.L >= 1) {
+            // Subband tiles write Q, base tiles Y (both on chip).
+            for (int t = tid; t < P.tile_end; t += nt) {
+                const TileJob j = P.merged ? fixed : decode_tile(P, t, TR, TC);
+                if (!j.valid) continue;
+                float w[KK];
+                load_weights<K>(sm + j.wts, w);
+                const float b0 = j.base ? sm[P.bias] : 0.f;
                 float* out = sm + j.out;
                 const int os = j.ostride;
                 conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
                     *reinterpret_cast<float4*>(out + o * os) = make_float4(a[0].x, a[0].y, a[1].x, a[1].y);
                 });
-            } else {
-                // L = 0: the base branch is the whole output.
-                const size_t es = act_es<GENERAL>(P);
+            }
+        } else {
+            // L = 0: every tile is a base tile, and the base branch is the
+            // whole output.
+            const size_t es = act_es<GENERAL>(P);
+            for (int t = tid; t < P.tile_end; t += nt) {
+                const TileJob j = P.merged ? fixed : decode_tile(P, t, TR, TC);
+                if (!j.valid) continue;
+                float w[KK];
+                load_weights<K>(sm + j.wts, w);
+                const float b0 = sm[P.bias];
                 T* yo = y + cx.rows_of(cur_b, cur_c) + (size_t)j.out * es;
                 const int h0 = j.row0;
                 conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
@@ -1304,6 +1315,18 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
             cnt = min(P.tpt, P.cls_tiles[cl] - first);
         }
         const int lvl = cl <= 0 ? kMaxL : ((cl - 1) >> 2);
+        // The correlation class's x-window buffer (XS or SS) and dy-tile
+        // buffer (the interior of X or S), selected once: one tile call site.
+        int wb = 0, ws = 0, db = 0, dsd = 0;
+        if constexpr (CORR) {
+            if (cl == 0) {
+                wb = P.XS.base; ws = P.XS.stride; db = P.X.base + p * P.X.stride + p; dsd = P.X.stride;
+            } else if (cl > 0) {
+                const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
+                wb = P.SS[l].base + s2 * P.SS[l].sub; ws = P.SS[l].stride;
+                db = P.S[l].base + s2 * P.S[l].sub + p * P.S[l].stride + p; dsd = P.S[l].stride;
+            }
+        }
         using Acc = typename CorrAcc<K>::type;
         Acc acc[CORR ? KK : 1];
 #pragma unroll
@@ -1367,18 +1390,8 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
                 for (int k = 0; k < cnt; ++k) {
                     const int local = first + k;
                     const int tr = fdiv(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
-                    if (cl == 0) {
-                        corr_tile<K, TR, TC, DLD>(sm + P.XS.base + tr * TR * P.XS.stride + tc * TC, P.XS.stride,
-                                                  X0 + tr * TR * P.X.stride + tc * TC, P.X.stride, acc);
-                    } else {
-                        const int l = (cl - 1) >> 2, s2 = (cl - 1) & 3;
-                        const Buf& SS = P.SS[l];
-                        const Buf& S = P.S[l];
-                        corr_tile<K, TR, TC, DLD>(sm + SS.base + s2 * SS.sub + tr * TR * SS.stride + tc * TC,
-                                                  SS.stride,
-                                                  sm + S.base + s2 * S.sub + (tr * TR + p) * S.stride + tc * TC + p,
-                                                  S.stride, acc);
-                    }
+                    corr_tile<K, TR, TC, DLD>(sm + wb + tr * TR * ws + tc * TC, ws, sm + db + tr * TR * dsd + tc * TC,
+                                              dsd, acc);
                 }
             }
             prev_b = b;
