@@ -106,8 +106,8 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
                   "wtconv_launch.h", "wtconv_api.cu", "wtconv_k1.cu", "wtconv_k3.cu", "wtconv_k5.cu", "wtconv_k7.cu")
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
-    ("stage1", "bwd_w"): (79115520.0, "wtconv_bwdw_partial_kernel",
-                          "2bd88317e2d7dd9d0b7c3097343e5860fc9be86c1c8084d27d0d7540d444549e",
+    ("stage1", "bwd_w"): (79151104.0, "wtconv_bwdw_partial_kernel",
+                          "056a46ed48cb0049315ffb828356952f1db8d281503b4e79579256377c29bf30",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 
