@@ -178,6 +178,10 @@ SMALL = [
     Case("pad_17x8_k3_L1", 2, 3, 17, 8, 3, 1, "f32", 34, "normal", "normal"),
     Case("pad_bf16_13x16", 2, 3, 13, 16, 5, 2, "bf16", 35, "uniform", "normal"),
     Case("pad_strips_250x248", 1, 1, 250, 248, 5, 4, "f32", 36, "normal", "normal"),
+    # strips of L = 0 planes and of planes with levels past the one-pass pyramid (L = 5, 6)
+    Case("strips_256_L0", 1, 2, 256, 256, 5, 0, "f32", 42, "normal", "normal"),
+    Case("strips_256_L5", 1, 1, 256, 256, 5, 5, "f32", 43, "normal", "normal"),
+    Case("strips_512x64_L6_bf16", 1, 1, 512, 64, 5, 6, "bf16", 44, "normal", "normal"),
     # deepest levels, bf16 with k = 7, and one channel over many batch elements
     Case("L5_32_k3", 1, 2, 32, 32, 3, 5, "f32", 37, "normal", "normal"),
     Case("bf16_k7_L3", 2, 2, 24, 24, 7, 3, "bf16", 38, "uniform", "normal"),

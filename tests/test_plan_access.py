@@ -28,6 +28,9 @@ EDGE = [
     # clusters of 4 and 16 strips at the sweep's channel counts and batch rule
     (14, 128, 192, 192, 5, 1, 0), (7, 256, 192, 192, 3, 4, 0), (28, 64, 192, 192, 7, 1, 1),
     (10, 64, 320, 320, 3, 1, 0), (1, 512, 320, 320, 5, 1, 1),
+    # strips without the pyramid (L = 0) and with levels past it (L = 5, 6): halo rows sent after
+    # the analysis instead of from inside it
+    (1, 2, 256, 256, 5, 0, 0), (1, 2, 256, 256, 3, 0, 1), (1, 1, 256, 256, 5, 5, 0), (1, 1, 512, 64, 5, 6, 0),
 ]
 
 
