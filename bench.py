@@ -107,7 +107,7 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
     ("stage1", "bwd_w"): (79151104.0, "wtconv_bwdw_partial_kernel",
-                          "056a46ed48cb0049315ffb828356952f1db8d281503b4e79579256377c29bf30",
+                          "d2dfb44563fee3de439b3a2f8fd5532fdcb5b794b0a09e70e280fc51b1e067ac",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 

@@ -392,10 +392,12 @@ inline bool prefer_one_pass(const Plan& P, const Plan& Pin, const Plan& Pw) {
 
 // Chooses the fewest strips that fit (whole planes, else clusters of 2, 4,
 // 8, 16 strips), and for that count the tile height (7 or 8 rows) with the
-// lowest plan_cost.  Every cluster strip adds barriers and halo copies per
-// plane that the tile count does not show: at 128 x 128 (L = 2..4) two
+// lowest plan_cost.  Every cluster strip adds barriers and halo exchanges
+// per plane that the tile count does not show: at 128 x 128 (L = 2..4) two
 // strips measured 1.7-1.9x faster than eight, and at every shape measured
-// fewer strips were faster.
+// fewer strips were faster (also where twice the strips would fit two CTAs
+// per SM: 4 strips at 128 x 128 and 16 at 256 x 256, L = 1, measured within
+// 3% of 2 and 8).
 inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, int num_sms, Plan* P) {
     bool have = false;
     double best = 0.0;
