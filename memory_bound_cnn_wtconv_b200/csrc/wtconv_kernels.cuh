@@ -632,7 +632,7 @@ __device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const f
 template <bool GENERAL>
 __device__ __forceinline__ void plane_sync(const Plan& P) {
     if constexpr (GENERAL) {
-        if (P.nstrips > 1) {
+        if (cluster_ctas(P) > 1) {
             cg::this_cluster().sync();
             return;
         }
@@ -666,6 +666,29 @@ __device__ __forceinline__ void st_cluster4(unsigned addr, float4 v) {
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
                  "f"(v.w)
                  : "memory");
+}
+
+__device__ __forceinline__ void st_cluster2(unsigned addr, unsigned a, unsigned b) {
+    asm volatile("st.shared::cluster.v2.b32 [%0], {%1, %2};\n" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+
+// NHWC channel octets: 4 outputs of pixels px .. px + 3 (one row; px a
+// multiple of 4) of this CTA's channel into the output octet buffer of the
+// CTA that owns them.  oaddr: this CTA's output octet buffer (shared window
+// address); ocol: byte offset of this CTA's channel row in it.
+template <typename T>
+__device__ __forceinline__ void st_octet_out(const Plan& P, unsigned oaddr, unsigned ocol, int px, float4 v) {
+    const int owner = fdiv(px, P.div_opix), j = px - owner * P.opix;
+    unsigned dst;
+    asm("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(dst) : "r"(oaddr), "r"(owner));
+    dst += ocol + (unsigned)j * (unsigned)sizeof(T);
+    if constexpr (sizeof(T) == 4) {
+        st_cluster4(dst, v);
+    } else {
+        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+        __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+        st_cluster2(dst, *reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+    }
 }
 
 // One buffer's halo rows (see above), as row groups: for every direction d
@@ -797,7 +820,8 @@ __device__ __forceinline__ TileJob decode_tile(const Plan& P, int t, int TR, int
 // LL: the level count when the caller has dispatched on it (the Horner walk
 // then has no per-level tests), or 0 for any L (P.L).
 template <typename T, bool GUARD, int LL = 0>
-__device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp, int t, int rows) {
+__device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp, int t, int rows, unsigned oaddr = 0u,
+                                           unsigned ocol = 0u) {
     const int i = fdiv(t, P.div_q4), q = t - i * (P.W >> 2);
     const int j0 = 2 * q;
     const int L = LL > 0 ? LL : P.L;
@@ -846,11 +870,126 @@ __device__ __forceinline__ void synth_item(const float* sm, const Plan& P, T* yp
         T* yo = yp + (size_t)(2 * i) * P.Wr + 4 * q;
         gst4<T>(yo, top);
         gst4<T>(yo + P.Wr, bot);
+    } else if (oaddr != 0u) {
+        // Channel octets (whole planes): to the owners' output octet buffers.
+        const int px = (2 * i) * P.W + 4 * q;
+        st_octet_out<T>(P, oaddr, ocol, px, top);
+        st_octet_out<T>(P, oaddr, ocol, px + P.W, bot);
     } else if (4 * q < P.Wr) {
         const size_t es = act_es<true>(P);
         T* yo = yp + ((size_t)(2 * i) * P.Wr + 4 * q) * es;
         if (2 * i < rows) gst4s<T>(yo, top, es);
         if (2 * i + 1 < rows) gst4s<T>(yo + (size_t)P.Wr * es, bot, es);
+    }
+}
+
+// NHWC channel octets.  load_octet: this CTA's run of opix pixels (from
+// pixel crank * opix) of the 8 channels starting at `src` (channel 8o of
+// pixel 0 of the plane pair's batch element), 8 * esize contiguous bytes a
+// pixel, into the octet buffer by 16-byte cp.async (pixel j at byte
+// 8 * esize * j).
+__device__ __forceinline__ void load_octet(float* tb, const void* src, const Plan& P, int crank, int tid, int nt) {
+    const int cpp = P.esize / 2;  // 16-byte chunks a pixel: 2 (fp32) or 1 (bf16)
+    const size_t pstride = (size_t)P.C * P.esize;
+    const char* g = static_cast<const char*>(src) + (size_t)crank * P.opix * pstride;
+    char* t = reinterpret_cast<char*>(tb);
+    const int n = P.opix * cpp;
+    for (int ch = tid; ch < n; ch += nt) {
+        const int j = cpp == 2 ? ch >> 1 : ch, h = ch - j * cpp;
+        cp_async16(t + 16 * ch, g + (size_t)j * pstride + 16 * h);
+    }
+}
+
+// scatter_octet: channel q of the octet buffer's pixels into CTA q's
+// staging (pixel crank * opix + j of the plane, stored format), four pixels
+// a step as one 16-byte (fp32) or 8-byte (bf16) distributed shared store per
+// channel.  The cluster barrier after it makes the stores visible.
+__device__ __forceinline__ void scatter_octet(float* sm, const Plan& P, int crank, int tid, int nt) {
+    const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm + P.stg));
+    unsigned dst[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(dst[q]) : "r"(local), "r"(q));
+    const float* tb = sm + P.tbuf;
+    const int ng = P.opix >> 2;
+    for (int gq = tid; gq < ng; gq += nt) {
+        const int j = 4 * gq;
+        const unsigned off = (unsigned)(crank * P.opix + j) * (unsigned)P.esize;
+        if (P.esize == 4) {
+            const float4* t = reinterpret_cast<const float4*>(tb) + 2 * j;
+            float4 a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = t[2 * i];
+                b[i] = t[2 * i + 1];
+            }
+            st_cluster4(dst[0] + off, make_float4(a[0].x, a[1].x, a[2].x, a[3].x));
+            st_cluster4(dst[1] + off, make_float4(a[0].y, a[1].y, a[2].y, a[3].y));
+            st_cluster4(dst[2] + off, make_float4(a[0].z, a[1].z, a[2].z, a[3].z));
+            st_cluster4(dst[3] + off, make_float4(a[0].w, a[1].w, a[2].w, a[3].w));
+            st_cluster4(dst[4] + off, make_float4(b[0].x, b[1].x, b[2].x, b[3].x));
+            st_cluster4(dst[5] + off, make_float4(b[0].y, b[1].y, b[2].y, b[3].y));
+            st_cluster4(dst[6] + off, make_float4(b[0].z, b[1].z, b[2].z, b[3].z));
+            st_cluster4(dst[7] + off, make_float4(b[0].w, b[1].w, b[2].w, b[3].w));
+        } else {
+            // bf16: word w of a pixel holds channels 2w (low half) and 2w + 1.
+            const uint4* t = reinterpret_cast<const uint4*>(tb) + j;
+            const uint4 r0 = t[0], r1 = t[1], r2 = t[2], r3 = t[3];
+            const unsigned w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+            const unsigned w2[4] = {r2.x, r2.y, r2.z, r2.w}, w3[4] = {r3.x, r3.y, r3.z, r3.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const unsigned sel = (q & 1) ? 0x7632u : 0x5410u;
+                st_cluster2(dst[q] + off, __byte_perm(w0[q >> 1], w1[q >> 1], sel),
+                            __byte_perm(w2[q >> 1], w3[q >> 1], sel));
+            }
+        }
+    }
+}
+
+// stream_octet_out: this CTA's pixels (crank * opix + j) of the output
+// octet buffer ([8 channels][opix pixels], stored format) to y, the 8
+// channels of a pixel as one 32-byte (fp32) or 16-byte (bf16) run; `dst` is
+// channel 8o of pixel 0 of the plane's batch element.
+template <typename T>
+__device__ __forceinline__ void stream_octet_out(const float* sm, const Plan& P, T* dst, int crank, int tid, int nt) {
+    const size_t pstride = (size_t)P.C;
+    T* g = dst + (size_t)crank * P.opix * pstride;
+    const T* ob = reinterpret_cast<const T*>(sm + P.obuf);
+    const int ng = P.opix >> 2;
+    for (int gq = tid; gq < ng; gq += nt) {
+        const int j = 4 * gq;
+        if constexpr (sizeof(T) == 4) {
+            float4 c[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) c[q] = *reinterpret_cast<const float4*>(ob + (size_t)q * P.opix + j);
+            float* o = reinterpret_cast<float*>(g + (size_t)j * pstride);
+            const size_t ps = pstride;
+            *reinterpret_cast<float4*>(o) = make_float4(c[0].x, c[1].x, c[2].x, c[3].x);
+            *reinterpret_cast<float4*>(o + 4) = make_float4(c[4].x, c[5].x, c[6].x, c[7].x);
+            *reinterpret_cast<float4*>(o + ps) = make_float4(c[0].y, c[1].y, c[2].y, c[3].y);
+            *reinterpret_cast<float4*>(o + ps + 4) = make_float4(c[4].y, c[5].y, c[6].y, c[7].y);
+            *reinterpret_cast<float4*>(o + 2 * ps) = make_float4(c[0].z, c[1].z, c[2].z, c[3].z);
+            *reinterpret_cast<float4*>(o + 2 * ps + 4) = make_float4(c[4].z, c[5].z, c[6].z, c[7].z);
+            *reinterpret_cast<float4*>(o + 3 * ps) = make_float4(c[0].w, c[1].w, c[2].w, c[3].w);
+            *reinterpret_cast<float4*>(o + 3 * ps + 4) = make_float4(c[4].w, c[5].w, c[6].w, c[7].w);
+        } else {
+            // bf16: channel q's 4 pixels are one 8-byte word pair (pixel i in
+            // half i & 1 of word i >> 1).
+            uint2 c[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) c[q] = *reinterpret_cast<const uint2*>(ob + (size_t)q * P.opix + j);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const unsigned sel = (i & 1) ? 0x7632u : 0x5410u;
+                auto w = [&](int q) { return (i >> 1) ? c[q].y : c[q].x; };
+                uint4 v;
+                v.x = __byte_perm(w(0), w(1), sel);
+                v.y = __byte_perm(w(2), w(3), sel);
+                v.z = __byte_perm(w(4), w(5), sel);
+                v.w = __byte_perm(w(6), w(7), sel);
+                *reinterpret_cast<uint4*>(g + (size_t)(j + i) * pstride) = v;
+            }
+        }
     }
 }
 
@@ -916,12 +1055,17 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
     constexpr int p = K / 2, KK = K * K, NP = TC / 2;
     static_assert(TC == 4, "4-column tiles");
     const int tid = threadIdx.x, nt = blockDim.x;
-    const long long units = (long long)P.B * P.C;
-    // With strips, the nstrips CTAs of a cluster walk the same planes.
+    const long long units = (long long)P.B * ((GENERAL && P.oct) ? P.C / 8 : P.C);
+    // With strips, the nstrips CTAs of a cluster walk the same planes; with
+    // channel octets (NHWC), the 8 CTAs of a cluster walk the same (b, octet)
+    // units, CTA r taking channel 8 * octet + r.
     const bool strips = GENERAL && P.nstrips > 1;
-    const int rank = strips ? (int)cg::this_cluster().block_rank() : 0;
-    const long long team = strips ? blockIdx.x / P.nstrips : blockIdx.x;
-    const long long teams = strips ? gridDim.x / P.nstrips : gridDim.x;
+    const bool oct = GENERAL && P.oct;
+    const int cs = GENERAL ? cluster_ctas(P) : 1;
+    const int crank = cs > 1 ? (int)cg::this_cluster().block_rank() : 0;
+    const int rank = strips ? crank : 0;  // strip of the plane
+    const long long team = cs > 1 ? blockIdx.x / cs : blockIdx.x;
+    const long long teams = cs > 1 ? gridDim.x / cs : gridDim.x;
     FusedCtx<K, T, BWD, GENERAL> cx{sm, P, x, base_w, base_b, base_scale, wt_w, wt_scale, units,
                            (int)((team * units) / teams), (int)(((team + 1) * units) / teams),
                            (size_t)P.Hr * P.Wr, (size_t)rank * P.H * P.Wr};
@@ -936,9 +1080,11 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
 
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
-    // (b, c) of the plane being analysed / tiled, of the previous plane, and of the next.
+    // (b, c) of the plane being analysed / tiled, of the previous plane, and of the next
+    // (with octets, c is the octet and chan(c) this CTA's channel).
     int cur_b = u0 % P.B, cur_c = u0 / P.B;
     int prev_b = 0, prev_c = 0;
+    auto chan = [&](int c) { return oct ? 8 * c + crank : c; };
     auto stage = [&](const T* src) {
         if constexpr (GENERAL) {
             stage_rows(sm + P.stg, src, P, myrows, tid, nt);
@@ -946,30 +1092,57 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
             stage_plane(sm + P.stg, src, P.plane_chunks, tid, nt);
         }
     };
-    if (u0 < u1) stage(cx.src(cur_b, cur_c));
-    cp_async_commit();
+    auto octet_src = [&](int b, int c) { return x + plane_origin<GENERAL>(P, b, 8 * c); };
+    // Octets with a synthesis (L >= 1): outputs go through the owners' output
+    // octet buffers (oaddr != 0), written out in phase B of the next plane.
+    const bool oct_out = oct && P.L >= 1;
+    const unsigned oaddr = oct_out ? static_cast<unsigned>(__cvta_generic_to_shared(sm + P.obuf)) : 0u;
+    const unsigned ocol = (unsigned)crank * (unsigned)P.opix * (unsigned)sizeof(T);
+    if (oct) {
+        // Octets: the first plane's octet run, then its scatter once every
+        // CTA of the cluster runs and has zeroed its shared memory.
+        if (u0 < u1) load_octet(sm + P.tbuf, octet_src(cur_b, cur_c), P, crank, tid, nt);
+        cp_async_commit();
+        cp_async_wait_all();
+        plane_sync<GENERAL>(P);
+        if (u0 < u1) scatter_octet(sm, P, crank, tid, nt);
+    } else {
+        if (u0 < u1) stage(cx.src(cur_b, cur_c));
+        cp_async_commit();
+    }
     int folded_c = -1;
     for (int u = u0; u <= u1; ++u) {
         cp_async_wait_all();
         plane_sync<GENERAL>(P);  // plane u staged; every tile of plane u-1 done (its halo rows are free)
+        int nb = cur_b + 1, nc = cur_c;
+        if (nb == P.B) {
+            nb = 0;
+            ++nc;
+        }
         // Phase A.
         if (u < u1) {
+            if (oct) {
+                // The next plane's octet run (the buffer's last reader, the
+                // scatter of phase B(u-1), is behind the barrier above).
+                if (u + 1 < u1) load_octet(sm + P.tbuf, octet_src(nb, nc), P, crank, tid, nt);
+                cp_async_commit();
+            }
             if (cur_c != folded_c) {
-                cx.fold(cur_c, nt, tid);
+                cx.fold(chan(cur_c), nt, tid);
                 folded_c = cur_c;
             }
             analyse_plane<T, p, false, kToS>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         }
         if (u > u0 && P.L >= 1) {
-            T* yp = y + cx.rows_of(prev_b, prev_c);
+            T* yp = y + cx.rows_of(prev_b, chan(prev_c));
             // One synthesis loop per level count (uniform dispatch), so that
             // the items' level walk is unrolled with no per-level tests.
             switch (P.L) {
-                case 1: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 1>(sm, P, yp, t, myrows); break;
-                case 2: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 2>(sm, P, yp, t, myrows); break;
-                case 3: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 3>(sm, P, yp, t, myrows); break;
-                case 4: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 4>(sm, P, yp, t, myrows); break;
-                default: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL>(sm, P, yp, t, myrows); break;
+                case 1: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 1>(sm, P, yp, t, myrows, oaddr, ocol); break;
+                case 2: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 2>(sm, P, yp, t, myrows, oaddr, ocol); break;
+                case 3: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 3>(sm, P, yp, t, myrows, oaddr, ocol); break;
+                case 4: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL, 4>(sm, P, yp, t, myrows, oaddr, ocol); break;
+                default: for (int t = ft; t < P.n_fin; t += nt) synth_item<T, GENERAL>(sm, P, yp, t, myrows, oaddr, ocol); break;
             }
         }
         if (u == u1) break;
@@ -977,15 +1150,19 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
             __syncthreads();  // this strip's X and S of plane u complete
             push_halos(sm, P, rank, tid, nt);
         }
+        if (oct) cp_async_wait_all();  // this thread's chunks of the next octet run
         plane_sync<GENERAL>(P);  // X, S and halo rows of plane u ready (every strip); Q and Y of plane u-1 consumed
         // Phase B.
-        int nb = cur_b + 1, nc = cur_c;
-        if (nb == P.B) {
-            nb = 0;
-            ++nc;
+        if (oct) {
+            // Every CTA of the cluster is past its analysis of plane u: the
+            // next plane goes into all eight stagings; and past its synthesis
+            // of plane u-1: this CTA's pixels of it are complete.
+            if (u + 1 < u1) scatter_octet(sm, P, crank, tid, nt);
+            if (oct_out && u > u0) stream_octet_out<T>(sm, P, y + plane_origin<GENERAL>(P, prev_b, 8 * prev_c), crank, tid, nt);
+        } else {
+            if (u + 1 < u1) stage(cx.src(nb, nc));
+            cp_async_commit();
         }
-        if (u + 1 < u1) stage(cx.src(nb, nc));
-        cp_async_commit();
         // One tile loop per output kind (a uniform branch), each with a
         // single conv-tile call site.
         if (P.L >= 1) {
@@ -1012,7 +1189,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
                 float w[KK];
                 load_weights<K>(sm + j.wts, w);
                 const float b0 = sm[P.bias];
-                T* yo = y + cx.rows_of(cur_b, cur_c) + (size_t)j.out * es;
+                T* yo = y + cx.rows_of(cur_b, chan(cur_c)) + (size_t)j.out * es;
                 const int h0 = j.row0;
                 conv_tile<K, TR, TC>(sm + j.win, j.wstride, w, make_float2(b0, b0), [&](int o, float2(&a)[NP]) {
                     if (h0 + o < myrows)
@@ -1026,6 +1203,10 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
         cur_c = nc;
     }
     cp_async_wait_all();
+    if (oct_out && u1 > u0) {
+        plane_sync<GENERAL>(P);  // the last plane's outputs are in every owner's buffer
+        stream_octet_out<T>(sm, P, y + plane_origin<GENERAL>(P, prev_b, 8 * prev_c), crank, tid, nt);
+    }
 }
 
 // ---------------------------------------------------------------------------

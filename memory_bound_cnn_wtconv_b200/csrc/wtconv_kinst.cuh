@@ -37,8 +37,8 @@ cudaError_t opt_in_smem(F* fn, std::atomic<bool> (&done)[kMaxDevices]) {
     return e;
 }
 
-// Launch configuration; planes split into strips run as clusters of
-// nstrips CTAs along x.
+// Launch configuration; planes split into strips (and NHWC channel octets)
+// run as clusters of cluster_ctas(P) CTAs along x.
 struct Launch {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
@@ -50,9 +50,9 @@ struct Launch {
         cfg.stream = s;
         cfg.attrs = attr;
         cfg.numAttrs = 0;
-        if (P.nstrips > 1) {
+        if (cluster_ctas(P) > 1) {
             attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = P.nstrips;
+            attr[0].val.clusterDim.x = cluster_ctas(P);
             attr[0].val.clusterDim.y = 1;
             attr[0].val.clusterDim.z = 1;
             cfg.numAttrs = 1;
@@ -66,13 +66,14 @@ cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
     auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD, GENERAL>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
-    // Persistent grid: every resident CTA slot (cluster slot, for strips) of
-    // the device, at most one CTA (cluster) per plane.
-    const long long units = (long long)P.B * P.C;
+    // Persistent grid: every resident CTA slot (cluster slot, for strips and
+    // octets) of the device, at most one CTA (cluster) per plane (octet).
+    const int cs = cluster_ctas(P);
+    const long long units = (long long)P.B * (P.oct ? P.C / 8 : P.C);
     long long teams = 0;
     Launch L(P, dim3(1), s);
-    if (P.nstrips > 1) {
-        L.cfg.gridDim = dim3(P.nstrips * 64);  // any multiple of the cluster size, for the query
+    if (cs > 1) {
+        L.cfg.gridDim = dim3(cs * 64);  // any multiple of the cluster size, for the query
         int clusters = 0;
         if ((e = cudaOccupancyMaxActiveClusters(&clusters, fn, &L.cfg)) != cudaSuccess) return e;
         if (clusters < 1) return cudaErrorInvalidConfiguration;
@@ -86,7 +87,7 @@ cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
             return e;
         teams = (long long)sms * std::max(per_sm, 1);
     }
-    L.cfg.gridDim = dim3((unsigned)(std::min<long long>(units, teams) * P.nstrips));
+    L.cfg.gridDim = dim3((unsigned)(std::min<long long>(units, teams) * cs));
     e = cudaLaunchKernelEx(&L.cfg, fn, static_cast<const T*>(a.x), a.base_w, a.base_b, a.base_scale, a.wt_w,
                            a.wt_scale, static_cast<T*>(a.y), P);
     if (e != cudaSuccess) return e;

@@ -90,6 +90,18 @@ struct Plan {
     // gathered element by element, C elements apart; the general
     // instantiations and the one-pass backward only).
     int nhwc;
+    // NHWC channel octets (forward / input gradient on whole planes, C a
+    // multiple of 8): clusters of 8 CTAs, CTA r of a cluster holding channel
+    // 8o + r of the planes (b, octet o) the cluster walks.  Each CTA loads
+    // its run of opix pixels of the plane's 8 channels (8 * esize contiguous
+    // bytes a pixel) into its octet buffer at tbuf (stg_floats floats, pixel
+    // j at 8 * esize * j bytes) and scatters channel q to CTA q's staging.
+    // The synthesis stores each output into the output octet buffer at obuf
+    // (stg_floats floats) of the CTA that owns its pixel, as row r of
+    // [8 channels][opix pixels] (stored format); the owner writes the 8
+    // channels of its pixels as whole runs.
+    int oct, opix, tbuf, obuf;
+    FastDiv div_opix;
     int parts;           // weight gradient: partial vectors per channel (groups * nstrips)
     int TR, TC;          // output tile: TR rows x TC cols per thread (TC = 4: two column pairs)
     int esize;           // bytes per stored activation (4 or 2)
@@ -148,5 +160,15 @@ struct Plan {
     FastDiv div_m[kMaxL];           // W >> (l+1)
     FastDiv div_ntc[kMaxL + 1];     // tile columns per tile row
 };
+
+// CTAs per cluster: the strips of a plane, or the 8 CTAs of a channel octet
+// (also compiled by host-only tools, without the CUDA qualifiers).
+#ifdef __CUDACC__
+#define WTC_HD __host__ __device__
+#else
+#define WTC_HD
+#endif
+inline WTC_HD int cluster_ctas(const Plan& P) { return P.oct ? 8 : P.nstrips; }
+#undef WTC_HD
 
 }  // namespace wtc

@@ -125,7 +125,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // num_sms (the device's SM count) sizes the persistent forward grid and the
 // weight gradient's batch groups.
 inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, int nstrips, int num_sms, Plan* P,
-                                     bool dy_stg = false) {
+                                     bool dy_stg = false, bool octets = true) {
     memset(P, 0, sizeof(*P));
     if (num_sms < 1) return WTCONV_ERR_UNSUPPORTED;
     // The plane the CTAs hold: H and W rounded up to multiples of 2^L.
@@ -223,6 +223,22 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         P->div_rowc = make_fastdiv(std::max(P->row_chunks, 1));
         P->stg = (int)off;
         off += (kind == kBackwardWeight || kind == kBackward ? 2LL : 1LL) * P->stg_floats;
+    }
+    // NHWC channel octets: a pixel's 8 channels are one 16- or 32-byte run,
+    // loaded once for the cluster's 8 planes instead of element by element
+    // per plane.  Whole, unpadded planes whose pixels split into 8 runs of a
+    // multiple of 4 pixels.
+    if (octets && (kind == kForward || kind == kBackwardInput) && P->nhwc && nstrips == 1 && !P->padded &&
+        d->C % 8 == 0 && ((long long)H * W) % 32 == 0) {
+        P->oct = 1;
+        P->opix = H * W / 8;
+        P->div_opix = make_fastdiv(P->opix);
+        P->tbuf = (int)off;
+        off += P->stg_floats;
+        if (L >= 1) {  // outputs of the synthesis (L = 0: the base tiles store y directly)
+            P->obuf = (int)off;
+            off += P->stg_floats;
+        }
     }
     if (dy_stg) {
         // The dy staging holds the strip as H rows of W floats: the DY layout
@@ -408,7 +424,11 @@ inline wtconv_status_t make_plan(const wtconv_desc_t* d, Kind kind, int num_sms,
         for (int alias = 0; alias < 2 && !have; ++alias) {
             if (alias && (kind != kBackwardWeight || n == 1)) break;
             for (int TR = 7; TR <= 8; ++TR) {
-                if (make_plan_for(d, kind, TR, n, num_sms, &cand, alias == 1) != WTCONV_OK) continue;
+                wtconv_status_t st = make_plan_for(d, kind, TR, n, num_sms, &cand, alias == 1);
+                // NHWC planes whose octet buffer does not fit: the element-by-element gather.
+                if (st != WTCONV_OK && n == 1 && d->layout == WTCONV_NHWC)
+                    st = make_plan_for(d, kind, TR, n, num_sms, &cand, alias == 1, false);
+                if (st != WTCONV_OK) continue;
                 const double c = plan_cost(cand, kind);
                 if (!have || c < best) {
                     best = c;

@@ -432,9 +432,55 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
         std::printf("FAIL smem size\n");
         std::exit(1);
     }
-    std::vector<Shadow> shs(NS, Shadow(P.smem_floats));
+    // NHWC channel octets: 8 CTAs a cluster, each on whole planes (strip 0),
+    // staging filled by the cluster's scatters from the octet buffers.
+    const int NC = cluster_ctas(P);
+    if (P.oct) {
+        if (!P.nhwc || NS != 1 || P.padded || P.C % 8 || P.opix * 8LL != (long long)H * W || P.opix % 4 ||
+            P.tbuf % 4 || P.tbuf < P.stg + P.stg_floats || P.tbuf + (long long)P.stg_floats > P.smem_floats ||
+            (kind != kForward && kind != kBackwardInput)) {
+            std::printf("FAIL octet plan: opix %d tbuf %d stg %d smem %d\n", P.opix, P.tbuf, P.stg, P.smem_floats);
+            std::exit(1);
+        }
+    } else if (P.nhwc && kind != kBackward && NS == 1 && !P.padded && P.C % 8 == 0 && ((long long)H * W) % 32 == 0 &&
+               P.smem_floats + (long long)P.stg_floats <= kSmemLimitFloats && (kind == kForward || kind == kBackwardInput)) {
+        std::printf("FAIL octet plan not taken where it fits\n");
+        std::exit(1);
+    }
+    std::vector<Shadow> shs(NC, Shadow(P.smem_floats));
     const long long all = P.smem_floats;
     if (P.grid < 1 || P.grid > (long long)P.B * P.C) shs[0].fail("grid", P.grid);
+    const int OCT = 400;  // tag of octet-buffer floats
+    // Octet run of CTA r (phase of the caller): 16-byte chunks of whole pixels
+    // from the last octet of the last batch element (bounds), into T once each.
+    auto octet_load = [&](Shadow& sh, int r) {
+        const int cpp = P.esize / 2;
+        const long long total = (long long)P.B * H * W * P.C;  // NHWC elements
+        const int o = P.C / 8 - 1, b = P.B - 1;
+        for (int ch = 0; ch < P.opix * cpp; ++ch) {
+            const int j = cpp == 2 ? ch >> 1 : ch, h = ch - j * cpp;
+            const long long e0 = ((long long)b * H * W + (long long)r * P.opix + j) * P.C + 8LL * o + 8 / cpp * h;
+            check_global(e0, total, "octet run first element");
+            check_global(e0 + 16 / P.esize - 1, total, "octet run last element");
+            if ((e0 * P.esize) % 16) sh.fail("octet chunk source not 16-byte aligned", e0);
+            for (int f = 0; f < 4; ++f)
+                sh.write(P.tbuf + 4LL * ch + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
+        }
+    };
+    // Scatter of CTA r: its pixels' channel q into CTA q's staging, four
+    // pixels a step (16 or 8 bytes a channel).
+    auto octet_scatter = [&](int r) {
+        Shadow& me = shs[r];
+        for (int f = 0; f < P.stg_floats; ++f) me.read(P.tbuf + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
+        const int per = 4 / P.esize;  // elements a staging float
+        for (int gq = 0; gq < P.opix / 4; ++gq) {
+            const long long e = (long long)r * P.opix + 4LL * gq;
+            if ((e * P.esize) % (4 * P.esize)) me.fail("scatter store misaligned", e);
+            for (int q = 0; q < 8; ++q)
+                for (long long f = e / per; f < (e + 4) / per; ++f)
+                    shs[q].write(P.stg + f, P.stg, P.stg + P.stg_floats, XT + 10, "scattered staging");
+        }
+    };
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
     const long long ylo = P.Y.base, yhi = P.Y.base + (long long)P.ntr[kMaxL] * TR * P.Y.stride;
@@ -443,8 +489,37 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     const int ntc = P.ntc[kMaxL];
     const long long plane = (long long)P.Hr * P.Wr;
 
+    // Channel octets with a synthesis: outputs go to the owners' output octet
+    // buffers ([8 channels][opix pixels], stored format; CTA r's channel row r).
+    const int OUT = 401;
+    const bool oct_out = P.oct && L >= 1;
+    if (oct_out && (P.obuf % 4 || P.obuf < P.tbuf + P.stg_floats || P.obuf + (long long)P.stg_floats > P.smem_floats))
+        shs[0].fail("output octet buffer", P.obuf);
+    auto octet_out = [&](int r, int px) {
+        const int owner = (int)fastdiv_host((uint32_t)px, P.div_opix), j = px - owner * P.opix;
+        if (owner != px / P.opix || owner < 0 || owner >= 8) shs[r].fail("output owner", px);
+        const long long e = (long long)r * P.opix + j;  // element of the owner's buffer
+        if ((e * P.esize) % (4 * P.esize)) shs[r].fail("output octet store misaligned", e);
+        const int per = 4 / P.esize;
+        for (long long f = e / per; f < (e + 4) / per; ++f)
+            shs[owner].write(P.obuf + f, P.obuf, P.obuf + P.stg_floats, OUT, "output octet buffer");
+    };
+    // The owner's pass over its buffer: every float read, its pixels' 8
+    // channels stored in y (last octet of the last batch element: bounds).
+    auto octet_stream = [&](int r) {
+        Shadow& me = shs[r];
+        for (int f = 0; f < P.stg_floats; ++f) me.read(P.obuf + f, P.obuf, P.obuf + P.stg_floats, OUT, "output octet buffer");
+        const long long total = (long long)P.B * H * W * P.C;
+        for (int j = 0; j < P.opix; ++j) {
+            const long long e0 = ((long long)(P.B - 1) * H * W + (long long)r * P.opix + j) * P.C + 8LL * (P.C / 8 - 1);
+            check_global(e0, total, "octet output run");
+            check_global(e0 + 7, total, "octet output run");
+            if ((e0 * P.esize) % 16) me.fail("octet output run not 16-byte aligned", e0);
+        }
+    };
+
     // Phase A's synthesis of the previous plane: rows 2i, 2i+1 x columns 4q..4q+3.
-    auto synthesis = [&](Shadow& sh, int rank) {
+    auto synthesis = [&](Shadow& sh, int rank, int crank) {
         for (int t = 0; t < P.n_fin; ++t) {
             const int i = (int)fastdiv_host(t, P.div_q4), q = t - i * (W / 4);
             if (i != t / (W / 4)) sh.fail("synthesis item division", t);
@@ -472,8 +547,9 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
                 const bool store = 2 * i + rr < real_rows_host(P, rank) && 4 * q < P.Wr;
                 for (int e = 0; e < 4; ++e) {
                     sh.read(a + e, ylo, yhi, YT, "Y read");
-                    if (store) check_global((long long)(rank * H + 2 * i + rr) * P.Wr + 4 * q + e, plane, "y store");
+                    if (store && !oct_out) check_global((long long)(rank * H + 2 * i + rr) * P.Wr + 4 * q + e, plane, "y store");
                 }
+                if (oct_out) octet_out(crank, (2 * i + rr) * W + 4 * q);
             }
         }
     };
@@ -481,15 +557,31 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     // The persistent walk over two planes and the final synthesis, with the
     // kernel's barriers (cluster-wide with strips) as phase boundaries:
     //   stage(0) | A(0) | [strips: halo push(0)] | B(0): stage(1), tiles(0) | A(1) | ... | A(end)
-    for (int r = 0; r < NS; ++r) {
-        shs[r].phase = "initial staging";
-        replay_stage(shs[r], P, P.stg, XT + 10, r);
+    if (P.oct) {
+        for (int r = 0; r < NC; ++r) {
+            shs[r].phase = "initial octet run";
+            octet_load(shs[r], r);
+        }
+        barrier_all(shs);
+        for (int r = 0; r < NC; ++r) {
+            shs[r].phase = "initial scatter";
+            octet_scatter(r);
+        }
+    } else {
+        for (int r = 0; r < NS; ++r) {
+            shs[r].phase = "initial staging";
+            replay_stage(shs[r], P, P.stg, XT + 10, r);
+        }
     }
     for (int unit = 0; unit <= 2; ++unit) {
         barrier_all(shs);
-        for (int r = 0; r < NS; ++r) {
+        for (int r = 0; r < NC; ++r) {
             Shadow& sh = shs[r];
             if (unit < 2) {
+                if (P.oct && unit + 1 < 2) {
+                    sh.phase = "A: next octet run";
+                    octet_load(sh, r);
+                }
                 sh.phase = "A: fold";
                 for (int cl = 0; cl < ncls; ++cl)
                     for (int t = 0; t < KK; ++t)
@@ -501,34 +593,51 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
         if (unit < 2) {
             // The analysis may have its own CTA barriers (levels computed one
             // at a time); the synthesis runs after its last one.
-            for (int r = 0; r < NS; ++r) {
+            for (int r = 0; r < NC; ++r) {
                 shs[r].phase = "A: analysis";
-                g_rank = r;
+                g_rank = P.oct ? 0 : r;
                 const int e0 = shs[r].epoch;
                 replay_analyse(shs[r], P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi,
                                XT, P.S, p, s_tag);
-                if (r + 1 < NS) shs[r].epoch = e0;  // replay the next strip from the same phase
-                else for (int q = 0; q + 1 < NS; ++q) shs[q].epoch = shs[r].epoch;
+                if (r + 1 < NC) shs[r].epoch = e0;  // replay the next strip from the same phase
+                else for (int q = 0; q + 1 < NC; ++q) shs[q].epoch = shs[r].epoch;
             }
         }
         if (unit > 0 && L >= 1)
-            for (int r = 0; r < NS; ++r) {
+            for (int r = 0; r < NC; ++r) {
                 shs[r].phase = "A: synthesis";
-                synthesis(shs[r], r);
+                synthesis(shs[r], P.oct ? 0 : r, r);
             }
-        if (unit == 2) break;
+        if (unit == 2) {
+            if (oct_out) {
+                barrier_all(shs);
+                for (int r = 0; r < NC; ++r) {
+                    shs[r].phase = "final output octets";
+                    octet_stream(r);
+                }
+            }
+            break;
+        }
         // Strips: CTA barrier, halo push, then the cluster barrier.
         if (NS > 1) {
             barrier_all(shs);
             replay_push(shs, P);
         }
         barrier_all(shs);
-        for (int r = 0; r < NS; ++r) {
+        for (int r = 0; r < NC; ++r) {
             shs[r].phase = "B: staging";
-            if (unit + 1 < 2) replay_stage(shs[r], P, P.stg, XT + 10, r);
+            if (unit + 1 < 2) {
+                if (P.oct) octet_scatter(r);
+                else replay_stage(shs[r], P, P.stg, XT + 10, r);
+            }
+            if (oct_out && unit > 0) {
+                shs[r].phase = "B: output octets";
+                octet_stream(r);
+            }
         }
-        for (int r = 0; r < NS; ++r) {
-            Shadow& sh = shs[r];
+        for (int rr = 0; rr < NC; ++rr) {
+            Shadow& sh = shs[rr];
+            const int r = P.oct ? 0 : rr;  // strip of the CTA
             sh.phase = "B: subband tiles";
             for (int cl = 1; cl < ncls; ++cl) {
                 const int l = (cl - 1) >> 2, s = (cl - 1) & 3;
@@ -572,8 +681,9 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
             }
         }
     }
-    std::printf("fused(kind %d): smem %d B, threads %d, TR %d, tiles %d+%d, merged %d, strips %d\n", (int)kind,
-                P.smem_floats * 4, P.nthreads, TR, P.n_sub_tiles, P.n_base_tiles, P.merged, NS);
+    std::printf("fused(kind %d): smem %d B, threads %d, TR %d, tiles %d+%d, merged %d, strips %d%s\n", (int)kind,
+                P.smem_floats * 4, P.nthreads, TR, P.n_sub_tiles, P.n_base_tiles, P.merged, NS,
+                P.oct ? ", channel octets" : "");
 }
 
 void check_bwdw(const wtconv_desc_t& d) {

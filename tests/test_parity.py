@@ -352,7 +352,16 @@ NHWC_SMALL = [
     Case("nhwc_strips_128_L2", 1, 3, 128, 128, 5, 2, "f32", 59, "normal", "normal"),
     Case("nhwc_strips_256_L3_bf16", 1, 2, 256, 256, 3, 3, "bf16", 60, "normal", "normal"),
     Case("nhwc_pad_strips_250x248", 1, 1, 250, 248, 5, 4, "f32", 61, "normal", "normal"),
+    # C a multiple of 8 on whole planes of a multiple of 32 pixels: the forward and input gradient
+    # run as clusters of 8 CTAs over channel octets (odd unit counts per cluster, bf16, L = 0,
+    # k = 1 and 7, a 64x64 plane at one CTA per SM)
+    Case("nhwc_octets_stage1_plane", 3, 16, 56, 56, 5, 3, "f32", 63, "normal", "normal"),
+    Case("nhwc_octets_bf16_32", 2, 8, 32, 32, 3, 2, "bf16", 64, "uniform", "normal"),
+    Case("nhwc_octets_L0_k7", 2, 16, 56, 56, 7, 0, "f32", 65, "normal", "normal"),
+    Case("nhwc_octets_k1_bf16", 5, 8, 16, 16, 1, 2, "bf16", 66, "normal", "normal"),
+    Case("nhwc_octets_64_L4", 1, 24, 64, 64, 5, 4, "f32", 67, "normal", "normal"),
 ]
+NHWC_OCTETS = [c for c in NHWC_SMALL if c.name.startswith("nhwc_octets")]
 
 
 @pytest.mark.parametrize("case", NHWC_SMALL, ids=lambda c: c.name)
@@ -361,7 +370,7 @@ def test_nhwc_small_case_all_outputs(oracle, case):
 
 
 @pytest.mark.parametrize("mode", ["auto", "one_pass"])
-@pytest.mark.parametrize("case", NHWC_SMALL[:8], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", NHWC_SMALL[:8] + NHWC_OCTETS[:2], ids=lambda c: c.name)
 def test_nhwc_small_case_fused_backward(oracle, case, mode):
     if mode == "one_pass" and not _one_pass_plan_exists(case, nhwc=True):
         pytest.skip("planes split into cluster strips have no one-pass plan")
@@ -373,9 +382,13 @@ def test_nhwc_full_size_workloads_sampled(oracle, case):
     check_sampled(oracle, case, nhwc=True)
 
 
-def test_nhwc_matches_nchw_bitwise():
-    # Same on-chip arithmetic in the same order: the layouts must agree bit for bit.
-    case = Case("nhwc_vs_nchw", 4, 6, 40, 36, 5, 3, "f32", 62, "normal", "normal")
+@pytest.mark.parametrize("case", [
+    Case("nhwc_vs_nchw", 4, 6, 40, 36, 5, 3, "f32", 62, "normal", "normal"),
+    Case("nhwc_vs_nchw_octets", 3, 16, 32, 32, 5, 3, "f32", 68, "normal", "normal"),
+], ids=lambda c: c.name)
+def test_nhwc_matches_nchw_bitwise(case):
+    # Same on-chip arithmetic in the same order: the layouts must agree bit for bit
+    # (element-by-element gather, and channel octets).
     inp = make_inputs(case)
     a = run_gpu(case, gpu_inputs(inp), ("fwd", "bwd_in", "bwd_w"))
     b = run_gpu(case, gpu_inputs(inp, nhwc=True), ("fwd", "bwd_in", "bwd_w"))

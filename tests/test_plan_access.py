@@ -68,6 +68,9 @@ NHWC = [
     (3, 5, 56, 56, 5, 3, 0), (2, 4, 56, 56, 5, 3, 1), (2, 3, 13, 12, 5, 2, 1), (1, 2, 12, 8, 1, 0, 0),
     (2, 3, 24, 40, 3, 3, 1), (1, 2, 128, 128, 5, 2, 0), (1, 1, 250, 248, 5, 4, 1), (3, 2, 30, 28, 5, 3, 0),
     (2, 2, 64, 64, 7, 4, 0), (5, 3, 20, 12, 5, 2, 1),
+    # channel octets (C a multiple of 8, whole planes of a multiple of 32 pixels)
+    (3, 16, 56, 56, 5, 3, 0), (2, 8, 32, 32, 3, 2, 1), (2, 16, 56, 56, 7, 0, 0), (5, 8, 16, 16, 1, 2, 1),
+    (1, 24, 64, 64, 5, 4, 0), (2, 8, 8, 8, 5, 1, 0), (32, 96, 56, 56, 5, 3, 0), (64, 96, 56, 56, 5, 3, 1),
 ]
 
 
@@ -76,6 +79,14 @@ def test_every_access_in_bounds_nhwc(checker, case):
     r = subprocess.run([checker, *map(str, case), "1"], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip().endswith("OK") and "each addressed once" in r.stdout, \
         r.stdout + r.stderr
+    # Channel octets exactly where C is a multiple of 8 on whole planes of a multiple of 32 pixels
+    # (every case here fits the octet buffer).
+    B, C, H, W, k, L, _ = case
+    m = 1 << L
+    whole = H % m == 0 and W % m == 0 and H * W <= 64 * 64
+    octets = C % 8 == 0 and whole and (H * W) % 32 == 0
+    fused = [l for l in r.stdout.splitlines() if l.startswith("fused(kind")]
+    assert fused and all(("channel octets" in l) == octets for l in fused), r.stdout
 
 
 @pytest.mark.parametrize("case,strips,alias", [
