@@ -629,10 +629,14 @@ __device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const f
 // Barrier of everything that shares a plane: the CTA, or the whole cluster
 // when the plane is split into strips (then it also orders the shared-memory
 // accesses of the cluster's CTAs to each other's strips).
-template <bool GENERAL>
+template <bool GENERAL, bool OCT = false>
 __device__ __forceinline__ void plane_sync(const Plan& P) {
+    if constexpr (OCT) {
+        cg::this_cluster().sync();
+        return;
+    }
     if constexpr (GENERAL) {
-        if (cluster_ctas(P) > 1) {
+        if (P.nstrips > 1) {
             cg::this_cluster().sync();
             return;
         }
@@ -901,35 +905,36 @@ __device__ __forceinline__ void load_octet(float* tb, const void* src, const Pla
 }
 
 // scatter_octet: channel q of the octet buffer's pixels into CTA q's
-// staging (pixel crank * opix + j of the plane, stored format), four pixels
+// staging at `stg` (pixel crank * opix + j of the plane, stored format), four pixels
 // a step as one 16-byte (fp32) or 8-byte (bf16) distributed shared store per
 // channel.  The cluster barrier after it makes the stores visible.
-__device__ __forceinline__ void scatter_octet(float* sm, const Plan& P, int crank, int tid, int nt) {
-    const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm + P.stg));
-    unsigned dst[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(dst[q]) : "r"(local), "r"(q));
+__device__ __forceinline__ void scatter_octet(float* sm, int stg, const Plan& P, int crank, int tid, int nt) {
+    const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm + stg));
+    // CTA q's copy of the staging (mapped per store: few registers live, the
+    // weight gradient's correlation sums stay in registers meanwhile).
+    auto remote = [&](int q) {
+        unsigned a;
+        asm("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(local), "r"(q));
+        return a;
+    };
     const float* tb = sm + P.tbuf;
     const int ng = P.opix >> 2;
     for (int gq = tid; gq < ng; gq += nt) {
         const int j = 4 * gq;
         const unsigned off = (unsigned)(crank * P.opix + j) * (unsigned)P.esize;
         if (P.esize == 4) {
+            // Pixel i's channels 0-3 at float4 2i, channels 4-7 at 2i + 1.
             const float4* t = reinterpret_cast<const float4*>(tb) + 2 * j;
-            float4 a[4], b[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a[i] = t[2 * i];
-                b[i] = t[2 * i + 1];
+            for (int h = 0; h < 2; ++h) {
+                float4 v[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) v[i] = t[2 * i + h];
+                st_cluster4(remote(4 * h) + off, make_float4(v[0].x, v[1].x, v[2].x, v[3].x));
+                st_cluster4(remote(4 * h + 1) + off, make_float4(v[0].y, v[1].y, v[2].y, v[3].y));
+                st_cluster4(remote(4 * h + 2) + off, make_float4(v[0].z, v[1].z, v[2].z, v[3].z));
+                st_cluster4(remote(4 * h + 3) + off, make_float4(v[0].w, v[1].w, v[2].w, v[3].w));
             }
-            st_cluster4(dst[0] + off, make_float4(a[0].x, a[1].x, a[2].x, a[3].x));
-            st_cluster4(dst[1] + off, make_float4(a[0].y, a[1].y, a[2].y, a[3].y));
-            st_cluster4(dst[2] + off, make_float4(a[0].z, a[1].z, a[2].z, a[3].z));
-            st_cluster4(dst[3] + off, make_float4(a[0].w, a[1].w, a[2].w, a[3].w));
-            st_cluster4(dst[4] + off, make_float4(b[0].x, b[1].x, b[2].x, b[3].x));
-            st_cluster4(dst[5] + off, make_float4(b[0].y, b[1].y, b[2].y, b[3].y));
-            st_cluster4(dst[6] + off, make_float4(b[0].z, b[1].z, b[2].z, b[3].z));
-            st_cluster4(dst[7] + off, make_float4(b[0].w, b[1].w, b[2].w, b[3].w));
         } else {
             // bf16: word w of a pixel holds channels 2w (low half) and 2w + 1.
             const uint4* t = reinterpret_cast<const uint4*>(tb) + j;
@@ -939,7 +944,7 @@ __device__ __forceinline__ void scatter_octet(float* sm, const Plan& P, int cran
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const unsigned sel = (q & 1) ? 0x7632u : 0x5410u;
-                st_cluster2(dst[q] + off, __byte_perm(w0[q >> 1], w1[q >> 1], sel),
+                st_cluster2(remote(q) + off, __byte_perm(w0[q >> 1], w1[q >> 1], sel),
                             __byte_perm(w2[q >> 1], w3[q >> 1], sel));
             }
         }
@@ -1045,7 +1050,7 @@ struct FusedCtx {
 // GENERAL: planes split into strips across a cluster and / or zero-padded on
 // chip (a separate instantiation, so the common walk of whole planes that
 // are multiples of 2^L carries none of that code).
-template <int K, int TR, int TC, typename T, bool BWD, bool GENERAL>
+template <int K, int TR, int TC, typename T, bool BWD, bool GENERAL, bool OCT = false>
 __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads, GENERAL ? 1 : 2) wtconv_fused_kernel(
     const T* __restrict__ x, const float* __restrict__ base_w, const float* __restrict__ base_b,
     const float* __restrict__ base_scale, const float* __restrict__ wt_w,
@@ -1055,13 +1060,14 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
     constexpr int p = K / 2, KK = K * K, NP = TC / 2;
     static_assert(TC == 4, "4-column tiles");
     const int tid = threadIdx.x, nt = blockDim.x;
-    const long long units = (long long)P.B * ((GENERAL && P.oct) ? P.C / 8 : P.C);
+    static_assert(!OCT || GENERAL, "channel octets run in the general walk");
+    const long long units = (long long)P.B * (OCT ? P.C / 8 : P.C);
     // With strips, the nstrips CTAs of a cluster walk the same planes; with
     // channel octets (NHWC), the 8 CTAs of a cluster walk the same (b, octet)
     // units, CTA r taking channel 8 * octet + r.
     const bool strips = GENERAL && P.nstrips > 1;
-    const bool oct = GENERAL && P.oct;
-    const int cs = GENERAL ? cluster_ctas(P) : 1;
+    constexpr bool oct = OCT;
+    const int cs = OCT ? 8 : (GENERAL ? P.nstrips : 1);
     const int crank = cs > 1 ? (int)cg::this_cluster().block_rank() : 0;
     const int rank = strips ? crank : 0;  // strip of the plane
     const long long team = cs > 1 ? blockIdx.x / cs : blockIdx.x;
@@ -1104,8 +1110,8 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
         if (u0 < u1) load_octet(sm + P.tbuf, octet_src(cur_b, cur_c), P, crank, tid, nt);
         cp_async_commit();
         cp_async_wait_all();
-        plane_sync<GENERAL>(P);
-        if (u0 < u1) scatter_octet(sm, P, crank, tid, nt);
+        plane_sync<GENERAL, OCT>(P);
+        if (u0 < u1) scatter_octet(sm, P.stg, P, crank, tid, nt);
     } else {
         if (u0 < u1) stage(cx.src(cur_b, cur_c));
         cp_async_commit();
@@ -1113,7 +1119,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
     int folded_c = -1;
     for (int u = u0; u <= u1; ++u) {
         cp_async_wait_all();
-        plane_sync<GENERAL>(P);  // plane u staged; every tile of plane u-1 done (its halo rows are free)
+        plane_sync<GENERAL, OCT>(P);  // plane u staged; every tile of plane u-1 done (its halo rows are free)
         int nb = cur_b + 1, nc = cur_c;
         if (nb == P.B) {
             nb = 0;
@@ -1151,13 +1157,13 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
             push_halos(sm, P, rank, tid, nt);
         }
         if (oct) cp_async_wait_all();  // this thread's chunks of the next octet run
-        plane_sync<GENERAL>(P);  // X, S and halo rows of plane u ready (every strip); Q and Y of plane u-1 consumed
+        plane_sync<GENERAL, OCT>(P);  // X, S and halo rows of plane u ready (every strip); Q and Y of plane u-1 consumed
         // Phase B.
         if (oct) {
             // Every CTA of the cluster is past its analysis of plane u: the
             // next plane goes into all eight stagings; and past its synthesis
             // of plane u-1: this CTA's pixels of it are complete.
-            if (u + 1 < u1) scatter_octet(sm, P, crank, tid, nt);
+            if (u + 1 < u1) scatter_octet(sm, P.stg, P, crank, tid, nt);
             if (oct_out && u > u0) stream_octet_out<T>(sm, P, y + plane_origin<GENERAL>(P, prev_b, 8 * prev_c), crank, tid, nt);
         } else {
             if (u + 1 < u1) stage(cx.src(nb, nc));
@@ -1204,7 +1210,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads,
     }
     cp_async_wait_all();
     if (oct_out && u1 > u0) {
-        plane_sync<GENERAL>(P);  // the last plane's outputs are in every owner's buffer
+        plane_sync<GENERAL, OCT>(P);  // the last plane's outputs are in every owner's buffer
         stream_octet_out<T>(sm, P, y + plane_origin<GENERAL>(P, prev_b, 8 * prev_c), crank, tid, nt);
     }
 }
@@ -1300,7 +1306,7 @@ __device__ __forceinline__ void finish_channel_if_last(float* sm, const Plan& P,
 // GENERAL: the plane is split into strips across a cluster and / or
 // zero-padded on chip (a separate instantiation, so whole-plane walks keep
 // every register for the sums).
-template <int K, int TR, int TC, typename T, bool GENERAL>
+template <int K, int TR, int TC, typename T, bool GENERAL, bool OCT = false>
 __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, GENERAL ? 1 : 2) wtconv_bwdw_partial_kernel(
     const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const GradArgs ga, const Plan P) {
     extern __shared__ float4 smem4[];
@@ -1308,9 +1314,13 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
     constexpr int p = K / 2, KK = K * K;
     constexpr int DLD = sizeof(T) == 2 ? 4 : 2;
     const int tid = threadIdx.x, nt = blockDim.x;
-    // blockIdx.x = c * nstrips + (strip rank within the cluster).
+    // blockIdx.x = c * nstrips + (strip rank within the cluster); with NHWC
+    // channel octets, clusters of the 8 channels of an octet (rank c mod 8).
+    static_assert(!OCT || GENERAL, "channel octets run in the general walk");
     const bool strips = GENERAL && P.nstrips > 1;
+    constexpr bool oct = OCT;
     const int rank = strips ? (int)cg::this_cluster().block_rank() : 0;
+    const int crank = oct ? (int)cg::this_cluster().block_rank() : 0;
     const int c = strips ? blockIdx.x / P.nstrips : blockIdx.x, g = blockIdx.y, G = P.groups;
     const size_t strip_off = (size_t)rank * P.H * P.Wr * act_es<GENERAL>(P);
     const int myrows = real_rows(P, rank);
@@ -1331,8 +1341,28 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
             stage_plane(sm + P.stg + P.stg_floats, dy + off, P.plane_chunks, tid, nt);
         }
     };
-    if (g < P.B) stage(plane_origin<GENERAL>(P, g, c) + strip_off, true);
-    cp_async_commit();
+    // Octets: the x and dy runs of the octet's planes go through one octet
+    // buffer in turn, each scattered into the cluster's stagings.
+    const size_t oct_off = (size_t)(c - crank);  // channel 8o: NHWC element offset of the octet
+    auto octet_run = [&](const T* src, int b) {
+        load_octet(sm + P.tbuf, src + plane_origin<GENERAL>(P, b, 0) + oct_off, P, crank, tid, nt);
+    };
+    if (oct) {
+        if (g < P.B) octet_run(x, g);
+        cp_async_commit();
+        cp_async_wait_all();
+        plane_sync<GENERAL, OCT>(P);  // every CTA of the cluster running, its shared memory zeroed; x run complete
+        if (g < P.B) scatter_octet(sm, P.stg, P, crank, tid, nt);
+        __syncthreads();  // the octet buffer consumed
+        if (g < P.B) octet_run(dy, g);
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncthreads();
+        if (g < P.B) scatter_octet(sm, P.stg + P.stg_floats, P, crank, tid, nt);
+    } else {
+        if (g < P.B) stage(plane_origin<GENERAL>(P, g, c) + strip_off, true);
+        cp_async_commit();
+    }
 
     // This thread's class and its run of that class's tiles.
     int cl = -1, first = 0, cnt = 0;
@@ -1363,7 +1393,11 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
     float* X0 = sm + P.X.base + p * P.X.stride + p;
     for (int b = g; b < P.B; b += G) {
         cp_async_wait_all();
-        plane_sync<GENERAL>(P);  // staged pair complete; previous correlations done (halo rows free)
+        plane_sync<GENERAL, OCT>(P);  // staged pair complete; previous correlations done (halo rows free)
+        if (oct) {
+            if (b + G < P.B) octet_run(x, b + G);  // the buffer's last reader is behind the barrier above
+            cp_async_commit();
+        }
         analyse_plane<T, p, false, kToS>(sm, P, sm + P.stg, X0, P.X.stride, p, nt, tid, csync);
         const float s = dys ? analyse_plane<T, 0, true, kToQ, false>(sm, P, sm + P.stg + P.stg_floats, sm + P.DY.base,
                                                                      P.DY.stride, 0, nt, tid, csync)
@@ -1382,8 +1416,15 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
             if (b + G < P.B) stage(plane_origin<GENERAL>(P, b + G, c) + strip_off, !dys);
             cp_async_commit();
             cluster_wait();  // every strip's X, S and halo rows ready
+        } else if (oct) {
+            cp_async_wait_all();     // this thread's chunks of the next x run
+            plane_sync<GENERAL, OCT>(P);  // both analyses complete in every CTA of the cluster
+            if (b + G < P.B) scatter_octet(sm, P.stg, P, crank, tid, nt);
+            __syncthreads();  // the octet buffer consumed
+            if (b + G < P.B) octet_run(dy, b + G);
+            cp_async_commit();
         } else {
-            plane_sync<GENERAL>(P);  // both analyses complete
+            plane_sync<GENERAL, OCT>(P);  // both analyses complete
             if (b + G < P.B) stage(plane_origin<GENERAL>(P, b + G, c) + strip_off, !dys);
             cp_async_commit();
         }
@@ -1391,6 +1432,11 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
             const int local = first + k;
             const int tr = fdiv(local, P.div_ntc[lvl]), tc = local - tr * P.ntc[lvl];
             corr_tile<K, TR, TC, DLD>(sm + wb + tr * TR * ws + tc * TC, ws, sm + db + tr * TR * dsd + tc * TC, dsd, acc);
+        }
+        if (oct) {
+            cp_async_wait_all();
+            __syncthreads();  // the next dy run complete
+            if (b + G < P.B) scatter_octet(sm, P.stg + P.stg_floats, P, crank, tid, nt);
         }
         if (dys) {
             __syncthreads();  // every dy tile read (dy is this CTA's own; no other CTA reads it)
@@ -1401,7 +1447,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
         }
     }
     cp_async_wait_all();
-    plane_sync<GENERAL>(P);  // the cluster leaves together
+    plane_sync<GENERAL, OCT>(P);  // the cluster leaves together
 
     // Fixed-order reduction of every class over its threads.
     float* red = sm + P.red;

@@ -60,10 +60,10 @@ struct Launch {
     }
 };
 
-template <int TR, typename T, bool BWD, bool GENERAL>
+template <int TR, typename T, bool BWD, bool GENERAL, bool OCT = false>
 cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
     static std::atomic<bool> done[kMaxDevices] = {};
-    auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD, GENERAL>;
+    auto* fn = wtconv_fused_kernel<WTC_K, TR, 4, T, BWD, GENERAL, OCT>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
     // Persistent grid: every resident CTA slot (cluster slot, for strips and
@@ -94,14 +94,14 @@ cudaError_t fused_typed(const Plan& P, const FusedArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <int TR, typename T, bool GENERAL>
+template <int TR, typename T, bool GENERAL, bool OCT = false>
 cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
     static std::atomic<bool> done[kMaxDevices] = {};
-    auto* fn = wtconv_bwdw_partial_kernel<WTC_K, TR, 4, T, GENERAL>;
+    auto* fn = wtconv_bwdw_partial_kernel<WTC_K, TR, 4, T, GENERAL, OCT>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
     Launch L(P, dim3(P.C * P.nstrips, P.groups), s);
-    if (P.nstrips > 1) {
+    if (cluster_ctas(P) > 1) {
         // A cluster that can never be resident is an error, not a hang.
         int clusters = 0;
         if ((e = cudaOccupancyMaxActiveClusters(&clusters, fn, &L.cfg)) != cudaSuccess) return e;
@@ -114,8 +114,10 @@ cudaError_t bwdw_typed(const Plan& P, const BwdwArgs& a, cudaStream_t s) {
 
 template <int TR, typename T>
 cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s) {
-    // The general instantiation for cluster strips, planes padded on chip
-    // and / or NHWC activations.
+    // NHWC channel octets, and the general instantiation for cluster
+    // strips, planes padded on chip and / or the NHWC gather.
+    if (P.oct)
+        return bwd ? fused_typed<TR, T, true, true, true>(P, a, s) : fused_typed<TR, T, false, true, true>(P, a, s);
     if (P.nstrips > 1 || P.padded || P.nhwc)
         return bwd ? fused_typed<TR, T, true, true>(P, a, s) : fused_typed<TR, T, false, true>(P, a, s);
     return bwd ? fused_typed<TR, T, true, false>(P, a, s) : fused_typed<TR, T, false, false>(P, a, s);
@@ -143,6 +145,8 @@ cudaError_t fused_tr(const Plan& P, int dtype, bool bwd, const FusedArgs& a, cud
 template <int TR>
 cudaError_t bwdw_tr(const Plan& P, int dtype, const BwdwArgs& a, cudaStream_t s) {
     const bool strips = P.nstrips > 1 || P.padded || P.nhwc;  // the general instantiation
+    if (P.oct)
+        return dtype == 0 ? bwdw_typed<TR, float, true, true>(P, a, s) : bwdw_typed<TR, __nv_bfloat16, true, true>(P, a, s);
     if (dtype == 0) return strips ? bwdw_typed<TR, float, true>(P, a, s) : bwdw_typed<TR, float, false>(P, a, s);
     return strips ? bwdw_typed<TR, __nv_bfloat16, true>(P, a, s) : bwdw_typed<TR, __nv_bfloat16, false>(P, a, s);
 }

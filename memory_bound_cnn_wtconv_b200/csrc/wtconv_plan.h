@@ -90,12 +90,13 @@ struct Plan {
     // gathered element by element, C elements apart; the general
     // instantiations and the one-pass backward only).
     int nhwc;
-    // NHWC channel octets (forward / input gradient on whole planes, C a
-    // multiple of 8): clusters of 8 CTAs, CTA r of a cluster holding channel
-    // 8o + r of the planes (b, octet o) the cluster walks.  Each CTA loads
-    // its run of opix pixels of the plane's 8 channels (8 * esize contiguous
-    // bytes a pixel) into its octet buffer at tbuf (stg_floats floats, pixel
-    // j at 8 * esize * j bytes) and scatters channel q to CTA q's staging.
+    // NHWC channel octets (whole planes, C a multiple of 8): clusters of 8
+    // CTAs, CTA r of a cluster holding channel 8o + r of the planes (b, octet
+    // o) the cluster walks.  Each CTA loads its run of opix pixels of the
+    // plane's 8 channels (8 * esize contiguous bytes a pixel) into its octet
+    // buffer at tbuf (stg_floats floats, pixel j at 8 * esize * j bytes) and
+    // scatters channel q to CTA q's staging (the weight gradient: the x run,
+    // then the dy run, through the same buffer).
     // The synthesis stores each output into the output octet buffer at obuf
     // (stg_floats floats) of the CTA that owns its pixel, as row r of
     // [8 channels][opix pixels] (stored format); the owner writes the 8

@@ -228,14 +228,15 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     // loaded once for the cluster's 8 planes instead of element by element
     // per plane.  Whole, unpadded planes whose pixels split into 8 runs of a
     // multiple of 4 pixels.
-    if (octets && (kind == kForward || kind == kBackwardInput) && P->nhwc && nstrips == 1 && !P->padded &&
-        d->C % 8 == 0 && ((long long)H * W) % 32 == 0) {
+    // The weight gradient's x and dy runs take the octet buffer in turn.
+    if (octets && (kind == kForward || kind == kBackwardInput || kind == kBackwardWeight) && P->nhwc &&
+        nstrips == 1 && !P->padded && !dy_stg && d->C % 8 == 0 && ((long long)H * W) % 32 == 0) {
         P->oct = 1;
         P->opix = H * W / 8;
         P->div_opix = make_fastdiv(P->opix);
         P->tbuf = (int)off;
         off += P->stg_floats;
-        if (L >= 1) {  // outputs of the synthesis (L = 0: the base tiles store y directly)
+        if (L >= 1 && kind != kBackwardWeight) {  // outputs of the synthesis (L = 0: the base tiles store y)
             P->obuf = (int)off;
             off += P->stg_floats;
         }
@@ -355,6 +356,10 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     if (kind == kBackwardWeight || kind == kBackward) off = std::max(off, (long long)P->nv + ncls * KK + 4);
     off = round4((int)std::min<long long>(off, 1LL << 30));
     if (off > kSmemLimitFloats) return WTCONV_ERR_UNSUPPORTED;
+    // The weight gradient's octets add two CTA barriers and a staging step
+    // after the tiles: measured slower than the gather at one CTA per SM
+    // (64 x 64, L = 4: 483 -> 534 us), faster at two (stage1: 178 -> 164 us).
+    if (P->oct && kind == kBackwardWeight && ctas_per_sm((int)off) < 2) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;
     if (kind == kBackwardWeight || kind == kBackward) {
         const long long slots = (long long)num_sms * resident_ctas(P->nthreads, P->smem_floats);

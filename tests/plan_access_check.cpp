@@ -395,6 +395,41 @@ void barrier_all(std::vector<Shadow>& shs) {
     for (auto& sh : shs) sh.barrier();
 }
 
+// NHWC channel octets.  The octet run of CTA r (pixels r*opix ..): 16-byte
+// chunks of whole pixels, from the last octet of the last batch element
+// (bounds), into the octet buffer once each.
+const int OCT = 400;  // tag of octet-buffer floats
+void replay_octet_load(Shadow& sh, const Plan& P, int r) {
+    const int cpp = P.esize / 2, H = P.H, W = P.W;
+    const long long total = (long long)P.B * H * W * P.C;  // NHWC elements
+    const int o = P.C / 8 - 1, b = P.B - 1;
+    if (P.tbuf % 4 || P.tbuf < P.stg) sh.fail("octet buffer", P.tbuf);
+    for (int ch = 0; ch < P.opix * cpp; ++ch) {
+        const int j = cpp == 2 ? ch >> 1 : ch, h = ch - j * cpp;
+        const long long e0 = ((long long)b * H * W + (long long)r * P.opix + j) * P.C + 8LL * o + 8 / cpp * h;
+        check_global(e0, total, "octet run first element");
+        check_global(e0 + 16 / P.esize - 1, total, "octet run last element");
+        if ((e0 * P.esize) % 16) sh.fail("octet chunk source not 16-byte aligned", e0);
+        for (int f = 0; f < 4; ++f) sh.write(P.tbuf + 4LL * ch + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
+    }
+}
+
+// Scatter of CTA r: its pixels' channel q into CTA q's staging at stg (tag
+// stag), four pixels a step (16 or 8 bytes a channel).
+void replay_octet_scatter(std::vector<Shadow>& shs, const Plan& P, int r, long long stg, int stag) {
+    Shadow& me = shs[r];
+    for (int f = 0; f < P.stg_floats; ++f) me.read(P.tbuf + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
+    const int per = 4 / P.esize;  // elements a staging float
+    if (stg % 4) me.fail("scattered staging not 16-byte aligned", stg);
+    for (int gq = 0; gq < P.opix / 4; ++gq) {
+        const long long e = (long long)r * P.opix + 4LL * gq;
+        if ((e * P.esize) % (4 * P.esize)) me.fail("scatter store misaligned", e);
+        for (int q = 0; q < 8; ++q)
+            for (long long f = e / per; f < (e + 4) / per; ++f)
+                shs[q].write(stg + f, stg, stg + P.stg_floats, stag, "scattered staging");
+    }
+}
+
 void check_fused(const wtconv_desc_t& d, Kind kind) {
     Plan P;
     const wtconv_status_t st = make_plan(&d, kind, kB200SMs, &P);
@@ -450,37 +485,8 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     std::vector<Shadow> shs(NC, Shadow(P.smem_floats));
     const long long all = P.smem_floats;
     if (P.grid < 1 || P.grid > (long long)P.B * P.C) shs[0].fail("grid", P.grid);
-    const int OCT = 400;  // tag of octet-buffer floats
-    // Octet run of CTA r (phase of the caller): 16-byte chunks of whole pixels
-    // from the last octet of the last batch element (bounds), into T once each.
-    auto octet_load = [&](Shadow& sh, int r) {
-        const int cpp = P.esize / 2;
-        const long long total = (long long)P.B * H * W * P.C;  // NHWC elements
-        const int o = P.C / 8 - 1, b = P.B - 1;
-        for (int ch = 0; ch < P.opix * cpp; ++ch) {
-            const int j = cpp == 2 ? ch >> 1 : ch, h = ch - j * cpp;
-            const long long e0 = ((long long)b * H * W + (long long)r * P.opix + j) * P.C + 8LL * o + 8 / cpp * h;
-            check_global(e0, total, "octet run first element");
-            check_global(e0 + 16 / P.esize - 1, total, "octet run last element");
-            if ((e0 * P.esize) % 16) sh.fail("octet chunk source not 16-byte aligned", e0);
-            for (int f = 0; f < 4; ++f)
-                sh.write(P.tbuf + 4LL * ch + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
-        }
-    };
-    // Scatter of CTA r: its pixels' channel q into CTA q's staging, four
-    // pixels a step (16 or 8 bytes a channel).
-    auto octet_scatter = [&](int r) {
-        Shadow& me = shs[r];
-        for (int f = 0; f < P.stg_floats; ++f) me.read(P.tbuf + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
-        const int per = 4 / P.esize;  // elements a staging float
-        for (int gq = 0; gq < P.opix / 4; ++gq) {
-            const long long e = (long long)r * P.opix + 4LL * gq;
-            if ((e * P.esize) % (4 * P.esize)) me.fail("scatter store misaligned", e);
-            for (int q = 0; q < 8; ++q)
-                for (long long f = e / per; f < (e + 4) / per; ++f)
-                    shs[q].write(P.stg + f, P.stg, P.stg + P.stg_floats, XT + 10, "scattered staging");
-        }
-    };
+    auto octet_load = [&](Shadow& sh, int r) { replay_octet_load(sh, P, r); };
+    auto octet_scatter = [&](int r) { replay_octet_scatter(shs, P, r, P.stg, XT + 10); };
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
     const long long ylo = P.Y.base, yhi = P.Y.base + (long long)P.ntr[kMaxL] * TR * P.Y.stride;
@@ -701,7 +707,15 @@ void check_bwdw(const wtconv_desc_t& d) {
     const int ncls = 1 + 4 * L, NS = P.nstrips;
     check_divs(P);
     check_div(P.div_w, W, (long long)(2 * p * 4) * W + 1, "W");
-    std::vector<Shadow> shs(NS, Shadow(P.smem_floats));
+    // NHWC channel octets: 8 CTAs a cluster on whole planes; the x run and
+    // then the dy run go through the one octet buffer.
+    const int NC = cluster_ctas(P);
+    if (P.oct && (!P.nhwc || NS != 1 || P.padded || P.dy_stg || P.C % 8 || P.opix * 8LL != (long long)H * W ||
+                  P.opix % 4 || P.tbuf < P.stg + 2LL * P.stg_floats || P.tbuf + (long long)P.stg_floats > P.smem_floats)) {
+        std::printf("FAIL weight-gradient octet plan\n");
+        std::exit(1);
+    }
+    std::vector<Shadow> shs(NC, Shadow(P.smem_floats));
     const int xrows = P.ntr[kMaxL] * TR + 2 * p;
     const long long xlo = P.X.base, xhi = P.X.base + (long long)xrows * P.X.stride;
     // dys: DY is the dy staging itself (strips of fp32 planes of whole tile
@@ -718,25 +732,44 @@ void check_bwdw(const wtconv_desc_t& d) {
     // Two planes in a row (the second must see the same zero padding), with
     // the kernel's barriers (cluster-wide with strips) as phase boundaries:
     //   stage(0) | analysis(0) | [strips: halo push(0), stage(1)] | [whole planes: stage(1)], correlation(0) | analysis(1) | ... | reduction
-    for (int r = 0; r < NS; ++r) {
-        shs[r].phase = "initial staging";
-        replay_stage(shs[r], P, P.stg, XT + 10, r);
-        replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
+    // Octets, per CTA r: x run | scatter x | dy run | scatter dy, each step
+    // behind a barrier.
+    auto octet_pair = [&](const char* what) {
+        for (int r = 0; r < NC; ++r) { shs[r].phase = what; replay_octet_load(shs[r], P, r); }
+        barrier_all(shs);
+        for (int r = 0; r < NC; ++r) replay_octet_scatter(shs, P, r, P.stg, XT + 10);
+        barrier_all(shs);
+        for (int r = 0; r < NC; ++r) replay_octet_load(shs[r], P, r);
+        barrier_all(shs);
+        for (int r = 0; r < NC; ++r) replay_octet_scatter(shs, P, r, P.stg + P.stg_floats, DYT + 10);
+    };
+    if (P.oct) {
+        octet_pair("initial octet runs");
+    } else {
+        for (int r = 0; r < NS; ++r) {
+            shs[r].phase = "initial staging";
+            replay_stage(shs[r], P, P.stg, XT + 10, r);
+            replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
+        }
     }
     for (int plane = 0; plane < 2; ++plane) {
         barrier_all(shs);
-        for (int r = 0; r < NS; ++r) {
+        for (int r = 0; r < NC; ++r) {
             Shadow& sh = shs[r];
+            if (P.oct && plane == 0) {
+                sh.phase = "next x run";
+                replay_octet_load(sh, P, r);
+            }
             sh.phase = "analysis";
-            g_rank = r;
+            g_rank = P.oct ? 0 : r;
             const int e0 = sh.epoch;
             replay_analyse(sh, P, P.stg, XT + 10, P.X.base + (long long)p * P.X.stride + p, P.X.stride, xlo, xhi, XT, P.S,
                            p, s_tag);
             g_copy_plane = !dys;
             replay_analyse(sh, P, P.stg + P.stg_floats, DYT + 10, P.DY.base, P.DY.stride, dlo, dhi, DYT, P.Q, 0, q_tag);
             g_copy_plane = true;
-            if (r + 1 < NS) sh.epoch = e0;
-            else for (int q = 0; q + 1 < NS; ++q) shs[q].epoch = sh.epoch;
+            if (r + 1 < NC) sh.epoch = e0;
+            else for (int q = 0; q + 1 < NC; ++q) shs[q].epoch = sh.epoch;
         }
         if (NS > 1) {
             barrier_all(shs);
@@ -744,16 +777,31 @@ void check_bwdw(const wtconv_desc_t& d) {
         } else {
             barrier_all(shs);
         }
-        for (int r = 0; r < NS; ++r) {
-            shs[r].phase = "staging";
-            if (plane == 0) {
-                replay_stage(shs[r], P, P.stg, XT + 10, r);
-                if (!dys) replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
+        if (P.oct) {
+            // Scatter the x run; behind a CTA barrier, the dy run (its
+            // scatter follows the correlation tiles).
+            for (int r = 0; r < NC; ++r) {
+                shs[r].phase = "x scatter";
+                if (plane == 0) replay_octet_scatter(shs, P, r, P.stg, XT + 10);
+            }
+            barrier_all(shs);
+            for (int r = 0; r < NC; ++r) {
+                shs[r].phase = "next dy run";
+                if (plane == 0) replay_octet_load(shs[r], P, r);
+            }
+        } else {
+            for (int r = 0; r < NS; ++r) {
+                shs[r].phase = "staging";
+                if (plane == 0) {
+                    replay_stage(shs[r], P, P.stg, XT + 10, r);
+                    if (!dys) replay_stage(shs[r], P, P.stg + P.stg_floats, DYT + 10, r);
+                }
             }
         }
         if (NS > 1) barrier_all(shs);
-        for (int r = 0; r < NS; ++r) {
-            Shadow& sh = shs[r];
+        for (int rr = 0; rr < NC; ++rr) {
+            Shadow& sh = shs[rr];
+            const int r = P.oct ? 0 : rr;  // strip of the CTA
             sh.phase = "correlation";
             int covered = 0;
             for (int tid = 0; tid < P.cls_thr[ncls]; ++tid)
@@ -790,10 +838,17 @@ void check_bwdw(const wtconv_desc_t& d) {
                 if (plane == 0) replay_stage(sh, P, P.stg + P.stg_floats, DYT + 10, r);
             }
         }
+        if (P.oct) {
+            barrier_all(shs);
+            for (int r = 0; r < NC; ++r) {
+                shs[r].phase = "dy scatter";
+                if (plane == 0) replay_octet_scatter(shs, P, r, P.stg + P.stg_floats, DYT + 10);
+            }
+        }
     }
     const long long red_end = (long long)P.red + (long long)P.nthreads * KK + P.nthreads;
     barrier_all(shs);
-    for (int r = 0; r < NS; ++r) {
+    for (int r = 0; r < NC; ++r) {
         Shadow& sh = shs[r];
         sh.phase = "reduction";
         if (red_end > P.smem_floats) sh.fail("reduction scratch", red_end);
@@ -803,7 +858,7 @@ void check_bwdw(const wtconv_desc_t& d) {
             sh.write(P.red + (long long)P.nthreads * KK + w, P.red, red_end, RED, "warp dy sums");
     }
     barrier_all(shs);
-    for (int r = 0; r < NS; ++r)
+    for (int r = 0; r < NC; ++r)
         for (int k2 = 0; k2 < ncls; ++k2)
             for (int th = P.cls_thr[k2]; th < P.cls_thr[k2 + 1]; ++th)
                 for (int t = 0; t < KK; ++t)
@@ -820,8 +875,9 @@ void check_bwdw(const wtconv_desc_t& d) {
     if ((long long)P.nthreads * KK + P.nthreads / 32 > P.smem_floats) sh.fail("sum-dy scratch", P.nthreads);
     if (P.nv != ncls * KK + 1) sh.fail("partial vector length", P.nv);
     if ((long long)P.nv + ncls * KK + 1 > P.smem_floats) sh.fail("final-step scratch", P.nv);
-    std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d (<= %d per thread), groups %d, strips %d%s\n",
-                P.smem_floats * 4, P.nthreads, TR, P.n_all_tiles, P.tpt, P.groups, NS, dys ? ", dy read from staging" : "");
+    std::printf("bwdw: smem %d B, threads %d, TR %d, tiles %d (<= %d per thread), groups %d, strips %d%s%s\n",
+                P.smem_floats * 4, P.nthreads, TR, P.n_all_tiles, P.tpt, P.groups, NS, dys ? ", dy read from staging" : "",
+                P.oct ? ", channel octets" : "");
 }
 
 // Fused backward: dx conv tiles (the input-gradient pass: dy in X / S, dx

@@ -86,7 +86,10 @@ def test_every_access_in_bounds_nhwc(checker, case):
     whole = H % m == 0 and W % m == 0 and H * W <= 64 * 64
     octets = C % 8 == 0 and whole and (H * W) % 32 == 0
     fused = [l for l in r.stdout.splitlines() if l.startswith("fused(kind")]
-    assert fused and all(("channel octets" in l) == octets for l in fused), r.stdout
+    assert len(fused) == 2 and all(("channel octets" in l) == octets for l in fused), r.stdout
+    # The weight gradient takes octets only where it still runs two CTAs an SM (the stage-1 planes).
+    bwdw = next(l for l in r.stdout.splitlines() if l.startswith("bwdw:"))
+    assert ("channel octets" in bwdw) == (octets and (H, W) != (64, 64)), bwdw
 
 
 @pytest.mark.parametrize("case,strips,alias", [
