@@ -106,8 +106,8 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
                   "wtconv_launch.h", "wtconv_api.cu", "wtconv_k1.cu", "wtconv_k3.cu", "wtconv_k5.cu", "wtconv_k7.cu")
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
-    ("stage1", "bwd_w"): (79151104.0, "wtconv_bwdw_partial_kernel",
-                          "d2dfb44563fee3de439b3a2f8fd5532fdcb5b794b0a09e70e280fc51b1e067ac",
+    ("stage1", "bwd_w"): (79382784.0, "wtconv_bwdw_partial_kernel",
+                          "c6cb26197c39e2bf7460f8f25b2e6bef1c5e738999cb531e5cb85f3d8094bb39",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 
@@ -394,14 +394,14 @@ class Workload:
         return times, wall, clk
 
 
-def call_record(case, per_call_ms: dict, peak: float) -> dict:
+def call_record(case, per_call_ms: dict, peak: float, nhwc: bool = False) -> dict:
     """GB/s, HBM fraction and FP32-pipe fraction of each call and of the step."""
     mb = modeled_bytes(case)
     alu_peak = SMS * FP32_LANES * 2 * MAX_SM_MHZ * 1e6 / 1e12
     step_ms = sum(per_call_ms[k] for k in mb)
     gbs = sum(mb.values()) / (step_ms * 1e-3) / 1e9
     return {
-        "workload": workload_name(case),
+        "workload": workload_name(case, nhwc),
         "us_per_call": {k: per_call_ms[k] * 1e3 for k in mb},
         "gbs_per_call": {k: mb[k] / (per_call_ms[k] * 1e-3) / 1e9 for k in mb},
         "hbm_frac_per_call": {k: mb[k] / (per_call_ms[k] * 1e-3) / 1e9 / peak for k in mb},
@@ -494,7 +494,7 @@ def run_ours(args, case):
                 "peak_source": peak_kind,
                 "bytes_per_launch": mb[dom]}
 
-    rec = call_record(case, per_call, peak)
+    rec = call_record(case, per_call, peak, args.nhwc)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -539,9 +539,7 @@ def run_ours(args, case):
             del_wl = Workload(wcase, dev, stream, 0, 1, nhwc=nhwc)
             t2, _, _ = del_wl.time_calls(del_wl.calls, K, args.warmup, flush)
             pc2 = {n: median(v) for n, v in t2.items()}
-            other[name] = call_record(wcase, pc2, peak)
-            if nhwc:
-                other[name]["workload"] += " (NHWC activations)"
+            other[name] = call_record(wcase, pc2, peak, nhwc)
             other[name]["fused_backward"], n_launch = backward_record(del_wl, wcase, pc2, KF, flush)
             line["gpu_launches"] += K * 3 + n_launch
             del del_wl

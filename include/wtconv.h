@@ -89,8 +89,11 @@ typedef enum {
 typedef enum { WTCONV_F32 = 0, WTCONV_BF16 = 1 } wtconv_dtype_t; /* activation storage */
 
 /* Activation layout: NCHW, or NHWC (channels last: element (b, c, h, w) at
- * ((b*H + h)*W + w)*C + c).  NHWC planes are gathered and scattered
- * element by element (C elements apart) by the same on-chip pass; the
+ * ((b*H + h)*W + w)*C + c).  With NHWC, where C is a multiple of 8 and a
+ * plane is held whole (H*W a multiple of 32, no zero padding), clusters of
+ * 8 CTAs move the 8 channels of a pixel as one 16- or 32-byte run; other
+ * NHWC planes are gathered and scattered element by element (C elements
+ * apart).  The on-chip pass, and so every result bit, is the NCHW one; the
  * parameters' layouts do not change. */
 typedef enum { WTCONV_NCHW = 0, WTCONV_NHWC = 1 } wtconv_layout_t;
 
