@@ -107,7 +107,7 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
     ("stage1", "bwd_w"): (79382784.0, "wtconv_bwdw_partial_kernel",
-                          "c6cb26197c39e2bf7460f8f25b2e6bef1c5e738999cb531e5cb85f3d8094bb39",
+                          "275e23ace03be6304c58ab3b487ed7c7b2de81471a7fd8b16778be94c963987f",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 

@@ -627,8 +627,9 @@ __device__ __forceinline__ float analyse_plane(float* sm, const Plan& P, const f
 // Planes split into strips across a thread-block cluster.
 // ---------------------------------------------------------------------------
 // Barrier of everything that shares a plane: the CTA, or the whole cluster
-// when the plane is split into strips (then it also orders the shared-memory
-// accesses of the cluster's CTAs to each other's strips).
+// when the plane is split into strips or the cluster holds a channel octet
+// (then it also orders the shared-memory accesses of the cluster's CTAs to
+// each other's buffers).
 template <bool GENERAL, bool OCT = false>
 __device__ __forceinline__ void plane_sync(const Plan& P) {
     if constexpr (OCT) {
@@ -1048,8 +1049,11 @@ struct FusedCtx {
 // Within a phase the buffers written (A: X, S, weights; B: staging, Q, Y) and
 // the buffers read (A: staging, Q, Y; B: S, X, weights) are disjoint.
 // GENERAL: planes split into strips across a cluster and / or zero-padded on
-// chip (a separate instantiation, so the common walk of whole planes that
-// are multiples of 2^L carries none of that code).
+// chip, or NHWC activations (a separate instantiation, so the common walk of
+// whole planes that are multiples of 2^L carries none of that code).  OCT
+// (with GENERAL): NHWC channel octets, the barriers cluster-wide, staging
+// by octet runs and scatters, outputs through the owners' output octet
+// buffers, written out in phase B of the next plane.
 template <int K, int TR, int TC, typename T, bool BWD, bool GENERAL, bool OCT = false>
 __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kFusedMaxThreads, GENERAL ? 1 : 2) wtconv_fused_kernel(
     const T* __restrict__ x, const float* __restrict__ base_w, const float* __restrict__ base_b,
@@ -1304,8 +1308,11 @@ __device__ __forceinline__ void finish_channel_if_last(float* sm, const Plan& P,
 // threads in a fixed order and writes one partial vector (plus sum dy).
 // ---------------------------------------------------------------------------
 // GENERAL: the plane is split into strips across a cluster and / or
-// zero-padded on chip (a separate instantiation, so whole-plane walks keep
-// every register for the sums).
+// zero-padded on chip, or NHWC activations (a separate instantiation, so
+// whole-plane walks keep every register for the sums).  OCT (with GENERAL):
+// NHWC channel octets, clusters of the 8 channels of an octet; the x run and
+// then the dy run of the next plane go through the octet buffer (the dy run
+// loaded during the correlation tiles and scattered after them).
 template <int K, int TR, int TC, typename T, bool GENERAL, bool OCT = false>
 __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, GENERAL ? 1 : 2) wtconv_bwdw_partial_kernel(
     const T* __restrict__ x, const T* __restrict__ dy, float* __restrict__ part, const GradArgs ga, const Plan P) {
