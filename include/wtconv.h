@@ -90,7 +90,7 @@ typedef enum { WTCONV_F32 = 0, WTCONV_BF16 = 1 } wtconv_dtype_t; /* activation s
 
 /* Activation layout: NCHW, or NHWC (channels last: element (b, c, h, w) at
  * ((b*H + h)*W + w)*C + c).  With NHWC, where C is a multiple of 8 and a
- * plane is held whole (H*W a multiple of 32, no zero padding), clusters of
+ * plane is held whole (H*W a multiple of 16, no zero padding), clusters of
  * 8 CTAs move the 8 channels of a pixel as one 16- or 32-byte run; other
  * NHWC planes are gathered and scattered element by element (C elements
  * apart).  The on-chip pass, and so every result bit, is the NCHW one; the

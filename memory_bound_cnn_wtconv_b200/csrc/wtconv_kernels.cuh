@@ -677,22 +677,41 @@ __device__ __forceinline__ void st_cluster2(unsigned addr, unsigned a, unsigned 
     asm volatile("st.shared::cluster.v2.b32 [%0], {%1, %2};\n" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
+__device__ __forceinline__ void st_cluster1(unsigned addr, unsigned a) {
+    asm volatile("st.shared::cluster.b32 [%0], %1;\n" ::"r"(addr), "r"(a) : "memory");
+}
+
 // NHWC channel octets: 4 outputs of pixels px .. px + 3 (one row; px a
 // multiple of 4) of this CTA's channel into the output octet buffer of the
-// CTA that owns them.  oaddr: this CTA's output octet buffer (shared window
-// address); ocol: byte offset of this CTA's channel row in it.
+// CTA that owns them (og = 2: each pixel pair to its own owner, since a
+// run boundary may fall between them).  oaddr: this CTA's output octet
+// buffer (shared window address); ocol: byte offset of this CTA's channel
+// row in it.
 template <typename T>
 __device__ __forceinline__ void st_octet_out(const Plan& P, unsigned oaddr, unsigned ocol, int px, float4 v) {
-    const int owner = fdiv(px, P.div_opix), j = px - owner * P.opix;
-    unsigned dst;
-    asm("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(dst) : "r"(oaddr), "r"(owner));
-    dst += ocol + (unsigned)j * (unsigned)sizeof(T);
+    auto dst_of = [&](int x) {
+        const int owner = fdiv(x, P.div_opix), j = x - owner * P.opix;
+        unsigned d;
+        asm("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(d) : "r"(oaddr), "r"(owner));
+        return d + ocol + (unsigned)j * (unsigned)sizeof(T);
+    };
     if constexpr (sizeof(T) == 4) {
-        st_cluster4(dst, v);
+        if (P.og == 4) {
+            st_cluster4(dst_of(px), v);
+        } else {
+            st_cluster2(dst_of(px), __float_as_uint(v.x), __float_as_uint(v.y));
+            st_cluster2(dst_of(px + 2), __float_as_uint(v.z), __float_as_uint(v.w));
+        }
     } else {
         __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
         __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
-        st_cluster2(dst, *reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+        const unsigned ua = *reinterpret_cast<uint32_t*>(&a), ub = *reinterpret_cast<uint32_t*>(&b);
+        if (P.og == 4) {
+            st_cluster2(dst_of(px), ua, ub);
+        } else {
+            st_cluster1(dst_of(px), ua);
+            st_cluster1(dst_of(px + 2), ub);
+        }
     }
 }
 
@@ -906,9 +925,10 @@ __device__ __forceinline__ void load_octet(float* tb, const void* src, const Pla
 }
 
 // scatter_octet: channel q of the octet buffer's pixels into CTA q's
-// staging at `stg` (pixel crank * opix + j of the plane, stored format), four pixels
-// a step as one 16-byte (fp32) or 8-byte (bf16) distributed shared store per
-// channel.  The cluster barrier after it makes the stores visible.
+// staging at `stg` (pixel crank * opix + j of the plane, stored format), og
+// pixels a step as one distributed shared store per channel (og = 4: 16
+// bytes in fp32, 8 in bf16; og = 2: 8 or 4).  The cluster barrier after it
+// makes the stores visible.
 __device__ __forceinline__ void scatter_octet(float* sm, int stg, const Plan& P, int crank, int tid, int nt) {
     const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm + stg));
     // CTA q's copy of the staging (mapped per store: few registers live, the
@@ -919,6 +939,33 @@ __device__ __forceinline__ void scatter_octet(float* sm, int stg, const Plan& P,
         return a;
     };
     const float* tb = sm + P.tbuf;
+    if (P.og == 2) {
+        // Two pixels a step: 8-byte (fp32) or 4-byte (bf16) stores.
+        for (int gq = tid; gq < (P.opix >> 1); gq += nt) {
+            const int j = 2 * gq;
+            const unsigned off = (unsigned)(crank * P.opix + j) * (unsigned)P.esize;
+            if (P.esize == 4) {
+                const float4* t = reinterpret_cast<const float4*>(tb) + 2 * j;
+                const float4 a0 = t[0], b0 = t[1], a1 = t[2], b1 = t[3];
+                st_cluster2(remote(0) + off, __float_as_uint(a0.x), __float_as_uint(a1.x));
+                st_cluster2(remote(1) + off, __float_as_uint(a0.y), __float_as_uint(a1.y));
+                st_cluster2(remote(2) + off, __float_as_uint(a0.z), __float_as_uint(a1.z));
+                st_cluster2(remote(3) + off, __float_as_uint(a0.w), __float_as_uint(a1.w));
+                st_cluster2(remote(4) + off, __float_as_uint(b0.x), __float_as_uint(b1.x));
+                st_cluster2(remote(5) + off, __float_as_uint(b0.y), __float_as_uint(b1.y));
+                st_cluster2(remote(6) + off, __float_as_uint(b0.z), __float_as_uint(b1.z));
+                st_cluster2(remote(7) + off, __float_as_uint(b0.w), __float_as_uint(b1.w));
+            } else {
+                const uint4* t = reinterpret_cast<const uint4*>(tb) + j;
+                const uint4 r0 = t[0], r1 = t[1];
+                const unsigned w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    st_cluster1(remote(q) + off, __byte_perm(w0[q >> 1], w1[q >> 1], (q & 1) ? 0x7632u : 0x5410u));
+            }
+        }
+        return;
+    }
     const int ng = P.opix >> 2;
     for (int gq = tid; gq < ng; gq += nt) {
         const int j = 4 * gq;
@@ -953,14 +1000,45 @@ __device__ __forceinline__ void scatter_octet(float* sm, int stg, const Plan& P,
 }
 
 // stream_octet_out: this CTA's pixels (crank * opix + j) of the output
-// octet buffer ([8 channels][opix pixels], stored format) to y, the 8
-// channels of a pixel as one 32-byte (fp32) or 16-byte (bf16) run; `dst` is
-// channel 8o of pixel 0 of the plane's batch element.
+// octet buffer ([8 channels][opix pixels], stored format) to y, og pixels a
+// step, the 8 channels of a pixel as one 32-byte (fp32) or 16-byte (bf16)
+// run; `dst` is channel 8o of pixel 0 of the plane's batch element.
 template <typename T>
 __device__ __forceinline__ void stream_octet_out(const float* sm, const Plan& P, T* dst, int crank, int tid, int nt) {
     const size_t pstride = (size_t)P.C;
     T* g = dst + (size_t)crank * P.opix * pstride;
     const T* ob = reinterpret_cast<const T*>(sm + P.obuf);
+    if (P.og == 2) {
+        // Two pixels a step.
+        for (int gq = tid; gq < (P.opix >> 1); gq += nt) {
+            const int j = 2 * gq;
+            if constexpr (sizeof(T) == 4) {
+                float2 c[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) c[q] = *reinterpret_cast<const float2*>(ob + (size_t)q * P.opix + j);
+                float* o = reinterpret_cast<float*>(g + (size_t)j * pstride);
+                *reinterpret_cast<float4*>(o) = make_float4(c[0].x, c[1].x, c[2].x, c[3].x);
+                *reinterpret_cast<float4*>(o + 4) = make_float4(c[4].x, c[5].x, c[6].x, c[7].x);
+                *reinterpret_cast<float4*>(o + pstride) = make_float4(c[0].y, c[1].y, c[2].y, c[3].y);
+                *reinterpret_cast<float4*>(o + pstride + 4) = make_float4(c[4].y, c[5].y, c[6].y, c[7].y);
+            } else {
+                unsigned c[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) c[q] = *reinterpret_cast<const unsigned*>(ob + (size_t)q * P.opix + j);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const unsigned sel = i ? 0x7632u : 0x5410u;
+                    uint4 v;
+                    v.x = __byte_perm(c[0], c[1], sel);
+                    v.y = __byte_perm(c[2], c[3], sel);
+                    v.z = __byte_perm(c[4], c[5], sel);
+                    v.w = __byte_perm(c[6], c[7], sel);
+                    *reinterpret_cast<uint4*>(g + (size_t)(j + i) * pstride) = v;
+                }
+            }
+        }
+        return;
+    }
     const int ng = P.opix >> 2;
     for (int gq = tid; gq < ng; gq += nt) {
         const int j = 4 * gq;

@@ -101,7 +101,9 @@ struct Plan {
     // (stg_floats floats) of the CTA that owns its pixel, as row r of
     // [8 channels][opix pixels] (stored format); the owner writes the 8
     // channels of its pixels as whole runs.
-    int oct, opix, tbuf, obuf;
+    // og: pixels a scatter / write-out step moves (4, or 2 where opix is not
+    // a multiple of 4).
+    int oct, opix, tbuf, obuf, og;
     FastDiv div_opix;
     int parts;           // weight gradient: partial vectors per channel (groups * nstrips)
     int TR, TC;          // output tile: TR rows x TC cols per thread (TC = 4: two column pairs)

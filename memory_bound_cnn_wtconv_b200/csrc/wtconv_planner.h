@@ -226,13 +226,15 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     }
     // NHWC channel octets: a pixel's 8 channels are one 16- or 32-byte run,
     // loaded once for the cluster's 8 planes instead of element by element
-    // per plane.  Whole, unpadded planes whose pixels split into 8 runs of a
-    // multiple of 4 pixels.
+    // per plane.  Whole, unpadded planes whose pixels split into 8 runs of an
+    // even number of pixels (moved 4 at a time, or 2 where the run is not a
+    // multiple of 4: 28 x 28 planes, 98 pixels a run).
     // The weight gradient's x and dy runs take the octet buffer in turn.
     if (octets && (kind == kForward || kind == kBackwardInput || kind == kBackwardWeight) && P->nhwc &&
-        nstrips == 1 && !P->padded && !dy_stg && d->C % 8 == 0 && ((long long)H * W) % 32 == 0) {
+        nstrips == 1 && !P->padded && !dy_stg && d->C % 8 == 0 && ((long long)H * W) % 16 == 0) {
         P->oct = 1;
         P->opix = H * W / 8;
+        P->og = P->opix % 4 == 0 ? 4 : 2;
         P->div_opix = make_fastdiv(P->opix);
         P->tbuf = (int)off;
         off += P->stg_floats;

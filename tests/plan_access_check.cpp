@@ -415,17 +415,18 @@ void replay_octet_load(Shadow& sh, const Plan& P, int r) {
 }
 
 // Scatter of CTA r: its pixels' channel q into CTA q's staging at stg (tag
-// stag), four pixels a step (16 or 8 bytes a channel).
+// stag), og pixels a step (og * esize bytes a channel, aligned to that).
 void replay_octet_scatter(std::vector<Shadow>& shs, const Plan& P, int r, long long stg, int stag) {
     Shadow& me = shs[r];
     for (int f = 0; f < P.stg_floats; ++f) me.read(P.tbuf + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
-    const int per = 4 / P.esize;  // elements a staging float
+    const int per = 4 / P.esize, og = P.og;  // elements a staging float; pixels a step
     if (stg % 4) me.fail("scattered staging not 16-byte aligned", stg);
-    for (int gq = 0; gq < P.opix / 4; ++gq) {
-        const long long e = (long long)r * P.opix + 4LL * gq;
-        if ((e * P.esize) % (4 * P.esize)) me.fail("scatter store misaligned", e);
+    if (og != (P.opix % 4 == 0 ? 4 : 2) || P.opix % og) me.fail("octet step", og);
+    for (int gq = 0; gq < P.opix / og; ++gq) {
+        const long long e = (long long)r * P.opix + (long long)og * gq;
+        if ((e * P.esize) % (og * P.esize)) me.fail("scatter store misaligned", e);
         for (int q = 0; q < 8; ++q)
-            for (long long f = e / per; f < (e + 4) / per; ++f)
+            for (long long f = e / per; f < (e + og) / per; ++f)
                 shs[q].write(stg + f, stg, stg + P.stg_floats, stag, "scattered staging");
     }
 }
@@ -471,13 +472,13 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     // staging filled by the cluster's scatters from the octet buffers.
     const int NC = cluster_ctas(P);
     if (P.oct) {
-        if (!P.nhwc || NS != 1 || P.padded || P.C % 8 || P.opix * 8LL != (long long)H * W || P.opix % 4 ||
+        if (!P.nhwc || NS != 1 || P.padded || P.C % 8 || P.opix * 8LL != (long long)H * W || P.opix % 2 ||
             P.tbuf % 4 || P.tbuf < P.stg + P.stg_floats || P.tbuf + (long long)P.stg_floats > P.smem_floats ||
             (kind != kForward && kind != kBackwardInput)) {
             std::printf("FAIL octet plan: opix %d tbuf %d stg %d smem %d\n", P.opix, P.tbuf, P.stg, P.smem_floats);
             std::exit(1);
         }
-    } else if (P.nhwc && kind != kBackward && NS == 1 && !P.padded && P.C % 8 == 0 && ((long long)H * W) % 32 == 0 &&
+    } else if (P.nhwc && kind != kBackward && NS == 1 && !P.padded && P.C % 8 == 0 && ((long long)H * W) % 16 == 0 &&
                P.smem_floats + (long long)P.stg_floats <= kSmemLimitFloats && (kind == kForward || kind == kBackwardInput)) {
         std::printf("FAIL octet plan not taken where it fits\n");
         std::exit(1);
@@ -501,14 +502,18 @@ void check_fused(const wtconv_desc_t& d, Kind kind) {
     const bool oct_out = P.oct && L >= 1;
     if (oct_out && (P.obuf % 4 || P.obuf < P.tbuf + P.stg_floats || P.obuf + (long long)P.stg_floats > P.smem_floats))
         shs[0].fail("output octet buffer", P.obuf);
-    auto octet_out = [&](int r, int px) {
-        const int owner = (int)fastdiv_host((uint32_t)px, P.div_opix), j = px - owner * P.opix;
-        if (owner != px / P.opix || owner < 0 || owner >= 8) shs[r].fail("output owner", px);
-        const long long e = (long long)r * P.opix + j;  // element of the owner's buffer
-        if ((e * P.esize) % (4 * P.esize)) shs[r].fail("output octet store misaligned", e);
-        const int per = 4 / P.esize;
-        for (long long f = e / per; f < (e + 4) / per; ++f)
-            shs[owner].write(P.obuf + f, P.obuf, P.obuf + P.stg_floats, OUT, "output octet buffer");
+    // Four outputs from pixel px (og = 2: two pixel pairs, each to its own owner).
+    auto octet_out = [&](int r, int px4) {
+        for (int px = px4; px < px4 + 4; px += P.og) {
+            const int owner = (int)fastdiv_host((uint32_t)px, P.div_opix), j = px - owner * P.opix;
+            if (owner != px / P.opix || owner < 0 || owner >= 8) shs[r].fail("output owner", px);
+            if ((px + P.og - 1) / P.opix != owner) shs[r].fail("output store crosses a run", px);
+            const long long e = (long long)r * P.opix + j;  // element of the owner's buffer
+            if ((e * P.esize) % (P.og * P.esize)) shs[r].fail("output octet store misaligned", e);
+            const int per = 4 / P.esize;
+            for (long long f = e / per; f < (e + P.og) / per; ++f)
+                shs[owner].write(P.obuf + f, P.obuf, P.obuf + P.stg_floats, OUT, "output octet buffer");
+        }
     };
     // The owner's pass over its buffer: every float read, its pixels' 8
     // channels stored in y (last octet of the last batch element: bounds).
@@ -711,7 +716,7 @@ void check_bwdw(const wtconv_desc_t& d) {
     // then the dy run go through the one octet buffer.
     const int NC = cluster_ctas(P);
     if (P.oct && (!P.nhwc || NS != 1 || P.padded || P.dy_stg || P.C % 8 || P.opix * 8LL != (long long)H * W ||
-                  P.opix % 4 || P.tbuf < P.stg + 2LL * P.stg_floats || P.tbuf + (long long)P.stg_floats > P.smem_floats)) {
+                  P.opix % 2 || P.tbuf < P.stg + 2LL * P.stg_floats || P.tbuf + (long long)P.stg_floats > P.smem_floats)) {
         std::printf("FAIL weight-gradient octet plan\n");
         std::exit(1);
     }

@@ -360,6 +360,10 @@ NHWC_SMALL = [
     Case("nhwc_octets_L0_k7", 2, 16, 56, 56, 7, 0, "f32", 65, "normal", "normal"),
     Case("nhwc_octets_k1_bf16", 5, 8, 16, 16, 1, 2, "bf16", 66, "normal", "normal"),
     Case("nhwc_octets_64_L4", 1, 24, 64, 64, 5, 4, "f32", 67, "normal", "normal"),
+    # runs of an even number of pixels that is not a multiple of 4 (98 at 28x28, 30 at 20x12)
+    Case("nhwc_octets_28_stage2_plane", 3, 16, 28, 28, 5, 2, "f32", 69, "normal", "normal"),
+    Case("nhwc_octets_28_bf16_L0", 2, 8, 28, 28, 3, 0, "bf16", 70, "normal", "normal"),
+    Case("nhwc_octets_20x12_bf16", 5, 8, 20, 12, 3, 1, "bf16", 71, "uniform", "normal"),
 ]
 NHWC_OCTETS = [c for c in NHWC_SMALL if c.name.startswith("nhwc_octets")]
 
@@ -370,14 +374,14 @@ def test_nhwc_small_case_all_outputs(oracle, case):
 
 
 @pytest.mark.parametrize("mode", ["auto", "one_pass"])
-@pytest.mark.parametrize("case", NHWC_SMALL[:8] + NHWC_OCTETS[:2], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", NHWC_SMALL[:8] + NHWC_OCTETS[:2] + NHWC_OCTETS[-2:], ids=lambda c: c.name)
 def test_nhwc_small_case_fused_backward(oracle, case, mode):
     if mode == "one_pass" and not _one_pass_plan_exists(case, nhwc=True):
         pytest.skip("planes split into cluster strips have no one-pass plan")
     check_full(oracle, case, ("bwd_in", "bwd_w"), fused_bwd=mode, nhwc=True)
 
 
-@pytest.mark.parametrize("case", [STAGE1, TRAIN_BF16], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", [STAGE1, STAGE2, TRAIN_BF16], ids=lambda c: c.name)
 def test_nhwc_full_size_workloads_sampled(oracle, case):
     check_sampled(oracle, case, nhwc=True)
 
@@ -385,6 +389,7 @@ def test_nhwc_full_size_workloads_sampled(oracle, case):
 @pytest.mark.parametrize("case", [
     Case("nhwc_vs_nchw", 4, 6, 40, 36, 5, 3, "f32", 62, "normal", "normal"),
     Case("nhwc_vs_nchw_octets", 3, 16, 32, 32, 5, 3, "f32", 68, "normal", "normal"),
+    Case("nhwc_vs_nchw_octets_28", 3, 16, 28, 28, 5, 2, "f32", 72, "normal", "normal"),
 ], ids=lambda c: c.name)
 def test_nhwc_matches_nchw_bitwise(case):
     # Same on-chip arithmetic in the same order: the layouts must agree bit for bit

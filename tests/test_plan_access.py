@@ -71,6 +71,9 @@ NHWC = [
     # channel octets (C a multiple of 8, whole planes of a multiple of 32 pixels)
     (3, 16, 56, 56, 5, 3, 0), (2, 8, 32, 32, 3, 2, 1), (2, 16, 56, 56, 7, 0, 0), (5, 8, 16, 16, 1, 2, 1),
     (1, 24, 64, 64, 5, 4, 0), (2, 8, 8, 8, 5, 1, 0), (32, 96, 56, 56, 5, 3, 0), (64, 96, 56, 56, 5, 3, 1),
+    # runs of an even number of pixels that is not a multiple of 4 (two pixels a step)
+    (3, 16, 28, 28, 5, 2, 0), (2, 8, 28, 28, 3, 2, 1), (32, 192, 28, 28, 5, 2, 0), (2, 8, 28, 28, 7, 0, 0),
+    (2, 8, 12, 12, 3, 1, 1), (5, 8, 20, 12, 3, 1, 0),
 ]
 
 
@@ -79,12 +82,12 @@ def test_every_access_in_bounds_nhwc(checker, case):
     r = subprocess.run([checker, *map(str, case), "1"], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip().endswith("OK") and "each addressed once" in r.stdout, \
         r.stdout + r.stderr
-    # Channel octets exactly where C is a multiple of 8 on whole planes of a multiple of 32 pixels
+    # Channel octets exactly where C is a multiple of 8 on whole planes of a multiple of 16 pixels
     # (every case here fits the octet buffer).
     B, C, H, W, k, L, _ = case
     m = 1 << L
     whole = H % m == 0 and W % m == 0 and H * W <= 64 * 64
-    octets = C % 8 == 0 and whole and (H * W) % 32 == 0
+    octets = C % 8 == 0 and whole and (H * W) % 16 == 0
     fused = [l for l in r.stdout.splitlines() if l.startswith("fused(kind")]
     assert len(fused) == 2 and all(("channel octets" in l) == octets for l in fused), r.stdout
     # The weight gradient takes octets only where it still runs two CTAs an SM (the stage-1 planes).
