@@ -106,8 +106,8 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
                   "wtconv_launch.h", "wtconv_api.cu", "wtconv_k1.cu", "wtconv_k3.cu", "wtconv_k5.cu", "wtconv_k7.cu")
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
-    ("stage1", "bwd_w"): (79382784.0, "wtconv_bwdw_partial_kernel",
-                          "275e23ace03be6304c58ab3b487ed7c7b2de81471a7fd8b16778be94c963987f",
+    ("stage1", "bwd_w"): (79442176.0, "wtconv_bwdw_partial_kernel",
+                          "eda254bffe737d55937000ba15c42b2ae4c82792990c3d9943f2a2485fb64ede",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 
