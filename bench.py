@@ -323,8 +323,8 @@ class Workload:
         self.dx = torch.empty_like(g["dy"])
         self.grads = grads = {k: torch.empty_like(g[k]) for k in ("base_w", "base_b", "base_scale", "wt_w", "wt_scale")}
         self.flat = torch.empty(sum(v.numel() for v in grads.values()), device=dev)
-        self.ws = torch.empty(max(16, wt.workspace_bytes(g["x"].shape, case.k, L, g["x"].dtype)), dtype=torch.uint8,
-                              device=dev)
+        self.ws = torch.empty(max(16, wt.workspace_bytes(g["x"].shape, case.k, L, g["x"].dtype, channels_last=nhwc)),
+                              dtype=torch.uint8, device=dev)
 
         def fwd():
             wt.forward(g["x"], g["base_w"], g["base_b"], g["base_scale"], g["wt_w"], g["wt_scale"], L, y=self.y,

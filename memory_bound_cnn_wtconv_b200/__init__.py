@@ -165,9 +165,14 @@ def _params(x, base_w, base_b, base_scale, wt_w, wt_scale, L):
     return k
 
 
-def workspace_bytes(x_shape, k: int, L: int, dtype=torch.float32) -> int:
+def workspace_bytes(x_shape, k: int, L: int, dtype=torch.float32, channels_last: bool = False) -> int:
+    """Workspace of ``backward_weight`` / ``backward`` for activations of this
+    shape (NCHW), dtype and layout (``channels_last``: NHWC).  An NHWC plan
+    never needs more than the NCHW one of the same shape (its channel-octet
+    buffers only lower the batch groups), so the NCHW size serves both."""
     B, C, H, W = x_shape
-    d = Desc(B, C, H, W, int(k), int(L), F32 if dtype == torch.float32 else BF16)
+    d = Desc(B, C, H, W, int(k), int(L), F32 if dtype == torch.float32 else BF16,
+             NHWC if channels_last else NCHW)
     return int(load_library().wtconv_workspace_bytes(ctypes.byref(d)))
 
 
