@@ -56,8 +56,7 @@
  *     workspace size) are made for the SM count of the device current at the
  *     call and for the descriptor's layout; make the wtconv_workspace_bytes
  *     call and the call that uses the workspace with the same device current.
- *     An NHWC plan never needs more workspace than the NCHW plan of the same
- *     shape, so a workspace sized for NCHW serves both layouts.
+ *     Both layouts of a shape need the same workspace size.
  *   - L = 0 is the base branch only; wt_w and wt_scale may then be NULL.
  *   - Calls are reentrant; apart from the fixed scratch array of
  *     wtconv_backward_weight_noalloc (see there), the library holds no

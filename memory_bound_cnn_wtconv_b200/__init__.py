@@ -167,9 +167,8 @@ def _params(x, base_w, base_b, base_scale, wt_w, wt_scale, L):
 
 def workspace_bytes(x_shape, k: int, L: int, dtype=torch.float32, channels_last: bool = False) -> int:
     """Workspace of ``backward_weight`` / ``backward`` for activations of this
-    shape (NCHW), dtype and layout (``channels_last``: NHWC).  An NHWC plan
-    never needs more than the NCHW one of the same shape (its channel-octet
-    buffers only lower the batch groups), so the NCHW size serves both."""
+    shape (NCHW), dtype and layout (``channels_last``: NHWC; both layouts of a
+    shape need the same size)."""
     B, C, H, W = x_shape
     d = Desc(B, C, H, W, int(k), int(L), F32 if dtype == torch.float32 else BF16,
              NHWC if channels_last else NCHW)

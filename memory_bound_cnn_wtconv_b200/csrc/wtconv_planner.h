@@ -364,7 +364,11 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     if (P->oct && kind == kBackwardWeight && ctas_per_sm((int)off) < 2) return WTCONV_ERR_UNSUPPORTED;
     P->smem_floats = (int)off;
     if (kind == kBackwardWeight || kind == kBackward) {
-        const long long slots = (long long)num_sms * resident_ctas(P->nthreads, P->smem_floats);
+        // The groups (and so the workspace) are chosen without the octet
+        // buffer, so that both layouts of a shape get the same workspace size
+        // (the choice is not monotone in the slots).
+        const int smem_groups = P->smem_floats - (P->oct ? P->stg_floats : 0);
+        const long long slots = (long long)num_sms * resident_ctas(P->nthreads, smem_groups);
         P->groups = pick_groups(P->B, P->C * nstrips, slots);
         P->parts = P->groups * nstrips;
     } else {

@@ -72,16 +72,16 @@ def test_sizes_not_multiples_of_2L_are_planned(cuda_lib, kw):
 @pytest.mark.parametrize("shape,k,L,dtype", [
     ((32, 96, 56, 56), 5, 3, 0), ((64, 96, 56, 56), 5, 3, 1), ((32, 192, 28, 28), 5, 2, 0),
     ((256, 64, 32, 32), 3, 1, 0), ((64, 16, 56, 56), 7, 0, 0), ((1024, 64, 32, 32), 3, 1, 0),
-    ((2, 5, 56, 56), 5, 3, 0),
+    ((2, 5, 56, 56), 5, 3, 0), ((4, 192, 28, 28), 5, 2, 0), ((6, 192, 32, 32), 3, 1, 1),
 ])
-def test_nhwc_workspace_never_exceeds_nchw(cuda_lib, shape, k, L, dtype):
-    # Channel octets only lower the weight gradient's batch groups (more shared memory a CTA),
-    # so a workspace sized for NCHW also serves NHWC; the binding's query takes the layout.
+def test_nhwc_workspace_equals_nchw(cuda_lib, shape, k, L, dtype):
+    # The weight gradient's batch groups are chosen without the channel-octet buffer, so both
+    # layouts of a shape need the same workspace; the binding's query takes the layout.
     import torch
     B, C, H, W = shape
     nchw = cuda_lib.wtconv_workspace_bytes(ctypes.byref(_desc(B, C, H, W, k, L, dtype, 0)))
     nhwc = cuda_lib.wtconv_workspace_bytes(ctypes.byref(_desc(B, C, H, W, k, L, dtype, 1)))
-    assert 0 < nhwc <= nchw
+    assert 0 < nhwc == nchw
     tdt = torch.bfloat16 if dtype else torch.float32
     assert w.workspace_bytes(shape, k, L, tdt, channels_last=True) == nhwc
     assert w.workspace_bytes(shape, k, L, tdt) == nchw
