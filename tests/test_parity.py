@@ -364,6 +364,9 @@ NHWC_SMALL = [
     Case("nhwc_octets_28_stage2_plane", 3, 16, 28, 28, 5, 2, "f32", 69, "normal", "normal"),
     Case("nhwc_octets_28_bf16_L0", 2, 8, 28, 28, 3, 0, "bf16", 70, "normal", "normal"),
     Case("nhwc_octets_20x12_bf16", 5, 8, 20, 12, 3, 1, "bf16", 71, "uniform", "normal"),
+    # levels past the pyramid (L = 5: CTA barriers inside the analysis of an octet walk)
+    Case("nhwc_octets_64_L5", 2, 8, 64, 64, 3, 5, "f32", 73, "normal", "normal"),
+    Case("nhwc_octets_32_L5_bf16", 2, 16, 32, 32, 5, 5, "bf16", 74, "normal", "normal"),
 ]
 NHWC_OCTETS = [c for c in NHWC_SMALL if c.name.startswith("nhwc_octets")]
 
@@ -374,7 +377,7 @@ def test_nhwc_small_case_all_outputs(oracle, case):
 
 
 @pytest.mark.parametrize("mode", ["auto", "one_pass"])
-@pytest.mark.parametrize("case", NHWC_SMALL[:8] + NHWC_OCTETS[:2] + NHWC_OCTETS[-2:], ids=lambda c: c.name)
+@pytest.mark.parametrize("case", NHWC_SMALL[:8] + NHWC_OCTETS[:2] + NHWC_OCTETS[-4:], ids=lambda c: c.name)
 def test_nhwc_small_case_fused_backward(oracle, case, mode):
     if mode == "one_pass" and not _one_pass_plan_exists(case, nhwc=True):
         pytest.skip("planes split into cluster strips have no one-pass plan")

@@ -74,6 +74,8 @@ NHWC = [
     # runs of an even number of pixels that is not a multiple of 4 (two pixels a step)
     (3, 16, 28, 28, 5, 2, 0), (2, 8, 28, 28, 3, 2, 1), (32, 192, 28, 28, 5, 2, 0), (2, 8, 28, 28, 7, 0, 0),
     (2, 8, 12, 12, 3, 1, 1), (5, 8, 20, 12, 3, 1, 0),
+    # levels past the pyramid
+    (2, 8, 64, 64, 3, 5, 0), (2, 16, 32, 32, 5, 5, 1),
 ]
 
 
