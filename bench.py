@@ -107,7 +107,7 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
     ("stage1", "bwd_w"): (79442176.0, "wtconv_bwdw_partial_kernel",
-                          "d942cf440744de65b0ea40840758f593d945ba8e31ee6852098a7c0c3456a552",
+                          "579a36cf751da5b5ede5d7d557a6bb168ab2f96946f73b3150435933cfa9d38a",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 

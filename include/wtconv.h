@@ -164,9 +164,9 @@ wtconv_status_t wtconv_backward_weight(const wtconv_desc_t *d, const void *x, co
  * wtconv_backward_one_pass where its plan exists and the planner's cost
  * (conv-tile rows on the busiest SM sub-partition) is below that of the two
  * passes together, or equal to it while one of the two passes runs one CTA
- * per SM, or the activations are NHWC and both passes would gather them
- * element by element (no channel octets); else wtconv_backward_input then
- * wtconv_backward_weight.  Both paths give the same results.  dx:
+ * per SM, or the activations are NHWC and either both passes would gather
+ * them element by element or the one pass holds them on channel octets;
+ * else wtconv_backward_input then wtconv_backward_weight.  Both paths give the same results.  dx:
  * [B][C][H][W] in desc->dtype, not overlapping x or dy.  Workspace as for
  * wtconv_backward_weight.  Every argument is checked before either pass is
  * enqueued. */

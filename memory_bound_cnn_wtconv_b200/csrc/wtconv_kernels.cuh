@@ -924,12 +924,14 @@ __device__ __forceinline__ void load_octet(float* tb, const void* src, const Pla
     }
 }
 
-// scatter_octet: channel q of the octet buffer's pixels into CTA q's
+// scatter_octet: channel q of the octet buffer's pixels (the buffer at
+// tbuf, P.tbuf if negative) into CTA q's
 // staging at `stg` (pixel crank * opix + j of the plane, stored format), og
 // pixels a step as one distributed shared store per channel (og = 4: 16
 // bytes in fp32, 8 in bf16; og = 2: 8 or 4).  The cluster barrier after it
 // makes the stores visible.
-__device__ __forceinline__ void scatter_octet(float* sm, int stg, const Plan& P, int crank, int tid, int nt) {
+__device__ __forceinline__ void scatter_octet(float* sm, int stg, const Plan& P, int crank, int tid, int nt,
+                                              int tbuf = -1) {
     const unsigned local = static_cast<unsigned>(__cvta_generic_to_shared(sm + stg));
     // CTA q's copy of the staging (mapped per store: few registers live, the
     // weight gradient's correlation sums stay in registers meanwhile).
@@ -938,7 +940,7 @@ __device__ __forceinline__ void scatter_octet(float* sm, int stg, const Plan& P,
         asm("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(local), "r"(q));
         return a;
     };
-    const float* tb = sm + P.tbuf;
+    const float* tb = sm + (tbuf >= 0 ? tbuf : P.tbuf);
     if (P.og == 2) {
         // Two pixels a step: 8-byte (fp32) or 4-byte (bf16) stores.
         for (int gq = tid; gq < (P.opix >> 1); gq += nt) {
@@ -1573,7 +1575,7 @@ __global__ void __launch_bounds__(GENERAL ? kStripMaxThreads : kBwdwMaxThreads, 
 // registers.  After the walk: the last plane's synthesis, then the
 // fixed-order reduction of the correlation sums into one partial vector.
 // ---------------------------------------------------------------------------
-template <int K, int TR, int TC, typename T>
+template <int K, int TR, int TC, typename T, bool OCT = false>
 __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
     const T* __restrict__ x, const T* __restrict__ dy, const float* __restrict__ base_w,
     const float* __restrict__ base_b, const float* __restrict__ base_scale, const float* __restrict__ wt_w,
@@ -1595,12 +1597,37 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
     zero_smem(sm, P.smem_floats, tid, nt);
     __syncthreads();
     cx.fold(c, nt, tid);  // the channel is fixed: dx weights folded once
-    if (g < P.B) {
-        const size_t off = plane_origin<true>(P, g, c);
-        stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
-        stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
+    // NHWC channel octets: clusters of the 8 channels of an octet (rank c mod
+    // 8).  The x run and the dy run of the next plane are loaded into the two
+    // octet buffers during phase A and scattered in phase B by the dx-tile
+    // threads, which also write out the previous plane's dx from the output
+    // octet buffer; the plane barriers are cluster-wide.
+    const int crank = OCT ? (int)cg::this_cluster().block_rank() : 0;
+    const size_t oct_off = (size_t)(c - crank);  // channel 8o: NHWC element offset of the octet
+    auto octet_runs = [&](int b) {
+        load_octet(sm + P.tbuf, x + plane_origin<true>(P, b, 0) + oct_off, P, crank, tid, nt);
+        load_octet(sm + P.tbuf + P.stg_floats, dy + plane_origin<true>(P, b, 0) + oct_off, P, crank, tid, nt);
+    };
+    auto octet_scatter = [&](int ptid, int np) {
+        scatter_octet(sm, P.stg, P, crank, ptid, np, P.tbuf);
+        scatter_octet(sm, P.stg + P.stg_floats, P, crank, ptid, np, P.tbuf + P.stg_floats);
+    };
+    const unsigned oaddr = (OCT && P.L >= 1) ? static_cast<unsigned>(__cvta_generic_to_shared(sm + P.obuf)) : 0u;
+    const unsigned ocol = (unsigned)crank * (unsigned)P.opix * (unsigned)sizeof(T);
+    if constexpr (OCT) {
+        if (g < P.B) octet_runs(g);
+        cp_async_commit();
+        cp_async_wait_all();
+        cg::this_cluster().sync();  // every CTA of the cluster running, its shared memory zeroed; the runs complete
+        if (g < P.B) octet_scatter(tid, nt);
+    } else {
+        if (g < P.B) {
+            const size_t off = plane_origin<true>(P, g, c);
+            stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
+            stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
+        }
+        cp_async_commit();
     }
-    cp_async_commit();
 
     const bool x_side = tid < P.an_split;
     float* XS0 = sm + P.XS.base + p * P.XS.stride + p;
@@ -1648,8 +1675,15 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
         for (int b = g;; b += G) {
             const bool have = b < P.B;
             cp_async_wait_all();
-            __syncthreads();  // staged pair complete; every tile of the previous plane done
+            // Staged pair complete (octets: scattered by every CTA of the
+            // cluster, and the previous output write-outs done); every tile
+            // of the previous plane done.
+            if constexpr (OCT) cg::this_cluster().sync(); else __syncthreads();
             // Phase A.
+            if constexpr (OCT) {
+                if (have && b + G < P.B) octet_runs(b + G);  // the buffers' last readers are behind the barrier above
+                cp_async_commit();
+            }
             if (have) {
                 if (x_side) {
                     analyse_plane<T, p, false, kToSS>(sm, P, sm + P.stg, XS0, P.XS.stride, p, P.an_split, tid, csync);
@@ -1664,17 +1698,33 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
             }
             if (prev_b >= 0 && P.L >= 1) {
                 T* yp = dx + plane_origin<true>(P, prev_b, c);
-                for (int t = tid; t < P.n_fin; t += nt) synth_item<T, true>(sm, P, yp, t, myrows);
+                for (int t = tid; t < P.n_fin; t += nt) synth_item<T, true>(sm, P, yp, t, myrows, oaddr, ocol);
             }
             if (!have) break;
-            __syncthreads();  // both analyses complete; the previous plane's Q and Y consumed
-            // Phase B.
-            if (b + G < P.B) {
-                const size_t off = plane_origin<true>(P, b + G, c);
-                stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
-                stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
+            // Both analyses complete (octets: in every CTA of the cluster, and
+            // their dx outputs of the previous plane stored); the previous
+            // plane's Q and Y consumed.
+            if constexpr (OCT) {
+                cp_async_wait_all();
+                cg::this_cluster().sync();
+            } else {
+                __syncthreads();
             }
-            cp_async_commit();
+            // Phase B.
+            if constexpr (OCT) {
+                if constexpr (!CORR) {
+                    if (b + G < P.B) octet_scatter(tid, P.corr0);
+                    if (P.L >= 1 && prev_b >= 0)
+                        stream_octet_out<T>(sm, P, dx + plane_origin<true>(P, prev_b, 0) + oct_off, crank, tid, P.corr0);
+                }
+            } else {
+                if (b + G < P.B) {
+                    const size_t off = plane_origin<true>(P, b + G, c);
+                    stage_rows(sm + P.stg, x + off, P, myrows, tid, nt);
+                    stage_rows(sm + P.stg + P.stg_floats, dy + off, P, myrows, tid, nt);
+                }
+                cp_async_commit();
+            }
             if constexpr (!CORR) {
                 if (job.valid) {
                     float w[KK];
@@ -1709,7 +1759,14 @@ __global__ void __launch_bounds__(kBwdMaxThreads, 1) wtconv_backward_kernel(
             prev_b = b;
         }
         cp_async_wait_all();
-        __syncthreads();  // the last synthesis done: the buffers are free
+        if constexpr (OCT) {
+            cg::this_cluster().sync();  // the last plane's dx outputs in every owner's buffer
+            if constexpr (!CORR) {
+                if (P.L >= 1 && prev_b >= 0)
+                    stream_octet_out<T>(sm, P, dx + plane_origin<true>(P, prev_b, 0) + oct_off, crank, tid, P.corr0);
+            }
+        }
+        __syncthreads();  // the last synthesis (and write-out) done: the buffers are free
         if constexpr (CORR) {
             if (ct < ncorr) {
 #pragma unroll

@@ -123,16 +123,27 @@ cudaError_t fused_t(const Plan& P, bool bwd, const FusedArgs& a, cudaStream_t s)
     return bwd ? fused_typed<TR, T, true, false>(P, a, s) : fused_typed<TR, T, false, false>(P, a, s);
 }
 
-template <int TR, typename T>
+template <int TR, typename T, bool OCT = false>
 cudaError_t bwd_typed(const Plan& P, const BwdArgs& a, cudaStream_t s) {
     static std::atomic<bool> done[kMaxDevices] = {};
-    auto* fn = wtconv_backward_kernel<WTC_K, TR, 4, T>;
+    auto* fn = wtconv_backward_kernel<WTC_K, TR, 4, T, OCT>;
     cudaError_t e = opt_in_smem(fn, done);
     if (e != cudaSuccess) return e;
     const GradArgs& g = a.ga;
-    fn<<<dim3(P.C, P.groups), P.nthreads, (size_t)P.smem_floats * 4, s>>>(
-        static_cast<const T*>(a.x), static_cast<const T*>(a.dy), g.base_w, g.base_b, g.base_scale, g.wt_w,
-        g.wt_scale, static_cast<T*>(a.dx), a.part, g, P);
+    if constexpr (OCT) {
+        // Clusters of the 8 channels of an octet (grid.x = C, a multiple of 8).
+        Launch L(P, dim3(P.C, P.groups), s);
+        int clusters = 0;
+        if ((e = cudaOccupancyMaxActiveClusters(&clusters, fn, &L.cfg)) != cudaSuccess) return e;
+        if (clusters < 1) return cudaErrorInvalidConfiguration;
+        e = cudaLaunchKernelEx(&L.cfg, fn, static_cast<const T*>(a.x), static_cast<const T*>(a.dy), g.base_w,
+                               g.base_b, g.base_scale, g.wt_w, g.wt_scale, static_cast<T*>(a.dx), a.part, g, P);
+        if (e != cudaSuccess) return e;
+    } else {
+        fn<<<dim3(P.C, P.groups), P.nthreads, (size_t)P.smem_floats * 4, s>>>(
+            static_cast<const T*>(a.x), static_cast<const T*>(a.dy), g.base_w, g.base_b, g.base_scale, g.wt_w,
+            g.wt_scale, static_cast<T*>(a.dx), a.part, g, P);
+    }
     return cudaGetLastError();
 }
 
@@ -164,8 +175,12 @@ cudaError_t WTC_CAT(launch_fused_k, WTC_K)(const Plan& P, int dtype, bool bwd, c
 
 cudaError_t WTC_CAT(launch_bwd_k, WTC_K)(const Plan& P, int dtype, const BwdArgs& a, cudaStream_t s) {
     switch (P.TR) {
-        case 7: return dtype == 0 ? bwd_typed<7, float>(P, a, s) : bwd_typed<7, __nv_bfloat16>(P, a, s);
-        case 8: return dtype == 0 ? bwd_typed<8, float>(P, a, s) : bwd_typed<8, __nv_bfloat16>(P, a, s);
+        case 7:
+            if (P.oct) return dtype == 0 ? bwd_typed<7, float, true>(P, a, s) : bwd_typed<7, __nv_bfloat16, true>(P, a, s);
+            return dtype == 0 ? bwd_typed<7, float>(P, a, s) : bwd_typed<7, __nv_bfloat16>(P, a, s);
+        case 8:
+            if (P.oct) return dtype == 0 ? bwd_typed<8, float, true>(P, a, s) : bwd_typed<8, __nv_bfloat16, true>(P, a, s);
+            return dtype == 0 ? bwd_typed<8, float>(P, a, s) : bwd_typed<8, __nv_bfloat16>(P, a, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -229,19 +229,24 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
     // per plane.  Whole, unpadded planes whose pixels split into 8 runs of an
     // even number of pixels (moved 4 at a time, or 2 where the run is not a
     // multiple of 4: 28 x 28 planes, 98 pixels a run).
-    // The weight gradient's x and dy runs take the octet buffer in turn.
-    if (octets && (kind == kForward || kind == kBackwardInput || kind == kBackwardWeight) && P->nhwc &&
-        nstrips == 1 && !P->padded && !dy_stg && d->C % 8 == 0 && ((long long)H * W) % 16 == 0) {
+    // The weight gradient's x and dy runs take the octet buffer in turn; the
+    // fused backward holds both (x run at tbuf, dy run after it).
+    // The fused backward only with 4 pixels a step (28 x 28 planes, 2 a
+    // step, measured 149.5 -> 191.5 us against its gather).
+    long long oct_floats = 0;  // shared memory of the octet buffers
+    if (octets && P->nhwc && nstrips == 1 && !P->padded && !dy_stg && d->C % 8 == 0 &&
+        ((long long)H * W) % (kind == kBackward ? 32 : 16) == 0) {
         P->oct = 1;
         P->opix = H * W / 8;
         P->og = P->opix % 4 == 0 ? 4 : 2;
         P->div_opix = make_fastdiv(P->opix);
         P->tbuf = (int)off;
-        off += P->stg_floats;
-        if (L >= 1 && kind != kBackwardWeight) {  // outputs of the synthesis (L = 0: the base tiles store y)
-            P->obuf = (int)off;
-            off += P->stg_floats;
+        oct_floats = (kind == kBackward ? 2LL : 1LL) * P->stg_floats;
+        if (L >= 1 && kind != kBackwardWeight) {  // outputs of the synthesis (L = 0: the base tiles store them)
+            P->obuf = (int)(off + oct_floats);
+            oct_floats += P->stg_floats;
         }
+        off += oct_floats;
     }
     if (dy_stg) {
         // The dy staging holds the strip as H rows of W floats: the DY layout
@@ -367,7 +372,7 @@ inline wtconv_status_t make_plan_for(const wtconv_desc_t* d, Kind kind, int TR, 
         // The groups (and so the workspace) are chosen without the octet
         // buffer, so that both layouts of a shape get the same workspace size
         // (the choice is not monotone in the slots).
-        const int smem_groups = P->smem_floats - (P->oct ? P->stg_floats : 0);
+        const int smem_groups = P->smem_floats - (int)oct_floats;
         const long long slots = (long long)num_sms * resident_ctas(P->nthreads, smem_groups);
         P->groups = pick_groups(P->B, P->C * nstrips, slots);
         P->parts = P->groups * nstrips;
@@ -411,9 +416,15 @@ inline double plan_cost(const Plan& P, Kind kind) {
 // (32x32 at L = 4, k = 3 is within 1% either way).  NHWC planes that both
 // passes gather element by element (no channel octets): the one pass, which
 // gathers x and dy once where the two passes gather dy twice; measured 1.2-1.45x
-// faster at six shapes (16x16 to 64x64, L = 1 to 4, C = 6 to 100).
+// faster at six shapes (16x16 to 64x64, L = 1 to 4, C = 6 to 100).  NHWC planes
+// that the one pass holds on channel octets: the one pass (below).
 inline bool prefer_one_pass(const Plan& P, const Plan& Pin, const Plan& Pw) {
     if (P.nhwc && !Pin.oct && !Pw.oct) return true;
+    // NHWC with the one pass on channel octets: measured 0.51-1.01x the two
+    // passes at eleven shapes (32x32 to 64x64, L = 1 to 4, stage1 fp32 and
+    // bf16), the one pass moving one run of x and one of dy a plane where the
+    // two passes move dy twice.
+    if (P.nhwc && P.oct) return true;
     const double c1 = plan_cost(P, kBackward);
     const double c2 = plan_cost(Pin, kBackwardInput) + plan_cost(Pw, kBackwardWeight);
     if (c1 < c2 * (1.0 - 1e-9)) return true;

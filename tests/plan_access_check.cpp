@@ -399,26 +399,28 @@ void barrier_all(std::vector<Shadow>& shs) {
 // chunks of whole pixels, from the last octet of the last batch element
 // (bounds), into the octet buffer once each.
 const int OCT = 400;  // tag of octet-buffer floats
-void replay_octet_load(Shadow& sh, const Plan& P, int r) {
+void replay_octet_load(Shadow& sh, const Plan& P, int r, long long tbuf = -1) {
     const int cpp = P.esize / 2, H = P.H, W = P.W;
     const long long total = (long long)P.B * H * W * P.C;  // NHWC elements
     const int o = P.C / 8 - 1, b = P.B - 1;
-    if (P.tbuf % 4 || P.tbuf < P.stg) sh.fail("octet buffer", P.tbuf);
+    if (tbuf < 0) tbuf = P.tbuf;
+    if (tbuf % 4 || tbuf < P.stg) sh.fail("octet buffer", tbuf);
     for (int ch = 0; ch < P.opix * cpp; ++ch) {
         const int j = cpp == 2 ? ch >> 1 : ch, h = ch - j * cpp;
         const long long e0 = ((long long)b * H * W + (long long)r * P.opix + j) * P.C + 8LL * o + 8 / cpp * h;
         check_global(e0, total, "octet run first element");
         check_global(e0 + 16 / P.esize - 1, total, "octet run last element");
         if ((e0 * P.esize) % 16) sh.fail("octet chunk source not 16-byte aligned", e0);
-        for (int f = 0; f < 4; ++f) sh.write(P.tbuf + 4LL * ch + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
+        for (int f = 0; f < 4; ++f) sh.write(tbuf + 4LL * ch + f, tbuf, tbuf + P.stg_floats, OCT, "octet buffer");
     }
 }
 
 // Scatter of CTA r: its pixels' channel q into CTA q's staging at stg (tag
 // stag), og pixels a step (og * esize bytes a channel, aligned to that).
-void replay_octet_scatter(std::vector<Shadow>& shs, const Plan& P, int r, long long stg, int stag) {
+void replay_octet_scatter(std::vector<Shadow>& shs, const Plan& P, int r, long long stg, int stag, long long tbuf = -1) {
     Shadow& me = shs[r];
-    for (int f = 0; f < P.stg_floats; ++f) me.read(P.tbuf + f, P.tbuf, P.tbuf + P.stg_floats, OCT, "octet buffer");
+    if (tbuf < 0) tbuf = P.tbuf;
+    for (int f = 0; f < P.stg_floats; ++f) me.read(tbuf + f, tbuf, tbuf + P.stg_floats, OCT, "octet buffer");
     const int per = 4 / P.esize, og = P.og;  // elements a staging float; pixels a step
     if (stg % 4) me.fail("scattered staging not 16-byte aligned", stg);
     if (og != (P.opix % 4 == 0 ? 4 : 2) || P.opix % og) me.fail("octet step", og);
@@ -888,6 +890,99 @@ void check_bwdw(const wtconv_desc_t& d) {
 // Fused backward: dx conv tiles (the input-gradient pass: dy in X / S, dx
 // in Q / Y) and correlation tiles (x windows in XS / SS against dy tiles at
 // the interior of X / S) in one walk.
+// Fused backward on NHWC channel octets: the octet buffers (x run at tbuf,
+// dy run after it, the dx output buffer at obuf) and the two stagings of the
+// cluster's 8 CTAs, over two planes: every staging float written once a
+// plane by the cluster's scatters, every output float once by the owners'
+// synthesis items, no phase race on them, and the global runs in bounds.
+// The rest of the walk is the whole-plane one, replayed by check_bwd.
+void check_bwd_octets(const Plan& P) {
+    const int H = P.H, W = P.W, L = P.L, per = 4 / P.esize;
+    const long long T0 = P.tbuf, T1 = P.tbuf + P.stg_floats;
+    std::vector<Shadow> shs(8, Shadow(P.smem_floats));
+    if (P.tbuf < P.stg + 2LL * P.stg_floats || (L >= 1 && P.obuf != P.tbuf + 2LL * P.stg_floats) ||
+        (L >= 1 ? P.obuf : T1) + (long long)P.stg_floats > P.smem_floats || P.opix * 8LL != (long long)H * W ||
+        P.og != (P.opix % 4 == 0 ? 4 : 2) || P.opix % P.og)
+        shs[0].fail("octet buffers of the fused backward", P.tbuf);
+    const int OUTB = 402;
+    auto loads = [&](const char* what) {
+        for (int r = 0; r < 8; ++r) {
+            shs[r].phase = what;
+            replay_octet_load(shs[r], P, r, T0);
+            replay_octet_load(shs[r], P, r, T1);
+        }
+    };
+    auto scatters = [&]() {
+        for (int r = 0; r < 8; ++r) {
+            shs[r].phase = "scatter";
+            replay_octet_scatter(shs, P, r, P.stg, XT + 10, T0);
+            replay_octet_scatter(shs, P, r, P.stg + P.stg_floats, DYT + 10, T1);
+        }
+    };
+    auto analyses = [&]() {  // every staging float read by the two analyses
+        for (int r = 0; r < 8; ++r) {
+            shs[r].phase = "analysis reads";
+            for (int f = 0; f < P.stg_floats; ++f) {
+                shs[r].read(P.stg + f, P.stg, P.stg + P.stg_floats, XT + 10, "x staging");
+                shs[r].read(P.stg + P.stg_floats + f, P.stg + P.stg_floats, P.stg + 2LL * P.stg_floats, DYT + 10,
+                            "dy staging");
+            }
+        }
+    };
+    auto outputs = [&]() {  // the synthesis items of every CTA into the owners' output buffers
+        if (L < 1) return;
+        for (int r = 0; r < 8; ++r) {
+            shs[r].phase = "dx outputs";
+            for (int t = 0; t < P.n_fin; ++t) {
+                const int i = t / (W / 4), q = t - i * (W / 4);
+                for (int rr = 0; rr < 2; ++rr)
+                    for (int px = (2 * i + rr) * W + 4 * q; px < (2 * i + rr) * W + 4 * q + 4; px += P.og) {
+                        const int owner = (int)fastdiv_host((uint32_t)px, P.div_opix), j = px - owner * P.opix;
+                        if (owner != px / P.opix || owner >= 8 || (px + P.og - 1) / P.opix != owner)
+                            shs[r].fail("dx output owner", px);
+                        const long long e = (long long)r * P.opix + j;
+                        for (long long f = e / per; f < (e + P.og) / per; ++f)
+                            shs[owner].write(P.obuf + f, P.obuf, P.obuf + P.stg_floats, OUTB, "dx output buffer");
+                    }
+            }
+        }
+    };
+    auto streams = [&]() {
+        if (L < 1) return;
+        const long long total = (long long)P.B * H * W * P.C;
+        for (int r = 0; r < 8; ++r) {
+            shs[r].phase = "dx write-out";
+            for (int f = 0; f < P.stg_floats; ++f)
+                shs[r].read(P.obuf + f, P.obuf, P.obuf + P.stg_floats, OUTB, "dx output buffer");
+            for (int j = 0; j < P.opix; ++j) {
+                const long long e0 = ((long long)(P.B - 1) * H * W + (long long)r * P.opix + j) * P.C + 8LL * (P.C / 8 - 1);
+                check_global(e0 + 7, total, "dx output run");
+            }
+        }
+    };
+    // prologue: runs, cluster barrier, scatters; then per plane: [barrier] A:
+    // next runs, analyses, outputs of the previous plane; [barrier] B:
+    // scatters, write-out of the previous plane; the last outputs behind a
+    // final barrier.
+    loads("initial runs");
+    barrier_all(shs);
+    scatters();
+    for (int plane = 0; plane <= 2; ++plane) {
+        barrier_all(shs);
+        if (plane < 2) {
+            if (plane + 1 < 2) loads("next runs");
+            analyses();
+        }
+        if (plane > 0) outputs();
+        if (plane == 2) break;
+        barrier_all(shs);
+        if (plane + 1 < 2) scatters();
+        if (plane > 0) streams();
+    }
+    barrier_all(shs);
+    streams();
+}
+
 void check_bwd(const wtconv_desc_t& d) {
     Plan P;
     const wtconv_status_t st = make_plan(&d, kBackward, kB200SMs, &P);
@@ -905,6 +1000,7 @@ void check_bwd(const wtconv_desc_t& d) {
     Shadow sh(P.smem_floats);
     const long long all = P.smem_floats;
     if (P.nstrips != 1) sh.fail("strips in the fused backward", P.nstrips);
+    if (P.oct) check_bwd_octets(P);
     if (P.nthreads > kBwdMaxThreads || P.nthreads % 32 || P.corr0 % 32 || P.corr0 < P.tile_end) sh.fail("threads", P.nthreads);
     const int ncorr = P.cls_thr[ncls];
     if (P.corr0 + ncorr > P.nthreads) sh.fail("correlation threads", ncorr);
@@ -1055,8 +1151,9 @@ void check_bwd(const wtconv_desc_t& d) {
     Plan Pin, Pw;
     const bool one = make_plan(&d, kBackwardInput, kB200SMs, &Pin) == WTCONV_OK &&
                      make_plan(&d, kBackwardWeight, kB200SMs, &Pw) == WTCONV_OK && prefer_one_pass(P, Pin, Pw);
-    std::printf("bwd: smem %d B, threads %d (%d conv + %d correlation), TR %d, groups %d, library picks %s\n",
-                P.smem_floats * 4, P.nthreads, P.corr0, ncorr, TR, P.groups, one ? "one pass" : "two passes");
+    std::printf("bwd: smem %d B, threads %d (%d conv + %d correlation), TR %d, groups %d, library picks %s%s\n",
+                P.smem_floats * 4, P.nthreads, P.corr0, ncorr, TR, P.groups, one ? "one pass" : "two passes",
+                P.oct ? ", channel octets" : "");
 }
 
 // NHWC: the kernels address element e (plane-relative, row-major over the
