@@ -107,7 +107,7 @@ KERNEL_SOURCES = ("wtconv_kernels.cuh", "wtconv_kinst.cuh", "wtconv_plan.h", "wt
 MEASURED_TRAFFIC = {
     # (workload, call): (bytes per launch, kernel, source digest, profile)
     ("stage1", "bwd_w"): (79442176.0, "wtconv_bwdw_partial_kernel",
-                          "579a36cf751da5b5ede5d7d557a6bb168ab2f96946f73b3150435933cfa9d38a",
+                          "3955a401d12ac3da446d06c2d26f646631dd5e28b326d479e49c854035394e2e",
                           "profiles/wtconv_bwdw_partial_kernel_stage1.md"),
 }
 

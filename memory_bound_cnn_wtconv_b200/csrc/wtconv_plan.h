@@ -96,9 +96,11 @@ struct Plan {
     // plane's 8 channels (8 * esize contiguous bytes a pixel) into its octet
     // buffer at tbuf (stg_floats floats, pixel j at 8 * esize * j bytes) and
     // scatters channel q to CTA q's staging (the weight gradient: the x run,
-    // then the dy run, through the same buffer).
-    // The synthesis stores each output into the output octet buffer at obuf
-    // (stg_floats floats) of the CTA that owns its pixel, as row r of
+    // then the dy run, through the same buffer; the fused backward: the x
+    // run at tbuf and the dy run at tbuf + stg_floats).
+    // The synthesis (forward, input gradient, fused backward) stores each
+    // output into the output octet buffer at obuf (stg_floats floats) of the
+    // CTA that owns its pixel, as row r of
     // [8 channels][opix pixels] (stored format); the owner writes the 8
     // channels of its pixels as whole runs.
     // og: pixels a scatter / write-out step moves (4, or 2 where opix is not
